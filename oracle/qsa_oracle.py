@@ -1,0 +1,278 @@
+"""Plain CPU oracle of the QSA (Qwen Sparse Attention) decode hot path.
+
+TEST INFRASTRUCTURE ONLY. Only tests/, __graft_entry__.smoke() and bench.py's
+CPU-baseline / reference leg may import or call this module. The product path
+(the CUDA library and its Python binding) never imports it and shares no code
+with it; the only module both sides use is `synth` (seeded inputs, no method
+arithmetic).
+
+Everything is float64 numpy, written for a reader to check against the pages by
+eye: no blocking, fusion or reordering beyond the definitions below. A library
+matmul serves as the dot-product step.
+
+Sources (web pages; cited below by short name and section):
+  Part 10  = "第10回 EVO-X2（Ryzen AI Max+ 395 / 128GB）+ Qwen3.8-Flash-Next用の
+             llama.cpp改造で長コンテキストのTGを高速化した話" (qiita, ariera)
+     §QSA indexer         : section "QSAとQSA indexerについて", subsection "QSA indexer"
+     §COMMON-004          : section "incremental pooled-key cache（COMMON-004）"
+     §FA-scaling          : section "なぜFlash Attentionがcontext長に比例していたのか"
+     §COMMON-005          : section "selected QSA K/V gather（COMMON-005）"
+     §COMMON-006          : section "block-domain top-k（COMMON-006）実装は見送り"
+
+What the method computes (Part 10 §QSA indexer, §COMMON-004..006):
+  1. indexer keys are summarised per 4-token micro-block: mean pool -> RMS norm ->
+     RoPE at the block position; completed summaries are cached per layer and only
+     new blocks are computed (COMMON-004);
+  2. the current query is scored against every completed block; the top-k blocks
+     covering indexer_top_k tokens are chosen, plus the still-open tail block
+     (at most 2048 + 4 - 1 = 2051 cells);
+  3. only those K/V cells are gathered (COMMON-005) and
+  4. ordinary (GQA) softmax attention runs over them.
+
+Readings taken where the pages are silent (each one is listed in the design notes):
+  R1 score_b = sum_h w_h * ReLU(q~_h . p_b) / sqrt(d_idx)  (the pages give no formula);
+     one pooled key per block is shared by all indexer heads.
+  R2 RoPE is the NeoX half-split rotation over all d dims: pair (i, i + d/2),
+     theta_i = base^(-2i/d), base 10000; z_i = x_i + j*x_{i+d/2} is multiplied by
+     exp(j * pos * theta_i).
+  R3 the position of block b is its first token, pos(b) = 4b; the query sits at
+     position n-1 (n = context length including the current token).
+  R4 RMS norm r = m / sqrt(mean(m^2) + eps) * g with eps 1e-6, unit gain unless a
+     gain vector is given.
+  R5 pooled summaries are stored as f16 (round to nearest even), like the cache.
+  R6 top-k ties go to the lower block index; if B <= K every block is selected; the
+     selected blocks are returned in ascending order.
+  R7 the tail is the n mod 4 tokens of the open block; a block that has just
+     completed is scored like any other, not force-included.
+  R8 attention: scale 1/sqrt(D), query head i uses KV head floor(i / (Hq/Hkv)), no
+     extra mask, sink, gate or softcap.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import numpy as np
+
+BLOCK = 4  # micro-block size = compression ratio 4 (Part 10 §QSA indexer)
+
+
+@dataclass(frozen=True)
+class QsaShape:
+    """Layer shapes the oracle needs (its own copy; it imports nothing from the product)."""
+
+    d_idx: int
+    n_idx_heads: int
+    top_k_tokens: int
+    n_q_heads: int
+    n_kv_heads: int
+    head_dim: int
+    rope_base: float = 10000.0
+    rms_eps: float = 1e-6
+
+    @property
+    def k_blocks(self) -> int:
+        # indexer_top_k tokens / compression ratio 4 (Part 10 §FA-scaling)
+        return self.top_k_tokens // BLOCK
+
+    @classmethod
+    def of(cls, wl) -> "QsaShape":
+        return cls(wl.d_idx, wl.n_idx_heads, wl.top_k_tokens, wl.n_q_heads, wl.n_kv_heads,
+                   wl.head_dim, wl.rope_base, wl.rms_eps)
+
+
+def to_f16(x) -> np.ndarray:
+    """Round float64 values to f16, nearest-even, directly from double (reading R5)."""
+    return np.asarray(x, dtype=np.float64).astype(np.float16)
+
+
+# ---------------------------------------------------------------------------
+# Step 1: pooled summaries (Part 10 §QSA indexer: average pooling -> RMS norm -> RoPE)
+# ---------------------------------------------------------------------------
+
+def rope_frequencies(dim: int, base: float) -> np.ndarray:
+    """theta_i = base^(-2i/dim), i < dim/2 (reading R2)."""
+    i = np.arange(dim // 2, dtype=np.float64)
+    return base ** (-2.0 * i / dim)
+
+
+def rope(x, pos, base: float) -> np.ndarray:
+    """NeoX half-split RoPE of the last axis of x at position(s) pos (reading R2).
+
+    x has shape [..., d]; pos is a scalar or broadcasts against x[..., 0].
+    Pair (x_i, x_{i+d/2}) is rotated by the angle pos * theta_i.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    half = x.shape[-1] // 2
+    angle = np.multiply.outer(np.asarray(pos, dtype=np.float64), rope_frequencies(2 * half, base))
+    c, s = np.cos(angle), np.sin(angle)
+    x1, x2 = x[..., :half], x[..., half:]
+    return np.concatenate([x1 * c - x2 * s, x1 * s + x2 * c], axis=-1)
+
+
+def mean_pool(raw_block) -> np.ndarray:
+    """Average of the 4 indexer keys of a micro-block: [..., 4, d] -> [..., d]."""
+    raw = np.asarray(raw_block, dtype=np.float64)
+    return raw.sum(axis=-2) / BLOCK
+
+
+def rms_normalize(m, eps: float, gain=None) -> np.ndarray:
+    """r = m / sqrt(mean(m^2) + eps) * g over the last axis (reading R4)."""
+    m = np.asarray(m, dtype=np.float64)
+    r = m / np.sqrt(np.mean(m * m, axis=-1, keepdims=True) + eps)
+    return r if gain is None else r * np.asarray(gain, dtype=np.float64)
+
+
+def block_position(b):
+    """Position of micro-block b = its first token (reading R3)."""
+    return BLOCK * np.asarray(b)
+
+
+def pooled_summaries(raw_idx, first_block: int, last_block: int, shape: QsaShape,
+                     gain=None) -> np.ndarray:
+    """f16 summaries p_b of blocks [first_block, last_block) from the raw indexer keys."""
+    d = shape.d_idx
+    blocks = np.arange(first_block, last_block)
+    raw = np.asarray(raw_idx[BLOCK * first_block:BLOCK * last_block]).reshape(-1, BLOCK, d)
+    m = mean_pool(raw)
+    r = rms_normalize(m, shape.rms_eps, gain)
+    p = rope(r, block_position(blocks), shape.rope_base)
+    return to_f16(p)
+
+
+def pooled_cache_full(raw_idx, n: int, shape: QsaShape, gain=None) -> np.ndarray:
+    """The old per-step path: every completed block recomputed (Part 10 §COMMON-004, 従来)."""
+    return pooled_summaries(raw_idx, 0, n // BLOCK, shape, gain)
+
+
+class PooledKeyCache:
+    """Persistent per-layer pooled-key cache, updated incrementally (Part 10 §COMMON-004).
+
+    Only blocks that completed (or were invalidated) since the last update are
+    computed; rows below `n_pooled` are reused as they are.
+    """
+
+    def __init__(self, max_blocks: int, d_idx: int):
+        self.rows = np.zeros((max_blocks, d_idx), dtype=np.float16)
+        self.n_pooled = 0
+
+    def update(self, raw_idx, n: int, shape: QsaShape, gain=None) -> int:
+        b_done = n // BLOCK
+        new = max(0, b_done - self.n_pooled)
+        if new:
+            self.rows[self.n_pooled:b_done] = pooled_summaries(raw_idx, self.n_pooled, b_done,
+                                                               shape, gain)
+            self.n_pooled = b_done
+        return new
+
+    def invalidate(self, from_block: int) -> None:
+        """State load / sequence edit: rows from `from_block` on are no longer trusted."""
+        self.n_pooled = min(self.n_pooled, max(0, from_block))
+
+
+# ---------------------------------------------------------------------------
+# Step 2: indexer scores and block-domain top-k (Part 10 §QSA indexer, §COMMON-006)
+# ---------------------------------------------------------------------------
+
+def indexer_query(q_idx, n: int, shape: QsaShape) -> np.ndarray:
+    """q~_h = RoPE(q_h, n-1): the current token's indexer query (readings R2, R3)."""
+    return rope(np.asarray(q_idx, dtype=np.float64), n - 1, shape.rope_base)
+
+
+def block_scores(pooled, q_idx, w, n: int, shape: QsaShape) -> np.ndarray:
+    """s_b = sum_h w_h * ReLU(q~_h . p_b) / sqrt(d_idx) for every completed block b < n/4 (R1)."""
+    b_done = n // BLOCK
+    p = np.asarray(pooled[:b_done], dtype=np.float64)             # [B, d]
+    q = indexer_query(q_idx, n, shape)                             # [H, d]
+    dots = p @ q.T                                                 # [B, H]
+    return (np.maximum(dots, 0.0) @ np.asarray(w, dtype=np.float64)) / np.sqrt(shape.d_idx)
+
+
+def topk_blocks(scores, k_blocks: int) -> np.ndarray:
+    """The k_blocks highest-scoring blocks, ties to the lower index, ascending (R6)."""
+    s = np.asarray(scores, dtype=np.float64)
+    if not np.all(np.isfinite(s)):
+        raise ValueError("indexer scores must be finite")
+    order = np.lexsort((np.arange(s.size), -s))   # by score descending, then index ascending
+    return np.sort(order[:min(k_blocks, s.size)]).astype(np.int64)
+
+
+def expand_cells(sel_blocks, n: int) -> np.ndarray:
+    """Selected blocks -> their 4 cells each, then the open tail [4B, n) (Part 10 §COMMON-006, R7)."""
+    sel = np.asarray(sel_blocks, dtype=np.int64)
+    cells = (BLOCK * sel[:, None] + np.arange(BLOCK)[None, :]).reshape(-1)
+    tail = np.arange(BLOCK * (n // BLOCK), n, dtype=np.int64)
+    return np.concatenate([cells, tail])
+
+
+# ---------------------------------------------------------------------------
+# Step 3+4: selected K/V gather and GQA attention (Part 10 §COMMON-005, reading R8)
+# ---------------------------------------------------------------------------
+
+def sparse_attention(q, k_cache, v_cache, cells, shape: QsaShape) -> np.ndarray:
+    """o_i = sum_c softmax_c(q_i . K[c, g] / sqrt(D)) V[c, g], g = i // (Hq/Hkv), over `cells`."""
+    q = np.asarray(q, dtype=np.float64)
+    cells = np.asarray(cells, dtype=np.int64)
+    group = shape.n_q_heads // shape.n_kv_heads
+    out = np.zeros((shape.n_q_heads, shape.head_dim), dtype=np.float64)
+    for i in range(shape.n_q_heads):
+        g = i // group
+        kc = np.asarray(k_cache[cells, g], dtype=np.float64)     # gathered rows [n_c, D]
+        vc = np.asarray(v_cache[cells, g], dtype=np.float64)
+        logits = kc @ q[i] / np.sqrt(shape.head_dim)
+        e = np.exp(logits - logits.max())
+        out[i] = (e @ vc) / e.sum()
+    return out
+
+
+# ---------------------------------------------------------------------------
+# One layer, step by step (mirrors the library's calls)
+# ---------------------------------------------------------------------------
+
+class OracleLayer:
+    """One QSA layer's caches and the decode-step calls, in plain numpy."""
+
+    def __init__(self, shape: QsaShape, max_ctx: int, gain=None):
+        self.shape = shape
+        self.max_ctx = max_ctx
+        self.gain = gain
+        self.k = np.zeros((max_ctx, shape.n_kv_heads, shape.head_dim), dtype=np.float16)
+        self.v = np.zeros_like(self.k)
+        self.idx = np.zeros((max_ctx, shape.d_idx), dtype=np.float16)
+        self.pooled = PooledKeyCache(max_ctx // BLOCK, shape.d_idx)
+        self.n = 0
+
+    def append_tokens(self, k, v, idx) -> None:
+        k = np.asarray(k, np.float16).reshape(-1, self.shape.n_kv_heads, self.shape.head_dim)
+        m = k.shape[0]
+        if self.n + m > self.max_ctx:
+            raise ValueError("context capacity exceeded")
+        self.k[self.n:self.n + m] = k
+        self.v[self.n:self.n + m] = np.asarray(v, np.float16).reshape(k.shape)
+        self.idx[self.n:self.n + m] = np.asarray(idx, np.float16).reshape(m, self.shape.d_idx)
+        self.n += m
+
+    def update_pooled_cache(self) -> int:
+        return self.pooled.update(self.idx, self.n, self.shape, self.gain)
+
+    def scores(self, q_idx, w) -> np.ndarray:
+        if self.pooled.n_pooled != self.n // BLOCK:
+            raise ValueError("pooled cache is stale")
+        return block_scores(self.pooled.rows, q_idx, w, self.n, self.shape)
+
+    def index_topk(self, q_idx, w):
+        s = self.scores(q_idx, w)
+        return topk_blocks(s, self.shape.k_blocks), s
+
+    def gather_cells(self, sel_blocks) -> np.ndarray:
+        return expand_cells(sel_blocks, self.n)
+
+    def attend(self, q, cells) -> np.ndarray:
+        return sparse_attention(q, self.k, self.v, cells, self.shape)
+
+    def decode_step(self, k, v, idx, q_idx, w, q):
+        """append -> incremental pooled update -> scores + top-k -> cells -> attention."""
+        self.append_tokens(k[None], v[None], idx[None])
+        self.update_pooled_cache()
+        sel, s = self.index_topk(q_idx, w)
+        cells = self.gather_cells(sel)
+        return {"sel": sel, "scores": s, "cells": cells, "out": self.attend(q, cells)}

@@ -1,0 +1,162 @@
+"""Seeded synthetic inputs for the QSA decode hot path.
+
+This module is the only code shared by the CPU oracle side (tests, the CPU baseline)
+and the CUDA side (tests, bench): it draws inputs and holds workload shapes, and it
+contains none of the method's arithmetic (no pooling, normalisation, rotation,
+scoring, selection or attention).
+
+Distributions follow the workloads the source pages measure on (a real long
+Japanese summarisation prompt on a trained model, which is not available here):
+keys, values, indexer keys and queries are f16 draws from N(0, 1); per-head indexer
+weights w_h are f32 draws from U(0, 1). Token counts are the pages' inputs
+61,789 / 126,253 / 255,181 ("Part 10", section 検証環境, main inputs).
+
+Every array is keyed by (seed, workload, layer, tensor, chunk) through numpy's
+SeedSequence, so any subset can be regenerated independently and the result does
+not depend on how many threads draw it.
+"""
+from __future__ import annotations
+
+import concurrent.futures as _cf
+import os
+from dataclasses import dataclass, replace
+
+import numpy as np
+
+SEED_BASE = 0x51A2026
+BLOCK = 4  # tokens per micro-block (compression ratio 4)
+
+# tensor ids used in the seed key
+_T_K, _T_V, _T_IDX, _T_QIDX, _T_W, _T_Q, _T_CELLS, _T_POOLED = range(8)
+_CHUNK_ROWS = 4096
+
+
+@dataclass(frozen=True)
+class Workload:
+    """Shapes of one decode workload (one QSA layer type, n_layers copies)."""
+
+    name: str
+    wid: int                 # numeric id used in the seed key
+    n_layers: int
+    n_prefill: int           # tokens already in the cache before the first step
+    n_steps: int             # decode steps (one appended token each)
+    d_idx: int               # indexer key width
+    n_idx_heads: int         # indexer heads H
+    top_k_tokens: int        # indexer_top_k (tokens); blocks = top_k_tokens / 4
+    n_q_heads: int
+    n_kv_heads: int
+    head_dim: int
+    rope_base: float = 10000.0
+    rms_eps: float = 1e-6
+
+    @property
+    def k_blocks(self) -> int:
+        return self.top_k_tokens // BLOCK
+
+    @property
+    def max_ctx(self) -> int:
+        # room for every decode step, rounded up to a whole block
+        n = self.n_prefill + self.n_steps
+        return ((n + BLOCK - 1) // BLOCK) * BLOCK
+
+    @property
+    def max_cells(self) -> int:
+        return BLOCK * self.k_blocks + BLOCK - 1
+
+
+_LAYER = dict(d_idx=128, n_idx_heads=16, top_k_tokens=2048, n_q_heads=32, n_kv_heads=4, head_dim=128)
+
+WORKLOADS = {
+    # 1 layer, 1,024-token context, 8 decode steps, small shapes
+    "tiny": Workload("tiny", 1, 1, 1024, 8, d_idx=64, n_idx_heads=4, top_k_tokens=256,
+                     n_q_heads=8, n_kv_heads=1, head_dim=64),
+    # single QSA layer at the pages' 64k input
+    "ctx64k": Workload("ctx64k", 2, 1, 61789, 1, **_LAYER),
+    # single QSA layer at the pages' 128k input, 64 decode steps
+    "ctx128k": Workload("ctx128k", 3, 1, 126253, 64, **_LAYER),
+    # all 12 QSA layers of the 48-layer hybrid at the pages' 256k input, one step
+    "ctx256k_12l": Workload("ctx256k_12l", 4, 12, 255181, 1, **_LAYER),
+    # streaming: 512 steps from the 256k prefill, all 12 layers
+    "stream256k_12l": Workload("stream256k_12l", 5, 12, 255181, 512, **_LAYER),
+}
+
+
+def workload(name: str, **overrides) -> Workload:
+    wl = WORKLOADS[name]
+    return replace(wl, **overrides) if overrides else wl
+
+
+def _rng(wl: Workload, layer: int, tensor: int, *extra: int) -> np.random.Generator:
+    key = [SEED_BASE, wl.wid, layer, tensor, *extra]
+    return np.random.Generator(np.random.PCG64(np.random.SeedSequence(key)))
+
+
+def _normal_f16(wl, layer, tensor, rows, row_shape, first_row=0, threads=None):
+    """N(0,1) draws rounded to f16, rows [first_row, first_row+rows), chunk-keyed."""
+    width = int(np.prod(row_shape))
+    out = np.empty((rows, width), np.float16)
+    if rows == 0:
+        return out.reshape((0, *row_shape))
+    c0 = first_row // _CHUNK_ROWS
+    c1 = (first_row + rows - 1) // _CHUNK_ROWS
+
+    def fill(c):
+        g = _rng(wl, layer, tensor, c)
+        chunk = g.standard_normal((_CHUNK_ROWS, width), dtype=np.float32)
+        lo = max(first_row, c * _CHUNK_ROWS)
+        hi = min(first_row + rows, (c + 1) * _CHUNK_ROWS)
+        out[lo - first_row:hi - first_row] = chunk[lo - c * _CHUNK_ROWS:hi - c * _CHUNK_ROWS]
+
+    n_threads = threads or min(32, os.cpu_count() or 1)
+    if c1 == c0 or n_threads == 1:
+        for c in range(c0, c1 + 1):
+            fill(c)
+    else:
+        with _cf.ThreadPoolExecutor(n_threads) as ex:
+            list(ex.map(fill, range(c0, c1 + 1)))
+    return out.reshape((rows, *row_shape))
+
+
+def prefill_tokens(wl: Workload, layer: int, n: int | None = None, first: int = 0):
+    """K, V and indexer keys of token positions [first, first+n) for one layer.
+
+    Returns dict k [n, Hkv, D] f16, v [n, Hkv, D] f16, idx [n, d_idx] f16.
+    Token position p always gets the same values, whatever range it is drawn in.
+    """
+    n = wl.n_prefill - first if n is None else n
+    return {
+        "k": _normal_f16(wl, layer, _T_K, n, (wl.n_kv_heads, wl.head_dim), first),
+        "v": _normal_f16(wl, layer, _T_V, n, (wl.n_kv_heads, wl.head_dim), first),
+        "idx": _normal_f16(wl, layer, _T_IDX, n, (wl.d_idx,), first),
+    }
+
+
+def step_inputs(wl: Workload, layer: int, step: int):
+    """Inputs of decode step `step` (0-based) of one layer.
+
+    The appended token sits at position n_prefill + step. Returns dict with
+    k, v [Hkv, D] f16, idx [d_idx] f16 (the appended token), q_idx [H, d_idx] f16
+    (un-rotated indexer query), w [H] f32 (indexer head weights, U(0,1)) and
+    q [Hq, D] f16 (attention query, already position-encoded by the model).
+    """
+    pos = wl.n_prefill + step
+    tok = prefill_tokens(wl, layer, 1, pos)
+    g = _rng(wl, layer, _T_QIDX, step)
+    q_idx = g.standard_normal((wl.n_idx_heads, wl.d_idx), dtype=np.float32).astype(np.float16)
+    w = _rng(wl, layer, _T_W, step).random(wl.n_idx_heads, dtype=np.float32)
+    q = _rng(wl, layer, _T_Q, step).standard_normal((wl.n_q_heads, wl.head_dim),
+                                                      dtype=np.float32).astype(np.float16)
+    return {"k": tok["k"][0], "v": tok["v"][0], "idx": tok["idx"][0], "q_idx": q_idx, "w": w, "q": q}
+
+
+def random_cells(wl: Workload, layer: int, n_ctx: int, n_cells: int, salt: int = 0):
+    """A sorted set of `n_cells` distinct cell ids in [0, n_ctx) (stage-isolated attention input)."""
+    g = _rng(wl, layer, _T_CELLS, salt)
+    n_cells = min(n_cells, n_ctx)
+    return np.sort(g.choice(n_ctx, size=n_cells, replace=False)).astype(np.int32)
+
+
+def random_pooled(wl: Workload, layer: int, n_blocks: int, salt: int = 0):
+    """An f16 table [n_blocks, d_idx] drawn from N(0,1) (stage-isolated scan input)."""
+    g = _rng(wl, layer, _T_POOLED, salt)
+    return g.standard_normal((n_blocks, wl.d_idx), dtype=np.float32).astype(np.float16)

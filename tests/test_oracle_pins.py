@@ -1,0 +1,342 @@
+"""Pins of the CPU oracle against facts fixed outside it.
+
+Each test checks the oracle against something other than itself: values the
+pages print (tests/golden/pages_constants.json), closed forms, independent
+formulations (complex exponentials, rank counting, exact fractions), a library
+routine (torch's scaled_dot_product_attention in float64) and invariants the
+pages state (the incremental cache equals a full recompute; a selection that
+covers every block equals dense attention). A plausible mistake in the oracle
+(a dropped term, a wrong sign, position or index) fails at least one of them.
+"""
+import json
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import qsa_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+SMALL = O.QsaShape(d_idx=16, n_idx_heads=3, top_k_tokens=16, n_q_heads=4, n_kv_heads=2, head_dim=8)
+
+
+def _pages():
+    with open(os.path.join(GOLDEN, "pages_constants.json")) as f:
+        return json.load(f)
+
+
+# ---------------------------------------------------------------- f16 storage
+
+def test_f16_rounding_is_direct_nearest_even():
+    x = np.array([1 + 2**-11, 1 + 3 * 2**-11, 1 + 2**-11 + 2**-40, -(1 + 2**-11)])
+    got = O.to_f16(x).astype(np.float64)
+    # ties go to the even mantissa; a value just above a tie rounds up (no double rounding)
+    assert got.tolist() == [1.0, 1 + 2**-9, 1 + 2**-10, -1.0]
+
+
+# ---------------------------------------------------------------- RoPE
+
+def test_rope_equals_complex_exponential():
+    rng = np.random.default_rng(1)
+    d, base = 32, 10000.0
+    x = rng.standard_normal((5, d))
+    pos = np.array([0, 1, 7, 4096, 255181])
+    z = x[:, : d // 2] + 1j * x[:, d // 2:]
+    freq = np.power(base, -np.arange(0, d, 2, dtype=np.float64) / d)
+    zr = z * np.exp(1j * pos[:, None] * freq[None, :])
+    want = np.concatenate([zr.real, zr.imag], axis=1)
+    np.testing.assert_allclose(O.rope(x, pos, base), want, rtol=0, atol=1e-12)
+
+
+def test_rope_equals_rotate_half_form():
+    rng = np.random.default_rng(2)
+    d = 16
+    x = rng.standard_normal(d)
+    inv = 1.0 / (10000.0 ** (np.arange(0, d, 2) / d))
+    emb = np.concatenate([inv, inv]) * 9
+    rot = np.concatenate([-x[d // 2:], x[: d // 2]])
+    want = x * np.cos(emb) + rot * np.sin(emb)
+    np.testing.assert_allclose(O.rope(x, 9, 10000.0), want, atol=1e-13)
+
+
+def test_rope_identity_norms_and_relative_position():
+    rng = np.random.default_rng(3)
+    a, b = rng.standard_normal(64), rng.standard_normal(64)
+    np.testing.assert_array_equal(O.rope(a, 0, 1e4), a)
+    ra = O.rope(a, 1234, 1e4)
+    pair = lambda v: v[:32] ** 2 + v[32:] ** 2
+    np.testing.assert_allclose(pair(ra), pair(a), rtol=1e-12)
+    for m, n in [(5, 5), (100, 3), (4 * 63000, 255180)]:
+        lhs = O.rope(a, m, 1e4) @ O.rope(b, n, 1e4)
+        rhs = a @ O.rope(b, n - m, 1e4)
+        assert abs(lhs - rhs) <= 1e-9 * (np.abs(a).sum() * np.abs(b).sum())
+
+
+# ---------------------------------------------------------------- pool + RMS norm
+
+def test_mean_pool_is_exact_mean():
+    rng = np.random.default_rng(4)
+    raw = rng.standard_normal((4, 8)).astype(np.float16)
+    got = O.mean_pool(raw)
+    for j in range(8):
+        exact = sum(Fraction(float(raw[i, j])) for i in range(4)) / 4
+        assert Fraction(float(got[j])) == exact
+    u = rng.standard_normal(8).astype(np.float16)
+    np.testing.assert_array_equal(O.mean_pool(np.stack([u] * 4)), u.astype(np.float64))
+
+
+def test_rms_norm_closed_forms():
+    rng = np.random.default_rng(5)
+    m = rng.standard_normal(128) * 3
+    eps = 1e-6
+    r = O.rms_normalize(m, eps)
+    ms = np.mean(m * m)
+    assert abs(np.sum(r * r) - 128 * ms / (ms + eps)) < 1e-10
+    np.testing.assert_allclose(O.rms_normalize(7.0 * m, 0.0), O.rms_normalize(m, 0.0), rtol=1e-13)
+    c = np.full(8, 0.5)
+    np.testing.assert_allclose(O.rms_normalize(c, eps), c / np.sqrt(0.25 + eps), rtol=1e-15)
+    g = rng.random(128)
+    np.testing.assert_allclose(O.rms_normalize(m, eps, g), r * g, rtol=1e-15)
+
+
+# ---------------------------------------------------------------- incremental cache (COMMON-004)
+
+def test_incremental_cache_equals_full_recompute():
+    rng = np.random.default_rng(6)
+    shape = O.QsaShape(64, 4, 64, 8, 1, 64)
+    raw = rng.standard_normal((400, 64)).astype(np.float16)
+    cache = O.PooledKeyCache(100, 64)
+    n = 0
+    for step in [1, 3, 4, 5, 17, 2, 1, 1, 1, 64, 100, 7]:
+        n += step
+        cache.update(raw, n, shape)
+        full = O.pooled_cache_full(raw, n, shape)
+        assert cache.n_pooled == n // 4
+        np.testing.assert_array_equal(cache.rows[: n // 4], full)
+    cache.invalidate(30)
+    assert cache.n_pooled == 30
+    cache.rows[30:] = 0
+    cache.update(raw, n, shape)
+    np.testing.assert_array_equal(cache.rows[: n // 4], O.pooled_cache_full(raw, n, shape))
+
+
+def test_pooled_summary_of_constant_block():
+    rng = np.random.default_rng(7)
+    u = rng.standard_normal(16).astype(np.float16)
+    raw = np.stack([u] * 8)             # blocks 0 and 1, every key equal to u
+    p = O.pooled_summaries(raw, 0, 2, SMALL)
+    uu = u.astype(np.float64)
+    r = uu / np.sqrt(np.mean(uu * uu) + SMALL.rms_eps)
+    for b in (0, 1):
+        z = (r[:8] + 1j * r[8:]) * np.exp(1j * 4 * b * np.power(1e4, -np.arange(0, 16, 2) / 16))
+        want = np.concatenate([z.real, z.imag])
+        np.testing.assert_allclose(p[b].astype(np.float64), want, rtol=0, atol=2e-3)
+
+
+# ---------------------------------------------------------------- indexer scores
+
+def test_scores_match_relative_complex_form():
+    """s_b from the complex form: <RoPE(q, n-1), RoPE(r, 4b)> = Re sum conj(zq) zr e^{j(4b-n+1)theta}."""
+    rng = np.random.default_rng(8)
+    shape = SMALL
+    d, H = shape.d_idx, shape.n_idx_heads
+    n = 4 * 9 + 2
+    raw = rng.standard_normal((n, d)).astype(np.float16)
+    pooled = O.pooled_cache_full(raw, n, shape)
+    q = rng.standard_normal((H, d)).astype(np.float16)
+    w = np.array([0.25, 0.0, 1.5])
+    got = O.block_scores(pooled, q, w, n, shape)
+    assert got.shape == (n // 4,)
+    theta = np.power(1e4, -np.arange(0, d, 2) / d)
+    for b in range(n // 4):
+        # undo the block rotation on the stored f16 row to get r_b, then rotate by the offset
+        p = pooled[b].astype(np.float64)
+        zp = (p[: d // 2] + 1j * p[d // 2:]) * np.exp(-1j * 4 * b * theta)
+        s = 0.0
+        for h in range(H):
+            zq = q[h, : d // 2].astype(np.float64) + 1j * q[h, d // 2:].astype(np.float64)
+            dot = np.real(np.sum(np.conj(zq) * zp * np.exp(1j * (4 * b - (n - 1)) * theta)))
+            s += w[h] * max(dot, 0.0)
+        assert abs(got[b] - s / np.sqrt(d)) <= 1e-10 * (1 + abs(s))
+
+
+def test_scores_properties():
+    rng = np.random.default_rng(9)
+    shape = SMALL
+    n = 4 * 20 + 3
+    pooled = rng.standard_normal((n // 4, 16)).astype(np.float16)
+    q = rng.standard_normal((3, 16)).astype(np.float16)
+    w = rng.random(3)
+    s = O.block_scores(pooled, q, w, n, shape)
+    assert np.all(s >= 0)
+    # positive homogeneity in the weights and linearity over heads
+    np.testing.assert_allclose(O.block_scores(pooled, q, 3 * w, n, shape), 3 * s, rtol=1e-13)
+    parts = sum(O.block_scores(pooled, q, np.eye(3)[h] * w[h], n, shape) for h in range(3))
+    np.testing.assert_allclose(parts, s, rtol=1e-12)
+    # a head whose query is negated keeps only the dots the other sign dropped
+    s_pos = O.block_scores(pooled, q, np.array([1.0, 0, 0]), n, shape)
+    qn = q.copy()
+    qn[0] = -qn[0]
+    s_neg = O.block_scores(pooled, qn, np.array([1.0, 0, 0]), n, shape)
+    dots_abs = np.abs(pooled.astype(np.float64) @ O.rope(q[0].astype(np.float64), n - 1, 1e4))
+    np.testing.assert_allclose(s_pos + s_neg, dots_abs / 4.0, rtol=1e-12)
+
+
+def test_needle_blocks_are_selected():
+    """Blocks whose keys point along the rotated query must win the top-k (pos(b)=4b, query n-1)."""
+    rng = np.random.default_rng(10)
+    shape = O.QsaShape(d_idx=64, n_idx_heads=2, top_k_tokens=12, n_q_heads=2, n_kv_heads=1, head_dim=16)
+    n = 4 * 200 + 1
+    raw = rng.standard_normal((n, 64)).astype(np.float16)
+    q = rng.standard_normal((2, 64)).astype(np.float16)
+    needles = [3, 77, 150]
+    for b in needles:
+        # r_b = RoPE(q_0, (n-1) - 4b) so that RoPE(r_b, 4b) = RoPE(q_0, n-1)
+        key = O.rope(q[0].astype(np.float64), (n - 1) - 4 * b, 1e4)
+        raw[4 * b:4 * b + 4] = key.astype(np.float16)
+    pooled = O.pooled_cache_full(raw, n, shape)
+    s = O.block_scores(pooled, q, np.array([1.0, 0.0]), n, shape)
+    sel = O.topk_blocks(s, 3)
+    assert sel.tolist() == needles
+
+
+# ---------------------------------------------------------------- top-k (COMMON-006 form)
+
+def _rank_count_selection(s, k):
+    """Brute force: b is selected iff fewer than k blocks beat it (higher score, or equal and lower index)."""
+    B = len(s)
+    out = []
+    for b in range(B):
+        beaten_by = sum(1 for c in range(B) if s[c] > s[b] or (s[c] == s[b] and c < b))
+        if beaten_by < k:
+            out.append(b)
+    return out
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_topk_equals_rank_counting(seed):
+    rng = np.random.default_rng(100 + seed)
+    B = int(rng.integers(1, 90))
+    s = np.round(rng.random(B) * 8) / 8        # coarse values force many exact ties
+    k = int(rng.integers(1, 40))
+    assert O.topk_blocks(s, k).tolist() == _rank_count_selection(s.tolist(), k)
+
+
+def test_topk_ties_lower_index_and_small_b():
+    s = np.array([1.0, 2.0, 2.0, 2.0, 0.5, 2.0])
+    assert O.topk_blocks(s, 2).tolist() == [1, 2]
+    assert O.topk_blocks(s, 5).tolist() == [0, 1, 2, 3, 5]
+    assert O.topk_blocks(s, 6).tolist() == [0, 1, 2, 3, 4, 5]
+    assert O.topk_blocks(s, 100).tolist() == list(range(6))
+    assert O.topk_blocks(np.zeros(0), 4).tolist() == []
+    with pytest.raises(ValueError):
+        O.topk_blocks(np.array([1.0, np.nan]), 1)
+
+
+# ---------------------------------------------------------------- cells
+
+def test_cells_count_order_and_tail():
+    for n, sel in [(0, []), (3, []), (4, [0]), (23, [0, 2, 4]), (26, [5])]:
+        cells = O.expand_cells(np.array(sel, dtype=np.int64), n)
+        assert len(cells) == 4 * len(sel) + n % 4
+        assert np.all(np.diff(cells) > 0) and (len(cells) == 0 or cells[-1] < n)
+        assert set(range(4 * (n // 4), n)) <= set(cells.tolist())
+
+
+def test_pages_max_cells():
+    pg = _pages()
+    k_tokens = pg["indexer_top_k"]["value"]
+    ratio = pg["compression_ratio"]["value"]
+    assert ratio == O.BLOCK
+    k = k_tokens // ratio
+    # the worst case: at least k completed blocks and a tail of 3
+    for n in pg["input_tokens"]["value"] + [255182, 255183, 255184]:
+        n_cells = len(O.expand_cells(np.arange(min(k, n // 4)), n))
+        assert n_cells <= pg["max_cells"]["value"]
+    assert len(O.expand_cells(np.arange(k), 4 * 1000 + 3)) == pg["max_cells"]["value"]
+
+
+def test_pages_kv_cache_size_matches_layer_shapes():
+    """2 x Hkv x D x f16 per token and layer, over 12 QSA layers, gives the pages' 6,144 MiB at 262,144."""
+    pg = _pages()
+    wl = synth.workload("ctx256k_12l")
+    per_tok = 2 * wl.n_kv_heads * wl.head_dim * 2 * pg["qsa_layers"]["value"]
+    assert per_tok * pg["kv_cache_mib"]["ctx"] == pg["kv_cache_mib"]["normal_kv"] * 2**20
+
+
+# ---------------------------------------------------------------- attention (COMMON-005)
+
+def _dense_sdpa(q, k, v, shape):
+    """torch scaled_dot_product_attention in float64 over all tokens (GQA by head grouping)."""
+    qt = torch.from_numpy(np.asarray(q, np.float64)).reshape(1, shape.n_q_heads, 1, shape.head_dim)
+    kt = torch.from_numpy(np.asarray(k, np.float64)).permute(1, 0, 2).unsqueeze(0)
+    vt = torch.from_numpy(np.asarray(v, np.float64)).permute(1, 0, 2).unsqueeze(0)
+    out = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, enable_gqa=True)
+    return out.reshape(shape.n_q_heads, shape.head_dim).numpy()
+
+
+def test_full_selection_equals_dense_attention():
+    wl = synth.workload("tiny")
+    shape = O.QsaShape.of(wl)
+    layer = O.OracleLayer(shape, max_ctx=wl.max_ctx)
+    n0 = 4 * shape.k_blocks - 2          # every block fits in the top-k
+    pre = synth.prefill_tokens(wl, 0, n0)
+    layer.append_tokens(pre["k"], pre["v"], pre["idx"])
+    layer.update_pooled_cache()
+    st = synth.step_inputs(wl, 0, 0)
+    res = layer.decode_step(st["k"], st["v"], st["idx"], st["q_idx"], st["w"], st["q"])
+    n = n0 + 1
+    assert res["cells"].tolist() == list(range(n))
+    want = _dense_sdpa(st["q"], layer.k[:n], layer.v[:n], shape)
+    np.testing.assert_allclose(res["out"], want, rtol=0, atol=1e-12)
+
+
+def test_attention_special_cases():
+    rng = np.random.default_rng(11)
+    shape = SMALL
+    k = rng.standard_normal((20, 2, 8)).astype(np.float16)
+    v = rng.standard_normal((20, 2, 8)).astype(np.float16)
+    q = rng.standard_normal((4, 8)).astype(np.float16)
+    out = O.sparse_attention(q, k, v, np.array([13]), shape)
+    for i in range(4):
+        np.testing.assert_array_equal(out[i], v[13, i // 2].astype(np.float64))
+    k_same = np.broadcast_to(k[:1], k.shape)
+    out = O.sparse_attention(q, k_same, v, np.array([1, 4, 9]), shape)
+    for i in range(4):
+        np.testing.assert_allclose(out[i], v[[1, 4, 9], i // 2].astype(np.float64).mean(0), atol=1e-14)
+
+
+# ---------------------------------------------------------------- chain
+
+def test_decode_chain_invariants_tiny():
+    wl = synth.workload("tiny")
+    shape = O.QsaShape.of(wl)
+    layer = O.OracleLayer(shape, max_ctx=wl.max_ctx)
+    pre = synth.prefill_tokens(wl, 0)
+    layer.append_tokens(pre["k"], pre["v"], pre["idx"])
+    layer.update_pooled_cache()
+    for step in range(wl.n_steps):
+        st = synth.step_inputs(wl, 0, step)
+        res = layer.decode_step(st["k"], st["v"], st["idx"], st["q_idx"], st["w"], st["q"])
+        n = wl.n_prefill + step + 1
+        assert len(res["sel"]) == min(shape.k_blocks, n // 4)
+        assert len(res["cells"]) == 4 * len(res["sel"]) + n % 4 <= wl.max_cells
+        np.testing.assert_array_equal(layer.pooled.rows[: n // 4],
+                                      O.pooled_cache_full(layer.idx, n, shape))
+        assert np.all(np.isfinite(res["out"]))
+
+
+def test_golden_tiny_chain_regression():
+    """The oracle still reproduces the committed tiny-workload chain (tests/golden/make_golden.py)."""
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("make_golden", os.path.join(GOLDEN, "make_golden.py"))
+    mg = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mg)
+    want = np.load(os.path.join(GOLDEN, "tiny_chain.npz"))
+    got = mg.tiny_chain()
+    assert sorted(want.files) == sorted(got)
+    for key in want.files:
+        np.testing.assert_allclose(got[key], want[key], rtol=1e-12, atol=0, err_msg=key)
