@@ -1,0 +1,192 @@
+/*
+ * qsa.h — C ABI of the B200 (sm_100a) QSA decode hot path.
+ *
+ * QSA (Qwen Sparse Attention) decode, as described on the web page
+ * "第10回 EVO-X2（Ryzen AI Max+ 395 / 128GB）+ Qwen3.8-Flash-Next用のllama.cpp改造で
+ * 長コンテキストのTGを高速化した話" ("Part 10" below), runs in four stages per layer:
+ *   1. indexer keys are summarised per 4-token micro-block (mean pool -> RMS norm ->
+ *      RoPE at the block position) into a persistent pooled-key cache that is only
+ *      extended by newly completed blocks            (Part 10, section COMMON-004);
+ *   2. the current indexer query scores every completed block and the top-k blocks
+ *      covering indexer_top_k tokens are chosen      (Part 10, sections "QSA indexer",
+ *                                                      COMMON-006);
+ *   3. their cells plus the open tail block are gathered (at most 2048 + 4 - 1 = 2051)
+ *                                                     (Part 10, section COMMON-005);
+ *   4. GQA softmax attention runs over those cells only.
+ *
+ * Conventions shared by every call:
+ *  - All data pointers are DEVICE pointers unless stated otherwise. Every buffer is
+ *    owned by the caller (e.g. allocated with PyTorch); the library never allocates
+ *    device memory and owns only the host-side context.
+ *  - Every call that takes a stream is asynchronous on that stream (NULL = legacy
+ *    default stream) and returns after HOST-side argument validation only; kernels are
+ *    launched with programmatic dependent launch so that consecutive calls on one
+ *    stream overlap their launch latency, and all of them are safe to capture in a
+ *    CUDA graph.
+ *  - The sequence state of each layer (context length n_ctx and number of pooled
+ *    blocks n_pooled) lives in DEVICE memory inside the layer's workspace and is
+ *    advanced by the kernels themselves, so a captured decode step can be replayed.
+ *  - Conditions that depend on that device state (capacity exceeded, a stale pooled
+ *    cache, an out-of-range cell or block id) never fault: the kernel skips the
+ *    offending work, writes empty outputs and records the first error code in the
+ *    layer's device status word, which qsa_read_layer_state() returns.
+ *  - f16 means IEEE binary16; f32 means IEEE binary32. Every pointer must be 16-byte
+ *    aligned; rows are tightly packed (row-major, innermost index last).
+ *  - No call throws across the ABI. A failed call returns a non-zero qsa_status and
+ *    stores a message retrievable with qsa_last_error().
+ */
+#ifndef QSA_H_
+#define QSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA stream (cudaStream_t). NULL selects the legacy default stream. */
+typedef struct CUstream_st* qsa_stream_t;
+
+typedef enum {
+  QSA_OK = 0,
+  QSA_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad layer id, bad size      */
+  QSA_ERR_CAPACITY = 2,      /* more tokens than max_ctx                              */
+  QSA_ERR_STATE = 3,         /* layer not bound, or pooled cache behind the context   */
+  QSA_ERR_CUDA = 4,          /* a CUDA runtime call failed (message has the detail)   */
+  QSA_ERR_UNSUPPORTED = 5,   /* shape outside what the kernels are built for          */
+  QSA_ERR_BAD_INDEX = 6      /* device status only: a block or cell id out of range   */
+} qsa_status;
+
+/* Static shape of every layer of one model (Part 10, section "QSA indexer"). */
+typedef struct {
+  int32_t n_layers;       /* QSA layers held by one context (12 in the pages' model)    */
+  int32_t max_ctx;        /* token capacity per layer; a multiple of 4, <= 1,048,576    */
+  int32_t d_idx;          /* indexer key width: 64 or 128                               */
+  int32_t n_idx_heads;    /* indexer heads H: 1, 2, 4, 8 or 16                          */
+  int32_t top_k_tokens;   /* indexer_top_k in tokens, a multiple of 4 (2048 on pages)   */
+  int32_t n_q_heads;      /* attention query heads Hq                                   */
+  int32_t n_kv_heads;     /* attention KV heads Hkv; Hq / Hkv in {1, 2, 4, 8}          */
+  int32_t head_dim;       /* attention head dimension D: 64 or 128                      */
+  float rope_base;        /* RoPE base (10000)                                          */
+  float rms_eps;          /* RMS-norm epsilon inside the square root (1e-6)             */
+} qsa_config;
+
+/* Caller-owned device buffers of one layer. Sizes come from qsa_buffer_bytes(). */
+typedef struct {
+  void* k_cache;          /* [max_ctx][n_kv_heads][head_dim] f16, token-major           */
+  void* v_cache;          /* [max_ctx][n_kv_heads][head_dim] f16, token-major           */
+  void* idx_cache;        /* [max_ctx][d_idx] f16: raw per-token indexer keys           */
+  void* pooled_cache;     /* [max_ctx/4][d_idx] f16: pooled summaries p_b               */
+  const float* rms_gain;  /* [d_idx] f32 RMS-norm gain, or NULL for unit gain           */
+  void* workspace;        /* device state + scratch; QSA_BUF_WORKSPACE bytes            */
+} qsa_layer_buffers;
+
+enum {
+  QSA_BUF_KV = 0,         /* bytes of k_cache (v_cache has the same size) */
+  QSA_BUF_IDX = 1,        /* bytes of idx_cache                           */
+  QSA_BUF_POOLED = 2,     /* bytes of pooled_cache                        */
+  QSA_BUF_WORKSPACE = 3,  /* bytes of workspace                           */
+  QSA_BUF_MAX_CELLS = 4   /* not bytes: max cells per step = 4*(top_k_tokens/4) + 3 */
+};
+
+typedef struct qsa_ctx qsa_ctx;
+
+/* Size in bytes of one of a layer's buffers (see QSA_BUF_*); 0 if cfg is invalid. */
+size_t qsa_buffer_bytes(const qsa_config* cfg, int32_t which);
+
+/* Validate cfg and create a host context bound to the CURRENT CUDA device.
+ * Returns QSA_ERR_UNSUPPORTED for shapes the kernels are not built for. */
+qsa_status qsa_create(const qsa_config* cfg, qsa_ctx** out);
+
+/* Free the host context. Does not touch any device buffer. NULL is a no-op. */
+void qsa_destroy(qsa_ctx* ctx);
+
+/* Message of the last failed call on ctx (host string owned by ctx), "" if none. */
+const char* qsa_last_error(const qsa_ctx* ctx);
+
+/* Attach a layer's buffers and reset its device state to an empty sequence
+ * (n_ctx = n_pooled = 0, status = 0), asynchronously on `stream`. Also encodes the
+ * TMA descriptor of the pooled cache. May be called again to rebind. */
+qsa_status qsa_bind_layer(qsa_ctx* ctx, int32_t layer, const qsa_layer_buffers* buf,
+                          qsa_stream_t stream);
+
+/* State load (Part 10, section COMMON-004: a cache that can no longer be trusted after a
+ * state load is invalidated and rebuilt when next needed). Sets the device state to
+ * n_ctx tokens of which the first n_pooled blocks already hold valid summaries; the
+ * caller has written the K/V/indexer caches (and pooled rows < n_pooled). Requires
+ * 0 <= n_pooled <= n_ctx/4 and n_ctx <= max_ctx. Clears the status word. */
+qsa_status qsa_restore_layer(qsa_ctx* ctx, int32_t layer, int32_t n_ctx, int32_t n_pooled,
+                             qsa_stream_t stream);
+
+/* Synchronise `stream` and read the layer's device state. Any output pointer may be
+ * NULL. If clear != 0 the status word is reset to 0 afterwards. */
+qsa_status qsa_read_layer_state(qsa_ctx* ctx, int32_t layer, int32_t* n_ctx,
+                                int32_t* n_pooled, int32_t* device_status, int32_t clear,
+                                qsa_stream_t stream);
+
+/* Append one token at position n_ctx: k, v [n_kv_heads][head_dim] f16 and the raw
+ * indexer key idx_key [d_idx] f16 (Part 10, section COMMON-004: the raw indexer K cache
+ * is the source of pooling). Device status QSA_ERR_CAPACITY (and no write) if the
+ * layer is full. */
+qsa_status qsa_append_token(qsa_ctx* ctx, int32_t layer, const void* k, const void* v,
+                            const void* idx_key, qsa_stream_t stream);
+
+/* Append n >= 1 tokens (prefill): k, v [n][n_kv_heads][head_dim] f16,
+ * idx_key [n][d_idx] f16. All-or-nothing: nothing is written if they do not fit. */
+qsa_status qsa_append_tokens(qsa_ctx* ctx, int32_t layer, int32_t n, const void* k,
+                             const void* v, const void* idx_key, qsa_stream_t stream);
+
+/* Incremental pooled-key cache update (Part 10, section COMMON-004): computes p_b for
+ * exactly the blocks b in [n_pooled, n_ctx/4) — mean of the 4 raw indexer keys,
+ * RMS norm (eps, gain), NeoX RoPE at position 4b, stored as f16 — and sets
+ * n_pooled = n_ctx/4. In decode this is one block every 4th token, else nothing. */
+qsa_status qsa_update_pooled_cache(qsa_ctx* ctx, int32_t layer, qsa_stream_t stream);
+
+/* Sequence edit / state load: summaries from block `from_block` on are no longer
+ * trusted; sets n_pooled = min(n_pooled, from_block). The next update rebuilds them. */
+qsa_status qsa_invalidate_pooled_cache(qsa_ctx* ctx, int32_t layer, int32_t from_block,
+                                       qsa_stream_t stream);
+
+/* Indexer scan + block-domain top-k (Part 10, sections "QSA indexer" and COMMON-006).
+ *   q_idx  [n_idx_heads][d_idx] f16: the current token's indexer query, NOT yet
+ *          rotated; the library applies RoPE at position n_ctx-1.
+ *   w      [n_idx_heads] f32: per-head weights.
+ *   score_b = sum_h w_h * max(0, RoPE(q_h, n_ctx-1) . p_b) / sqrt(d_idx)
+ *   for every completed block b < n_ctx/4, accumulated in f32.
+ * Outputs: sel_blocks [top_k_tokens/4] i32 — the min(K, B) highest-scoring blocks,
+ * ties to the lower block index, in ascending order; n_sel — a device i32 scalar
+ * with their count; scores [max_ctx/4] f32 (optional, may be NULL) — every score.
+ * Requires the pooled cache to be current (n_pooled == n_ctx/4); otherwise device
+ * status QSA_ERR_STATE and n_sel = 0. */
+qsa_status qsa_index_topk(qsa_ctx* ctx, int32_t layer, const void* q_idx, const float* w,
+                          int32_t* sel_blocks, int32_t* n_sel, float* scores,
+                          qsa_stream_t stream);
+
+/* Selected K/V gather (Part 10, section COMMON-005). Expands the selected blocks into
+ * their cells 4b..4b+3 and appends the open tail block [4*(n_ctx/4), n_ctx):
+ *   cells [4*(top_k_tokens/4)+3] i32 (ascending when sel_blocks is ascending),
+ *   n_cells device i32 scalar = 4*n_sel + n_ctx mod 4.
+ * If k_compact / v_compact are non-NULL, also copies the selected rows into them:
+ * [max_cells][n_kv_heads][head_dim] f16 each (the literal compact K/V). Block ids out
+ * of range are dropped and reported as device status QSA_ERR_BAD_INDEX. */
+qsa_status qsa_gather_kv(qsa_ctx* ctx, int32_t layer, const int32_t* sel_blocks,
+                         const int32_t* n_sel, int32_t* cells, int32_t* n_cells,
+                         void* k_compact, void* v_compact, qsa_stream_t stream);
+
+/* GQA attention over the selected cells, reading K/V rows straight from the cache
+ * (the gather fused into a split-KV flash-decode; Part 10, section COMMON-005).
+ *   q     [n_q_heads][head_dim] f16, already position-encoded by the model;
+ *   cells [n_cells] i32 device ids in [0, n_ctx); n_cells device i32 scalar
+ *         (<= max cells); out [n_q_heads][head_dim] f32.
+ *   out_i = sum_c softmax_c(q_i . K[c][g] / sqrt(D)) V[c][g], g = i / (Hq/Hkv),
+ *   with f32 softmax and accumulation. An empty cell set gives out = 0; ids out of
+ *   range are skipped and reported as device status QSA_ERR_BAD_INDEX. */
+qsa_status qsa_sparse_attend(qsa_ctx* ctx, int32_t layer, const void* q, const int32_t* cells,
+                             const int32_t* n_cells, float* out, qsa_stream_t stream);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif  /* QSA_H_ */

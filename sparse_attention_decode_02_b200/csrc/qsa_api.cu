@@ -1,0 +1,287 @@
+// C ABI of the QSA decode hot path: host-side validation, the host context and the
+// dispatch of each call to its kernels. The device-side sequence state lives in the
+// layer workspace (see qsa_internal.h); nothing here allocates device memory.
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <string>
+#include <vector>
+
+#include "../../include/qsa.h"
+#include "qsa_internal.h"
+
+using namespace qsa;
+
+namespace {
+
+struct Layer {
+  bool bound = false;
+  qsa_layer_buffers buf{};
+  // Upper bound on blocks the next pooled update may have to compute; it only sizes
+  // the update's grid (the kernel itself reads the exact range from device state).
+  long long pending_blocks = 0;
+};
+
+bool is_pow2_upto(int v, int hi) { return v >= 1 && v <= hi && (v & (v - 1)) == 0; }
+
+const char* config_problem(const qsa_config& c) {
+  if (c.n_layers < 1) return "n_layers must be >= 1";
+  if (c.max_ctx < kBlock || c.max_ctx % kBlock) return "max_ctx must be a positive multiple of 4";
+  if (c.max_ctx > kBlock * kTopkCluster * kTopkMaxPerCta) return "max_ctx above 1,048,576";
+  if (c.d_idx != 64 && c.d_idx != 128) return "d_idx must be 64 or 128";
+  if (!is_pow2_upto(c.n_idx_heads, 16)) return "n_idx_heads must be 1, 2, 4, 8 or 16";
+  if (c.top_k_tokens < kBlock || c.top_k_tokens % kBlock) return "top_k_tokens must be a positive multiple of 4";
+  if (c.head_dim != 64 && c.head_dim != 128) return "head_dim must be 64 or 128";
+  if (c.n_kv_heads < 1 || c.n_q_heads < 1 || c.n_q_heads % c.n_kv_heads) return "n_q_heads must be a multiple of n_kv_heads";
+  if (!is_pow2_upto(c.n_q_heads / c.n_kv_heads, 8)) return "n_q_heads / n_kv_heads must be 1, 2, 4 or 8";
+  if (!(c.rope_base > 1.0f)) return "rope_base must be > 1";
+  if (!(c.rms_eps >= 0.0f)) return "rms_eps must be >= 0";
+  return nullptr;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+}  // namespace
+
+struct qsa_ctx {
+  qsa_config cfg{};
+  int device = 0;
+  int n_sms = 0;
+  AttnSplit split{};
+  WorkspaceLayout ws{};
+  std::vector<Layer> layers;
+  std::string last_error;
+
+  qsa_status fail(qsa_status st, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    last_error = buf;
+    return st;
+  }
+  qsa_status cuda(cudaError_t e, const char* what) {
+    if (e == cudaSuccess) return QSA_OK;
+    return fail(QSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  }
+  qsa_status layer_ok(int32_t layer) {
+    if (layer < 0 || layer >= cfg.n_layers) return fail(QSA_ERR_INVALID_ARG, "layer %d out of range", layer);
+    if (!layers[layer].bound) return fail(QSA_ERR_STATE, "layer %d has no buffers bound", layer);
+    return QSA_OK;
+  }
+  LayerView view(int32_t layer) const {
+    const Layer& l = layers[layer];
+    char* wsp = static_cast<char*>(l.buf.workspace);
+    LayerView v;
+    v.cfg = cfg;
+    v.k_cache = l.buf.k_cache;
+    v.v_cache = l.buf.v_cache;
+    v.idx_cache = l.buf.idx_cache;
+    v.pooled_cache = l.buf.pooled_cache;
+    v.rms_gain = l.buf.rms_gain;
+    v.state = reinterpret_cast<DevState*>(wsp + ws.state);
+    v.scores = reinterpret_cast<float*>(wsp + ws.scores);
+    v.part_o = reinterpret_cast<float*>(wsp + ws.part_o);
+    v.part_ml = reinterpret_cast<float*>(wsp + ws.part_ml);
+    v.split = split;
+    v.n_sms = n_sms;
+    return v;
+  }
+};
+
+#define QSA_CHECK_PTR(p, a, name)                                                         \
+  do {                                                                                    \
+    if (!(p) || !aligned((p), (a)))                                                       \
+      return ctx->fail(QSA_ERR_INVALID_ARG, "%s must be a non-null %d-byte aligned pointer", \
+                       name, (int)(a));                                                   \
+  } while (0)
+
+extern "C" {
+
+size_t qsa_buffer_bytes(const qsa_config* cfg, int32_t which) {
+  if (!cfg || config_problem(*cfg)) return 0;
+  const qsa_config& c = *cfg;
+  switch (which) {
+    case QSA_BUF_KV: return size_t(c.max_ctx) * c.n_kv_heads * c.head_dim * 2;
+    case QSA_BUF_IDX: return size_t(c.max_ctx) * c.d_idx * 2;
+    case QSA_BUF_POOLED: return size_t(c.max_ctx / kBlock) * c.d_idx * 2;
+    case QSA_BUF_WORKSPACE: {
+      int dev = 0, sms = 0;
+      if (cudaGetDevice(&dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
+        sms = 148;
+      // the largest split count any device could choose (one SM per CTA)
+      const AttnSplit worst = attn_split(c, sms > 148 ? sms : 148);
+      const AttnSplit here = attn_split(c, sms);
+      const int n_splits = worst.n_splits > here.n_splits ? worst.n_splits : here.n_splits;
+      return workspace_layout(c, n_splits).total;
+    }
+    case QSA_BUF_MAX_CELLS: return size_t(max_cells_of(c));
+    default: return 0;
+  }
+}
+
+qsa_status qsa_create(const qsa_config* cfg, qsa_ctx** out) {
+  if (!cfg || !out) return QSA_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (config_problem(*cfg)) return QSA_ERR_UNSUPPORTED;
+  qsa_ctx* ctx = new (std::nothrow) qsa_ctx();
+  if (!ctx) return QSA_ERR_INVALID_ARG;
+  ctx->cfg = *cfg;
+  if (cudaGetDevice(&ctx->device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&ctx->n_sms, cudaDevAttrMultiProcessorCount, ctx->device) != cudaSuccess) {
+    delete ctx;
+    return QSA_ERR_CUDA;
+  }
+  ctx->split = attn_split(*cfg, ctx->n_sms);
+  const AttnSplit worst = attn_split(*cfg, ctx->n_sms > 148 ? ctx->n_sms : 148);
+  ctx->ws = workspace_layout(*cfg, worst.n_splits > ctx->split.n_splits ? worst.n_splits : ctx->split.n_splits);
+  ctx->layers.resize(cfg->n_layers);
+  *out = ctx;
+  return QSA_OK;
+}
+
+void qsa_destroy(qsa_ctx* ctx) { delete ctx; }
+
+const char* qsa_last_error(const qsa_ctx* ctx) { return ctx ? ctx->last_error.c_str() : "null context"; }
+
+qsa_status qsa_bind_layer(qsa_ctx* ctx, int32_t layer, const qsa_layer_buffers* buf, qsa_stream_t stream) {
+  if (!ctx) return QSA_ERR_INVALID_ARG;
+  if (!buf) return ctx->fail(QSA_ERR_INVALID_ARG, "buffers must not be null");
+  if (layer < 0 || layer >= ctx->cfg.n_layers) return ctx->fail(QSA_ERR_INVALID_ARG, "layer %d out of range", layer);
+  QSA_CHECK_PTR(buf->k_cache, 16, "k_cache");
+  QSA_CHECK_PTR(buf->v_cache, 16, "v_cache");
+  QSA_CHECK_PTR(buf->idx_cache, 16, "idx_cache");
+  QSA_CHECK_PTR(buf->pooled_cache, 16, "pooled_cache");
+  QSA_CHECK_PTR(buf->workspace, 256, "workspace");
+  if (buf->rms_gain && !aligned(buf->rms_gain, 16))
+    return ctx->fail(QSA_ERR_INVALID_ARG, "rms_gain must be 16-byte aligned");
+  Layer& l = ctx->layers[layer];
+  l.buf = *buf;
+  l.bound = true;
+  l.pending_blocks = 0;
+  qsa_status st = ctx->cuda(launch_set_state(ctx->view(layer), 0, 0, kSetReset, (cudaStream_t)stream), "bind_layer");
+  if (st != QSA_OK) l.bound = false;
+  return st;
+}
+
+qsa_status qsa_restore_layer(qsa_ctx* ctx, int32_t layer, int32_t n_ctx, int32_t n_pooled, qsa_stream_t stream) {
+  if (!ctx) return QSA_ERR_INVALID_ARG;
+  if (qsa_status st = ctx->layer_ok(layer)) return st;
+  if (n_ctx < 0 || n_ctx > ctx->cfg.max_ctx)
+    return ctx->fail(QSA_ERR_CAPACITY, "n_ctx %d outside [0, max_ctx=%d]", n_ctx, ctx->cfg.max_ctx);
+  if (n_pooled < 0 || n_pooled > n_ctx / kBlock)
+    return ctx->fail(QSA_ERR_INVALID_ARG, "n_pooled %d outside [0, n_ctx/4]", n_pooled);
+  ctx->layers[layer].pending_blocks = n_ctx / kBlock - n_pooled;
+  return ctx->cuda(launch_set_state(ctx->view(layer), n_ctx, n_pooled, kSetRestore, (cudaStream_t)stream),
+                   "restore_layer");
+}
+
+qsa_status qsa_read_layer_state(qsa_ctx* ctx, int32_t layer, int32_t* n_ctx, int32_t* n_pooled,
+                                int32_t* device_status, int32_t clear, qsa_stream_t stream) {
+  if (!ctx) return QSA_ERR_INVALID_ARG;
+  if (qsa_status st = ctx->layer_ok(layer)) return st;
+  LayerView v = ctx->view(layer);
+  if (qsa_status st = ctx->cuda(cudaStreamSynchronize((cudaStream_t)stream), "read_layer_state: sync")) return st;
+  DevState h;
+  if (qsa_status st = ctx->cuda(cudaMemcpy(&h, v.state, sizeof h, cudaMemcpyDeviceToHost), "read_layer_state: copy"))
+    return st;
+  if (n_ctx) *n_ctx = h.n_ctx;
+  if (n_pooled) *n_pooled = h.n_pooled;
+  if (device_status) *device_status = h.status;
+  if (clear) {
+    if (qsa_status st = ctx->cuda(launch_set_state(v, 0, 0, kSetClearStatus, (cudaStream_t)stream), "clear status"))
+      return st;
+    return ctx->cuda(cudaStreamSynchronize((cudaStream_t)stream), "read_layer_state: sync");
+  }
+  return QSA_OK;
+}
+
+qsa_status qsa_append_tokens(qsa_ctx* ctx, int32_t layer, int32_t n, const void* k, const void* v,
+                             const void* idx_key, qsa_stream_t stream) {
+  if (!ctx) return QSA_ERR_INVALID_ARG;
+  if (qsa_status st = ctx->layer_ok(layer)) return st;
+  if (n < 1 || n > ctx->cfg.max_ctx) return ctx->fail(QSA_ERR_CAPACITY, "cannot append %d tokens", n);
+  QSA_CHECK_PTR(k, 16, "k");
+  QSA_CHECK_PTR(v, 16, "v");
+  QSA_CHECK_PTR(idx_key, 16, "idx_key");
+  Layer& l = ctx->layers[layer];
+  l.pending_blocks += n / kBlock + 1;
+  if (l.pending_blocks > ctx->cfg.max_ctx / kBlock) l.pending_blocks = ctx->cfg.max_ctx / kBlock;
+  return ctx->cuda(launch_append(ctx->view(layer), n, k, v, idx_key, ctx->n_sms * 4, (cudaStream_t)stream),
+                   "append_tokens");
+}
+
+qsa_status qsa_append_token(qsa_ctx* ctx, int32_t layer, const void* k, const void* v, const void* idx_key,
+                            qsa_stream_t stream) {
+  return qsa_append_tokens(ctx, layer, 1, k, v, idx_key, stream);
+}
+
+qsa_status qsa_update_pooled_cache(qsa_ctx* ctx, int32_t layer, qsa_stream_t stream) {
+  if (!ctx) return QSA_ERR_INVALID_ARG;
+  if (qsa_status st = ctx->layer_ok(layer)) return st;
+  Layer& l = ctx->layers[layer];
+  // 8 warps per CTA, one block per warp per iteration
+  long long grid = (l.pending_blocks + 7) / 8;
+  if (grid < 1) grid = 1;
+  if (grid > ctx->n_sms * 8) grid = ctx->n_sms * 8;
+  l.pending_blocks = 0;
+  return ctx->cuda(launch_pool_update(ctx->view(layer), (int)grid, (cudaStream_t)stream), "update_pooled_cache");
+}
+
+qsa_status qsa_invalidate_pooled_cache(qsa_ctx* ctx, int32_t layer, int32_t from_block, qsa_stream_t stream) {
+  if (!ctx) return QSA_ERR_INVALID_ARG;
+  if (qsa_status st = ctx->layer_ok(layer)) return st;
+  if (from_block < 0) return ctx->fail(QSA_ERR_INVALID_ARG, "from_block must be >= 0");
+  Layer& l = ctx->layers[layer];
+  l.pending_blocks = ctx->cfg.max_ctx / kBlock - (from_block < ctx->cfg.max_ctx / kBlock ? from_block : 0);
+  return ctx->cuda(launch_set_state(ctx->view(layer), 0, from_block, kSetInvalidate, (cudaStream_t)stream),
+                   "invalidate_pooled_cache");
+}
+
+qsa_status qsa_index_topk(qsa_ctx* ctx, int32_t layer, const void* q_idx, const float* w, int32_t* sel_blocks,
+                          int32_t* n_sel, float* scores, qsa_stream_t stream) {
+  if (!ctx) return QSA_ERR_INVALID_ARG;
+  if (qsa_status st = ctx->layer_ok(layer)) return st;
+  QSA_CHECK_PTR(q_idx, 16, "q_idx");
+  QSA_CHECK_PTR(w, 16, "w");
+  QSA_CHECK_PTR(sel_blocks, 16, "sel_blocks");
+  QSA_CHECK_PTR(n_sel, 4, "n_sel");
+  if (scores && !aligned(scores, 16)) return ctx->fail(QSA_ERR_INVALID_ARG, "scores must be 16-byte aligned");
+  LayerView v = ctx->view(layer);
+  float* s = scores ? scores : v.scores;
+  if (qsa_status st = ctx->cuda(launch_index_scan(v, q_idx, w, s, (cudaStream_t)stream), "index scan")) return st;
+  return ctx->cuda(launch_topk(v, s, sel_blocks, n_sel, (cudaStream_t)stream), "block top-k");
+}
+
+qsa_status qsa_gather_kv(qsa_ctx* ctx, int32_t layer, const int32_t* sel_blocks, const int32_t* n_sel,
+                         int32_t* cells, int32_t* n_cells, void* k_compact, void* v_compact, qsa_stream_t stream) {
+  if (!ctx) return QSA_ERR_INVALID_ARG;
+  if (qsa_status st = ctx->layer_ok(layer)) return st;
+  QSA_CHECK_PTR(sel_blocks, 16, "sel_blocks");
+  QSA_CHECK_PTR(n_sel, 4, "n_sel");
+  QSA_CHECK_PTR(cells, 16, "cells");
+  QSA_CHECK_PTR(n_cells, 4, "n_cells");
+  if ((k_compact && !aligned(k_compact, 16)) || (v_compact && !aligned(v_compact, 16)))
+    return ctx->fail(QSA_ERR_INVALID_ARG, "compact K/V must be 16-byte aligned");
+  return ctx->cuda(launch_gather(ctx->view(layer), sel_blocks, n_sel, cells, n_cells, k_compact, v_compact,
+                                 (cudaStream_t)stream),
+                   "gather_kv");
+}
+
+qsa_status qsa_sparse_attend(qsa_ctx* ctx, int32_t layer, const void* q, const int32_t* cells,
+                             const int32_t* n_cells, float* out, qsa_stream_t stream) {
+  if (!ctx) return QSA_ERR_INVALID_ARG;
+  if (qsa_status st = ctx->layer_ok(layer)) return st;
+  QSA_CHECK_PTR(q, 16, "q");
+  QSA_CHECK_PTR(cells, 16, "cells");
+  QSA_CHECK_PTR(n_cells, 4, "n_cells");
+  QSA_CHECK_PTR(out, 16, "out");
+  return ctx->cuda(launch_attend(ctx->view(layer), q, cells, n_cells, out, (cudaStream_t)stream), "sparse_attend");
+}
+
+}  // extern "C"

@@ -1,0 +1,303 @@
+// Selected K/V gather and GQA sparse attention.
+//
+// Web page "Part 10" (第10回 EVO-X2 ... 長コンテキストのTGを高速化した話):
+//  - section "なぜFlash Attentionがcontext長に比例していたのか": with indexer_top_k = 2048
+//    and compression ratio 4, at most 2048 + 4 - 1 = 2051 cells are attended (the
+//    selected blocks plus the still-open tail block);
+//  - section "selected QSA K/V gather（COMMON-005）": attend only over the selected rows
+//    of K/V (the pages materialise compact K/V with get_rows and then run ordinary flash
+//    attention). Here the gather is fused into a split-KV flash-decode kernel that reads
+//    the selected rows straight from the f16 cache; qsa_gather_kv can still materialise
+//    the compact K/V.
+#include <cuda_fp16.h>
+
+#include "qsa_device.cuh"
+
+namespace qsa {
+
+// ---------------------------------------------------------------------------------
+// Cell expansion: block b -> cells 4b..4b+3, then the open tail [4*(n/4), n).
+// ---------------------------------------------------------------------------------
+__global__ void __launch_bounds__(1024) expand_cells_kernel(DevState* st, const int32_t* __restrict__ sel,
+                                                            const int32_t* __restrict__ n_sel,
+                                                            int32_t* __restrict__ cells,
+                                                            int32_t* __restrict__ n_cells, int k_blocks) {
+  pdl_wait();
+  const int n = ld_volatile(&st->n_ctx);
+  const int n_blocks = n / kBlock;
+  int ns = *n_sel;
+  if (ns < 0 || ns > k_blocks) {
+    if (threadIdx.x == 0) record_status(st, QSA_ERR_BAD_INDEX);
+    ns = ns < 0 ? 0 : k_blocks;
+  }
+  const int tail = n - kBlock * n_blocks;
+  const int total = kBlock * ns + tail;
+  for (int t = threadIdx.x; t < total; t += blockDim.x) {
+    int cell;
+    if (t < kBlock * ns) {
+      const int b = sel[t / kBlock];
+      if (b < 0 || b >= n_blocks) {
+        record_status(st, QSA_ERR_BAD_INDEX);
+        cell = -1;  // skipped by the attention kernel
+      } else {
+        cell = kBlock * b + (t % kBlock);
+      }
+    } else {
+      cell = kBlock * n_blocks + (t - kBlock * ns);
+    }
+    cells[t] = cell;
+  }
+  if (threadIdx.x == 0) *n_cells = total;
+}
+
+// Literal compact K/V (the pages' get_rows(K), get_rows(V)): row c of k_out/v_out is
+// the cache row of cells[c]; invalid cells give zero rows.
+__global__ void __launch_bounds__(256) gather_rows_kernel(DevState* st, const int32_t* __restrict__ cells,
+                                                          const int32_t* __restrict__ n_cells,
+                                                          const uint4* __restrict__ kc, const uint4* __restrict__ vc,
+                                                          uint4* __restrict__ k_out, uint4* __restrict__ v_out,
+                                                          int row_units, int max_cells) {
+  pdl_wait();
+  const int n = ld_volatile(&st->n_ctx);
+  int nc = *n_cells;
+  nc = nc < 0 ? 0 : (nc > max_cells ? max_cells : nc);
+  const size_t total = size_t(nc) * row_units;
+  for (size_t e = size_t(blockIdx.x) * blockDim.x + threadIdx.x; e < total; e += size_t(gridDim.x) * blockDim.x) {
+    const int c = int(e / row_units), u = int(e % row_units);
+    const int cell = cells[c];
+    uint4 kv = make_uint4(0, 0, 0, 0), vv = kv;
+    if (cell >= 0 && cell < n) {
+      kv = kc[size_t(cell) * row_units + u];
+      vv = vc[size_t(cell) * row_units + u];
+    }
+    if (k_out) k_out[e] = kv;
+    if (v_out) v_out[e] = vv;
+  }
+}
+
+cudaError_t launch_gather(const LayerView& L, const int32_t* sel, const int32_t* n_sel, int32_t* cells,
+                          int32_t* n_cells, void* k_compact, void* v_compact, cudaStream_t s) {
+  cudaError_t e = launch_pdl(expand_cells_kernel, dim3(1), dim3(1024), 0, s, 1, L.state, sel, n_sel, cells,
+                             n_cells, L.cfg.top_k_tokens / kBlock);
+  if (e != cudaSuccess || (!k_compact && !v_compact)) return e;
+  const int row_units = L.cfg.n_kv_heads * L.cfg.head_dim * 2 / 16;
+  const int max_cells = max_cells_of(L.cfg);
+  int grid = int((size_t(max_cells) * row_units + 255) / 256);
+  if (grid > L.n_sms * 4) grid = L.n_sms * 4;
+  return launch_pdl(gather_rows_kernel, dim3(grid), dim3(256), 0, s, 1, L.state, (const int32_t*)cells,
+                    (const int32_t*)n_cells, (const uint4*)L.k_cache, (const uint4*)L.v_cache, (uint4*)k_compact,
+                    (uint4*)v_compact, row_units, max_cells);
+}
+
+// ---------------------------------------------------------------------------------
+// Split-KV flash decode with the gather fused in. CTA (split s, KV head g) takes cells
+// [s*Lc, (s+1)*Lc) of the cell list; warp w takes every 8th of them. Lane l owns dims
+// [l*VPL, (l+1)*VPL) of K, V and of the G query heads that share KV head g, so each
+// warp reads every selected 2*D-byte K and V row of its cells with one coalesced load.
+// Logits -> per-head max/sum over the CTA's cells (f32) -> unnormalised partial output
+// with its (max, sum) pair; a second kernel merges the splits.
+// ---------------------------------------------------------------------------------
+template <int D, int G>
+__global__ void __launch_bounds__(256) attn_split_kernel(DevState* st, const __half* __restrict__ q,
+                                                         const int32_t* __restrict__ cells,
+                                                         const int32_t* __restrict__ n_cells,
+                                                         const __half* __restrict__ kc, const __half* __restrict__ vc,
+                                                         float* __restrict__ part_o, float* __restrict__ part_ml,
+                                                         int n_kv_heads, int cells_per_cta, int max_cells) {
+  constexpr int VPL = D / 32;
+  constexpr int W = kAttnWarps;
+  constexpr int JMAX = kAttnMaxCells / W;
+  constexpr int GR = G < 32 ? G : 32;  // heads reduced across lanes at once
+  static_assert(G <= 8, "at most 8 query heads per KV head");
+  __shared__ float s_p[G][kAttnMaxCells];
+  __shared__ float s_o[W][G][D];
+  __shared__ float s_m[G], s_l[G];
+
+  const int split = blockIdx.x, g = blockIdx.y;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int n_q_heads = n_kv_heads * G;
+
+  pdl_wait();
+  const int n = ld_volatile(&st->n_ctx);
+  int nc = *n_cells;
+  if (nc < 0 || nc > max_cells) {
+    if (split == 0 && g == 0 && threadIdx.x == 0) record_status(st, QSA_ERR_BAD_INDEX);
+    nc = nc < 0 ? 0 : max_cells;
+  }
+  const int c0 = split * cells_per_cta;
+  const int my_cells = max(0, min(cells_per_cta, nc - c0));
+
+  // this warp's cells: local index j*W + warp
+  int cid[JMAX];
+  bool valid[JMAX];
+#pragma unroll
+  for (int j = 0; j < JMAX; ++j) {
+    const int lc = j * W + warp;
+    cid[j] = lc < my_cells ? cells[c0 + lc] : -1;
+    valid[j] = lc < my_cells && cid[j] >= 0 && cid[j] < n;
+    if (lc < my_cells && !valid[j] && lane == 0) record_status(st, QSA_ERR_BAD_INDEX);
+  }
+  // issue every K and V row load before any arithmetic
+  float kv_k[JMAX][VPL], kv_v[JMAX][VPL];
+#pragma unroll
+  for (int j = 0; j < JMAX; ++j) {
+    if (valid[j]) {
+      const size_t off = (size_t(cid[j]) * n_kv_heads + g) * D + lane * VPL;
+      if constexpr (VPL == 4) {
+        const uint2 rk = *reinterpret_cast<const uint2*>(kc + off);
+        const uint2 rv = *reinterpret_cast<const uint2*>(vc + off);
+        const float2 k0 = __half22float2(*reinterpret_cast<const __half2*>(&rk.x));
+        const float2 k1 = __half22float2(*reinterpret_cast<const __half2*>(&rk.y));
+        const float2 v0 = __half22float2(*reinterpret_cast<const __half2*>(&rv.x));
+        const float2 v1 = __half22float2(*reinterpret_cast<const __half2*>(&rv.y));
+        kv_k[j][0] = k0.x; kv_k[j][1] = k0.y; kv_k[j][2] = k1.x; kv_k[j][3] = k1.y;
+        kv_v[j][0] = v0.x; kv_v[j][1] = v0.y; kv_v[j][2] = v1.x; kv_v[j][3] = v1.y;
+      } else {
+        const float2 k0 = __half22float2(*reinterpret_cast<const __half2*>(kc + off));
+        const float2 v0 = __half22float2(*reinterpret_cast<const __half2*>(vc + off));
+        kv_k[j][0] = k0.x; kv_k[j][1] = k0.y;
+        kv_v[j][0] = v0.x; kv_v[j][1] = v0.y;
+      }
+    } else {
+#pragma unroll
+      for (int x = 0; x < VPL; ++x) kv_k[j][x] = kv_v[j][x] = 0.0f;
+    }
+  }
+  float qv[G][VPL];
+#pragma unroll
+  for (int h = 0; h < G; ++h)
+#pragma unroll
+    for (int x = 0; x < VPL; ++x) qv[h][x] = __half2float(q[(size_t(g) * G + h) * D + lane * VPL + x]);
+
+  const float scale = 1.0f / sqrtf((float)D);
+  // logits
+#pragma unroll
+  for (int j = 0; j < JMAX; ++j) {
+    const int lc = j * W + warp;
+    if (lc < my_cells) {  // warp-uniform
+      float dot[GR];
+#pragma unroll
+      for (int h = 0; h < GR; ++h) {
+        float a = 0.0f;
+#pragma unroll
+        for (int x = 0; x < VPL; ++x) a = fmaf(qv[h][x], kv_k[j][x], a);
+        dot[h] = a;
+      }
+      const float mine = transpose_reduce<GR>(dot, lane);
+      const int h = head_of_lane<GR>(lane);
+      if ((lane & (32 / GR - 1)) == 0) s_p[h][lc] = valid[j] ? mine * scale : -INFINITY;
+    }
+  }
+  __syncthreads();
+  // per-head max and sum over this CTA's cells
+  for (int h = warp; h < G; h += W) {
+    float m = -INFINITY;
+    for (int c = lane; c < my_cells; c += 32) m = fmaxf(m, s_p[h][c]);
+    m = warp_max(m);
+    float l = 0.0f;
+    for (int c = lane; c < my_cells; c += 32) {
+      const float p = m == -INFINITY ? 0.0f : expf(s_p[h][c] - m);
+      s_p[h][c] = p;
+      l += p;
+    }
+    l = warp_sum(l);
+    if (lane == 0) {
+      s_m[h] = m;
+      s_l[h] = l;
+    }
+  }
+  __syncthreads();
+  // unnormalised P.V over this warp's cells
+  float o[G][VPL];
+#pragma unroll
+  for (int h = 0; h < G; ++h)
+#pragma unroll
+    for (int x = 0; x < VPL; ++x) o[h][x] = 0.0f;
+#pragma unroll
+  for (int j = 0; j < JMAX; ++j) {
+    const int lc = j * W + warp;
+    if (lc < my_cells) {
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const float p = s_p[h][lc];
+#pragma unroll
+        for (int x = 0; x < VPL; ++x) o[h][x] = fmaf(p, kv_v[j][x], o[h][x]);
+      }
+    }
+  }
+#pragma unroll
+  for (int h = 0; h < G; ++h)
+#pragma unroll
+    for (int x = 0; x < VPL; ++x) s_o[warp][h][lane * VPL + x] = o[h][x];
+  __syncthreads();
+  // sum over warps (fixed order) and store the partial of this split
+  for (int e = threadIdx.x; e < G * D; e += blockDim.x) {
+    const int h = e / D, d = e % D;
+    float acc = 0.0f;
+#pragma unroll
+    for (int w = 0; w < W; ++w) acc += s_o[w][h][d];
+    part_o[(size_t(split) * n_q_heads + g * G + h) * D + d] = acc;
+  }
+  if (threadIdx.x < G) {
+    const int h = threadIdx.x;
+    part_ml[(size_t(split) * n_q_heads + g * G + h) * 2 + 0] = s_m[h];
+    part_ml[(size_t(split) * n_q_heads + g * G + h) * 2 + 1] = s_l[h];
+  }
+}
+
+// Merge the splits of one query head: out = sum_s e^(m_s-M) o_s / sum_s e^(m_s-M) l_s.
+__global__ void __launch_bounds__(128) attn_combine_kernel(const float* __restrict__ part_o,
+                                                           const float* __restrict__ part_ml,
+                                                           float* __restrict__ out, int n_q_heads, int D,
+                                                           int n_splits) {
+  pdl_wait();
+  const int i = blockIdx.x;
+  float M = -INFINITY;
+  for (int s = 0; s < n_splits; ++s) M = fmaxf(M, part_ml[(size_t(s) * n_q_heads + i) * 2]);
+  for (int d = threadIdx.x; d < D; d += blockDim.x) {
+    float acc = 0.0f, den = 0.0f;
+    if (M != -INFINITY) {
+      for (int s = 0; s < n_splits; ++s) {
+        const float m = part_ml[(size_t(s) * n_q_heads + i) * 2];
+        if (m == -INFINITY) continue;
+        const float e = expf(m - M);
+        acc = fmaf(e, part_o[(size_t(s) * n_q_heads + i) * D + d], acc);
+        den = fmaf(e, part_ml[(size_t(s) * n_q_heads + i) * 2 + 1], den);
+      }
+    }
+    out[size_t(i) * D + d] = den > 0.0f ? acc / den : 0.0f;
+  }
+}
+
+template <int D>
+static cudaError_t launch_attn_d(const LayerView& L, const void* q, const int32_t* cells, const int32_t* n_cells,
+                                 cudaStream_t s) {
+  const dim3 grid(L.split.n_splits, L.cfg.n_kv_heads), block(kAttnWarps * 32);
+  const int G = L.cfg.n_q_heads / L.cfg.n_kv_heads;
+  const int mc = L.split.n_splits * L.split.cells_per_cta;
+  const int maxc = max_cells_of(L.cfg) < mc ? max_cells_of(L.cfg) : mc;
+#define QSA_ATTN_CASE(GG)                                                                                   \
+  case GG:                                                                                                  \
+    return launch_pdl(attn_split_kernel<D, GG>, grid, block, 0, s, 1, L.state, (const __half*)q, cells,     \
+                      n_cells, (const __half*)L.k_cache, (const __half*)L.v_cache, L.part_o, L.part_ml,     \
+                      L.cfg.n_kv_heads, L.split.cells_per_cta, maxc);
+  switch (G) {
+    QSA_ATTN_CASE(1)
+    QSA_ATTN_CASE(2)
+    QSA_ATTN_CASE(4)
+    QSA_ATTN_CASE(8)
+    default: return cudaErrorInvalidValue;
+  }
+#undef QSA_ATTN_CASE
+}
+
+cudaError_t launch_attend(const LayerView& L, const void* q, const int32_t* cells, const int32_t* n_cells,
+                          float* out, cudaStream_t s) {
+  cudaError_t e = L.cfg.head_dim == 128 ? launch_attn_d<128>(L, q, cells, n_cells, s)
+                                        : launch_attn_d<64>(L, q, cells, n_cells, s);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(attn_combine_kernel, dim3(L.cfg.n_q_heads), dim3(128), 0, s, 1, (const float*)L.part_o,
+                    (const float*)L.part_ml, out, L.cfg.n_q_heads, L.cfg.head_dim, L.split.n_splits);
+}
+
+}  // namespace qsa

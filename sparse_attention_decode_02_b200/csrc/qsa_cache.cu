@@ -1,0 +1,175 @@
+// Sequence state, token append and the incremental pooled-key cache.
+//
+// Incremental pooled-key cache: web page "Part 10" (第10回 EVO-X2 ... 長コンテキストのTGを
+// 高速化した話), section "incremental pooled-key cache（COMMON-004）": completed-block
+// summaries are kept per layer and only blocks that completed (or were invalidated)
+// since the last update are computed. Summary of block b (section "QSA indexer"):
+// mean of its 4 raw indexer keys -> RMS norm -> RoPE at the block position 4b, stored
+// as f16. RoPE is the NeoX half-split rotation of pair (i, i+d/2) by angle
+// pos * base^(-2i/d); angles and their sine/cosine are taken in double precision so that
+// positions near 2.6e5 keep full accuracy, then the rotation itself runs in f32.
+#include <cuda_fp16.h>
+
+#include "qsa_device.cuh"
+
+namespace qsa {
+
+__global__ void set_state_kernel(DevState* st, int n_ctx, int n_pooled, int mode) {
+  pdl_wait();
+  if (threadIdx.x != 0) return;
+  if (mode == kSetReset) {
+    st->n_ctx = 0;
+    st->n_pooled = 0;
+    st->status = 0;
+    st->ticket_append = 0;
+    st->ticket_pool = 0;
+  } else if (mode == kSetRestore) {
+    st->n_ctx = n_ctx;
+    st->n_pooled = n_pooled;
+    st->status = 0;
+    st->ticket_append = 0;
+    st->ticket_pool = 0;
+  } else if (mode == kSetInvalidate) {
+    if (st->n_pooled > n_pooled) st->n_pooled = n_pooled;
+  } else {
+    st->status = 0;
+  }
+}
+
+cudaError_t launch_set_state(const LayerView& L, int n_ctx, int n_pooled, int mode, cudaStream_t s) {
+  return launch_pdl(set_state_kernel, dim3(1), dim3(32), 0, s, 1, L.state, n_ctx, n_pooled, mode);
+}
+
+// Appends n tokens at position n_ctx: three contiguous copies (token-major caches), in
+// 16-byte units. All CTAs read n_ctx before any of them can change it: the last CTA to
+// finish (atomic ticket) publishes n_ctx + n.
+__global__ void __launch_bounds__(256) append_kernel(DevState* st, uint4* kc, uint4* vc, uint4* ic,
+                                                     const uint4* k, const uint4* v, const uint4* idx,
+                                                     int n, int kv_units, int idx_units, int max_ctx) {
+  pdl_wait();
+  const int base = ld_volatile(&st->n_ctx);
+  const bool fits = base >= 0 && base + n <= max_ctx;
+  if (fits) {
+    const size_t nkv = size_t(n) * kv_units, nidx = size_t(n) * idx_units;
+    const size_t okv = size_t(base) * kv_units, oidx = size_t(base) * idx_units;
+    const size_t stride = size_t(gridDim.x) * blockDim.x;
+    for (size_t i = size_t(blockIdx.x) * blockDim.x + threadIdx.x; i < nkv; i += stride) {
+      kc[okv + i] = k[i];
+      vc[okv + i] = v[i];
+    }
+    for (size_t i = size_t(blockIdx.x) * blockDim.x + threadIdx.x; i < nidx; i += stride)
+      ic[oidx + i] = idx[i];
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    const unsigned t = atomicAdd(&st->ticket_append, 1u);
+    if (t == gridDim.x - 1) {
+      if (fits) st->n_ctx = base + n;
+      else record_status(st, QSA_ERR_CAPACITY);
+      st->ticket_append = 0;
+      __threadfence();
+    }
+  }
+}
+
+cudaError_t launch_append(const LayerView& L, int n, const void* k, const void* v, const void* idx,
+                          int grid_hint, cudaStream_t s) {
+  const int kv_units = L.cfg.n_kv_heads * L.cfg.head_dim * 2 / 16;
+  const int idx_units = L.cfg.d_idx * 2 / 16;
+  long long work = (long long)n * kv_units;
+  int grid = int((work + 256 * 4 - 1) / (256 * 4));
+  if (grid < 1) grid = 1;
+  if (grid > grid_hint) grid = grid_hint;
+  return launch_pdl(append_kernel, dim3(grid), dim3(256), 0, s, 1, L.state, (uint4*)L.k_cache,
+                    (uint4*)L.v_cache, (uint4*)L.idx_cache, (const uint4*)k, (const uint4*)v,
+                    (const uint4*)idx, n, kv_units, idx_units, L.cfg.max_ctx);
+}
+
+// One warp per block summary. Lane `lane` owns the rotation pairs i = lane*P + j (j < P,
+// P = D/64) and their partners i + D/2.
+template <int D>
+__global__ void __launch_bounds__(256) pool_update_kernel(DevState* st, const __half* __restrict__ ic,
+                                                          __half* __restrict__ pc,
+                                                          const float* __restrict__ gain, float eps,
+                                                          float rope_base) {
+  constexpr int P = D / 64;
+  constexpr int HALF = D / 2;
+  pdl_wait();
+  const int n = ld_volatile(&st->n_ctx);
+  const int b_first = ld_volatile(&st->n_pooled);
+  const int b_end = n / kBlock;
+  const int lane = threadIdx.x & 31;
+  const int warps = blockDim.x >> 5;
+  const int gw = blockIdx.x * warps + (threadIdx.x >> 5);
+
+  double theta[P];
+  float g1[P], g2[P];
+#pragma unroll
+  for (int j = 0; j < P; ++j) {
+    const int i = lane * P + j;
+    theta[j] = pow((double)rope_base, -2.0 * (double)i / (double)D);
+    g1[j] = gain ? gain[i] : 1.0f;
+    g2[j] = gain ? gain[i + HALF] : 1.0f;
+  }
+
+  for (int b = b_first + gw; b < b_end; b += gridDim.x * warps) {
+    float m1[P], m2[P];
+#pragma unroll
+    for (int j = 0; j < P; ++j) m1[j] = m2[j] = 0.0f;
+    // mean of the 4 raw indexer keys, summed in token order
+#pragma unroll
+    for (int t = 0; t < kBlock; ++t) {
+      const __half* row = ic + (size_t(b) * kBlock + t) * D;
+#pragma unroll
+      for (int j = 0; j < P; ++j) {
+        m1[j] += __half2float(row[lane * P + j]);
+        m2[j] += __half2float(row[lane * P + j + HALF]);
+      }
+    }
+    float ss = 0.0f;
+#pragma unroll
+    for (int j = 0; j < P; ++j) {
+      m1[j] *= 0.25f;
+      m2[j] *= 0.25f;
+      ss += m1[j] * m1[j] + m2[j] * m2[j];
+    }
+    ss = warp_sum(ss);
+    const float inv_rms = 1.0f / sqrtf(ss / (float)D + eps);
+    const double pos = (double)(b * kBlock);
+#pragma unroll
+    for (int j = 0; j < P; ++j) {
+      const float r1 = m1[j] * inv_rms * g1[j];
+      const float r2 = m2[j] * inv_rms * g2[j];
+      double sd, cd;
+      sincos(pos * theta[j], &sd, &cd);
+      const float c = (float)cd, s = (float)sd;
+      const int i = lane * P + j;
+      pc[size_t(b) * D + i] = __float2half_rn(r1 * c - r2 * s);
+      pc[size_t(b) * D + i + HALF] = __float2half_rn(r1 * s + r2 * c);
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    const unsigned t = atomicAdd(&st->ticket_pool, 1u);
+    if (t == gridDim.x - 1) {
+      if (b_end > b_first) st->n_pooled = b_end;
+      st->ticket_pool = 0;
+      __threadfence();
+    }
+  }
+}
+
+cudaError_t launch_pool_update(const LayerView& L, int grid_hint, cudaStream_t s) {
+  const int grid = grid_hint < 1 ? 1 : grid_hint;
+  if (L.cfg.d_idx == 128)
+    return launch_pdl(pool_update_kernel<128>, dim3(grid), dim3(256), 0, s, 1, L.state,
+                      (const __half*)L.idx_cache, (__half*)L.pooled_cache, L.rms_gain, L.cfg.rms_eps,
+                      L.cfg.rope_base);
+  return launch_pdl(pool_update_kernel<64>, dim3(grid), dim3(256), 0, s, 1, L.state,
+                    (const __half*)L.idx_cache, (__half*)L.pooled_cache, L.rms_gain, L.cfg.rms_eps,
+                    L.cfg.rope_base);
+}
+
+}  // namespace qsa

@@ -1,0 +1,107 @@
+// Internal declarations shared by the library's translation units: the device-side
+// sequence state, the workspace layout and the kernel launchers.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/qsa.h"
+
+namespace qsa {
+
+constexpr int kBlock = 4;             // tokens per micro-block (compression ratio 4)
+constexpr int kTopkCluster = 8;       // CTAs in the top-k cluster
+constexpr int kTopkThreads = 1024;
+constexpr int kTopkMaxPerCta = 32768; // keys held in shared memory per top-k CTA
+constexpr int kAttnWarps = 8;         // warps per attention CTA
+constexpr int kAttnMaxCells = 64;     // cells per attention CTA (split size cap)
+
+// Device-resident sequence state of one layer; lives at the start of the workspace.
+struct DevState {
+  int32_t n_ctx;          // tokens in the caches
+  int32_t n_pooled;       // completed blocks whose summaries are valid
+  int32_t status;         // first device-side error (qsa_status), 0 if none
+  uint32_t ticket_append; // last-CTA tickets of multi-CTA kernels (reset by the last CTA)
+  uint32_t ticket_pool;
+  int32_t reserved[59];
+};
+static_assert(sizeof(DevState) == 256, "DevState must stay 256 bytes");
+
+// Byte offsets inside a layer's workspace (all 256-byte aligned).
+struct WorkspaceLayout {
+  size_t state, scores, part_o, part_ml, total;
+};
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Attention split: each CTA of the split-KV kernel takes `cells_per_cta` cells of one
+// KV head; `n_splits` CTAs per KV head cover the largest cell set.
+struct AttnSplit {
+  int cells_per_cta;
+  int n_splits;
+};
+
+inline int max_cells_of(const qsa_config& c) { return kBlock * (c.top_k_tokens / kBlock) + kBlock - 1; }
+
+inline AttnSplit attn_split(const qsa_config& c, int n_sms) {
+  int max_cells = max_cells_of(c);
+  int per_head = n_sms / c.n_kv_heads;
+  if (per_head < 1) per_head = 1;
+  int l = (max_cells + per_head - 1) / per_head;
+  l = (l + 7) / 8 * 8;
+  if (l < 8) l = 8;
+  if (l > kAttnMaxCells) l = kAttnMaxCells;
+  return AttnSplit{l, (max_cells + l - 1) / l};
+}
+
+inline WorkspaceLayout workspace_layout(const qsa_config& c, int n_splits) {
+  WorkspaceLayout w{};
+  size_t off = 0;
+  w.state = off;
+  off += align256(sizeof(DevState));
+  w.scores = off;
+  off += align256(size_t(c.max_ctx / kBlock) * sizeof(float));
+  w.part_o = off;
+  off += align256(size_t(n_splits) * c.n_q_heads * c.head_dim * sizeof(float));
+  w.part_ml = off;
+  off += align256(size_t(n_splits) * c.n_q_heads * 2 * sizeof(float));
+  w.total = off;
+  return w;
+}
+
+// Everything a launcher needs about one bound layer.
+struct LayerView {
+  qsa_config cfg;
+  void* k_cache;
+  void* v_cache;
+  void* idx_cache;
+  void* pooled_cache;
+  const float* rms_gain;
+  DevState* state;
+  float* scores;          // workspace scores
+  float* part_o;
+  float* part_ml;
+  AttnSplit split;
+  int n_sms;
+};
+
+// ---- launchers (return the launch's cudaError_t) ----
+cudaError_t launch_set_state(const LayerView& L, int n_ctx, int n_pooled, int mode, cudaStream_t s);
+cudaError_t launch_append(const LayerView& L, int n, const void* k, const void* v,
+                          const void* idx, int grid_hint, cudaStream_t s);
+cudaError_t launch_pool_update(const LayerView& L, int grid_hint, cudaStream_t s);
+cudaError_t launch_index_scan(const LayerView& L, const void* q_idx, const float* w,
+                              float* scores, cudaStream_t s);
+cudaError_t launch_topk(const LayerView& L, const float* scores, int32_t* sel, int32_t* n_sel,
+                        cudaStream_t s);
+cudaError_t launch_gather(const LayerView& L, const int32_t* sel, const int32_t* n_sel,
+                          int32_t* cells, int32_t* n_cells, void* k_compact, void* v_compact,
+                          cudaStream_t s);
+cudaError_t launch_attend(const LayerView& L, const void* q, const int32_t* cells,
+                          const int32_t* n_cells, float* out, cudaStream_t s);
+
+// set_state modes
+enum { kSetReset = 0, kSetRestore = 1, kSetInvalidate = 2, kSetClearStatus = 3 };
+
+}  // namespace qsa

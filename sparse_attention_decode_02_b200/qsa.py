@@ -1,0 +1,209 @@
+"""Thin ctypes binding of libqsa.so (include/qsa.h): argument marshalling only.
+
+Every call takes torch tensors that already live on the GPU and passes their device
+pointers and the stream handle to the C ABI; every step of the decode path runs in
+the library's CUDA kernels. There is no fallback: if libqsa.so is missing or cannot be
+loaded, importing the binding's library raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from ctypes import c_float, c_int32, c_size_t, c_void_p
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libqsa.so")
+
+QSA_OK = 0
+STATUS_NAMES = {0: "QSA_OK", 1: "QSA_ERR_INVALID_ARG", 2: "QSA_ERR_CAPACITY", 3: "QSA_ERR_STATE",
+                4: "QSA_ERR_CUDA", 5: "QSA_ERR_UNSUPPORTED", 6: "QSA_ERR_BAD_INDEX"}
+QSA_BUF_KV, QSA_BUF_IDX, QSA_BUF_POOLED, QSA_BUF_WORKSPACE, QSA_BUF_MAX_CELLS = range(5)
+
+
+class QsaError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+class QsaConfig(ctypes.Structure):
+    _fields_ = [("n_layers", c_int32), ("max_ctx", c_int32), ("d_idx", c_int32),
+                ("n_idx_heads", c_int32), ("top_k_tokens", c_int32), ("n_q_heads", c_int32),
+                ("n_kv_heads", c_int32), ("head_dim", c_int32), ("rope_base", c_float),
+                ("rms_eps", c_float)]
+
+
+class QsaLayerBuffers(ctypes.Structure):
+    _fields_ = [("k_cache", c_void_p), ("v_cache", c_void_p), ("idx_cache", c_void_p),
+                ("pooled_cache", c_void_p), ("rms_gain", c_void_p), ("workspace", c_void_p)]
+
+
+_P = c_void_p
+_I = c_int32
+# name -> (restype, argtypes); must list every function include/qsa.h declares
+SIGNATURES = {
+    "qsa_buffer_bytes": (c_size_t, [ctypes.POINTER(QsaConfig), _I]),
+    "qsa_create": (_I, [ctypes.POINTER(QsaConfig), ctypes.POINTER(_P)]),
+    "qsa_destroy": (None, [_P]),
+    "qsa_last_error": (ctypes.c_char_p, [_P]),
+    "qsa_bind_layer": (_I, [_P, _I, ctypes.POINTER(QsaLayerBuffers), _P]),
+    "qsa_restore_layer": (_I, [_P, _I, _I, _I, _P]),
+    "qsa_read_layer_state": (_I, [_P, _I, ctypes.POINTER(_I), ctypes.POINTER(_I), ctypes.POINTER(_I), _I, _P]),
+    "qsa_append_token": (_I, [_P, _I, _P, _P, _P, _P]),
+    "qsa_append_tokens": (_I, [_P, _I, _I, _P, _P, _P, _P]),
+    "qsa_update_pooled_cache": (_I, [_P, _I, _P]),
+    "qsa_invalidate_pooled_cache": (_I, [_P, _I, _I, _P]),
+    "qsa_index_topk": (_I, [_P, _I, _P, _P, _P, _P, _P, _P]),
+    "qsa_gather_kv": (_I, [_P, _I, _P, _P, _P, _P, _P, _P, _P]),
+    "qsa_sparse_attend": (_I, [_P, _I, _P, _P, _P, _P, _P]),
+}
+
+_lib = None
+
+
+def load_library(path: str | None = None) -> ctypes.CDLL:
+    """Load libqsa.so and declare its signatures. Raises if it is missing."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise ImportError(f"{p} is missing: build it with `python -m sparse_attention_decode_02_b200.build`")
+    lib = ctypes.CDLL(p)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def _ptr(t):
+    """Device pointer of a torch tensor (None -> NULL)."""
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensors passed to the QSA library must live on the GPU")
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to the QSA library must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return getattr(stream, "cuda_stream", stream)
+
+
+def make_config(n_layers, max_ctx, d_idx, n_idx_heads, top_k_tokens, n_q_heads, n_kv_heads, head_dim,
+                rope_base=10000.0, rms_eps=1e-6) -> QsaConfig:
+    return QsaConfig(n_layers, max_ctx, d_idx, n_idx_heads, top_k_tokens, n_q_heads, n_kv_heads, head_dim,
+                     rope_base, rms_eps)
+
+
+def buffer_bytes(cfg: QsaConfig, which: int) -> int:
+    return int(load_library().qsa_buffer_bytes(ctypes.byref(cfg), which))
+
+
+class Qsa:
+    """One library context (qsa_ctx) on the current CUDA device. Method names follow the C ABI."""
+
+    def __init__(self, cfg: QsaConfig):
+        self.lib = load_library()
+        self.cfg = cfg
+        h = c_void_p()
+        st = self.lib.qsa_create(ctypes.byref(cfg), ctypes.byref(h))
+        if st != QSA_OK:
+            raise QsaError(st, "qsa_create rejected the configuration")
+        self.handle = h
+
+    def close(self):
+        if getattr(self, "handle", None):
+            self.lib.qsa_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def _check(self, st):
+        if st != QSA_OK:
+            msg = self.lib.qsa_last_error(self.handle)
+            raise QsaError(st, msg.decode() if msg else "")
+
+    def buffer_bytes(self, which: int) -> int:
+        return buffer_bytes(self.cfg, which)
+
+    def bind_layer(self, layer, k_cache, v_cache, idx_cache, pooled_cache, workspace, rms_gain=None,
+                   stream=None):
+        b = QsaLayerBuffers(_ptr(k_cache), _ptr(v_cache), _ptr(idx_cache), _ptr(pooled_cache),
+                            _ptr(rms_gain), _ptr(workspace))
+        self._check(self.lib.qsa_bind_layer(self.handle, layer, ctypes.byref(b), _stream(stream)))
+
+    def restore_layer(self, layer, n_ctx, n_pooled, stream=None):
+        self._check(self.lib.qsa_restore_layer(self.handle, layer, n_ctx, n_pooled, _stream(stream)))
+
+    def read_layer_state(self, layer, clear=False, stream=None):
+        n, p, s = c_int32(), c_int32(), c_int32()
+        self._check(self.lib.qsa_read_layer_state(self.handle, layer, ctypes.byref(n), ctypes.byref(p),
+                                                  ctypes.byref(s), int(clear), _stream(stream)))
+        return n.value, p.value, s.value
+
+    def append_token(self, layer, k, v, idx_key, stream=None):
+        self._check(self.lib.qsa_append_token(self.handle, layer, _ptr(k), _ptr(v), _ptr(idx_key),
+                                              _stream(stream)))
+
+    def append_tokens(self, layer, k, v, idx_key, stream=None):
+        self._check(self.lib.qsa_append_tokens(self.handle, layer, int(k.shape[0]), _ptr(k), _ptr(v),
+                                               _ptr(idx_key), _stream(stream)))
+
+    def update_pooled_cache(self, layer, stream=None):
+        self._check(self.lib.qsa_update_pooled_cache(self.handle, layer, _stream(stream)))
+
+    def invalidate_pooled_cache(self, layer, from_block, stream=None):
+        self._check(self.lib.qsa_invalidate_pooled_cache(self.handle, layer, from_block, _stream(stream)))
+
+    def index_topk(self, layer, q_idx, w, sel_blocks, n_sel, scores=None, stream=None):
+        self._check(self.lib.qsa_index_topk(self.handle, layer, _ptr(q_idx), _ptr(w), _ptr(sel_blocks),
+                                            _ptr(n_sel), _ptr(scores), _stream(stream)))
+
+    def gather_kv(self, layer, sel_blocks, n_sel, cells, n_cells, k_compact=None, v_compact=None,
+                  stream=None):
+        self._check(self.lib.qsa_gather_kv(self.handle, layer, _ptr(sel_blocks), _ptr(n_sel), _ptr(cells),
+                                           _ptr(n_cells), _ptr(k_compact), _ptr(v_compact), _stream(stream)))
+
+    def sparse_attend(self, layer, q, cells, n_cells, out, stream=None):
+        self._check(self.lib.qsa_sparse_attend(self.handle, layer, _ptr(q), _ptr(cells), _ptr(n_cells),
+                                               _ptr(out), _stream(stream)))
+
+
+def alloc_layer(cfg: QsaConfig, device="cuda"):
+    """Allocate one layer's buffers with torch (the caller owns them)."""
+    import torch
+    kv_elems = buffer_bytes(cfg, QSA_BUF_KV) // 2
+    return {
+        "k_cache": torch.zeros(kv_elems, dtype=torch.float16, device=device).view(
+            cfg.max_ctx, cfg.n_kv_heads, cfg.head_dim),
+        "v_cache": torch.zeros(kv_elems, dtype=torch.float16, device=device).view(
+            cfg.max_ctx, cfg.n_kv_heads, cfg.head_dim),
+        "idx_cache": torch.zeros(cfg.max_ctx, cfg.d_idx, dtype=torch.float16, device=device),
+        "pooled_cache": torch.zeros(cfg.max_ctx // 4, cfg.d_idx, dtype=torch.float16, device=device),
+        "workspace": torch.zeros(buffer_bytes(cfg, QSA_BUF_WORKSPACE), dtype=torch.uint8, device=device),
+    }
+
+
+def alloc_step_outputs(cfg: QsaConfig, device="cuda"):
+    """Per-step output buffers: selected blocks, cells, counts and the attention output."""
+    import torch
+    k_blocks = cfg.top_k_tokens // 4
+    return {
+        "sel": torch.zeros(k_blocks, dtype=torch.int32, device=device),
+        "n_sel": torch.zeros(4, dtype=torch.int32, device=device),
+        "cells": torch.zeros(4 * k_blocks + 3, dtype=torch.int32, device=device),
+        "n_cells": torch.zeros(4, dtype=torch.int32, device=device),
+        "out": torch.zeros(cfg.n_q_heads, cfg.head_dim, dtype=torch.float32, device=device),
+    }

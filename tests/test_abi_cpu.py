@@ -1,0 +1,76 @@
+"""C-ABI library checks that need no GPU: it loads, exports every declared symbol, and
+validates configurations and sizes on the host."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import sparse_attention_decode_02_b200 as qsa_pkg
+from sparse_attention_decode_02_b200 import build as qbuild
+from sparse_attention_decode_02_b200 import qsa as Q
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for h in os.listdir(os.path.join(ROOT, "include")):
+        if h.endswith(".h"):
+            txt = open(os.path.join(ROOT, "include", h)).read()
+            txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+            names |= set(re.findall(r"\b(qsa_[a-z0-9_]+)\s*\(", txt))
+    return names
+
+
+@pytest.fixture(scope="module")
+def lib():
+    qbuild.build()
+    return Q.load_library()
+
+
+def test_library_exports_every_declared_function(lib):
+    declared = _declared()
+    assert len(declared) >= 14
+    for name in sorted(declared):
+        assert hasattr(lib, name), f"libqsa.so does not export {name}"
+    # the binding declares a signature for every function of the header
+    assert declared <= set(Q.SIGNATURES), declared - set(Q.SIGNATURES)
+
+
+def test_buffer_sizes(lib):
+    cfg = Q.make_config(12, 255184 + 512, 128, 16, 2048, 32, 4, 128)
+    assert Q.buffer_bytes(cfg, Q.QSA_BUF_KV) == cfg.max_ctx * 4 * 128 * 2
+    assert Q.buffer_bytes(cfg, Q.QSA_BUF_IDX) == cfg.max_ctx * 128 * 2
+    assert Q.buffer_bytes(cfg, Q.QSA_BUF_POOLED) == cfg.max_ctx // 4 * 128 * 2
+    assert Q.buffer_bytes(cfg, Q.QSA_BUF_MAX_CELLS) == 2051
+    ws = Q.buffer_bytes(cfg, Q.QSA_BUF_WORKSPACE)
+    assert ws % 256 == 0 and ws >= 256 + cfg.max_ctx // 4 * 4
+
+
+@pytest.mark.parametrize("bad", [
+    dict(d_idx=96), dict(n_idx_heads=3), dict(n_idx_heads=32), dict(top_k_tokens=2046),
+    dict(head_dim=256), dict(n_q_heads=32, n_kv_heads=2), dict(max_ctx=1026), dict(max_ctx=4 << 20),
+    dict(n_layers=0),
+])
+def test_unsupported_configs_are_rejected(lib, bad):
+    base = dict(n_layers=1, max_ctx=4096, d_idx=128, n_idx_heads=16, top_k_tokens=2048, n_q_heads=32,
+                n_kv_heads=4, head_dim=128)
+    base.update(bad)
+    cfg = Q.make_config(**base)
+    assert Q.buffer_bytes(cfg, Q.QSA_BUF_KV) == 0
+    h = ctypes.c_void_p()
+    assert lib.qsa_create(ctypes.byref(cfg), ctypes.byref(h)) == 5  # QSA_ERR_UNSUPPORTED
+    assert not h.value
+
+
+def test_null_arguments_are_rejected(lib):
+    assert lib.qsa_create(None, None) == 1
+    lib.qsa_destroy(None)  # no-op
+    assert lib.qsa_last_error(None) == b"null context"
+
+
+def test_binding_has_no_fallback(tmp_path):
+    with pytest.raises(ImportError):
+        Q.load_library(str(tmp_path / "missing.so"))
+    assert qsa_pkg.Qsa is Q.Qsa
