@@ -163,13 +163,23 @@ qsa_status qsa_index_topk(qsa_ctx* ctx, int32_t layer, const void* q_idx, const 
                           int32_t* sel_blocks, int32_t* n_sel, float* scores,
                           qsa_stream_t stream);
 
+/* The two halves of qsa_index_topk, for callers that want the scores alone or want to
+ * select from scores they computed. qsa_index_scores writes scores [n_ctx/4] f32 (same
+ * definition and requirements as above); qsa_select_topk selects from scores [n_ctx/4]
+ * f32 with the same rule and outputs (NaN ranks lowest; -0 equals +0). */
+qsa_status qsa_index_scores(qsa_ctx* ctx, int32_t layer, const void* q_idx, const float* w,
+                            float* scores, qsa_stream_t stream);
+qsa_status qsa_select_topk(qsa_ctx* ctx, int32_t layer, const float* scores, int32_t* sel_blocks,
+                           int32_t* n_sel, qsa_stream_t stream);
+
 /* Selected K/V gather (Part 10, section COMMON-005). Expands the selected blocks into
  * their cells 4b..4b+3 and appends the open tail block [4*(n_ctx/4), n_ctx):
  *   cells [4*(top_k_tokens/4)+3] i32 (ascending when sel_blocks is ascending),
  *   n_cells device i32 scalar = 4*n_sel + n_ctx mod 4.
  * If k_compact / v_compact are non-NULL, also copies the selected rows into them:
  * [max_cells][n_kv_heads][head_dim] f16 each (the literal compact K/V). Block ids out
- * of range are dropped and reported as device status QSA_ERR_BAD_INDEX. */
+ * of range are reported as device status QSA_ERR_BAD_INDEX and their cells written as
+ * -1, which qsa_sparse_attend skips. */
 qsa_status qsa_gather_kv(qsa_ctx* ctx, int32_t layer, const int32_t* sel_blocks,
                          const int32_t* n_sel, int32_t* cells, int32_t* n_cells,
                          void* k_compact, void* v_compact, qsa_stream_t stream);

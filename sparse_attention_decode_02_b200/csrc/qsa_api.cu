@@ -258,6 +258,26 @@ qsa_status qsa_index_topk(qsa_ctx* ctx, int32_t layer, const void* q_idx, const 
   return ctx->cuda(launch_topk(v, s, sel_blocks, n_sel, (cudaStream_t)stream), "block top-k");
 }
 
+qsa_status qsa_index_scores(qsa_ctx* ctx, int32_t layer, const void* q_idx, const float* w, float* scores,
+                            qsa_stream_t stream) {
+  if (!ctx) return QSA_ERR_INVALID_ARG;
+  if (qsa_status st = ctx->layer_ok(layer)) return st;
+  QSA_CHECK_PTR(q_idx, 16, "q_idx");
+  QSA_CHECK_PTR(w, 16, "w");
+  QSA_CHECK_PTR(scores, 16, "scores");
+  return ctx->cuda(launch_index_scan(ctx->view(layer), q_idx, w, scores, (cudaStream_t)stream), "index scan");
+}
+
+qsa_status qsa_select_topk(qsa_ctx* ctx, int32_t layer, const float* scores, int32_t* sel_blocks, int32_t* n_sel,
+                           qsa_stream_t stream) {
+  if (!ctx) return QSA_ERR_INVALID_ARG;
+  if (qsa_status st = ctx->layer_ok(layer)) return st;
+  QSA_CHECK_PTR(scores, 16, "scores");
+  QSA_CHECK_PTR(sel_blocks, 16, "sel_blocks");
+  QSA_CHECK_PTR(n_sel, 4, "n_sel");
+  return ctx->cuda(launch_topk(ctx->view(layer), scores, sel_blocks, n_sel, (cudaStream_t)stream), "block top-k");
+}
+
 qsa_status qsa_gather_kv(qsa_ctx* ctx, int32_t layer, const int32_t* sel_blocks, const int32_t* n_sel,
                          int32_t* cells, int32_t* n_cells, void* k_compact, void* v_compact, qsa_stream_t stream) {
   if (!ctx) return QSA_ERR_INVALID_ARG;

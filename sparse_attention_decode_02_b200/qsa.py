@@ -54,6 +54,8 @@ SIGNATURES = {
     "qsa_update_pooled_cache": (_I, [_P, _I, _P]),
     "qsa_invalidate_pooled_cache": (_I, [_P, _I, _I, _P]),
     "qsa_index_topk": (_I, [_P, _I, _P, _P, _P, _P, _P, _P]),
+    "qsa_index_scores": (_I, [_P, _I, _P, _P, _P, _P]),
+    "qsa_select_topk": (_I, [_P, _I, _P, _P, _P, _P]),
     "qsa_gather_kv": (_I, [_P, _I, _P, _P, _P, _P, _P, _P, _P]),
     "qsa_sparse_attend": (_I, [_P, _I, _P, _P, _P, _P, _P]),
 }
@@ -170,6 +172,14 @@ class Qsa:
     def index_topk(self, layer, q_idx, w, sel_blocks, n_sel, scores=None, stream=None):
         self._check(self.lib.qsa_index_topk(self.handle, layer, _ptr(q_idx), _ptr(w), _ptr(sel_blocks),
                                             _ptr(n_sel), _ptr(scores), _stream(stream)))
+
+    def index_scores(self, layer, q_idx, w, scores, stream=None):
+        self._check(self.lib.qsa_index_scores(self.handle, layer, _ptr(q_idx), _ptr(w), _ptr(scores),
+                                              _stream(stream)))
+
+    def select_topk(self, layer, scores, sel_blocks, n_sel, stream=None):
+        self._check(self.lib.qsa_select_topk(self.handle, layer, _ptr(scores), _ptr(sel_blocks), _ptr(n_sel),
+                                             _stream(stream)))
 
     def gather_kv(self, layer, sel_blocks, n_sel, cells, n_cells, k_compact=None, v_compact=None,
                   stream=None):
