@@ -1,0 +1,510 @@
+#!/usr/bin/env python
+"""QSA decode benchmark: steps/s per layer and achieved HBM bandwidth on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one decode token through every layer of the workload: for each layer,
+append the token (K/V + indexer key) -> incremental pooled-key update -> indexer
+scan + block top-k -> cell expansion -> sparse GQA attention over the selected cells.
+Each step is one CUDA-graph replay of the library's kernels (launched through the C
+ABI while capturing). The headline workload is all 12 QSA layers at the pages' 256k
+input (255,181 tokens); 64k and 128k single-layer lines (rotated over enough layer
+replicas that the working set exceeds L2) are reported under "by_ctx".
+
+Timing: W untimed warm-up steps, then exactly K steps bracketed by a barrier and
+torch.cuda.synchronize(), timed with CUDA events on the launching stream; the max over
+ranks is reported. Inputs are larger than L2 (12 layers x ~20.6 MB per step), so no
+flush is needed for the headline. For N > 1 every rank runs its own replica of the
+workload (weak scaling, no collective on the data path).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "QSA decode steps/s per layer (256k ctx, 12 layers)"
+UNIT = "layer-steps/s"
+STAGES = ("append", "pool_update", "index_scan", "block_topk", "cell_expand", "sparse_attend")
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default="ctx256k_12l")
+    ap.add_argument("--no-by-ctx", action="store_true", help="skip the 64k/128k lines")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=300)
+    ap.add_argument("--profile-case", action="store_true",
+                    help="small case for ncu: 1 layer at 256k, few steps, no extras")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs, copy burst)"
+    return 6650.0, "fallback (6.65 TB/s pool measurement)"
+
+
+class ClockSampler:
+    """nvidia-smi samples (200 ms) of SM clock and throttle reasons during a region."""
+
+    QUERY = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                                          "-lms", "200", "-i", str(self.gpu_index)],
+                                         stdout=self.file, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.6)
+
+    def mark(self, begin: bool):
+        if begin:
+            self.t0 = time.time()
+        else:
+            self.t1 = time.time()
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        time.sleep(0.3)
+        self.proc.terminate()
+        self.proc.wait(timeout=10)
+        self.file.flush()
+        self.file.seek(0)
+        rows = [ln.strip().split(", ") for ln in self.file if ln.strip()]
+        os.unlink(self.file.name)
+        sm, smax, reasons, in_win = [], None, set(), 0
+        for r in rows:
+            if len(r) < 10:
+                continue
+            try:
+                ts = time.mktime(time.strptime(r[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                ts += float("0." + r[0].split(".")[1]) if "." in r[0] else 0.0
+            except ValueError:
+                continue
+            smax = float(r[3])
+            if self.t0 is not None and self.t0 - 0.25 <= ts <= self.t1 + 0.25:
+                in_win += 1
+                sm.append(float(r[2]))
+                for name, col in (("hw_slowdown", 6), ("hw_thermal_slowdown", 7), ("sw_thermal_slowdown", 8),
+                                  ("sw_power_cap", 9)):
+                    if r[col].strip() == "Active":
+                        reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": in_win}
+
+
+def dist_setup(n_gpus):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------- our implementation
+
+class Workbench:
+    """L bound layers prefilled with the workload's context and graph-captured steps."""
+
+    def __init__(self, wl, n_layers, n_graph_steps, extra_steps, rank):
+        import torch
+
+        import synth
+        import sparse_attention_decode_02_b200 as Q
+        self.torch, self.Q, self.wl, self.L = torch, Q, wl, n_layers
+        max_ctx = int(math.ceil((wl.n_prefill + n_graph_steps + extra_steps + 8) / 4) * 4)
+        self.cfg = Q.make_config(n_layers, max_ctx, wl.d_idx, wl.n_idx_heads, wl.top_k_tokens, wl.n_q_heads,
+                                 wl.n_kv_heads, wl.head_dim, wl.rope_base, wl.rms_eps)
+        self.qsa = Q.Qsa(self.cfg)
+        self.bufs, self.outs = [], []
+        for layer in range(n_layers):
+            b = Q.alloc_layer(self.cfg)
+            self.qsa.bind_layer(layer, **b)
+            pre = synth.device_prefill(wl, layer, rank=rank)
+            self.qsa.append_tokens(layer, pre["k"], pre["v"], pre["idx"])
+            self.qsa.update_pooled_cache(layer)
+            del pre
+            self.bufs.append(b)
+            self.outs.append(Q.alloc_step_outputs(self.cfg))
+        # all layers' attention outputs in one tensor: one device->host copy per step
+        self.out_all = torch.zeros((n_layers, wl.n_q_heads, wl.head_dim), dtype=torch.float32, device="cuda")
+        for layer in range(n_layers):
+            self.outs[layer]["out"] = self.out_all[layer]
+        torch.cuda.synchronize()
+        for layer in range(n_layers):
+            n, p, st = self.qsa.read_layer_state(layer)
+            assert (n, p, st) == (wl.n_prefill, wl.n_prefill // 4, 0), (n, p, st)
+        # per-step inputs of every graph-captured step, plus a staging slot
+        self.packed, self.views = synth.device_steps(wl, n_layers, n_graph_steps + 1, rank=rank)
+        self.stage = n_graph_steps          # index of the staging slot
+        self.launches_per_layer = 7         # append, pool, scan, top-k, expand, attn split, attn merge
+
+    def _chain(self, s, layer, ev=None):
+        q, o, v = self.qsa, self.outs[layer], self.views
+        t = lambda name: v[name][s, layer]
+        q.append_token(layer, t("k"), t("v"), t("idx"))
+        if ev: ev[0].record()
+        q.update_pooled_cache(layer)
+        if ev: ev[1].record()
+        q.index_scores(layer, t("q_idx"), t("w"), o["scores"] if "scores" in o else self._scores(layer))
+        if ev: ev[2].record()
+        q.select_topk(layer, self._scores(layer), o["sel"], o["n_sel"])
+        if ev: ev[3].record()
+        q.gather_kv(layer, o["sel"], o["n_sel"], o["cells"], o["n_cells"])
+        if ev: ev[4].record()
+        q.sparse_attend(layer, t("q"), o["cells"], o["n_cells"], o["out"])
+        if ev: ev[5].record()
+
+    def _scores(self, layer):
+        o = self.outs[layer]
+        if "scores_buf" not in o:
+            o["scores_buf"] = self.torch.zeros(self.cfg.max_ctx // 4, dtype=self.torch.float32, device="cuda")
+        return o["scores_buf"]
+
+    def capture(self, slots):
+        """One CUDA graph running the given step slots back to back (all layers each)."""
+        torch = self.torch
+        for layer in range(self.L):
+            self._scores(layer)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for s in slots:
+                for layer in range(self.L):
+                    self._chain(s, layer)
+        return g
+
+    def capture_instrumented(self):
+        """One step from the staging slot with timing events between the stages."""
+        torch = self.torch
+        evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(6)] for _ in range(self.L)]
+        start = torch.cuda.Event(enable_timing=True, external=True)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            start.record()
+            for layer in range(self.L):
+                self._chain(self.stage, layer, evs[layer])
+        return g, start, evs
+
+    def n_ctx(self):
+        return self.qsa.read_layer_state(0)[0]
+
+
+def run_ours(wl, n_layers, K, W, rank, world, e2e_steps, sample_clocks, local):
+    import torch
+    G = max(d for d in range(1, 33) if K % d == 0)       # steps per timed graph
+    wb = Workbench(wl, n_layers, W + K, extra_steps=e2e_steps + 64, rank=rank)
+    warm = [wb.capture([s]) for s in range(W)]
+    timed = [wb.capture(list(range(W + j * G, W + (j + 1) * G))) for j in range(K // G)]
+    torch.cuda.synchronize()
+    for g in warm:
+        g.replay()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local) if sample_clocks else None
+    if clocks:
+        clocks.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if clocks:
+        clocks.mark(True)
+    t0.record(stream)
+    for g in timed:
+        g.replay()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if clocks:
+        clocks.mark(False)
+    barrier(world)
+    ms = max_over_ranks(t0.elapsed_time(t1), world)
+    clk = clocks.stop() if clocks else None
+    n_after = wb.n_ctx()
+    assert n_after == wl.n_prefill + W + K, n_after
+    for layer in range(n_layers):
+        assert wb.qsa.read_layer_state(layer)[2] == 0
+
+    # per-stage breakdown from an instrumented graph (events break the launch overlap,
+    # so these are serialised per-kernel durations, used for the roofline)
+    ig, start, evs = wb.capture_instrumented()
+    reps = 10
+    acc = {s: 0.0 for s in STAGES}
+    for _ in range(reps):
+        wb.packed[wb.stage].copy_(wb.packed[W + K - 1])
+        ig.replay()
+        torch.cuda.synchronize()
+        prev = start
+        for layer in range(n_layers):
+            for i, name in enumerate(STAGES):
+                acc[name] += prev.elapsed_time(evs[layer][i])
+                prev = evs[layer][i]
+    per_launch_us = {s: 1e3 * acc[s] / (reps * n_layers) for s in STAGES}
+    n_ctx_instr = wb.n_ctx()
+
+    # end to end through the public API: pinned host inputs in, attention outputs out
+    e2e = None
+    if e2e_steps > 0:
+        eg = wb.capture([wb.stage])
+        host_in = wb.packed[W:W + e2e_steps].cpu().pin_memory() if e2e_steps <= K else \
+            torch.cat([wb.packed[W:W + K]] * math.ceil(e2e_steps / K))[:e2e_steps].cpu().pin_memory()
+        host_out = torch.empty((e2e_steps, *wb.out_all.shape), dtype=torch.float32).pin_memory()
+        torch.cuda.synchronize()
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for s in range(e2e_steps):
+            wb.packed[wb.stage].copy_(host_in[s], non_blocking=True)
+            eg.replay()
+            host_out[s].copy_(wb.out_all, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+        e2e = {"value": world * n_layers * e2e_steps / (e_ms / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": int(host_in[0].numel()), "d2h_bytes_per_step": int(host_out[0].numel() * 4),
+               "steps": e2e_steps}
+    return {"ms": ms, "clocks": clk, "per_launch_us": per_launch_us, "n_ctx_instr": n_ctx_instr,
+            "n_layers": n_layers, "launches_per_step": n_layers * wb.launches_per_layer, "e2e": e2e,
+            "graph_steps": G}
+
+
+def stage_bytes(wl, n_ctx):
+    """Algorithmic HBM bytes per launch of each stage at context n_ctx (per layer)."""
+    B = n_ctx // 4
+    kv_row = wl.n_kv_heads * wl.head_dim * 2
+    n_cells = 4 * min(wl.k_blocks, B) + n_ctx % 4
+    return {
+        "append": 2 * kv_row + wl.d_idx * 2 + 2 * kv_row + wl.d_idx * 2,        # read inputs, write caches
+        "pool_update": (4 * wl.d_idx * 2 + wl.d_idx * 2) / 4.0,                  # one block every 4th step
+        "index_scan": B * wl.d_idx * 2 + B * 4 + wl.n_idx_heads * (wl.d_idx * 2 + 4),
+        "block_topk": B * 4 + wl.k_blocks * 4,
+        "cell_expand": wl.k_blocks * 4 + n_cells * 4,
+        "sparse_attend": n_cells * (4 + 2 * kv_row) + wl.n_q_heads * wl.head_dim * (2 + 4),
+    }
+
+
+def cpu_baseline(wl, budget_s=12.0, max_steps=400):
+    """The oracle as it stands, one layer of the workload on this host's cores."""
+    import numpy as np
+
+    import synth
+    from oracle import qsa_oracle as O
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:  # pragma: no cover
+        threads = os.cpu_count() or 1
+    shape = O.QsaShape.of(wl)
+    layer = O.OracleLayer(shape, max_ctx=int(math.ceil((wl.n_prefill + max_steps + 8) / 4) * 4))
+    pre = synth.prefill_tokens(wl, 0)
+    layer.append_tokens(pre["k"], pre["v"], pre["idx"])
+    layer.update_pooled_cache()
+    steps = [synth.step_inputs(wl, 0, s) for s in range(8)]
+    done, t0 = 0, time.perf_counter()
+    while done < max_steps:
+        st = steps[done % len(steps)]
+        layer.decode_step(st["k"], st["v"], st["idx"], st["q_idx"], st["w"], st["q"])
+        done += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": done / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{done} decode steps of 1 of the {wl.n_layers} layers at {wl.n_prefill:,}-token context "
+                      f"(numpy float64, {threads} BLAS threads)"}
+
+
+def main_ours(args):
+    import torch
+
+    import synth
+    from sparse_attention_decode_02_b200 import build as qbuild
+    world, rank, local = dist_setup(args.gpus)
+    if rank == 0 or world == 1:
+        qbuild.build()
+    barrier(world)
+    wl = synth.workload(args.workload)
+    K, W = args.steps, args.warmup
+    if args.profile_case:
+        wl = synth.workload(args.workload, n_layers=1)
+        args.no_by_ctx, args.no_cpu_baseline = True, True
+    assert W >= 3, "at least 3 warm-up steps"
+    peak, peak_src = measured_peaks()
+
+    main = run_ours(wl, wl.n_layers, K, W, rank, world, 0 if args.profile_case else args.e2e_steps,
+                    sample_clocks=not args.profile_case, local=local)
+    layer_steps = world * wl.n_layers * K
+    value = layer_steps / (main["ms"] / 1e3)
+
+    sb = stage_bytes(wl, main["n_ctx_instr"])
+    per = main["per_launch_us"]
+    dominant = max(STAGES, key=lambda s: per[s])
+    achieved = {s: sb[s] / (per[s] * 1e-6) / 1e9 for s in STAGES}
+    hot = ("index_scan", "block_topk", "cell_expand", "sparse_attend")
+    hot_bytes = sum(sb[s] for s in hot)
+    hot_us = sum(per[s] for s in hot)
+    roofline = {"bound": "hbm", "kernel": dominant, "achieved": round(achieved[dominant], 1), "peak": peak,
+                "unit": "GB/s", "frac": round(achieved[dominant] / peak, 4), "traffic": None,
+                "peak_source": peak_src,
+                "bytes_per_launch": int(sb[dominant]), "us_per_launch": round(per[dominant], 3),
+                "stages_us": {s: round(per[s], 3) for s in STAGES},
+                "stages_gbs": {s: round(achieved[s], 1) for s in STAGES},
+                "scan_attn_path": {"bytes": int(hot_bytes), "us": round(hot_us, 3),
+                                   "gbs": round(hot_bytes / (hot_us * 1e-6) / 1e9, 1),
+                                   "frac": round(hot_bytes / (hot_us * 1e-6) / 1e9 / peak, 4)}}
+
+    by_ctx = {}
+    if not args.no_by_ctx:
+        for name, reps in (("ctx64k", 24), ("ctx128k", 16)):
+            w2 = synth.workload(name)
+            k2 = max(50, min(K // 4, 500))
+            k2 -= k2 % 10
+            r = run_ours(w2, reps, k2, 5, rank, world, 0, sample_clocks=False, local=local)
+            v2 = world * reps * k2 / (r["ms"] / 1e3)
+            b2 = stage_bytes(w2, r["n_ctx_instr"])
+            hb = sum(b2[s] for s in hot)
+            hu = sum(r["per_launch_us"][s] for s in hot)
+            by_ctx[name] = {"ctx": w2.n_prefill, "layer_replicas": reps, "steps": k2,
+                            "value": round(v2, 1), "unit": UNIT,
+                            "ms_per_step": round(r["ms"] / k2, 4),
+                            "stages_us": {s: round(r["per_launch_us"][s], 3) for s in STAGES},
+                            "scan_attn_gbs": round(hb / (hu * 1e-6) / 1e9, 1)}
+            torch.cuda.empty_cache()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
+            "ms_per_step": round(main["ms"] / K, 5), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f16", "data": "synthetic (seeded N(0,1) f16 K/V/keys/queries, U(0,1) w)",
+            "config": {"workload": wl.name, "ctx_prefill": wl.n_prefill, "layers": wl.n_layers,
+                       "d_idx": wl.d_idx, "idx_heads": wl.n_idx_heads, "top_k_tokens": wl.top_k_tokens,
+                       "q_heads": wl.n_q_heads, "kv_heads": wl.n_kv_heads, "head_dim": wl.head_dim,
+                       "batch": 1, "parallelism": f"replicas x{world}",
+                       "l2": "inputs larger than L2 (each step reads ~20.6 MB per layer x 12 layers)",
+                       "graph_steps_per_replay": main["graph_steps"]},
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "clocks": main["clocks"],
+            "e2e": main["e2e"],
+            "gpu_launches": main["launches_per_step"] * K,
+            "by_ctx": by_ctx,
+            "hbm_gbs_step": round(world * wl.n_layers * K * sum(sb.values()) / (main["ms"] / 1e3) / 1e9, 1),
+        }
+        print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def main_reference(args):
+    """The oracle (the plain CPU definition of the path) timed on this host's cores."""
+    import synth
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    wl = synth.workload(args.workload)
+    import numpy as np  # noqa: F401
+    from oracle import qsa_oracle as O
+    shape = O.QsaShape.of(wl)
+    # Each step is one layer's decode step (a bounded sample of the 12-layer step); the
+    # run stops after K steps or a 60 s budget, whichever comes first, and reports the
+    # steps it timed.
+    K, W, budget = args.steps, min(args.warmup, 3), 60.0
+    layer = O.OracleLayer(shape, max_ctx=int(math.ceil((wl.n_prefill + K + W + 8) / 4) * 4))
+    pre = synth.prefill_tokens(wl, 0)
+    layer.append_tokens(pre["k"], pre["v"], pre["idx"])
+    layer.update_pooled_cache()
+    steps = [synth.step_inputs(wl, 0, s) for s in range(16)]
+    for i in range(W):
+        st = steps[i % 16]
+        layer.decode_step(st["k"], st["v"], st["idx"], st["q_idx"], st["w"], st["q"])
+    t0 = time.perf_counter()
+    done = 0
+    while done < K and (time.perf_counter() - t0) < budget:
+        st = steps[done % 16]
+        layer.decode_step(st["k"], st["v"], st["idx"], st["q_idx"], st["w"], st["q"])
+        done += 1
+    dt = time.perf_counter() - t0
+    K = done
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:  # pragma: no cover
+        threads = os.cpu_count() or 1
+    value = K / dt
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
+        "steps": K, "warmup": W, "ms_per_step": round(1e3 * dt / K, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded, host)",
+        "config": {"workload": wl.name, "ctx_prefill": wl.n_prefill, "layers_sampled": 1,
+                   "layers": wl.n_layers},
+        "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": f"{K} decode steps of 1 of {wl.n_layers} layers at {wl.n_prefill:,} tokens"},
+        "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }))
+
+
+if __name__ == "__main__":
+    a = parse_args()
+    if a.impl == "reference":
+        main_reference(a)
+    else:
+        main_ours(a)

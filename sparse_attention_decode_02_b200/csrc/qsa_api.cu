@@ -137,6 +137,10 @@ qsa_status qsa_create(const qsa_config* cfg, qsa_ctx** out) {
     delete ctx;
     return QSA_ERR_CUDA;
   }
+  if (init_kernel_attributes() != cudaSuccess) {
+    delete ctx;
+    return QSA_ERR_CUDA;
+  }
   ctx->split = attn_split(*cfg, ctx->n_sms);
   const AttnSplit worst = attn_split(*cfg, ctx->n_sms > 148 ? ctx->n_sms : 148);
   ctx->ws = workspace_layout(*cfg, worst.n_splits > ctx->split.n_splits ? worst.n_splits : ctx->split.n_splits);

@@ -287,17 +287,17 @@ __global__ void __launch_bounds__(kTopkThreads, 1) block_topk_kernel(DevState* s
   cluster.sync();  // keep this CTA's shared memory alive until every remote read is done
 }
 
+cudaError_t init_kernel_attributes() {
+  // shared-memory opt-in of the top-k cluster (set once per process and device, before
+  // any launch, so that no attribute call happens while a stream is being captured)
+  return cudaFuncSetAttribute(block_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              kTopkMaxPerCta * (int)sizeof(uint32_t));
+}
+
 cudaError_t launch_topk(const LayerView& L, const float* scores, int32_t* sel, int32_t* n_sel, cudaStream_t s) {
   const int max_blocks = L.cfg.max_ctx / kBlock;
   const int chunk = (max_blocks + kTopkCluster - 1) / kTopkCluster;
   const size_t smem = size_t(chunk) * sizeof(uint32_t);
-  static bool attr_done = false;
-  if (!attr_done) {
-    cudaError_t e = cudaFuncSetAttribute(block_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kTopkMaxPerCta * (int)sizeof(uint32_t));
-    if (e != cudaSuccess) return e;
-    attr_done = true;
-  }
   return launch_pdl(block_topk_kernel, dim3(kTopkCluster), dim3(kTopkThreads), smem, s, kTopkCluster,
                     L.state, scores, sel, n_sel, L.cfg.top_k_tokens / kBlock);
 }

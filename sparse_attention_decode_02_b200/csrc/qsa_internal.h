@@ -87,6 +87,7 @@ struct LayerView {
 };
 
 // ---- launchers (return the launch's cudaError_t) ----
+cudaError_t init_kernel_attributes();  // once per context creation, outside any capture
 cudaError_t launch_set_state(const LayerView& L, int n_ctx, int n_pooled, int mode, cudaStream_t s);
 cudaError_t launch_append(const LayerView& L, int n, const void* k, const void* v,
                           const void* idx, int grid_hint, cudaStream_t s);

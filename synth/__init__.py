@@ -160,3 +160,64 @@ def random_pooled(wl: Workload, layer: int, n_blocks: int, salt: int = 0):
     """An f16 table [n_blocks, d_idx] drawn from N(0,1) (stage-isolated scan input)."""
     g = _rng(wl, layer, _T_POOLED, salt)
     return g.standard_normal((n_blocks, wl.d_idx), dtype=np.float32).astype(np.float16)
+
+
+# ---------------------------------------------------------------------------------
+# Device-side draws (torch's seeded CUDA generator) for the timing workloads, where
+# host generation of 12 x 255k tokens would dominate the bench's set-up time. Same
+# distributions as above; the values differ from the host draws, so parity tests use
+# the host generators.
+# ---------------------------------------------------------------------------------
+
+def _torch_gen(wl: Workload, layer: int, tensor: int, rank: int, device):
+    import torch
+    g = torch.Generator(device=device)
+    key = np.random.SeedSequence([SEED_BASE, wl.wid, layer, tensor, rank]).generate_state(1, np.uint64)[0]
+    g.manual_seed(int(key) & ((1 << 63) - 1))
+    return g
+
+
+def device_prefill(wl: Workload, layer: int, n: int | None = None, device="cuda", rank: int = 0):
+    """k, v [n, Hkv, D] f16 and idx [n, d_idx] f16 drawn on the GPU from N(0,1)."""
+    import torch
+    n = wl.n_prefill if n is None else n
+    out = {}
+    for name, tid, shape in (("k", _T_K, (n, wl.n_kv_heads, wl.head_dim)),
+                             ("v", _T_V, (n, wl.n_kv_heads, wl.head_dim)),
+                             ("idx", _T_IDX, (n, wl.d_idx))):
+        g = _torch_gen(wl, layer, tid, rank, device)
+        out[name] = torch.randn(shape, generator=g, device=device, dtype=torch.float32).half()
+    return out
+
+
+def device_steps(wl: Workload, n_layers: int, n_steps: int, device="cuda", rank: int = 0):
+    """Per-step inputs of n_steps x n_layers drawn on the GPU, packed so that step s of
+    every layer is one contiguous byte range (one copy stages a whole step).
+
+    Returns (packed, views): packed is uint8 [n_steps, step_bytes]; views[name] is a
+    typed view [n_steps, n_layers, elems] of it for name in k, v, idx (the appended
+    token), q_idx, w, q (same meaning as step_inputs); views[name][s, l] is contiguous.
+    """
+    import torch
+    fields = [("k", torch.float16, wl.n_kv_heads * wl.head_dim, _T_K, "normal"),
+              ("v", torch.float16, wl.n_kv_heads * wl.head_dim, _T_V, "normal"),
+              ("idx", torch.float16, wl.d_idx, _T_IDX, "normal"),
+              ("q_idx", torch.float16, wl.n_idx_heads * wl.d_idx, _T_QIDX, "normal"),
+              ("w", torch.float32, wl.n_idx_heads, _T_W, "uniform"),
+              ("q", torch.float16, wl.n_q_heads * wl.head_dim, _T_Q, "normal")]
+    esz = {torch.float16: 2, torch.float32: 4}
+    slots = [(cnt * esz[dt] + 255) // 256 * 256 for _, dt, cnt, _, _ in fields]   # 256-byte aligned
+    layer_bytes = sum(slots)
+    packed = torch.empty((n_steps, n_layers * layer_bytes), dtype=torch.uint8, device=device)
+    per_layer = packed.view(n_steps, n_layers, layer_bytes)
+    views, off = {}, 0
+    for (name, dt, cnt, tid, kind), nb in zip(fields, slots):
+        g = _torch_gen(wl, 1000 + n_layers, tid, rank, device)
+        shape = (n_steps, n_layers, cnt)
+        vals = (torch.rand(shape, generator=g, device=device, dtype=torch.float32) if kind == "uniform"
+                else torch.randn(shape, generator=g, device=device, dtype=torch.float32)).to(dt)
+        raw = per_layer[:, :, off:off + cnt * esz[dt]]
+        raw.copy_(vals.view(torch.uint8).view(n_steps, n_layers, cnt * esz[dt]))
+        views[name] = raw.view(dt)
+        off += nb
+    return packed, views
