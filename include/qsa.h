@@ -195,6 +195,36 @@ qsa_status qsa_gather_kv(qsa_ctx* ctx, int32_t layer, const int32_t* sel_blocks,
 qsa_status qsa_sparse_attend(qsa_ctx* ctx, int32_t layer, const void* q, const int32_t* cells,
                              const int32_t* n_cells, float* out, qsa_stream_t stream);
 
+/* Size of the fixed scratch array behind qsa_sparse_attend_noalloc (1 MiB). */
+#define QSA_NOALLOC_SCRATCH_BYTES (1u << 20)
+
+/* qsa_sparse_attend without a context, a workspace or any other scratch from the caller.
+ * The pages have no counterpart: it exists for callers that cannot call cudaMalloc —
+ * for instance a plugin inside a serving runtime that reserves all device memory in
+ * its own arena and forbids further allocations, or a process under a hard
+ * device-memory cap — and so cannot provide the layer workspace that holds the
+ * split-KV partials. The caller passes only inputs and the output:
+ *   q [n_q_heads][head_dim] f16; k_cache, v_cache [>= n_ctx][n_kv_heads][head_dim] f16;
+ *   cells [n_cells] i32 device ids (ids outside [0, n_ctx) are skipped); n_cells a device
+ *   i32 scalar, at most 4*(top_k_tokens/4)+3; out [n_q_heads][head_dim] f32.
+ * The result is the same as qsa_sparse_attend's for the same inputs and shapes.
+ * Scratch: one array of QSA_NOALLOC_SCRATCH_BYTES compiled into the library; every GPU
+ * that loads the library holds it until the process exits. The first call on a device
+ * looks up the array's device address (make that first call before any stream capture).
+ * Every call shares the array and overwrites what the previous call left there, so
+ * calls whose kernels overlap on the GPU (on different streams, or from several host
+ * threads) race and must be serialised by the caller. Nothing here allocates: no
+ * cudaMalloc, cudaFree or allocating library routine is called.
+ * Returns QSA_ERR_INVALID_ARG for null or misaligned pointers or n_ctx < 0,
+ * QSA_ERR_UNSUPPORTED for shapes the kernels are not built for (head_dim 64/128,
+ * n_q_heads/n_kv_heads in {1,2,4,8}, top_k_tokens a positive multiple of 4),
+ * QSA_ERR_CAPACITY if the partials of these shapes would not fit in the array, and
+ * QSA_ERR_CUDA if a launch fails. Device-side problems are not reported. */
+qsa_status qsa_sparse_attend_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                                     int32_t n_ctx, const int32_t* cells, const int32_t* n_cells,
+                                     float* out, int32_t n_q_heads, int32_t n_kv_heads,
+                                     int32_t head_dim, int32_t top_k_tokens, qsa_stream_t stream);
+
 #ifdef __cplusplus
 }  /* extern "C" */
 #endif

@@ -4,4 +4,4 @@ The compute lives in csrc/ (hand-written CUDA for sm_100a behind the C ABI decla
 include/qsa.h); qsa.py only marshals torch device tensors and streams into that ABI.
 """
 from .qsa import (Qsa, QsaConfig, QsaError, alloc_layer, alloc_step_outputs, buffer_bytes,  # noqa: F401
-                  load_library, make_config)
+                  load_library, make_config, sparse_attend_noalloc)

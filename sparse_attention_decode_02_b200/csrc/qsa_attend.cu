@@ -11,6 +11,8 @@
 //    the compact K/V.
 #include <cuda_fp16.h>
 
+#include <mutex>
+
 #include "qsa_device.cuh"
 
 namespace qsa {
@@ -300,4 +302,87 @@ cudaError_t launch_attend(const LayerView& L, const void* q, const int32_t* cell
                     (const float*)L.part_ml, out, L.cfg.n_q_heads, L.cfg.head_dim, L.split.n_splits);
 }
 
+// ---------------------------------------------------------------------------------
+// Attention for callers that cannot allocate device memory (qsa_sparse_attend_noalloc).
+// The split-KV partials and the small state block that the attention kernels use as
+// scratch live in one fixed array compiled into the library, so the caller passes only
+// its inputs and its output. Every GPU that loads the library holds this array until
+// the process exits, and all calls on a device share it.
+// ---------------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_noalloc_scratch[QSA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kMaxDevices];  // device address of g_noalloc_scratch, per device
+int g_noalloc_sms[kMaxDevices];
+
+// Once per device, with that device current: look up the array's device address (host
+// code cannot use the symbol itself, which is only a host-side stand-in).
+cudaError_t noalloc_setup(void** addr, int* n_sms) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    int sms = 0;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_noalloc_sms[dev] = sms;
+    g_noalloc_addr[dev] = p;
+  }
+  *addr = g_noalloc_addr[dev];
+  *n_sms = g_noalloc_sms[dev];
+  return cudaSuccess;
+}
+
+bool aligned_to(const void* p, uintptr_t a) { return p && (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+}  // namespace
+
 }  // namespace qsa
+
+extern "C" qsa_status qsa_sparse_attend_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                                                int32_t n_ctx, const int32_t* cells, const int32_t* n_cells,
+                                                float* out, int32_t n_q_heads, int32_t n_kv_heads,
+                                                int32_t head_dim, int32_t top_k_tokens, qsa_stream_t stream) {
+  using namespace qsa;
+  if (!aligned_to(q, 16) || !aligned_to(k_cache, 16) || !aligned_to(v_cache, 16) || !aligned_to(cells, 16) ||
+      !aligned_to(n_cells, 4) || !aligned_to(out, 16) || n_ctx < 0)
+    return QSA_ERR_INVALID_ARG;
+  if ((head_dim != 64 && head_dim != 128) || n_kv_heads < 1 || n_q_heads < 1 || n_q_heads % n_kv_heads ||
+      top_k_tokens < kBlock || top_k_tokens % kBlock)
+    return QSA_ERR_UNSUPPORTED;
+  const int g = n_q_heads / n_kv_heads;
+  if (g != 1 && g != 2 && g != 4 && g != 8) return QSA_ERR_UNSUPPORTED;
+  void* base = nullptr;
+  int n_sms = 0;
+  if (noalloc_setup(&base, &n_sms) != cudaSuccess) return QSA_ERR_CUDA;
+
+  LayerView v{};
+  v.cfg.n_layers = 1;
+  v.cfg.max_ctx = n_ctx;
+  v.cfg.top_k_tokens = top_k_tokens;
+  v.cfg.n_q_heads = n_q_heads;
+  v.cfg.n_kv_heads = n_kv_heads;
+  v.cfg.head_dim = head_dim;
+  v.k_cache = const_cast<void*>(k_cache);
+  v.v_cache = const_cast<void*>(v_cache);
+  v.split = attn_split(v.cfg, n_sms);
+  v.n_sms = n_sms;
+  // scratch layout: state block | (max, sum) pairs | partial outputs
+  const size_t ml_bytes = align256(size_t(v.split.n_splits) * n_q_heads * 2 * sizeof(float));
+  const size_t o_bytes = size_t(v.split.n_splits) * n_q_heads * head_dim * sizeof(float);
+  if (sizeof(DevState) + ml_bytes + o_bytes > QSA_NOALLOC_SCRATCH_BYTES) return QSA_ERR_CAPACITY;
+  char* p = static_cast<char*>(base);
+  v.state = reinterpret_cast<DevState*>(p);
+  v.part_ml = reinterpret_cast<float*>(p + sizeof(DevState));
+  v.part_o = reinterpret_cast<float*>(p + sizeof(DevState) + ml_bytes);
+  // the state block keeps the previous call's contents: set n_ctx and clear the status
+  if (launch_set_state(v, n_ctx, 0, kSetRestore, (cudaStream_t)stream) != cudaSuccess) return QSA_ERR_CUDA;
+  if (launch_attend(v, q, cells, n_cells, out, (cudaStream_t)stream) != cudaSuccess) return QSA_ERR_CUDA;
+  return QSA_OK;
+}

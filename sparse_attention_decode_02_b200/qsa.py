@@ -58,6 +58,7 @@ SIGNATURES = {
     "qsa_select_topk": (_I, [_P, _I, _P, _P, _P, _P]),
     "qsa_gather_kv": (_I, [_P, _I, _P, _P, _P, _P, _P, _P, _P]),
     "qsa_sparse_attend": (_I, [_P, _I, _P, _P, _P, _P, _P]),
+    "qsa_sparse_attend_noalloc": (_I, [_P, _P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _P]),
 }
 
 _lib = None
@@ -189,6 +190,17 @@ class Qsa:
     def sparse_attend(self, layer, q, cells, n_cells, out, stream=None):
         self._check(self.lib.qsa_sparse_attend(self.handle, layer, _ptr(q), _ptr(cells), _ptr(n_cells),
                                                _ptr(out), _stream(stream)))
+
+
+def sparse_attend_noalloc(q, k_cache, v_cache, n_ctx, cells, n_cells, out, n_q_heads, n_kv_heads, head_dim,
+                          top_k_tokens, stream=None):
+    """qsa_sparse_attend_noalloc: attention with the library's fixed scratch array (no
+    context, no workspace). Raises QsaError with the returned status on failure."""
+    st = load_library().qsa_sparse_attend_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), int(n_ctx), _ptr(cells),
+                                                  _ptr(n_cells), _ptr(out), n_q_heads, n_kv_heads, head_dim,
+                                                  top_k_tokens, _stream(stream))
+    if st != QSA_OK:
+        raise QsaError(st, "qsa_sparse_attend_noalloc failed")
 
 
 def alloc_layer(cfg: QsaConfig, device="cuda"):
