@@ -36,7 +36,7 @@ if ROOT not in sys.path:
 
 METRIC = "QSA decode steps/s per layer (256k ctx, 12 layers)"
 UNIT = "layer-steps/s"
-STAGES = ("append", "pool_update", "index_scan", "block_topk", "cell_expand", "sparse_attend")
+STAGES = ("append", "pool_update", "index_scan", "block_topk", "sparse_attend")
 
 
 def parse_args():
@@ -192,7 +192,7 @@ class Workbench:
         # per-step inputs of every graph-captured step, plus a staging slot
         self.packed, self.views = synth.device_steps(wl, n_layers, n_graph_steps + 1, rank=rank)
         self.stage = n_graph_steps          # index of the staging slot
-        self.launches_per_layer = 7         # append, pool, scan, top-k, expand, attn split, attn merge
+        self.launches_per_layer = 5         # append, pool update, scan, top-k, attention (expansion fused)
 
     def _chain(self, s, layer, ev=None):
         q, o, v = self.qsa, self.outs[layer], self.views
@@ -205,10 +205,8 @@ class Workbench:
         if ev: ev[2].record()
         q.select_topk(layer, self._scores(layer), o["sel"], o["n_sel"])
         if ev: ev[3].record()
-        q.gather_kv(layer, o["sel"], o["n_sel"], o["cells"], o["n_cells"])
+        q.sparse_attend_selected(layer, t("q"), o["sel"], o["n_sel"], o["out"])
         if ev: ev[4].record()
-        q.sparse_attend(layer, t("q"), o["cells"], o["n_cells"], o["out"])
-        if ev: ev[5].record()
 
     def _scores(self, layer):
         o = self.outs[layer]
@@ -231,7 +229,8 @@ class Workbench:
     def capture_instrumented(self):
         """One step from the staging slot with timing events between the stages."""
         torch = self.torch
-        evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(6)] for _ in range(self.L)]
+        evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(STAGES))]
+               for _ in range(self.L)]
         start = torch.cuda.Event(enable_timing=True, external=True)
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
@@ -332,8 +331,8 @@ def stage_bytes(wl, n_ctx):
         "pool_update": (4 * wl.d_idx * 2 + wl.d_idx * 2) / 4.0,                  # one block every 4th step
         "index_scan": B * wl.d_idx * 2 + B * 4 + wl.n_idx_heads * (wl.d_idx * 2 + 4),
         "block_topk": B * 4 + wl.k_blocks * 4,
-        "cell_expand": wl.k_blocks * 4 + n_cells * 4,
-        "sparse_attend": n_cells * (4 + 2 * kv_row) + wl.n_q_heads * wl.head_dim * (2 + 4),
+        "sparse_attend": wl.k_blocks * 4 + n_cells * 2 * (kv_row // wl.n_kv_heads) * wl.n_kv_heads
+                         + wl.n_q_heads * wl.head_dim * (2 + 4),
     }
 
 
@@ -393,7 +392,7 @@ def main_ours(args):
     per = main["per_launch_us"]
     dominant = max(STAGES, key=lambda s: per[s])
     achieved = {s: sb[s] / (per[s] * 1e-6) / 1e9 for s in STAGES}
-    hot = ("index_scan", "block_topk", "cell_expand", "sparse_attend")
+    hot = ("index_scan", "block_topk", "sparse_attend")
     hot_bytes = sum(sb[s] for s in hot)
     hot_us = sum(per[s] for s in hot)
     roofline = {"bound": "hbm", "kernel": dominant, "achieved": round(achieved[dominant], 1), "peak": peak,

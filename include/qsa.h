@@ -55,7 +55,9 @@ typedef enum {
   QSA_ERR_STATE = 3,         /* layer not bound, or pooled cache behind the context   */
   QSA_ERR_CUDA = 4,          /* a CUDA runtime call failed (message has the detail)   */
   QSA_ERR_UNSUPPORTED = 5,   /* shape outside what the kernels are built for          */
-  QSA_ERR_BAD_INDEX = 6      /* device status only: a block or cell id out of range   */
+  QSA_ERR_BAD_INDEX = 6,     /* device status only: a block or cell id out of range   */
+  QSA_ERR_TIMEOUT = 7        /* device status only: a bounded wait inside a kernel gave
+                                up (the kernel skipped its remaining work and returned) */
 } qsa_status;
 
 /* Static shape of every layer of one model (Part 10, section "QSA indexer"). */
@@ -194,6 +196,17 @@ qsa_status qsa_gather_kv(qsa_ctx* ctx, int32_t layer, const int32_t* sel_blocks,
  *   range are skipped and reported as device status QSA_ERR_BAD_INDEX. */
 qsa_status qsa_sparse_attend(qsa_ctx* ctx, int32_t layer, const void* q, const int32_t* cells,
                              const int32_t* n_cells, float* out, qsa_stream_t stream);
+
+/* qsa_gather_kv's cell expansion fused into qsa_sparse_attend (Part 10, sections
+ * COMMON-005 and COMMON-006: expand only the chosen blocks into cells, add the tail
+ * index, attend over those rows). Takes the selection straight from qsa_index_topk /
+ * qsa_select_topk: sel_blocks [n_sel] i32 ascending block ids (< n_ctx/4), n_sel a
+ * device i32 scalar (<= top_k_tokens/4). The cell set is {4b..4b+3 : b in sel} plus
+ * [4*(n_ctx/4), n_ctx), exactly as qsa_gather_kv writes it; output as qsa_sparse_attend.
+ * Out-of-range block ids are skipped and reported as device status QSA_ERR_BAD_INDEX. */
+qsa_status qsa_sparse_attend_selected(qsa_ctx* ctx, int32_t layer, const void* q,
+                                      const int32_t* sel_blocks, const int32_t* n_sel, float* out,
+                                      qsa_stream_t stream);
 
 /* Size of the fixed scratch array behind qsa_sparse_attend_noalloc (1 MiB). */
 #define QSA_NOALLOC_SCRATCH_BYTES (1u << 20)

@@ -20,6 +20,7 @@ namespace {
 struct Layer {
   bool bound = false;
   qsa_layer_buffers buf{};
+  CUtensorMap pooled_map{};
   // Upper bound on blocks the next pooled update may have to compute; it only sizes
   // the update's grid (the kernel itself reads the exact range from device state).
   long long pending_blocks = 0;
@@ -51,6 +52,7 @@ struct qsa_ctx {
   int device = 0;
   int n_sms = 0;
   AttnSplit split{};
+  int attn_cluster = 0, attn_cells_per_cta = 0;
   WorkspaceLayout ws{};
   std::vector<Layer> layers;
   std::string last_error;
@@ -89,6 +91,9 @@ struct qsa_ctx {
     v.part_ml = reinterpret_cast<float*>(wsp + ws.part_ml);
     v.split = split;
     v.n_sms = n_sms;
+    v.pooled_map = l.pooled_map;
+    v.attn_cluster = attn_cluster;
+    v.attn_cells_per_cta = attn_cells_per_cta;
     return v;
   }
 };
@@ -137,9 +142,13 @@ qsa_status qsa_create(const qsa_config* cfg, qsa_ctx** out) {
     delete ctx;
     return QSA_ERR_CUDA;
   }
-  if (init_kernel_attributes() != cudaSuccess) {
+  if (init_kernel_attributes() != cudaSuccess || init_scan_attributes() != cudaSuccess) {
     delete ctx;
     return QSA_ERR_CUDA;
+  }
+  if (plan_attention(*cfg, &ctx->attn_cluster, &ctx->attn_cells_per_cta) != cudaSuccess) {
+    delete ctx;
+    return QSA_ERR_UNSUPPORTED;
   }
   ctx->split = attn_split(*cfg, ctx->n_sms);
   const AttnSplit worst = attn_split(*cfg, ctx->n_sms > 148 ? ctx->n_sms : 148);
@@ -165,7 +174,11 @@ qsa_status qsa_bind_layer(qsa_ctx* ctx, int32_t layer, const qsa_layer_buffers* 
   if (buf->rms_gain && !aligned(buf->rms_gain, 16))
     return ctx->fail(QSA_ERR_INVALID_ARG, "rms_gain must be 16-byte aligned");
   Layer& l = ctx->layers[layer];
+  CUtensorMap map;
+  if (qsa_status st = ctx->cuda(encode_pooled_map(ctx->cfg, buf->pooled_cache, &map), "bind_layer: pooled TMA map"))
+    return st;
   l.buf = *buf;
+  l.pooled_map = map;
   l.bound = true;
   l.pending_blocks = 0;
   qsa_status st = ctx->cuda(launch_set_state(ctx->view(layer), 0, 0, kSetReset, (cudaStream_t)stream), "bind_layer");
@@ -306,6 +319,18 @@ qsa_status qsa_sparse_attend(qsa_ctx* ctx, int32_t layer, const void* q, const i
   QSA_CHECK_PTR(n_cells, 4, "n_cells");
   QSA_CHECK_PTR(out, 16, "out");
   return ctx->cuda(launch_attend(ctx->view(layer), q, cells, n_cells, out, (cudaStream_t)stream), "sparse_attend");
+}
+
+qsa_status qsa_sparse_attend_selected(qsa_ctx* ctx, int32_t layer, const void* q, const int32_t* sel_blocks,
+                                      const int32_t* n_sel, float* out, qsa_stream_t stream) {
+  if (!ctx) return QSA_ERR_INVALID_ARG;
+  if (qsa_status st = ctx->layer_ok(layer)) return st;
+  QSA_CHECK_PTR(q, 16, "q");
+  QSA_CHECK_PTR(sel_blocks, 16, "sel_blocks");
+  QSA_CHECK_PTR(n_sel, 4, "n_sel");
+  QSA_CHECK_PTR(out, 16, "out");
+  return ctx->cuda(launch_attend_selected(ctx->view(layer), q, sel_blocks, n_sel, out, (cudaStream_t)stream),
+                   "sparse_attend_selected");
 }
 
 }  // extern "C"

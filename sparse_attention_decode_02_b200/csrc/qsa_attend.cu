@@ -11,9 +11,13 @@
 //    the compact K/V.
 #include <cuda_fp16.h>
 
+#include <cooperative_groups.h>
+
 #include <mutex>
 
 #include "qsa_device.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace qsa {
 
@@ -293,13 +297,343 @@ static cudaError_t launch_attn_d(const LayerView& L, const void* q, const int32_
 #undef QSA_ATTN_CASE
 }
 
-cudaError_t launch_attend(const LayerView& L, const void* q, const int32_t* cells, const int32_t* n_cells,
-                          float* out, cudaStream_t s) {
+cudaError_t launch_attend_split(const LayerView& L, const void* q, const int32_t* cells, const int32_t* n_cells,
+                                float* out, cudaStream_t s) {
   cudaError_t e = L.cfg.head_dim == 128 ? launch_attn_d<128>(L, q, cells, n_cells, s)
                                         : launch_attn_d<64>(L, q, cells, n_cells, s);
   if (e != cudaSuccess) return e;
   return launch_pdl(attn_combine_kernel, dim3(L.cfg.n_q_heads), dim3(128), 0, s, 1, (const float*)L.part_o,
                     (const float*)L.part_ml, out, L.cfg.n_q_heads, L.cfg.head_dim, L.split.n_splits);
+}
+
+// ---------------------------------------------------------------------------------
+// Split-KV flash decode with the split merge done in distributed shared memory.
+// One cluster of CS CTAs per KV head g covers the whole cell set: CTA r stages the K
+// and V rows of cells [r*Lc, (r+1)*Lc) in shared memory (16-byte cp.async, straight
+// from the cache: the gather is fused), computes the f32 logits, softmax statistics and
+// unnormalised P.V of the G query heads that share g, then the CTAs merge their
+// (max, sum, output) partials through DSMEM and write the final output. In the
+// FROM_BLOCKS form the cell ids are expanded on the fly from the selected blocks and
+// the open tail (cell expansion fused in as well).
+// ---------------------------------------------------------------------------------
+constexpr int kAcThreads = 512;
+constexpr int kAcWarps = kAcThreads / 32;
+
+__device__ __forceinline__ void cp_async_16(void* smem_dst, const void* gsrc, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst))),
+               "l"(gsrc), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
+template <int D, int G>
+struct AcSmem {
+  // byte offsets inside the dynamic shared memory for Lc cells per CTA
+  __host__ __device__ static size_t k_off(int) { return 0; }
+  __host__ __device__ static size_t v_off(int lc) { return size_t(lc) * D * 2; }
+  __host__ __device__ static size_t p_off(int lc) { return size_t(lc) * D * 4; }
+  __host__ __device__ static size_t o_off(int lc) { return (p_off(lc) + size_t(G) * lc * 4 + 15) / 16 * 16; }
+  __host__ __device__ static size_t ml_off(int lc) { return o_off(lc) + size_t(G) * D * 4; }
+  __host__ __device__ static size_t cell_off(int lc) { return ml_off(lc) + 2 * G * 4; }
+  __host__ __device__ static size_t stage_off(int lc) { return (cell_off(lc) + size_t(lc) * 4 + 15) / 16 * 16; }
+  __host__ __device__ static size_t bytes(int lc, int cs) { return stage_off(lc) + size_t(cs) * G * 2 * 4; }
+};
+
+template <int D, int G, int CS, bool FROM_BLOCKS>
+__global__ void __launch_bounds__(kAcThreads, 1)
+attn_cluster_kernel(DevState* st, const __half* __restrict__ q, const int32_t* __restrict__ ids,
+                    const int32_t* __restrict__ n_ids, const __half* __restrict__ kc, const __half* __restrict__ vc,
+                    float* __restrict__ out, int n_kv_heads, int cells_per_cta, int max_cells, int k_blocks) {
+  using SM = AcSmem<D, G>;
+  constexpr int VPL = D / 32;
+  constexpr int CH = D * 2 / 16;  // 16-byte chunks per row
+  extern __shared__ __align__(16) unsigned char smem[];
+  const int Lc = cells_per_cta;
+  __half* sK = reinterpret_cast<__half*>(smem + SM::k_off(Lc));
+  __half* sV = reinterpret_cast<__half*>(smem + SM::v_off(Lc));
+  float* s_p = reinterpret_cast<float*>(smem + SM::p_off(Lc));
+  float* s_o = reinterpret_cast<float*>(smem + SM::o_off(Lc));
+  float* s_m = reinterpret_cast<float*>(smem + SM::ml_off(Lc));
+  float* s_l = s_m + G;
+  int* s_cell = reinterpret_cast<int*>(smem + SM::cell_off(Lc));
+  float* s_stage = reinterpret_cast<float*>(smem + SM::stage_off(Lc));  // [CS][G][2] merged (m, l)
+
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = int(cluster.block_rank());
+  const int g = blockIdx.x / CS;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+  pdl_wait();
+  const int n = ld_volatile(&st->n_ctx);
+  const int n_blocks = n / kBlock;
+  int total, ns = 0;
+  if constexpr (FROM_BLOCKS) {
+    ns = *n_ids;
+    if (ns < 0 || ns > k_blocks) {
+      if (blockIdx.x == 0 && tid == 0) record_status(st, QSA_ERR_BAD_INDEX);
+      ns = ns < 0 ? 0 : k_blocks;
+    }
+    total = kBlock * ns + (n - kBlock * n_blocks);
+  } else {
+    total = *n_ids;
+    if (total < 0 || total > max_cells) {
+      if (blockIdx.x == 0 && tid == 0) record_status(st, QSA_ERR_BAD_INDEX);
+      total = total < 0 ? 0 : max_cells;
+    }
+  }
+  const int c0 = rank * Lc;
+  const int cnt = max(0, min(Lc, total - c0));
+
+  for (int i = tid; i < cnt; i += kAcThreads) {
+    const int ci = c0 + i;
+    int cell;
+    if constexpr (FROM_BLOCKS) {
+      if (ci < kBlock * ns) {
+        const int b = ids[ci / kBlock];
+        cell = (b >= 0 && b < n_blocks) ? kBlock * b + ci % kBlock : -1;
+      } else {
+        cell = kBlock * n_blocks + (ci - kBlock * ns);
+      }
+    } else {
+      cell = ids[ci];
+    }
+    if (cell < 0 || cell >= n) {
+      record_status(st, QSA_ERR_BAD_INDEX);
+      cell = -1;
+    }
+    s_cell[i] = cell;
+  }
+  __syncthreads();
+  // stage the selected K and V rows (rows of invalid cells are zero-filled)
+  for (int e = tid; e < cnt * CH; e += kAcThreads) {
+    const int i = e / CH, ch = e % CH;
+    const int cell = s_cell[i];
+    const size_t off = cell >= 0 ? ((size_t(cell) * n_kv_heads + g) * D + ch * 8) : 0;
+    cp_async_16(sK + size_t(i) * D + ch * 8, kc + off, cell >= 0 ? 16 : 0);
+    cp_async_16(sV + size_t(i) * D + ch * 8, vc + off, cell >= 0 ? 16 : 0);
+  }
+  float qv[G][VPL];
+#pragma unroll
+  for (int h = 0; h < G; ++h)
+#pragma unroll
+    for (int x = 0; x < VPL; ++x) qv[h][x] = __half2float(q[(size_t(g) * G + h) * D + lane * VPL + x]);
+  cp_async_commit_wait_all();
+  __syncthreads();
+
+  // logits: warp w takes cells w, w + 16, ...
+  const float scale = 1.0f / sqrtf((float)D);
+  for (int i = warp; i < cnt; i += kAcWarps) {
+    float kx[VPL];
+    if constexpr (VPL == 4) {
+      const uint2 raw = *reinterpret_cast<const uint2*>(sK + size_t(i) * D + lane * 4);
+      const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
+      const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
+      kx[0] = a.x; kx[1] = a.y; kx[2] = b.x; kx[3] = b.y;
+    } else {
+      const float2 a = __half22float2(*reinterpret_cast<const __half2*>(sK + size_t(i) * D + lane * 2));
+      kx[0] = a.x; kx[1] = a.y;
+    }
+    float dot[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      float a = 0.0f;
+#pragma unroll
+      for (int x = 0; x < VPL; ++x) a = fmaf(qv[h][x], kx[x], a);
+      dot[h] = a;
+    }
+    const float mine = transpose_reduce<G>(dot, lane);
+    const int h = head_of_lane<G>(lane);
+    if ((lane & (32 / G - 1)) == 0) s_p[h * Lc + i] = s_cell[i] >= 0 ? mine * scale : -INFINITY;
+  }
+  __syncthreads();
+  // softmax statistics of this CTA's cells, per head
+  for (int h = warp; h < G; h += kAcWarps) {
+    float m = -INFINITY;
+    for (int i = lane; i < cnt; i += 32) m = fmaxf(m, s_p[h * Lc + i]);
+    m = warp_max(m);
+    float l = 0.0f;
+    for (int i = lane; i < cnt; i += 32) {
+      const float p = m == -INFINITY ? 0.0f : expf(s_p[h * Lc + i] - m);
+      s_p[h * Lc + i] = p;
+      l += p;
+    }
+    l = warp_sum(l);
+    if (lane == 0) {
+      s_m[h] = m;
+      s_l[h] = l;
+    }
+  }
+  __syncthreads();
+  // unnormalised P.V: thread -> (head, pair of dims), summed over the cells in order
+  for (int t = tid; t < G * (D / 2); t += kAcThreads) {
+    const int h = t / (D / 2), d2 = t % (D / 2);
+    float o0 = 0.0f, o1 = 0.0f;
+    const float* ph = s_p + h * Lc;
+    for (int i = 0; i < cnt; ++i) {
+      const float2 vv = __half22float2(*reinterpret_cast<const __half2*>(sV + size_t(i) * D + 2 * d2));
+      const float p = ph[i];
+      o0 = fmaf(p, vv.x, o0);
+      o1 = fmaf(p, vv.y, o1);
+    }
+    s_o[h * D + 2 * d2] = o0;
+    s_o[h * D + 2 * d2 + 1] = o1;
+  }
+  cluster.sync();
+  // merge the CS partials: (max, sum) of every CTA first, then this CTA's output slice
+  for (int t = tid; t < CS * G; t += kAcThreads) {
+    const int r = t / G, h = t % G;
+    const float* rm = cluster.map_shared_rank(s_m, r);
+    s_stage[(r * G + h) * 2] = rm[h];
+    s_stage[(r * G + h) * 2 + 1] = rm[G + h];
+  }
+  __syncthreads();
+  constexpr int PAIRS = G * (D / 2);
+  constexpr int PER = (PAIRS + CS - 1) / CS;
+  for (int t = tid; t < PER; t += kAcThreads) {
+    const int pidx = rank * PER + t;
+    if (pidx >= PAIRS) break;
+    const int h = pidx / (D / 2), d2 = pidx % (D / 2);
+    float M = -INFINITY;
+#pragma unroll
+    for (int r = 0; r < CS; ++r) M = fmaxf(M, s_stage[(r * G + h) * 2]);
+    float2 o[CS];
+#pragma unroll
+    for (int r = 0; r < CS; ++r) o[r] = *reinterpret_cast<const float2*>(cluster.map_shared_rank(s_o, r) + h * D + 2 * d2);
+    float a0 = 0.0f, a1 = 0.0f, den = 0.0f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int r = 0; r < CS; ++r) {
+        const float m = s_stage[(r * G + h) * 2];
+        const float e = m == -INFINITY ? 0.0f : expf(m - M);
+        a0 = fmaf(e, o[r].x, a0);
+        a1 = fmaf(e, o[r].y, a1);
+        den = fmaf(e, s_stage[(r * G + h) * 2 + 1], den);
+      }
+    }
+    float2 res = make_float2(0.0f, 0.0f);
+    if (den > 0.0f) res = make_float2(a0 / den, a1 / den);
+    *reinterpret_cast<float2*>(out + (size_t(g) * G + h) * D + 2 * d2) = res;
+  }
+  cluster.sync();  // keep this CTA's shared memory alive until every remote read is done
+}
+
+template <int D, int G, int CS, bool FB>
+static cudaError_t set_ac_attr(size_t smem) {
+  cudaError_t e = cudaFuncSetAttribute(attn_cluster_kernel<D, G, CS, FB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e == cudaSuccess && CS > 8)
+    e = cudaFuncSetAttribute(attn_cluster_kernel<D, G, CS, FB>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  return e;
+}
+
+template <int D, int G, int CS>
+static cudaError_t launch_ac(const LayerView& L, bool from_blocks, const void* q, const int32_t* ids,
+                             const int32_t* n_ids, float* out, cudaStream_t s) {
+  const int lc = L.attn_cells_per_cta;
+  const size_t smem = AcSmem<D, G>::bytes(lc, CS);
+  const dim3 grid(L.cfg.n_kv_heads * CS), block(kAcThreads);
+  const int mc = max_cells_of(L.cfg), kb = L.cfg.top_k_tokens / kBlock;
+  if (from_blocks)
+    return launch_pdl(attn_cluster_kernel<D, G, CS, true>, grid, block, smem, s, CS, L.state, (const __half*)q, ids,
+                      n_ids, (const __half*)L.k_cache, (const __half*)L.v_cache, out, L.cfg.n_kv_heads, lc, mc, kb);
+  return launch_pdl(attn_cluster_kernel<D, G, CS, false>, grid, block, smem, s, CS, L.state, (const __half*)q, ids,
+                    n_ids, (const __half*)L.k_cache, (const __half*)L.v_cache, out, L.cfg.n_kv_heads, lc, mc, kb);
+}
+
+template <int D, int G>
+static cudaError_t launch_ac_g(const LayerView& L, bool fb, const void* q, const int32_t* ids, const int32_t* n_ids,
+                               float* out, cudaStream_t s) {
+  return L.attn_cluster == 16 ? launch_ac<D, G, 16>(L, fb, q, ids, n_ids, out, s)
+                              : launch_ac<D, G, 8>(L, fb, q, ids, n_ids, out, s);
+}
+
+template <int D>
+static cudaError_t launch_ac_d(const LayerView& L, bool fb, const void* q, const int32_t* ids, const int32_t* n_ids,
+                               float* out, cudaStream_t s) {
+  switch (L.cfg.n_q_heads / L.cfg.n_kv_heads) {
+    case 1: return launch_ac_g<D, 1>(L, fb, q, ids, n_ids, out, s);
+    case 2: return launch_ac_g<D, 2>(L, fb, q, ids, n_ids, out, s);
+    case 4: return launch_ac_g<D, 4>(L, fb, q, ids, n_ids, out, s);
+    case 8: return launch_ac_g<D, 8>(L, fb, q, ids, n_ids, out, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_attend(const LayerView& L, const void* q, const int32_t* cells, const int32_t* n_cells, float* out,
+                          cudaStream_t s) {
+  return L.cfg.head_dim == 128 ? launch_ac_d<128>(L, false, q, cells, n_cells, out, s)
+                               : launch_ac_d<64>(L, false, q, cells, n_cells, out, s);
+}
+
+cudaError_t launch_attend_selected(const LayerView& L, const void* q, const int32_t* sel, const int32_t* n_sel,
+                                   float* out, cudaStream_t s) {
+  return L.cfg.head_dim == 128 ? launch_ac_d<128>(L, true, q, sel, n_sel, out, s)
+                               : launch_ac_d<64>(L, true, q, sel, n_sel, out, s);
+}
+
+// Cluster size and cells per CTA for a configuration, plus the kernel attributes they
+// need; called once per context, outside any stream capture.
+template <int D, int G>
+static cudaError_t plan_ac_g(const qsa_config& c, int* cluster, int* lc) {
+  const int mc = max_cells_of(c);
+  for (int cs : {16, 8}) {
+    const int l = (mc + cs - 1) / cs;
+    const size_t smem = AcSmem<D, G>::bytes(l, cs);
+    if (smem > 220 * 1024) continue;
+    cudaError_t e = cs == 16 ? set_ac_attr<D, G, 16, false>(smem) : set_ac_attr<D, G, 8, false>(smem);
+    if (e == cudaSuccess) e = cs == 16 ? set_ac_attr<D, G, 16, true>(smem) : set_ac_attr<D, G, 8, true>(smem);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      continue;
+    }
+    // every KV head's cluster must be able to run at the same time
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(c.n_kv_heads * cs);
+    cfg.blockDim = dim3(kAcThreads);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = cs;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    int active = 0;
+    e = cs == 16 ? cudaOccupancyMaxActiveClusters(&active, attn_cluster_kernel<D, G, 16, true>, &cfg)
+                 : cudaOccupancyMaxActiveClusters(&active, attn_cluster_kernel<D, G, 8, true>, &cfg);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      continue;
+    }
+    if (active >= (cs == 16 ? c.n_kv_heads : 1)) {
+      *cluster = cs;
+      *lc = l;
+      return cudaSuccess;
+    }
+  }
+  return cudaErrorNotSupported;
+}
+
+cudaError_t plan_attention(const qsa_config& c, int* cluster, int* cells_per_cta) {
+  const int G = c.n_q_heads / c.n_kv_heads;
+  if (c.head_dim == 128) {
+    switch (G) {
+      case 1: return plan_ac_g<128, 1>(c, cluster, cells_per_cta);
+      case 2: return plan_ac_g<128, 2>(c, cluster, cells_per_cta);
+      case 4: return plan_ac_g<128, 4>(c, cluster, cells_per_cta);
+      case 8: return plan_ac_g<128, 8>(c, cluster, cells_per_cta);
+    }
+  } else {
+    switch (G) {
+      case 1: return plan_ac_g<64, 1>(c, cluster, cells_per_cta);
+      case 2: return plan_ac_g<64, 2>(c, cluster, cells_per_cta);
+      case 4: return plan_ac_g<64, 4>(c, cluster, cells_per_cta);
+      case 8: return plan_ac_g<64, 8>(c, cluster, cells_per_cta);
+    }
+  }
+  return cudaErrorInvalidValue;
 }
 
 // ---------------------------------------------------------------------------------
@@ -383,6 +717,6 @@ extern "C" qsa_status qsa_sparse_attend_noalloc(const void* q, const void* k_cac
   v.part_o = reinterpret_cast<float*>(p + sizeof(DevState) + ml_bytes);
   // the state block keeps the previous call's contents: set n_ctx and clear the status
   if (launch_set_state(v, n_ctx, 0, kSetRestore, (cudaStream_t)stream) != cudaSuccess) return QSA_ERR_CUDA;
-  if (launch_attend(v, q, cells, n_cells, out, (cudaStream_t)stream) != cudaSuccess) return QSA_ERR_CUDA;
+  if (launch_attend_split(v, q, cells, n_cells, out, (cudaStream_t)stream) != cudaSuccess) return QSA_ERR_CUDA;
   return QSA_OK;
 }

@@ -1,4 +1,4 @@
-// Indexer scan and block-domain top-k.
+// Block-domain top-k (the indexer scan that produces the scores is in qsa_scan_tc.cu).
 //
 // Web page "Part 10" (第10回 EVO-X2 ... 長コンテキストのTGを高速化した話):
 //  - section "QSA indexer": the current query is scored against every completed
@@ -16,121 +16,6 @@
 namespace cg = cooperative_groups;
 
 namespace qsa {
-
-// ---------------------------------------------------------------------------------
-// Indexer scan on the CUDA cores. Each warp scores one block at a time (U blocks per
-// iteration for memory-level parallelism): lane l holds dims [l*VPL, (l+1)*VPL) of the
-// rotated query of every head, reads the same dims of the block's f16 summary (one
-// coalesced 2*D-byte row per warp), and a transposing reduction gives each lane one
-// head's dot product. Accumulation is f32.
-// ---------------------------------------------------------------------------------
-template <int D, int H>
-__global__ void __launch_bounds__(256) index_scan_kernel(DevState* st, const __half* __restrict__ pooled,
-                                                         const __half* __restrict__ q_idx,
-                                                         const float* __restrict__ w,
-                                                         float* __restrict__ scores, float rope_base) {
-  constexpr int VPL = D / 32;  // dims per lane
-  constexpr int U = 4;         // blocks in flight per warp
-  __shared__ float s_q[H][D];
-  __shared__ float s_cos[D / 2], s_sin[D / 2];
-
-  pdl_wait();
-  const int n = ld_volatile(&st->n_ctx);
-  const int n_blocks = n / kBlock;
-  if (ld_volatile(&st->n_pooled) != n_blocks) {
-    if (blockIdx.x == 0 && threadIdx.x == 0) record_status(st, QSA_ERR_STATE);
-    return;
-  }
-  // RoPE of the query at position n-1 (angles in double, rotation in f32)
-  for (int i = threadIdx.x; i < D / 2; i += blockDim.x) {
-    const double theta = pow((double)rope_base, -2.0 * (double)i / (double)D);
-    double sd, cd;
-    sincos((double)(n - 1) * theta, &sd, &cd);
-    s_cos[i] = (float)cd;
-    s_sin[i] = (float)sd;
-  }
-  __syncthreads();
-  for (int e = threadIdx.x; e < H * (D / 2); e += blockDim.x) {
-    const int h = e / (D / 2), i = e % (D / 2);
-    const float x1 = __half2float(q_idx[h * D + i]);
-    const float x2 = __half2float(q_idx[h * D + i + D / 2]);
-    s_q[h][i] = x1 * s_cos[i] - x2 * s_sin[i];
-    s_q[h][i + D / 2] = x1 * s_sin[i] + x2 * s_cos[i];
-  }
-  __syncthreads();
-
-  const int lane = threadIdx.x & 31;
-  float qr[H][VPL];
-#pragma unroll
-  for (int h = 0; h < H; ++h)
-#pragma unroll
-    for (int j = 0; j < VPL; ++j) qr[h][j] = s_q[h][lane * VPL + j];
-  const int my_head = head_of_lane<H>(lane);
-  const float w_mine = w[my_head];
-  const float sqrt_d = sqrtf((float)D);
-
-  const int warps = blockDim.x >> 5;
-  const int gw = blockIdx.x * warps + (threadIdx.x >> 5);
-  const int total_warps = gridDim.x * warps;
-  for (int b0 = gw * U; b0 < n_blocks; b0 += total_warps * U) {
-    float p[U][VPL];
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int b = b0 + u;
-      if (b < n_blocks) {
-        const __half* row = pooled + size_t(b) * D + lane * VPL;
-        if constexpr (VPL == 4) {
-          const uint2 raw = *reinterpret_cast<const uint2*>(row);
-          const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
-          const float2 c = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
-          p[u][0] = a.x; p[u][1] = a.y; p[u][2] = c.x; p[u][3] = c.y;
-        } else {
-          const float2 a = __half22float2(*reinterpret_cast<const __half2*>(row));
-          p[u][0] = a.x; p[u][1] = a.y;
-        }
-      } else {
-#pragma unroll
-        for (int j = 0; j < VPL; ++j) p[u][j] = 0.0f;
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      float dot[H];
-#pragma unroll
-      for (int h = 0; h < H; ++h) {
-        float acc = 0.0f;
-#pragma unroll
-        for (int j = 0; j < VPL; ++j) acc = fmaf(qr[h][j], p[u][j], acc);
-        dot[h] = acc;
-      }
-      const float mine = transpose_reduce<H>(dot, lane);
-      const float total = sum_over_heads<H>(w_mine * fmaxf(mine, 0.0f));
-      const int b = b0 + u;
-      if (lane == 0 && b < n_blocks) scores[b] = total / sqrt_d;
-    }
-  }
-}
-
-template <int D>
-static cudaError_t launch_scan_d(const LayerView& L, const void* q_idx, const float* w, float* scores,
-                                 cudaStream_t s) {
-  const dim3 grid(L.n_sms * 2), block(256);
-  const float base = L.cfg.rope_base;
-  switch (L.cfg.n_idx_heads) {
-    case 1: return launch_pdl(index_scan_kernel<D, 1>, grid, block, 0, s, 1, L.state, (const __half*)L.pooled_cache, (const __half*)q_idx, w, scores, base);
-    case 2: return launch_pdl(index_scan_kernel<D, 2>, grid, block, 0, s, 1, L.state, (const __half*)L.pooled_cache, (const __half*)q_idx, w, scores, base);
-    case 4: return launch_pdl(index_scan_kernel<D, 4>, grid, block, 0, s, 1, L.state, (const __half*)L.pooled_cache, (const __half*)q_idx, w, scores, base);
-    case 8: return launch_pdl(index_scan_kernel<D, 8>, grid, block, 0, s, 1, L.state, (const __half*)L.pooled_cache, (const __half*)q_idx, w, scores, base);
-    case 16: return launch_pdl(index_scan_kernel<D, 16>, grid, block, 0, s, 1, L.state, (const __half*)L.pooled_cache, (const __half*)q_idx, w, scores, base);
-    default: return cudaErrorInvalidValue;
-  }
-}
-
-cudaError_t launch_index_scan(const LayerView& L, const void* q_idx, const float* w, float* scores,
-                              cudaStream_t s) {
-  return L.cfg.d_idx == 128 ? launch_scan_d<128>(L, q_idx, w, scores, s)
-                            : launch_scan_d<64>(L, q_idx, w, scores, s);
-}
 
 // ---------------------------------------------------------------------------------
 // Block top-k: one cluster of kTopkCluster CTAs runs an exact radix select on 32-bit

@@ -2,6 +2,7 @@
 // sequence state, the workspace layout and the kernel launchers.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -84,10 +85,15 @@ struct LayerView {
   float* part_ml;
   AttnSplit split;
   int n_sms;
+  int attn_cluster;        // CTAs per KV head in the attention cluster (16 or 8)
+  int attn_cells_per_cta;  // cells each of them stages
+  CUtensorMap pooled_map;  // TMA descriptor of pooled_cache (encoded at bind time)
 };
 
 // ---- launchers (return the launch's cudaError_t) ----
 cudaError_t init_kernel_attributes();  // once per context creation, outside any capture
+cudaError_t init_scan_attributes();
+cudaError_t encode_pooled_map(const qsa_config& c, void* pooled, CUtensorMap* out);
 cudaError_t launch_set_state(const LayerView& L, int n_ctx, int n_pooled, int mode, cudaStream_t s);
 cudaError_t launch_append(const LayerView& L, int n, const void* k, const void* v,
                           const void* idx, int grid_hint, cudaStream_t s);
@@ -101,6 +107,11 @@ cudaError_t launch_gather(const LayerView& L, const int32_t* sel, const int32_t*
                           cudaStream_t s);
 cudaError_t launch_attend(const LayerView& L, const void* q, const int32_t* cells,
                           const int32_t* n_cells, float* out, cudaStream_t s);
+cudaError_t launch_attend_selected(const LayerView& L, const void* q, const int32_t* sel,
+                                   const int32_t* n_sel, float* out, cudaStream_t s);
+cudaError_t launch_attend_split(const LayerView& L, const void* q, const int32_t* cells,
+                                const int32_t* n_cells, float* out, cudaStream_t s);
+cudaError_t plan_attention(const qsa_config& c, int* cluster, int* cells_per_cta);
 
 // set_state modes
 enum { kSetReset = 0, kSetRestore = 1, kSetInvalidate = 2, kSetClearStatus = 3 };

@@ -1,0 +1,321 @@
+// Indexer scan on the 5th-generation tensor cores (tcgen05) with TMA streaming.
+//
+// Web page "Part 10" (第10回 EVO-X2 ... 長コンテキストのTGを高速化した話), section
+// "QSA indexer": the current indexer query is scored against every completed block's
+// pooled summary. This library's score (the pages give no formula):
+//    score_b = sum_h w_h * max(0, q~_h . p_b) / sqrt(d),   q~_h = RoPE(q_h, n-1).
+//
+// The dots q~_h . p_b for all B blocks and H heads form a dense [B x d] . [d x H]
+// contraction over f16 pooled rows, which at d = 128, H = 16 needs 8 FMA per byte read:
+// more than the CUDA cores sustain at HBM rate, so it runs on the tensor cores:
+//  - the rotated f32 query is split into two f16 matrices, q~ = hi + lo * 2^-12
+//    (hi = f16(q~), lo = f16((q~ - hi) * 2^12)); both are the B operand (N = 2H columns,
+//    padded to 16), so one MMA pass yields hi and lo dots accumulated in f32 and the
+//    epilogue adds them: the query keeps ~22 significant bits instead of f16's 11;
+//  - each CTA (one per SM) owns a contiguous range of pooled rows; warp 4 streams them
+//    with TMA (16-row boxes, 128-byte swizzle) into a 6-stage shared-memory ring,
+//    warp 5 issues tcgen05.mma (M = 128 rows) into one of 4 TMEM accumulators, and
+//    warps 0-3 read the accumulator back (one row per thread) and form the score.
+// No tile is re-read: every pooled byte crosses HBM once (plus at most 15 rows per CTA
+// of rounding to the 16-row box).
+#include <cuda.h>
+#include <cuda_fp16.h>
+
+#include "qsa_device.cuh"
+#include "qsa_sm100.cuh"
+
+namespace qsa {
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kStages = 6;       // shared-memory ring of 128-row tiles
+constexpr int kAcc = 4;          // TMEM accumulators
+constexpr int kBoxRows = 16;     // TMA box height
+constexpr int kThreads = 192;    // warps 0-3 epilogue, warp 4 TMA, warp 5 MMA + TMEM owner
+constexpr float kLoScale = 4096.0f;
+
+template <int D, int H>
+struct ScanShape {
+  static constexpr int HALVES = D / 64;                  // one 128-byte swizzle span = 64 f16
+  static constexpr int N = 2 * H < 16 ? 16 : 2 * H;      // MMA N: hi rows, lo rows, zero pad
+  static constexpr int TILE_BYTES = 128 * D * 2;         // A tile: 128 rows
+  static constexpr int HALF_BYTES = 128 * 128;           // 128 rows x 128 bytes
+  static constexpr int B_HALF_BYTES = N * 128;
+  static constexpr int B_BYTES = N * D * 2;
+  static constexpr int ACC_COLS = kAcc * N;
+  static constexpr int TMEM_COLS = ACC_COLS <= 32 ? 32 : ACC_COLS <= 64 ? 64 : ACC_COLS <= 128 ? 128 : 256;
+  static constexpr uint32_t IDESC = idesc_f16_f32(128, N);
+  static constexpr int CTRL_BYTES = 1024;                // barriers, TMEM address, flags, sin/cos
+  static constexpr size_t SMEM = 1024 + size_t(kStages) * TILE_BYTES + B_BYTES + CTRL_BYTES;
+  static_assert(N <= 32, "the epilogue reads at most 32 accumulator columns");
+  static_assert(TILE_BYTES % 1024 == 0 && B_HALF_BYTES % 1024 == 0, "1024-byte swizzle atoms");
+};
+
+// Byte offset of element (row n, column k) of a K-major operand in the 128-byte swizzle
+// layout (the layout TMA's SWIZZLE_128B writes): 64-column halves of `half_bytes` each,
+// 8-row atoms of 1024 bytes, 16-byte chunk index XOR (row % 8).
+__device__ __forceinline__ uint32_t sw128_offset(int n, int k, int half_bytes) {
+  const int j = k >> 6, c = k & 63;
+  return uint32_t(j * half_bytes + (n >> 3) * 1024 + (n & 7) * 128 + (((c >> 3) ^ (n & 7)) << 4) + ((c & 7) << 1));
+}
+
+}  // namespace
+
+template <int D, int H>
+__global__ void __launch_bounds__(kThreads, 1)
+index_scan_tc_kernel(const __grid_constant__ CUtensorMap pooled_map, DevState* st, const __half* __restrict__ q_idx,
+                     const float* __restrict__ w, float* __restrict__ scores, float rope_base) {
+  using S = ScanShape<D, H>;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  unsigned char* sA = smem;
+  unsigned char* sB = sA + size_t(kStages) * S::TILE_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + S::B_BYTES);
+  uint64_t* empty = full + kStages;
+  uint64_t* tfull = empty + kStages;
+  uint64_t* tempty = tfull + kAcc;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tempty + kAcc);
+  float* s_cos = reinterpret_cast<float*>(tmem_holder + 4);
+  float* s_sin = s_cos + D / 2;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < kAcc; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 128);
+    }
+    fence_mbar_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(tmem_holder, S::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 4 && lane == 0) tma_prefetch_desc(&pooled_map);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  pdl_wait();
+  const int n = ld_volatile(&st->n_ctx);
+  const int n_blocks = n / kBlock;
+  const bool stale = ld_volatile(&st->n_pooled) != n_blocks;
+  if (stale && blockIdx.x == 0 && threadIdx.x == 0) record_status(st, QSA_ERR_STATE);
+  const int r0 = int((long long)blockIdx.x * n_blocks / gridDim.x);
+  const int r1 = int((long long)(blockIdx.x + 1) * n_blocks / gridDim.x);
+  const int n_rows = stale ? 0 : r1 - r0;
+  const int n_tiles = (n_rows + 127) / 128;
+
+  if (n_tiles > 0) {
+    if (warp == 4) {
+      // ---------------- TMA producer ----------------
+      if (lane == 0) {
+        int issued = 0;
+        bool ok = true;
+        for (int t = 0; t < n_tiles && ok; ++t) {
+          const int s = t % kStages;
+          if (t >= kStages && !mbar_wait(&empty[s], ((t / kStages) - 1) & 1)) {
+            ok = false;
+            break;
+          }
+          const int rows = min(128, n_rows - t * 128);
+          const int boxes = (rows + kBoxRows - 1) / kBoxRows;
+          mbar_arrive_expect_tx(&full[s], uint32_t(boxes * kBoxRows * 128 * S::HALVES));
+          unsigned char* dst = sA + size_t(s) * S::TILE_BYTES;
+#pragma unroll
+          for (int j = 0; j < S::HALVES; ++j)
+            for (int b = 0; b < boxes; ++b)
+              tma_load_2d(dst + j * S::HALF_BYTES + b * kBoxRows * 128, &pooled_map, j * 64,
+                          r0 + t * 128 + b * kBoxRows, &full[s]);
+          ++issued;
+        }
+        if (!ok) record_status(st, QSA_ERR_TIMEOUT);
+        // every fill this thread started must land before the CTA's shared memory is released
+        for (int t = max(0, issued - kStages); t < issued; ++t) mbar_wait(&full[t % kStages], (t / kStages) & 1);
+      }
+    } else if (warp == 5) {
+      // ---------------- MMA issuer ----------------
+      named_bar_sync(1, 160);  // B operand written by warps 0-3
+      if (lane == 0) {
+        bool ok = true;
+        int last = -1;
+        for (int t = 0; t < n_tiles; ++t) {
+          const int s = t % kStages, a = t % kAcc;
+          if (!mbar_wait(&full[s], (t / kStages) & 1)) { ok = false; break; }
+          if (t >= kAcc && !mbar_wait(&tempty[a], ((t / kAcc) - 1) & 1)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t d_tmem = tmem_base + uint32_t(a * S::N);
+          const uint32_t a0 = smem_u32(sA + size_t(s) * S::TILE_BYTES);
+          const uint32_t b0 = smem_u32(sB);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const int j = kk >> 2, kin = kk & 3;  // 64-column half, 16-column step inside it
+            const uint64_t adesc = smem_desc_sw128(a0 + j * S::HALF_BYTES + kin * 32);
+            const uint64_t bdesc = smem_desc_sw128(b0 + j * S::B_HALF_BYTES + kin * 32);
+            mma_f16_ss(d_tmem, adesc, bdesc, S::IDESC, kk > 0 ? 1u : 0u);
+          }
+          tc_commit(&empty[s]);
+          tc_commit(&tfull[a]);
+          last = t;
+        }
+        if (!ok) record_status(st, QSA_ERR_TIMEOUT);
+        // the tensor core must be done with TMEM before it is freed
+        if (last >= 0) mbar_wait(&tfull[last % kAcc], (last / kAcc) & 1);
+      }
+      __syncwarp();
+    } else {
+      // ---------------- warps 0-3: rotated, split query -> B operand; then epilogue ----------------
+      const int tid = threadIdx.x;  // 0..127
+      for (int i = tid; i < D / 2; i += 128) {
+        const double theta = pow((double)rope_base, -2.0 * (double)i / (double)D);
+        double sd, cd;
+        sincos((double)(n - 1) * theta, &sd, &cd);
+        s_cos[i] = (float)cd;
+        s_sin[i] = (float)sd;
+      }
+      named_bar_sync(2, 128);
+      for (int e = tid; e < H * (D / 2); e += 128) {
+        const int h = e / (D / 2), i = e % (D / 2);
+        const float x1 = __half2float(q_idx[h * D + i]);
+        const float x2 = __half2float(q_idx[h * D + i + D / 2]);
+        const float r1 = x1 * s_cos[i] - x2 * s_sin[i];
+        const float r2 = x1 * s_sin[i] + x2 * s_cos[i];
+        const __half h1 = __float2half_rn(r1), h2 = __float2half_rn(r2);
+        const __half l1 = __float2half_rn((r1 - __half2float(h1)) * kLoScale);
+        const __half l2 = __float2half_rn((r2 - __half2float(h2)) * kLoScale);
+        *reinterpret_cast<__half*>(sB + sw128_offset(h, i, S::B_HALF_BYTES)) = h1;
+        *reinterpret_cast<__half*>(sB + sw128_offset(h, i + D / 2, S::B_HALF_BYTES)) = h2;
+        *reinterpret_cast<__half*>(sB + sw128_offset(H + h, i, S::B_HALF_BYTES)) = l1;
+        *reinterpret_cast<__half*>(sB + sw128_offset(H + h, i + D / 2, S::B_HALF_BYTES)) = l2;
+      }
+      for (int e = tid; e < (S::N - 2 * H) * D; e += 128)
+        *reinterpret_cast<__half*>(sB + sw128_offset(2 * H + e / D, e % D, S::B_HALF_BYTES)) = __float2half_rn(0.0f);
+      fence_proxy_async_smem();
+      named_bar_sync(1, 160);
+
+      float wr[H];
+#pragma unroll
+      for (int h = 0; h < H; ++h) wr[h] = w[h];
+      const float sqrt_d = sqrtf((float)D);
+      bool ok = true;
+      for (int t = 0; t < n_tiles; ++t) {
+        const int a = t % kAcc;
+        if (!mbar_wait(&tfull[a], (t / kAcc) & 1)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t taddr = tmem_base + (uint32_t(32 * warp) << 16) + uint32_t(a * S::N);
+        float acc[32];
+        if constexpr (S::N == 32) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(taddr, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int c = 0; c < 32; ++c) acc[c] = __uint_as_float(r[c]);
+        } else {
+          uint32_t r[16];
+          tmem_ld_32x32b_x16(taddr, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int c = 0; c < 16; ++c) acc[c] = __uint_as_float(r[c]);
+        }
+        tc_fence_before();
+        mbar_arrive(&tempty[a]);
+        const int row = r0 + t * 128 + tid;
+        if (row < r1) {
+          float s = 0.0f;
+#pragma unroll
+          for (int h = 0; h < H; ++h) s += wr[h] * fmaxf(acc[h] + acc[H + h] * (1.0f / kLoScale), 0.0f);
+          scores[row] = s / sqrt_d;
+        }
+      }
+      if (!ok && tid == 0) record_status(st, QSA_ERR_TIMEOUT);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, S::TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------------
+template <int D, int H>
+static cudaError_t set_scan_attr() {
+  return cudaFuncSetAttribute(index_scan_tc_kernel<D, H>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)ScanShape<D, H>::SMEM);
+}
+
+cudaError_t init_scan_attributes() {
+  cudaError_t e = cudaSuccess;
+#define QSA_SCAN_ATTR(DD)                                                                             \
+  if ((e = set_scan_attr<DD, 1>()) != cudaSuccess || (e = set_scan_attr<DD, 2>()) != cudaSuccess ||   \
+      (e = set_scan_attr<DD, 4>()) != cudaSuccess || (e = set_scan_attr<DD, 8>()) != cudaSuccess ||   \
+      (e = set_scan_attr<DD, 16>()) != cudaSuccess)                                                   \
+    return e;
+  QSA_SCAN_ATTR(64)
+  QSA_SCAN_ATTR(128)
+#undef QSA_SCAN_ATTR
+  return e;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// TMA descriptor of a layer's pooled cache: rows = max_ctx/4 blocks of d_idx f16,
+// 16-row x 64-column boxes written with the 128-byte swizzle.
+cudaError_t encode_pooled_map(const qsa_config& c, void* pooled, CUtensorMap* out) {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+    if (e != cudaSuccess) return e;
+    if (q != cudaDriverEntryPointSuccess || !p) return cudaErrorNotSupported;
+    fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  const cuuint64_t dims[2] = {cuuint64_t(c.d_idx), cuuint64_t(c.max_ctx / kBlock)};
+  const cuuint64_t strides[1] = {cuuint64_t(c.d_idx) * 2};
+  const cuuint32_t box[2] = {64, kBoxRows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(out, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, pooled, dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+template <int D>
+static cudaError_t launch_scan_tc_d(const LayerView& L, const void* q_idx, const float* w, float* scores,
+                                    cudaStream_t s) {
+  const dim3 grid(L.n_sms), block(kThreads);
+  const float base = L.cfg.rope_base;
+#define QSA_SCAN_CASE(HH)                                                                                  \
+  case HH:                                                                                                 \
+    return launch_pdl(index_scan_tc_kernel<D, HH>, grid, block, ScanShape<D, HH>::SMEM, s, 1, L.pooled_map, \
+                      L.state, (const __half*)q_idx, w, scores, base);
+  switch (L.cfg.n_idx_heads) {
+    QSA_SCAN_CASE(1)
+    QSA_SCAN_CASE(2)
+    QSA_SCAN_CASE(4)
+    QSA_SCAN_CASE(8)
+    QSA_SCAN_CASE(16)
+    default: return cudaErrorInvalidValue;
+  }
+#undef QSA_SCAN_CASE
+}
+
+cudaError_t launch_index_scan(const LayerView& L, const void* q_idx, const float* w, float* scores,
+                              cudaStream_t s) {
+  return L.cfg.d_idx == 128 ? launch_scan_tc_d<128>(L, q_idx, w, scores, s)
+                            : launch_scan_tc_d<64>(L, q_idx, w, scores, s);
+}
+
+}  // namespace qsa

@@ -16,7 +16,8 @@ LIB_PATH = os.path.join(_PKG, "libqsa.so")
 
 QSA_OK = 0
 STATUS_NAMES = {0: "QSA_OK", 1: "QSA_ERR_INVALID_ARG", 2: "QSA_ERR_CAPACITY", 3: "QSA_ERR_STATE",
-                4: "QSA_ERR_CUDA", 5: "QSA_ERR_UNSUPPORTED", 6: "QSA_ERR_BAD_INDEX"}
+                4: "QSA_ERR_CUDA", 5: "QSA_ERR_UNSUPPORTED", 6: "QSA_ERR_BAD_INDEX",
+                7: "QSA_ERR_TIMEOUT"}
 QSA_BUF_KV, QSA_BUF_IDX, QSA_BUF_POOLED, QSA_BUF_WORKSPACE, QSA_BUF_MAX_CELLS = range(5)
 
 
@@ -58,6 +59,7 @@ SIGNATURES = {
     "qsa_select_topk": (_I, [_P, _I, _P, _P, _P, _P]),
     "qsa_gather_kv": (_I, [_P, _I, _P, _P, _P, _P, _P, _P, _P]),
     "qsa_sparse_attend": (_I, [_P, _I, _P, _P, _P, _P, _P]),
+    "qsa_sparse_attend_selected": (_I, [_P, _I, _P, _P, _P, _P, _P]),
     "qsa_sparse_attend_noalloc": (_I, [_P, _P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _P]),
 }
 
@@ -186,6 +188,10 @@ class Qsa:
                   stream=None):
         self._check(self.lib.qsa_gather_kv(self.handle, layer, _ptr(sel_blocks), _ptr(n_sel), _ptr(cells),
                                            _ptr(n_cells), _ptr(k_compact), _ptr(v_compact), _stream(stream)))
+
+    def sparse_attend_selected(self, layer, q, sel_blocks, n_sel, out, stream=None):
+        self._check(self.lib.qsa_sparse_attend_selected(self.handle, layer, _ptr(q), _ptr(sel_blocks), _ptr(n_sel),
+                                                        _ptr(out), _stream(stream)))
 
     def sparse_attend(self, layer, q, cells, n_cells, out, stream=None):
         self._check(self.lib.qsa_sparse_attend(self.handle, layer, _ptr(q), _ptr(cells), _ptr(n_cells),

@@ -69,6 +69,10 @@ class GpuLayer:
         self.qsa.sparse_attend(self.layer, to_dev(q), o["cells"] if cells is None else cells,
                                o["n_cells"] if n_cells is None else n_cells, o["out"])
 
+    def attend_selected(self, q):
+        o = self.outs
+        self.qsa.sparse_attend_selected(self.layer, to_dev(q), o["sel"], o["n_sel"], o["out"])
+
     def step(self, st):
         """append -> pooled update -> scan + top-k -> cells -> attention (all on the stream)."""
         self.append(st["k"], st["v"], st["idx"])

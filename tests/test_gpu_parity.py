@@ -358,3 +358,42 @@ def test_full_size_layer_step(wl_name):
         H.assert_attention_close(res["out"], ref_out)
     print(f"{wl_name}: n={n} cells={len(ref_cells)} chain flips={flips}")
     assert g.state() == (n, n // 4, 0)
+
+
+def test_attend_selected_equals_oracle_chain_every_step():
+    """Cell expansion fused into attention: same result as the oracle's cells -> attention."""
+    wl = synth.workload("tiny")
+    qsa, g, ref = _prefilled(wl)
+    for step in range(wl.n_steps):
+        st = synth.step_inputs(wl, 0, step)
+        g.append(st["k"], st["v"], st["idx"])
+        g.update()
+        g.index_topk(st["q_idx"], st["w"])
+        g.attend_selected(st["q"])
+        res = g.fetch()
+        r = ref.decode_step(st["k"], st["v"], st["idx"], st["q_idx"], st["w"], st["q"])
+        if np.array_equal(res["sel"], r["sel"]):
+            H.assert_attention_close(res["out"], r["out"])
+    assert g.state()[2] == 0
+
+
+@pytest.mark.slow
+def test_attend_selected_full_size_256k():
+    """Fused expansion + attention on the oracle's selection at the 256k layer shape."""
+    wl = synth.workload("ctx256k_12l")
+    n = 255182
+    qsa = _qsa(wl, max_ctx=n + 2)
+    g = H.GpuLayer(qsa)
+    pre = synth.prefill_tokens(wl, 0, n)
+    g.append(pre["k"], pre["v"], pre["idx"])
+    qsa.restore_layer(0, n, 0)
+    shape = O.QsaShape.of(wl)
+    st = synth.step_inputs(wl, 0, 0)
+    sel = O.topk_blocks(synth.random_pooled(wl, 0, n // 4, salt=5)[:, 0].astype(np.float64), shape.k_blocks)
+    g.outs["sel"][: len(sel)] = H.to_dev(sel.astype(np.int32))
+    g.outs["n_sel"][0] = len(sel)
+    g.attend_selected(st["q"])
+    out = g.fetch()["out"]
+    ref = O.sparse_attention(st["q"], pre["k"], pre["v"], O.expand_cells(sel, n), shape)
+    H.assert_attention_close(out, ref)
+    assert g.state()[2] == 0
