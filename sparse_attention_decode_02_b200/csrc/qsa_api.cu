@@ -20,7 +20,7 @@ namespace {
 struct Layer {
   bool bound = false;
   qsa_layer_buffers buf{};
-  CUtensorMap pooled_map{};
+  CUtensorMap pooled_tile_map{}, pooled_box_map{};
   // Upper bound on blocks the next pooled update may have to compute; it only sizes
   // the update's grid (the kernel itself reads the exact range from device state).
   long long pending_blocks = 0;
@@ -35,6 +35,7 @@ const char* config_problem(const qsa_config& c) {
   if (c.d_idx != 64 && c.d_idx != 128) return "d_idx must be 64 or 128";
   if (!is_pow2_upto(c.n_idx_heads, 16)) return "n_idx_heads must be 1, 2, 4, 8 or 16";
   if (c.top_k_tokens < kBlock || c.top_k_tokens % kBlock) return "top_k_tokens must be a positive multiple of 4";
+  if (c.top_k_tokens / kBlock > kTopkMaxK) return "top_k_tokens above 4096";
   if (c.head_dim != 64 && c.head_dim != 128) return "head_dim must be 64 or 128";
   if (c.n_kv_heads < 1 || c.n_q_heads < 1 || c.n_q_heads % c.n_kv_heads) return "n_q_heads must be a multiple of n_kv_heads";
   if (!is_pow2_upto(c.n_q_heads / c.n_kv_heads, 8)) return "n_q_heads / n_kv_heads must be 1, 2, 4 or 8";
@@ -91,7 +92,8 @@ struct qsa_ctx {
     v.part_ml = reinterpret_cast<float*>(wsp + ws.part_ml);
     v.split = split;
     v.n_sms = n_sms;
-    v.pooled_map = l.pooled_map;
+    v.pooled_tile_map = l.pooled_tile_map;
+    v.pooled_box_map = l.pooled_box_map;
     v.attn_cluster = attn_cluster;
     v.attn_cells_per_cta = attn_cells_per_cta;
     return v;
@@ -174,11 +176,14 @@ qsa_status qsa_bind_layer(qsa_ctx* ctx, int32_t layer, const qsa_layer_buffers* 
   if (buf->rms_gain && !aligned(buf->rms_gain, 16))
     return ctx->fail(QSA_ERR_INVALID_ARG, "rms_gain must be 16-byte aligned");
   Layer& l = ctx->layers[layer];
-  CUtensorMap map;
-  if (qsa_status st = ctx->cuda(encode_pooled_map(ctx->cfg, buf->pooled_cache, &map), "bind_layer: pooled TMA map"))
+  CUtensorMap tile_map, box_map;
+  if (qsa_status st = ctx->cuda(encode_pooled_map(ctx->cfg, buf->pooled_cache, 128, &tile_map), "bind_layer: pooled TMA map"))
+    return st;
+  if (qsa_status st = ctx->cuda(encode_pooled_map(ctx->cfg, buf->pooled_cache, 16, &box_map), "bind_layer: pooled TMA map"))
     return st;
   l.buf = *buf;
-  l.pooled_map = map;
+  l.pooled_tile_map = tile_map;
+  l.pooled_box_map = box_map;
   l.bound = true;
   l.pending_blocks = 0;
   qsa_status st = ctx->cuda(launch_set_state(ctx->view(layer), 0, 0, kSetReset, (cudaStream_t)stream), "bind_layer");

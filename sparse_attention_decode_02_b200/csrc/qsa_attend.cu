@@ -365,6 +365,7 @@ attn_cluster_kernel(DevState* st, const __half* __restrict__ q, const int32_t* _
   const int g = blockIdx.x / CS;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
+  pdl_launch_dependents();
   pdl_wait();
   const int n = ld_volatile(&st->n_ctx);
   const int n_blocks = n / kBlock;
@@ -422,30 +423,47 @@ attn_cluster_kernel(DevState* st, const __half* __restrict__ q, const int32_t* _
   cp_async_commit_wait_all();
   __syncthreads();
 
-  // logits: warp w takes cells w, w + 16, ...
+  // logits: warp w takes cells w, w + 16, ..., four at a time so that the four
+  // transposing reductions (shuffle chains) interleave
   const float scale = 1.0f / sqrtf((float)D);
-  for (int i = warp; i < cnt; i += kAcWarps) {
-    float kx[VPL];
-    if constexpr (VPL == 4) {
-      const uint2 raw = *reinterpret_cast<const uint2*>(sK + size_t(i) * D + lane * 4);
-      const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
-      const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
-      kx[0] = a.x; kx[1] = a.y; kx[2] = b.x; kx[3] = b.y;
-    } else {
-      const float2 a = __half22float2(*reinterpret_cast<const __half2*>(sK + size_t(i) * D + lane * 2));
-      kx[0] = a.x; kx[1] = a.y;
-    }
-    float dot[G];
+  constexpr int UN = 4;
+  for (int i0 = warp; i0 < cnt; i0 += kAcWarps * UN) {
+    float dot[UN][G];
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      float a = 0.0f;
+    for (int u = 0; u < UN; ++u) {
+      const int i = i0 + u * kAcWarps;
+      float kx[VPL];
+      if (i < cnt) {
+        if constexpr (VPL == 4) {
+          const uint2 raw = *reinterpret_cast<const uint2*>(sK + size_t(i) * D + lane * 4);
+          const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
+          const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
+          kx[0] = a.x; kx[1] = a.y; kx[2] = b.x; kx[3] = b.y;
+        } else {
+          const float2 a = __half22float2(*reinterpret_cast<const __half2*>(sK + size_t(i) * D + lane * 2));
+          kx[0] = a.x; kx[1] = a.y;
+        }
+      } else {
 #pragma unroll
-      for (int x = 0; x < VPL; ++x) a = fmaf(qv[h][x], kx[x], a);
-      dot[h] = a;
+        for (int x = 0; x < VPL; ++x) kx[x] = 0.0f;
+      }
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        float a = 0.0f;
+#pragma unroll
+        for (int x = 0; x < VPL; ++x) a = fmaf(qv[h][x], kx[x], a);
+        dot[u][h] = a;
+      }
     }
-    const float mine = transpose_reduce<G>(dot, lane);
+    float mine[UN];
+#pragma unroll
+    for (int u = 0; u < UN; ++u) mine[u] = transpose_reduce<G>(dot[u], lane);
     const int h = head_of_lane<G>(lane);
-    if ((lane & (32 / G - 1)) == 0) s_p[h * Lc + i] = s_cell[i] >= 0 ? mine * scale : -INFINITY;
+#pragma unroll
+    for (int u = 0; u < UN; ++u) {
+      const int i = i0 + u * kAcWarps;
+      if (i < cnt && (lane & (32 / G - 1)) == 0) s_p[h * Lc + i] = s_cell[i] >= 0 ? mine[u] * scale : -INFINITY;
+    }
   }
   __syncthreads();
   // softmax statistics of this CTA's cells, per head
@@ -466,19 +484,30 @@ attn_cluster_kernel(DevState* st, const __half* __restrict__ q, const int32_t* _
     }
   }
   __syncthreads();
-  // unnormalised P.V: thread -> (head, pair of dims), summed over the cells in order
+  // unnormalised P.V: thread -> (head, pair of dims); four independent partial sums over
+  // the cells (cell i goes to partial i % 4, the cnt % 4 leftovers to partial 0), added in a fixed order
   for (int t = tid; t < G * (D / 2); t += kAcThreads) {
     const int h = t / (D / 2), d2 = t % (D / 2);
-    float o0 = 0.0f, o1 = 0.0f;
+    float o0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, o1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
     const float* ph = s_p + h * Lc;
-    for (int i = 0; i < cnt; ++i) {
+    int i = 0;
+    for (; i + 4 <= cnt; i += 4) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float2 vv = __half22float2(*reinterpret_cast<const __half2*>(sV + size_t(i + u) * D + 2 * d2));
+        const float p = ph[i + u];
+        o0[u] = fmaf(p, vv.x, o0[u]);
+        o1[u] = fmaf(p, vv.y, o1[u]);
+      }
+    }
+    for (; i < cnt; ++i) {  // the last cnt % 4 cells go to partial 0
       const float2 vv = __half22float2(*reinterpret_cast<const __half2*>(sV + size_t(i) * D + 2 * d2));
       const float p = ph[i];
-      o0 = fmaf(p, vv.x, o0);
-      o1 = fmaf(p, vv.y, o1);
+      o0[0] = fmaf(p, vv.x, o0[0]);
+      o1[0] = fmaf(p, vv.y, o1[0]);
     }
-    s_o[h * D + 2 * d2] = o0;
-    s_o[h * D + 2 * d2 + 1] = o1;
+    s_o[h * D + 2 * d2] = (o0[0] + o0[1]) + (o0[2] + o0[3]);
+    s_o[h * D + 2 * d2 + 1] = (o1[0] + o1[1]) + (o1[2] + o1[3]);
   }
   cluster.sync();
   // merge the CS partials: (max, sum) of every CTA first, then this CTA's output slice

@@ -15,6 +15,7 @@
 namespace qsa {
 
 __global__ void set_state_kernel(DevState* st, int n_ctx, int n_pooled, int mode) {
+  pdl_launch_dependents();
   pdl_wait();
   if (threadIdx.x != 0) return;
   if (mode == kSetReset) {
@@ -46,6 +47,7 @@ cudaError_t launch_set_state(const LayerView& L, int n_ctx, int n_pooled, int mo
 __global__ void __launch_bounds__(256) append_kernel(DevState* st, uint4* kc, uint4* vc, uint4* ic,
                                                      const uint4* k, const uint4* v, const uint4* idx,
                                                      int n, int kv_units, int idx_units, int max_ctx) {
+  pdl_launch_dependents();
   pdl_wait();
   const int base = ld_volatile(&st->n_ctx);
   const bool fits = base >= 0 && base + n <= max_ctx;
@@ -95,6 +97,7 @@ __global__ void __launch_bounds__(256) pool_update_kernel(DevState* st, const __
                                                           float rope_base) {
   constexpr int P = D / 64;
   constexpr int HALF = D / 2;
+  pdl_launch_dependents();
   pdl_wait();
   const int n = ld_volatile(&st->n_ctx);
   const int b_first = ld_volatile(&st->n_pooled);

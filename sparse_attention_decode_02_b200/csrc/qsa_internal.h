@@ -12,9 +12,10 @@
 namespace qsa {
 
 constexpr int kBlock = 4;             // tokens per micro-block (compression ratio 4)
-constexpr int kTopkCluster = 8;       // CTAs in the top-k cluster
-constexpr int kTopkThreads = 1024;
-constexpr int kTopkMaxPerCta = 32768; // keys held in shared memory per top-k CTA
+constexpr int kTopkCluster = 16;      // CTAs in the top-k cluster
+constexpr int kTopkThreads = 512;
+constexpr int kTopkMaxPerCta = kTopkThreads * 32;  // keys held in registers per top-k CTA
+constexpr int kTopkMaxK = kTopkThreads * 32 / kTopkCluster;  // largest top_k_tokens / 4 (1024)
 constexpr int kAttnWarps = 8;         // warps per attention CTA
 constexpr int kAttnMaxCells = 64;     // cells per attention CTA (split size cap)
 
@@ -87,13 +88,14 @@ struct LayerView {
   int n_sms;
   int attn_cluster;        // CTAs per KV head in the attention cluster (16 or 8)
   int attn_cells_per_cta;  // cells each of them stages
-  CUtensorMap pooled_map;  // TMA descriptor of pooled_cache (encoded at bind time)
+  CUtensorMap pooled_tile_map;  // TMA descriptors of pooled_cache (encoded at bind time):
+  CUtensorMap pooled_box_map;   // 128-row boxes for whole tiles, 16-row boxes for ragged ones
 };
 
 // ---- launchers (return the launch's cudaError_t) ----
 cudaError_t init_kernel_attributes();  // once per context creation, outside any capture
 cudaError_t init_scan_attributes();
-cudaError_t encode_pooled_map(const qsa_config& c, void* pooled, CUtensorMap* out);
+cudaError_t encode_pooled_map(const qsa_config& c, void* pooled, int box_rows, CUtensorMap* out);
 cudaError_t launch_set_state(const LayerView& L, int n_ctx, int n_pooled, int mode, cudaStream_t s);
 cudaError_t launch_append(const LayerView& L, int n, const void* k, const void* v,
                           const void* idx, int grid_hint, cudaStream_t s);

@@ -47,7 +47,9 @@ struct ScanShape {
   static constexpr int ACC_COLS = kAcc * N;
   static constexpr int TMEM_COLS = ACC_COLS <= 32 ? 32 : ACC_COLS <= 64 ? 64 : ACC_COLS <= 128 ? 128 : 256;
   static constexpr uint32_t IDESC = idesc_f16_f32(128, N);
-  static constexpr int CTRL_BYTES = 1024;                // barriers, TMEM address, flags, sin/cos
+  // barriers and TMEM address (256 B), sin/cos (D floats), RoPE frequencies (D/2 doubles),
+  // raw query (H*D f16)
+  static constexpr int CTRL_BYTES = 256 + D * 4 + D / 2 * 8 + H * D * 2;
   static constexpr size_t SMEM = 1024 + size_t(kStages) * TILE_BYTES + B_BYTES + CTRL_BYTES;
   static_assert(N <= 32, "the epilogue reads at most 32 accumulator columns");
   static_assert(TILE_BYTES % 1024 == 0 && B_HALF_BYTES % 1024 == 0, "1024-byte swizzle atoms");
@@ -65,8 +67,9 @@ __device__ __forceinline__ uint32_t sw128_offset(int n, int k, int half_bytes) {
 
 template <int D, int H>
 __global__ void __launch_bounds__(kThreads, 1)
-index_scan_tc_kernel(const __grid_constant__ CUtensorMap pooled_map, DevState* st, const __half* __restrict__ q_idx,
-                     const float* __restrict__ w, float* __restrict__ scores, float rope_base) {
+index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_constant__ CUtensorMap map_box,
+                     DevState* st, const __half* __restrict__ q_idx, const float* __restrict__ w,
+                     float* __restrict__ scores, float rope_base) {
   using S = ScanShape<D, H>;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -79,8 +82,11 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap pooled_map, DevState* s
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tempty + kAcc);
   float* s_cos = reinterpret_cast<float*>(tmem_holder + 4);
   float* s_sin = s_cos + D / 2;
+  double* s_theta = reinterpret_cast<double*>(s_sin + D / 2);         // D/2 doubles
+  __half* s_q = reinterpret_cast<__half*>(s_theta + D / 2);           // raw query, H x D
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_launch_dependents();
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
@@ -96,7 +102,12 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap pooled_map, DevState* s
     tmem_alloc(tmem_holder, S::TMEM_COLS);
     tmem_relinquish();
   }
-  if (warp == 4 && lane == 0) tma_prefetch_desc(&pooled_map);
+  if (warp == 4 && lane == 0) {
+    tma_prefetch_desc(&map_tile);
+    tma_prefetch_desc(&map_box);
+  }
+  // RoPE frequencies do not depend on the previous kernel: compute them before waiting on it
+  for (int i = threadIdx.x; i < D / 2; i += blockDim.x) s_theta[i] = pow((double)rope_base, -2.0 * (double)i / (double)D);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -125,14 +136,21 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap pooled_map, DevState* s
             break;
           }
           const int rows = min(128, n_rows - t * 128);
-          const int boxes = (rows + kBoxRows - 1) / kBoxRows;
-          mbar_arrive_expect_tx(&full[s], uint32_t(boxes * kBoxRows * 128 * S::HALVES));
           unsigned char* dst = sA + size_t(s) * S::TILE_BYTES;
+          if (rows == 128) {  // whole tile: one 128-row box per 64-column half
+            mbar_arrive_expect_tx(&full[s], uint32_t(S::TILE_BYTES));
 #pragma unroll
-          for (int j = 0; j < S::HALVES; ++j)
-            for (int b = 0; b < boxes; ++b)
-              tma_load_2d(dst + j * S::HALF_BYTES + b * kBoxRows * 128, &pooled_map, j * 64,
-                          r0 + t * 128 + b * kBoxRows, &full[s]);
+            for (int j = 0; j < S::HALVES; ++j)
+              tma_load_2d(dst + j * S::HALF_BYTES, &map_tile, j * 64, r0 + t * 128, &full[s]);
+          } else {            // ragged tail: 16-row boxes, at most 15 rows past the range
+            const int boxes = (rows + kBoxRows - 1) / kBoxRows;
+            mbar_arrive_expect_tx(&full[s], uint32_t(boxes * kBoxRows * 128 * S::HALVES));
+#pragma unroll
+            for (int j = 0; j < S::HALVES; ++j)
+              for (int b = 0; b < boxes; ++b)
+                tma_load_2d(dst + j * S::HALF_BYTES + b * kBoxRows * 128, &map_box, j * 64,
+                            r0 + t * 128 + b * kBoxRows, &full[s]);
+          }
           ++issued;
         }
         if (!ok) record_status(st, QSA_ERR_TIMEOUT);
@@ -172,18 +190,26 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap pooled_map, DevState* s
     } else {
       // ---------------- warps 0-3: rotated, split query -> B operand; then epilogue ----------------
       const int tid = threadIdx.x;  // 0..127
+      // raw query: H*D f16 = H*D/8 16-byte vectors, all loads in flight at once
+      constexpr int QV = H * D / 8;
+      uint4 qraw[(QV + 127) / 128];
+#pragma unroll
+      for (int k = 0; k < (QV + 127) / 128; ++k)
+        if (tid + k * 128 < QV) qraw[k] = reinterpret_cast<const uint4*>(q_idx)[tid + k * 128];
       for (int i = tid; i < D / 2; i += 128) {
-        const double theta = pow((double)rope_base, -2.0 * (double)i / (double)D);
         double sd, cd;
-        sincos((double)(n - 1) * theta, &sd, &cd);
+        sincos((double)(n - 1) * s_theta[i], &sd, &cd);
         s_cos[i] = (float)cd;
         s_sin[i] = (float)sd;
       }
+#pragma unroll
+      for (int k = 0; k < (QV + 127) / 128; ++k)
+        if (tid + k * 128 < QV) reinterpret_cast<uint4*>(s_q)[tid + k * 128] = qraw[k];
       named_bar_sync(2, 128);
       for (int e = tid; e < H * (D / 2); e += 128) {
         const int h = e / (D / 2), i = e % (D / 2);
-        const float x1 = __half2float(q_idx[h * D + i]);
-        const float x2 = __half2float(q_idx[h * D + i + D / 2]);
+        const float x1 = __half2float(s_q[h * D + i]);
+        const float x2 = __half2float(s_q[h * D + i + D / 2]);
         const float r1 = x1 * s_cos[i] - x2 * s_sin[i];
         const float r2 = x1 * s_sin[i] + x2 * s_cos[i];
         const __half h1 = __float2half_rn(r1), h2 = __float2half_rn(r2);
@@ -271,8 +297,8 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 // TMA descriptor of a layer's pooled cache: rows = max_ctx/4 blocks of d_idx f16,
-// 16-row x 64-column boxes written with the 128-byte swizzle.
-cudaError_t encode_pooled_map(const qsa_config& c, void* pooled, CUtensorMap* out) {
+// box_rows x 64-column boxes written with the 128-byte swizzle.
+cudaError_t encode_pooled_map(const qsa_config& c, void* pooled, int box_rows, CUtensorMap* out) {
   static EncodeTiledFn fn = nullptr;
   if (!fn) {
     void* p = nullptr;
@@ -284,7 +310,7 @@ cudaError_t encode_pooled_map(const qsa_config& c, void* pooled, CUtensorMap* ou
   }
   const cuuint64_t dims[2] = {cuuint64_t(c.d_idx), cuuint64_t(c.max_ctx / kBlock)};
   const cuuint64_t strides[1] = {cuuint64_t(c.d_idx) * 2};
-  const cuuint32_t box[2] = {64, kBoxRows};
+  const cuuint32_t box[2] = {64, cuuint32_t(box_rows)};
   const cuuint32_t estr[2] = {1, 1};
   const CUresult r = fn(out, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, pooled, dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -299,8 +325,8 @@ static cudaError_t launch_scan_tc_d(const LayerView& L, const void* q_idx, const
   const float base = L.cfg.rope_base;
 #define QSA_SCAN_CASE(HH)                                                                                  \
   case HH:                                                                                                 \
-    return launch_pdl(index_scan_tc_kernel<D, HH>, grid, block, ScanShape<D, HH>::SMEM, s, 1, L.pooled_map, \
-                      L.state, (const __half*)q_idx, w, scores, base);
+    return launch_pdl(index_scan_tc_kernel<D, HH>, grid, block, ScanShape<D, HH>::SMEM, s, 1, L.pooled_tile_map, \
+                      L.pooled_box_map, L.state, (const __half*)q_idx, w, scores, base);
   switch (L.cfg.n_idx_heads) {
     QSA_SCAN_CASE(1)
     QSA_SCAN_CASE(2)
