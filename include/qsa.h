@@ -145,6 +145,15 @@ qsa_status qsa_append_tokens(qsa_ctx* ctx, int32_t layer, int32_t n, const void*
  * n_pooled = n_ctx/4. In decode this is one block every 4th token, else nothing. */
 qsa_status qsa_update_pooled_cache(qsa_ctx* ctx, int32_t layer, qsa_stream_t stream);
 
+/* Decode form of the two calls above in one launch (Part 10, section COMMON-004: in
+ * decode only the block the new token completes is pooled): appends one token like
+ * qsa_append_token, then pools every block in [n_pooled, (n_ctx+1)/4) like
+ * qsa_update_pooled_cache — one block every 4th token, usually none. The result is
+ * bit-identical to the two calls. Device status QSA_ERR_CAPACITY (and no write) if the
+ * layer is full. */
+qsa_status qsa_decode_append(qsa_ctx* ctx, int32_t layer, const void* k, const void* v,
+                             const void* idx_key, qsa_stream_t stream);
+
 /* Sequence edit / state load: summaries from block `from_block` on are no longer
  * trusted; sets n_pooled = min(n_pooled, from_block). The next update rebuilds them. */
 qsa_status qsa_invalidate_pooled_cache(qsa_ctx* ctx, int32_t layer, int32_t from_block,

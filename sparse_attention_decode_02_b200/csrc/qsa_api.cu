@@ -243,6 +243,16 @@ qsa_status qsa_append_token(qsa_ctx* ctx, int32_t layer, const void* k, const vo
   return qsa_append_tokens(ctx, layer, 1, k, v, idx_key, stream);
 }
 
+qsa_status qsa_decode_append(qsa_ctx* ctx, int32_t layer, const void* k, const void* v, const void* idx_key,
+                             qsa_stream_t stream) {
+  if (!ctx) return QSA_ERR_INVALID_ARG;
+  if (qsa_status st = ctx->layer_ok(layer)) return st;
+  QSA_CHECK_PTR(k, 16, "k");
+  QSA_CHECK_PTR(v, 16, "v");
+  QSA_CHECK_PTR(idx_key, 16, "idx_key");
+  return ctx->cuda(launch_decode_append(ctx->view(layer), k, v, idx_key, (cudaStream_t)stream), "decode_append");
+}
+
 qsa_status qsa_update_pooled_cache(qsa_ctx* ctx, int32_t layer, qsa_stream_t stream) {
   if (!ctx) return QSA_ERR_INVALID_ARG;
   if (qsa_status st = ctx->layer_ok(layer)) return st;

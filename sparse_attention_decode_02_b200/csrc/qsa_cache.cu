@@ -88,15 +88,78 @@ cudaError_t launch_append(const LayerView& L, int n, const void* k, const void* 
                     (const uint4*)idx, n, kv_units, idx_units, L.cfg.max_ctx);
 }
 
-// One warp per block summary. Lane `lane` owns the rotation pairs i = lane*P + j (j < P,
-// P = D/64) and their partners i + D/2.
+// Summary of block b computed by one warp. Lane `lane` owns the rotation pairs
+// i = lane*P + j (j < P, P = D/64) and their partners i + D/2. theta/g1/g2 are the
+// lane's RoPE frequencies and gains (see pool_lane_consts).
+template <int D>
+struct PoolLane {
+  static constexpr int P = D / 64;
+  double theta[P];
+  float g1[P], g2[P];
+};
+
+template <int D>
+__device__ __forceinline__ PoolLane<D> pool_lane_consts(int lane, const float* __restrict__ gain, float rope_base) {
+  PoolLane<D> c;
+#pragma unroll
+  for (int j = 0; j < PoolLane<D>::P; ++j) {
+    const int i = lane * PoolLane<D>::P + j;
+    c.theta[j] = pow((double)rope_base, -2.0 * (double)i / (double)D);
+    c.g1[j] = gain ? gain[i] : 1.0f;
+    c.g2[j] = gain ? gain[i + D / 2] : 1.0f;
+  }
+  return c;
+}
+
+template <int D>
+// `ic` is deliberately not __restrict__: the fused decode kernel reads back a row it has
+// just written, which must not go through the non-coherent load path.
+__device__ __forceinline__ void pool_one_block(int b, int lane, const PoolLane<D>& c, const __half* ic,
+                                               __half* __restrict__ pc, float eps) {
+  constexpr int P = PoolLane<D>::P;
+  constexpr int HALF = D / 2;
+  float m1[P], m2[P];
+#pragma unroll
+  for (int j = 0; j < P; ++j) m1[j] = m2[j] = 0.0f;
+  // mean of the 4 raw indexer keys, summed in token order
+#pragma unroll
+  for (int t = 0; t < kBlock; ++t) {
+    const __half* row = ic + (size_t(b) * kBlock + t) * D;
+#pragma unroll
+    for (int j = 0; j < P; ++j) {
+      m1[j] += __half2float(row[lane * P + j]);
+      m2[j] += __half2float(row[lane * P + j + HALF]);
+    }
+  }
+  float ss = 0.0f;
+#pragma unroll
+  for (int j = 0; j < P; ++j) {
+    m1[j] *= 0.25f;
+    m2[j] *= 0.25f;
+    ss += m1[j] * m1[j] + m2[j] * m2[j];
+  }
+  ss = warp_sum(ss);
+  const float inv_rms = 1.0f / sqrtf(ss / (float)D + eps);
+  const double pos = (double)(b * kBlock);
+#pragma unroll
+  for (int j = 0; j < P; ++j) {
+    const float r1 = m1[j] * inv_rms * c.g1[j];
+    const float r2 = m2[j] * inv_rms * c.g2[j];
+    double sd, cd;
+    sincos(pos * c.theta[j], &sd, &cd);
+    const float cs = (float)cd, sn = (float)sd;
+    const int i = lane * P + j;
+    pc[size_t(b) * D + i] = __float2half_rn(r1 * cs - r2 * sn);
+    pc[size_t(b) * D + i + HALF] = __float2half_rn(r1 * sn + r2 * cs);
+  }
+}
+
+// Pools blocks [n_pooled, n_ctx/4), one warp per block, grid-stride.
 template <int D>
 __global__ void __launch_bounds__(256) pool_update_kernel(DevState* st, const __half* __restrict__ ic,
                                                           __half* __restrict__ pc,
                                                           const float* __restrict__ gain, float eps,
                                                           float rope_base) {
-  constexpr int P = D / 64;
-  constexpr int HALF = D / 2;
   pdl_launch_dependents();
   pdl_wait();
   const int n = ld_volatile(&st->n_ctx);
@@ -105,53 +168,8 @@ __global__ void __launch_bounds__(256) pool_update_kernel(DevState* st, const __
   const int lane = threadIdx.x & 31;
   const int warps = blockDim.x >> 5;
   const int gw = blockIdx.x * warps + (threadIdx.x >> 5);
-
-  double theta[P];
-  float g1[P], g2[P];
-#pragma unroll
-  for (int j = 0; j < P; ++j) {
-    const int i = lane * P + j;
-    theta[j] = pow((double)rope_base, -2.0 * (double)i / (double)D);
-    g1[j] = gain ? gain[i] : 1.0f;
-    g2[j] = gain ? gain[i + HALF] : 1.0f;
-  }
-
-  for (int b = b_first + gw; b < b_end; b += gridDim.x * warps) {
-    float m1[P], m2[P];
-#pragma unroll
-    for (int j = 0; j < P; ++j) m1[j] = m2[j] = 0.0f;
-    // mean of the 4 raw indexer keys, summed in token order
-#pragma unroll
-    for (int t = 0; t < kBlock; ++t) {
-      const __half* row = ic + (size_t(b) * kBlock + t) * D;
-#pragma unroll
-      for (int j = 0; j < P; ++j) {
-        m1[j] += __half2float(row[lane * P + j]);
-        m2[j] += __half2float(row[lane * P + j + HALF]);
-      }
-    }
-    float ss = 0.0f;
-#pragma unroll
-    for (int j = 0; j < P; ++j) {
-      m1[j] *= 0.25f;
-      m2[j] *= 0.25f;
-      ss += m1[j] * m1[j] + m2[j] * m2[j];
-    }
-    ss = warp_sum(ss);
-    const float inv_rms = 1.0f / sqrtf(ss / (float)D + eps);
-    const double pos = (double)(b * kBlock);
-#pragma unroll
-    for (int j = 0; j < P; ++j) {
-      const float r1 = m1[j] * inv_rms * g1[j];
-      const float r2 = m2[j] * inv_rms * g2[j];
-      double sd, cd;
-      sincos(pos * theta[j], &sd, &cd);
-      const float c = (float)cd, s = (float)sd;
-      const int i = lane * P + j;
-      pc[size_t(b) * D + i] = __float2half_rn(r1 * c - r2 * s);
-      pc[size_t(b) * D + i + HALF] = __float2half_rn(r1 * s + r2 * c);
-    }
-  }
+  const PoolLane<D> c = pool_lane_consts<D>(lane, gain, rope_base);
+  for (int b = b_first + gw; b < b_end; b += gridDim.x * warps) pool_one_block<D>(b, lane, c, ic, pc, eps);
   __syncthreads();
   if (threadIdx.x == 0) {
     __threadfence();
@@ -162,6 +180,55 @@ __global__ void __launch_bounds__(256) pool_update_kernel(DevState* st, const __
       __threadfence();
     }
   }
+}
+
+// Decode-step append fused with the incremental pooled update: one CTA writes the token
+// at position n_ctx, then pools every block in [n_pooled, (n_ctx+1)/4) (in decode: the
+// block this token completes, every 4th step, or nothing). Same result as
+// qsa_append_token followed by qsa_update_pooled_cache.
+template <int D>
+__global__ void __launch_bounds__(256) decode_append_kernel(DevState* st, uint4* kc, uint4* vc, uint4* ic,
+                                                            const uint4* k, const uint4* v, const uint4* idx,
+                                                            int kv_units, int max_ctx, __half* __restrict__ pc,
+                                                            const float* __restrict__ gain, float eps,
+                                                            float rope_base) {
+  constexpr int IDX_UNITS = D * 2 / 16;
+  pdl_launch_dependents();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  pdl_wait();
+  const PoolLane<D> c = pool_lane_consts<D>(lane, gain, rope_base);
+  const int n = ld_volatile(&st->n_ctx);
+  const int b_first = ld_volatile(&st->n_pooled);
+  if (n < 0 || n >= max_ctx) {
+    if (threadIdx.x == 0) record_status(st, QSA_ERR_CAPACITY);
+    return;
+  }
+  for (int i = threadIdx.x; i < kv_units; i += blockDim.x) {
+    kc[size_t(n) * kv_units + i] = k[i];
+    vc[size_t(n) * kv_units + i] = v[i];
+  }
+  if (threadIdx.x < IDX_UNITS) ic[size_t(n) * IDX_UNITS + threadIdx.x] = idx[threadIdx.x];
+  __syncthreads();  // the new indexer key is visible to every warp of the CTA
+  const int b_end = (n + 1) / kBlock;
+  const __half* ich = reinterpret_cast<const __half*>(ic);
+  for (int b = b_first + warp; b < b_end; b += blockDim.x >> 5) pool_one_block<D>(b, lane, c, ich, pc, eps);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    if (b_end > b_first) st->n_pooled = b_end;
+    st->n_ctx = n + 1;
+  }
+}
+
+cudaError_t launch_decode_append(const LayerView& L, const void* k, const void* v, const void* idx, cudaStream_t s) {
+  const int kv_units = L.cfg.n_kv_heads * L.cfg.head_dim * 2 / 16;
+  if (L.cfg.d_idx == 128)
+    return launch_pdl(decode_append_kernel<128>, dim3(1), dim3(256), 0, s, 1, L.state, (uint4*)L.k_cache,
+                      (uint4*)L.v_cache, (uint4*)L.idx_cache, (const uint4*)k, (const uint4*)v, (const uint4*)idx,
+                      kv_units, L.cfg.max_ctx, (__half*)L.pooled_cache, L.rms_gain, L.cfg.rms_eps,
+                      L.cfg.rope_base);
+  return launch_pdl(decode_append_kernel<64>, dim3(1), dim3(256), 0, s, 1, L.state, (uint4*)L.k_cache,
+                    (uint4*)L.v_cache, (uint4*)L.idx_cache, (const uint4*)k, (const uint4*)v, (const uint4*)idx,
+                    kv_units, L.cfg.max_ctx, (__half*)L.pooled_cache, L.rms_gain, L.cfg.rms_eps, L.cfg.rope_base);
 }
 
 cudaError_t launch_pool_update(const LayerView& L, int grid_hint, cudaStream_t s) {

@@ -100,6 +100,7 @@ cudaError_t launch_set_state(const LayerView& L, int n_ctx, int n_pooled, int mo
 cudaError_t launch_append(const LayerView& L, int n, const void* k, const void* v,
                           const void* idx, int grid_hint, cudaStream_t s);
 cudaError_t launch_pool_update(const LayerView& L, int grid_hint, cudaStream_t s);
+cudaError_t launch_decode_append(const LayerView& L, const void* k, const void* v, const void* idx, cudaStream_t s);
 cudaError_t launch_index_scan(const LayerView& L, const void* q_idx, const float* w,
                               float* scores, cudaStream_t s);
 cudaError_t launch_topk(const LayerView& L, const float* scores, int32_t* sel, int32_t* n_sel,

@@ -53,6 +53,7 @@ SIGNATURES = {
     "qsa_append_token": (_I, [_P, _I, _P, _P, _P, _P]),
     "qsa_append_tokens": (_I, [_P, _I, _I, _P, _P, _P, _P]),
     "qsa_update_pooled_cache": (_I, [_P, _I, _P]),
+    "qsa_decode_append": (_I, [_P, _I, _P, _P, _P, _P]),
     "qsa_invalidate_pooled_cache": (_I, [_P, _I, _I, _P]),
     "qsa_index_topk": (_I, [_P, _I, _P, _P, _P, _P, _P, _P]),
     "qsa_index_scores": (_I, [_P, _I, _P, _P, _P, _P]),
@@ -165,6 +166,9 @@ class Qsa:
     def append_tokens(self, layer, k, v, idx_key, stream=None):
         self._check(self.lib.qsa_append_tokens(self.handle, layer, int(k.shape[0]), _ptr(k), _ptr(v),
                                                _ptr(idx_key), _stream(stream)))
+
+    def decode_append(self, layer, k, v, idx_key, stream=None):
+        self._check(self.lib.qsa_decode_append(self.handle, layer, _ptr(k), _ptr(v), _ptr(idx_key), _stream(stream)))
 
     def update_pooled_cache(self, layer, stream=None):
         self._check(self.lib.qsa_update_pooled_cache(self.handle, layer, _stream(stream)))

@@ -397,3 +397,31 @@ def test_attend_selected_full_size_256k():
     ref = O.sparse_attention(st["q"], pre["k"], pre["v"], O.expand_cells(sel, n), shape)
     H.assert_attention_close(out, ref)
     assert g.state()[2] == 0
+
+
+def test_decode_append_equals_append_then_update():
+    """The fused decode append gives the same caches and state as the two separate calls."""
+    wl = synth.workload("tiny")
+    qa, ga, _ = _prefilled(wl, n=1021, max_ctx=1100)
+    qb, gb, _ = _prefilled(wl, n=1021, max_ctx=1100)
+    for step in range(11):
+        st = synth.step_inputs(wl, 0, step)
+        ga.append(st["k"], st["v"], st["idx"])
+        ga.update()
+        gb.qsa.decode_append(0, H.to_dev(st["k"]), H.to_dev(st["v"]), H.to_dev(st["idx"]))
+        assert ga.state() == gb.state()
+    n = ga.state()[0]
+    np.testing.assert_array_equal(ga.pooled_rows(0, n // 4), gb.pooled_rows(0, n // 4))
+    for key in ("k_cache", "v_cache", "idx_cache"):
+        np.testing.assert_array_equal(ga.buf[key].cpu().numpy(), gb.buf[key].cpu().numpy())
+    # a lagging cache (several blocks behind) is caught up by the fused call as well
+    pre = synth.prefill_tokens(wl, 0, 9, first=n)
+    ga.append(pre["k"], pre["v"], pre["idx"])
+    gb.append(pre["k"], pre["v"], pre["idx"])
+    st = synth.step_inputs(wl, 0, 20)
+    ga.append(st["k"], st["v"], st["idx"])
+    ga.update()
+    gb.qsa.decode_append(0, H.to_dev(st["k"]), H.to_dev(st["v"]), H.to_dev(st["idx"]))
+    assert ga.state() == gb.state() and ga.state()[1] == ga.state()[0] // 4
+    n = ga.state()[0]
+    np.testing.assert_array_equal(ga.pooled_rows(0, n // 4), gb.pooled_rows(0, n // 4))
