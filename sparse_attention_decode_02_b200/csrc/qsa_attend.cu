@@ -328,16 +328,49 @@ __device__ __forceinline__ void cp_async_commit_wait_all() {
   asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
 }
 
+// Warp-level tensor-core helpers (f16 inputs, f32 accumulation). The contractions here
+// are tiny (8 query heads x ~129 cells per CTA), below the 64/128-row tiles of tcgen05,
+// so the warp-synchronous m16n8k16 form is used; it keeps the logits and P.V off the
+// CUDA cores, whose issue rate bounded this kernel.
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(p))));
+}
+__device__ __forceinline__ void ldsm_x2(uint32_t (&r)[2], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];"
+               : "=r"(r[0]), "=r"(r[1])
+               : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(p))));
+}
+__device__ __forceinline__ void ldsm_x2_trans(uint32_t (&r)[2], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];"
+               : "=r"(r[0]), "=r"(r[1])
+               : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(p))));
+}
+
+// Shared memory of attn_cluster_kernel for Lc cells per CTA (LP = Lc rounded up to 16).
+// K and V rows are padded to D + 8 halves and P rows to LP + 8 halves so that the 8 row
+// addresses of every ldmatrix fall in distinct 16-byte bank groups.
 template <int D, int G>
 struct AcSmem {
-  // byte offsets inside the dynamic shared memory for Lc cells per CTA
+  static constexpr int RS = D + 8;  // K/V row stride (halves)
+  __host__ __device__ static int lp(int lc) { return (lc + 15) & ~15; }
+  __host__ __device__ static int ps(int lc) { return lp(lc) + 8; }  // P row stride (halves)
   __host__ __device__ static size_t k_off(int) { return 0; }
-  __host__ __device__ static size_t v_off(int lc) { return size_t(lc) * D * 2; }
-  __host__ __device__ static size_t p_off(int lc) { return size_t(lc) * D * 4; }
-  __host__ __device__ static size_t o_off(int lc) { return (p_off(lc) + size_t(G) * lc * 4 + 15) / 16 * 16; }
-  __host__ __device__ static size_t ml_off(int lc) { return o_off(lc) + size_t(G) * D * 4; }
-  __host__ __device__ static size_t cell_off(int lc) { return ml_off(lc) + 2 * G * 4; }
-  __host__ __device__ static size_t stage_off(int lc) { return (cell_off(lc) + size_t(lc) * 4 + 15) / 16 * 16; }
+  __host__ __device__ static size_t v_off(int lc) { return size_t(lp(lc)) * RS * 2; }
+  __host__ __device__ static size_t p_off(int lc) { return 2 * v_off(lc); }
+  __host__ __device__ static size_t o_off(int lc) { return p_off(lc) + size_t(8) * ps(lc) * 2; }
+  __host__ __device__ static size_t red_off(int lc) { return o_off(lc) + size_t(G) * D * 4; }     // 2 x 16 x 8 f32
+  __host__ __device__ static size_t ml_off(int lc) { return red_off(lc) + 2 * 16 * 8 * 4; }        // 2G f32
+  __host__ __device__ static size_t cell_off(int lc) { return ml_off(lc) + 16 * 4; }
+  __host__ __device__ static size_t stage_off(int lc) { return (cell_off(lc) + size_t(lp(lc)) * 4 + 15) / 16 * 16; }
   __host__ __device__ static size_t bytes(int lc, int cs) { return stage_off(lc) + size_t(cs) * G * 2 * 4; }
 };
 
@@ -347,15 +380,20 @@ attn_cluster_kernel(DevState* st, const __half* __restrict__ q, const int32_t* _
                     const int32_t* __restrict__ n_ids, const __half* __restrict__ kc, const __half* __restrict__ vc,
                     float* __restrict__ out, int n_kv_heads, int cells_per_cta, int max_cells, int k_blocks) {
   using SM = AcSmem<D, G>;
-  constexpr int VPL = D / 32;
+  constexpr int RS = SM::RS;
+  constexpr int KSTEPS = D / 16;
   constexpr int CH = D * 2 / 16;  // 16-byte chunks per row
+  static_assert(G <= 8, "the 8 rows of the MMA hold the query heads of one KV head");
   extern __shared__ __align__(16) unsigned char smem[];
   const int Lc = cells_per_cta;
+  const int LP = SM::lp(Lc), PS = SM::ps(Lc);
   __half* sK = reinterpret_cast<__half*>(smem + SM::k_off(Lc));
   __half* sV = reinterpret_cast<__half*>(smem + SM::v_off(Lc));
-  float* s_p = reinterpret_cast<float*>(smem + SM::p_off(Lc));
+  __half* sP = reinterpret_cast<__half*>(smem + SM::p_off(Lc));
   float* s_o = reinterpret_cast<float*>(smem + SM::o_off(Lc));
-  float* s_m = reinterpret_cast<float*>(smem + SM::ml_off(Lc));
+  float* s_rmax = reinterpret_cast<float*>(smem + SM::red_off(Lc));   // [16 warps][8 rows]
+  float* s_rsum = s_rmax + 16 * 8;
+  float* s_m = reinterpret_cast<float*>(smem + SM::ml_off(Lc));       // [G], then s_l [G]
   float* s_l = s_m + G;
   int* s_cell = reinterpret_cast<int*>(smem + SM::cell_off(Lc));
   float* s_stage = reinterpret_cast<float*>(smem + SM::stage_off(Lc));  // [CS][G][2] merged (m, l)
@@ -364,6 +402,7 @@ attn_cluster_kernel(DevState* st, const __half* __restrict__ q, const int32_t* _
   const int rank = int(cluster.block_rank());
   const int g = blockIdx.x / CS;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int gq = lane >> 2, tq = lane & 3;  // MMA fragment row (query head) and column pair
 
   pdl_launch_dependents();
   pdl_wait();
@@ -387,127 +426,122 @@ attn_cluster_kernel(DevState* st, const __half* __restrict__ q, const int32_t* _
   const int c0 = rank * Lc;
   const int cnt = max(0, min(Lc, total - c0));
 
-  for (int i = tid; i < cnt; i += kAcThreads) {
-    const int ci = c0 + i;
-    int cell;
-    if constexpr (FROM_BLOCKS) {
-      if (ci < kBlock * ns) {
-        const int b = ids[ci / kBlock];
-        cell = (b >= 0 && b < n_blocks) ? kBlock * b + ci % kBlock : -1;
+  for (int i = tid; i < LP; i += kAcThreads) {
+    int cell = -1;
+    if (i < cnt) {
+      const int ci = c0 + i;
+      if constexpr (FROM_BLOCKS) {
+        if (ci < kBlock * ns) {
+          const int b = ids[ci / kBlock];
+          cell = (b >= 0 && b < n_blocks) ? kBlock * b + ci % kBlock : -1;
+        } else {
+          cell = kBlock * n_blocks + (ci - kBlock * ns);
+        }
       } else {
-        cell = kBlock * n_blocks + (ci - kBlock * ns);
+        cell = ids[ci];
       }
-    } else {
-      cell = ids[ci];
-    }
-    if (cell < 0 || cell >= n) {
-      record_status(st, QSA_ERR_BAD_INDEX);
-      cell = -1;
+      if (cell < 0 || cell >= n) {
+        record_status(st, QSA_ERR_BAD_INDEX);
+        cell = -1;
+      }
     }
     s_cell[i] = cell;
   }
   __syncthreads();
-  // stage the selected K and V rows (rows of invalid cells are zero-filled)
-  for (int e = tid; e < cnt * CH; e += kAcThreads) {
+  // stage the selected K and V rows (rows of invalid or padding cells are zero-filled)
+  for (int e = tid; e < LP * CH; e += kAcThreads) {
     const int i = e / CH, ch = e % CH;
     const int cell = s_cell[i];
     const size_t off = cell >= 0 ? ((size_t(cell) * n_kv_heads + g) * D + ch * 8) : 0;
-    cp_async_16(sK + size_t(i) * D + ch * 8, kc + off, cell >= 0 ? 16 : 0);
-    cp_async_16(sV + size_t(i) * D + ch * 8, vc + off, cell >= 0 ? 16 : 0);
+    cp_async_16(sK + size_t(i) * RS + ch * 8, kc + off, cell >= 0 ? 16 : 0);
+    cp_async_16(sV + size_t(i) * RS + ch * 8, vc + off, cell >= 0 ? 16 : 0);
   }
-  float qv[G][VPL];
+  // query fragments (A operand, rows = the G heads of KV head g, rows >= G zero)
+  uint32_t qa[KSTEPS][2];
 #pragma unroll
-  for (int h = 0; h < G; ++h)
-#pragma unroll
-    for (int x = 0; x < VPL; ++x) qv[h][x] = __half2float(q[(size_t(g) * G + h) * D + lane * VPL + x]);
+  for (int ks = 0; ks < KSTEPS; ++ks) {
+    qa[ks][0] = qa[ks][1] = 0u;
+    if (gq < G) {
+      const __half* qr = q + (size_t(g) * G + gq) * D + ks * 16 + 2 * tq;
+      qa[ks][0] = *reinterpret_cast<const uint32_t*>(qr);
+      qa[ks][1] = *reinterpret_cast<const uint32_t*>(qr + 8);
+    }
+  }
   cp_async_commit_wait_all();
   __syncthreads();
 
-  // logits: warp w takes cells w, w + 16, ..., four at a time so that the four
-  // transposing reductions (shuffle chains) interleave
+  // ---- logits = Q K^T: warp w takes 8-cell tiles w and w + 16 ----
   const float scale = 1.0f / sqrtf((float)D);
-  constexpr int UN = 4;
-  for (int i0 = warp; i0 < cnt; i0 += kAcWarps * UN) {
-    float dot[UN][G];
+  const int NT = LP / 8;  // <= 32
+  float lg[2][2];
+  float rmax = -INFINITY;
 #pragma unroll
-    for (int u = 0; u < UN; ++u) {
-      const int i = i0 + u * kAcWarps;
-      float kx[VPL];
-      if (i < cnt) {
-        if constexpr (VPL == 4) {
-          const uint2 raw = *reinterpret_cast<const uint2*>(sK + size_t(i) * D + lane * 4);
-          const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
-          const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
-          kx[0] = a.x; kx[1] = a.y; kx[2] = b.x; kx[3] = b.y;
-        } else {
-          const float2 a = __half22float2(*reinterpret_cast<const __half2*>(sK + size_t(i) * D + lane * 2));
-          kx[0] = a.x; kx[1] = a.y;
-        }
-      } else {
+  for (int tt = 0; tt < 2; ++tt) {
+    lg[tt][0] = lg[tt][1] = -INFINITY;
+    const int nt = warp + 16 * tt;
+    if (nt >= NT) continue;  // warp-uniform
+    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    const __half* kb = sK + size_t(nt * 8 + (lane & 7)) * RS + (lane >> 3) * 8;
 #pragma unroll
-        for (int x = 0; x < VPL; ++x) kx[x] = 0.0f;
-      }
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        float a = 0.0f;
-#pragma unroll
-        for (int x = 0; x < VPL; ++x) a = fmaf(qv[h][x], kx[x], a);
-        dot[u][h] = a;
-      }
+    for (int ks = 0; ks < KSTEPS; ks += 2) {
+      uint32_t b[4];
+      ldsm_x4(b, kb + ks * 16);  // cells nt*8.., dims ks*16 + {0,8,16,24}..
+      mma_16816(acc, qa[ks][0], 0u, qa[ks][1], 0u, b[0], b[1]);
+      mma_16816(acc, qa[ks + 1][0], 0u, qa[ks + 1][1], 0u, b[2], b[3]);
     }
-    float mine[UN];
 #pragma unroll
-    for (int u = 0; u < UN; ++u) mine[u] = transpose_reduce<G>(dot[u], lane);
-    const int h = head_of_lane<G>(lane);
-#pragma unroll
-    for (int u = 0; u < UN; ++u) {
-      const int i = i0 + u * kAcWarps;
-      if (i < cnt && (lane & (32 / G - 1)) == 0) s_p[h * Lc + i] = s_cell[i] >= 0 ? mine[u] * scale : -INFINITY;
+    for (int c = 0; c < 2; ++c) {
+      const int i = nt * 8 + 2 * tq + c;
+      lg[tt][c] = (i < cnt && s_cell[i] >= 0) ? acc[c] * scale : -INFINITY;
+      rmax = fmaxf(rmax, lg[tt][c]);
     }
   }
+  rmax = fmaxf(rmax, __shfl_xor_sync(0xffffffffu, rmax, 1));
+  rmax = fmaxf(rmax, __shfl_xor_sync(0xffffffffu, rmax, 2));
+  if (tq == 0) s_rmax[warp * 8 + gq] = rmax;
   __syncthreads();
-  // softmax statistics of this CTA's cells, per head
-  for (int h = warp; h < G; h += kAcWarps) {
-    float m = -INFINITY;
-    for (int i = lane; i < cnt; i += 32) m = fmaxf(m, s_p[h * Lc + i]);
-    m = warp_max(m);
-    float l = 0.0f;
-    for (int i = lane; i < cnt; i += 32) {
-      const float p = m == -INFINITY ? 0.0f : expf(s_p[h * Lc + i] - m);
-      s_p[h * Lc + i] = p;
-      l += p;
-    }
-    l = warp_sum(l);
-    if (lane == 0) {
-      s_m[h] = m;
-      s_l[h] = l;
-    }
-  }
-  __syncthreads();
-  // unnormalised P.V: thread -> (head, pair of dims); four independent partial sums over
-  // the cells (cell i goes to partial i % 4, the cnt % 4 leftovers to partial 0), added in a fixed order
-  for (int t = tid; t < G * (D / 2); t += kAcThreads) {
-    const int h = t / (D / 2), d2 = t % (D / 2);
-    float o0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, o1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    const float* ph = s_p + h * Lc;
-    int i = 0;
-    for (; i + 4 <= cnt; i += 4) {
+  float m = -INFINITY;
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const float2 vv = __half22float2(*reinterpret_cast<const __half2*>(sV + size_t(i + u) * D + 2 * d2));
-        const float p = ph[i + u];
-        o0[u] = fmaf(p, vv.x, o0[u]);
-        o1[u] = fmaf(p, vv.y, o1[u]);
-      }
+  for (int w = 0; w < 16; ++w) m = fmaxf(m, s_rmax[w * 8 + gq]);
+  // probabilities, rounded to f16 for the P.V product; the row sums use the rounded values
+  float psum = 0.0f;
+#pragma unroll
+  for (int tt = 0; tt < 2; ++tt) {
+    const int nt = warp + 16 * tt;
+    if (nt >= NT) continue;
+    const float p0 = m == -INFINITY ? 0.0f : expf(lg[tt][0] - m);
+    const float p1 = m == -INFINITY ? 0.0f : expf(lg[tt][1] - m);
+    const __half2 h = __floats2half2_rn(p0, p1);
+    *reinterpret_cast<__half2*>(sP + size_t(gq) * PS + nt * 8 + 2 * tq) = h;
+    const float2 r = __half22float2(h);
+    psum += r.x + r.y;
+  }
+  psum += __shfl_xor_sync(0xffffffffu, psum, 1);
+  psum += __shfl_xor_sync(0xffffffffu, psum, 2);
+  if (tq == 0) s_rsum[warp * 8 + gq] = psum;
+  __syncthreads();
+  if (tid < G) {
+    float mm = -INFINITY, ll = 0.0f;
+#pragma unroll
+    for (int w = 0; w < 16; ++w) {
+      mm = fmaxf(mm, s_rmax[w * 8 + tid]);
+      ll += s_rsum[w * 8 + tid];
     }
-    for (; i < cnt; ++i) {  // the last cnt % 4 cells go to partial 0
-      const float2 vv = __half22float2(*reinterpret_cast<const __half2*>(sV + size_t(i) * D + 2 * d2));
-      const float p = ph[i];
-      o0[0] = fmaf(p, vv.x, o0[0]);
-      o1[0] = fmaf(p, vv.y, o1[0]);
+    s_m[tid] = mm;
+    s_l[tid] = ll;
+  }
+  // ---- unnormalised P.V: warp w takes output dims [8w, 8w+8), all cells ----
+  if (warp < D / 8) {
+    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    const __half* pb = sP + size_t(lane & 7) * PS + ((lane >> 3) & 1) * 8;
+    const __half* vb = sV + size_t((lane & 7) + ((lane >> 3) & 1) * 8) * RS + warp * 8;
+    for (int kc16 = 0; kc16 < LP / 16; ++kc16) {
+      uint32_t a[2], b[2];
+      ldsm_x2(a, pb + kc16 * 16);                     // P rows 0..7, cells kc16*16 + {0..7, 8..15}
+      ldsm_x2_trans(b, vb + size_t(kc16) * 16 * RS);  // V cells kc16*16 + {0..7, 8..15}, dims 8w..8w+7
+      mma_16816(acc, a[0], 0u, a[1], 0u, b[0], b[1]);
     }
-    s_o[h * D + 2 * d2] = (o0[0] + o0[1]) + (o0[2] + o0[3]);
-    s_o[h * D + 2 * d2 + 1] = (o1[0] + o1[1]) + (o1[2] + o1[3]);
+    if (gq < G) *reinterpret_cast<float2*>(s_o + gq * D + warp * 8 + 2 * tq) = make_float2(acc[0], acc[1]);
   }
   cluster.sync();
   // merge the CS partials: (max, sum) of every CTA first, then this CTA's output slice
@@ -534,8 +568,8 @@ attn_cluster_kernel(DevState* st, const __half* __restrict__ q, const int32_t* _
     if (M != -INFINITY) {
 #pragma unroll
       for (int r = 0; r < CS; ++r) {
-        const float m = s_stage[(r * G + h) * 2];
-        const float e = m == -INFINITY ? 0.0f : expf(m - M);
+        const float mr = s_stage[(r * G + h) * 2];
+        const float e = mr == -INFINITY ? 0.0f : expf(mr - M);
         a0 = fmaf(e, o[r].x, a0);
         a1 = fmaf(e, o[r].y, a1);
         den = fmaf(e, s_stage[(r * G + h) * 2 + 1], den);
@@ -610,7 +644,7 @@ static cudaError_t plan_ac_g(const qsa_config& c, int* cluster, int* lc) {
   for (int cs : {16, 8}) {
     const int l = (mc + cs - 1) / cs;
     const size_t smem = AcSmem<D, G>::bytes(l, cs);
-    if (smem > 220 * 1024) continue;
+    if (smem > 220 * 1024 || AcSmem<D, G>::lp(l) > 256) continue;
     cudaError_t e = cs == 16 ? set_ac_attr<D, G, 16, false>(smem) : set_ac_attr<D, G, 8, false>(smem);
     if (e == cudaSuccess) e = cs == 16 ? set_ac_attr<D, G, 16, true>(smem) : set_ac_attr<D, G, 8, true>(smem);
     if (e != cudaSuccess) {
