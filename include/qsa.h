@@ -66,7 +66,7 @@ typedef struct {
   int32_t max_ctx;        /* token capacity per layer; a multiple of 4, <= 1,048,576    */
   int32_t d_idx;          /* indexer key width: 64 or 128                               */
   int32_t n_idx_heads;    /* indexer heads H: 1, 2, 4, 8 or 16                          */
-  int32_t top_k_tokens;   /* indexer_top_k in tokens, a multiple of 4 (2048 on pages)   */
+  int32_t top_k_tokens;   /* indexer_top_k in tokens: a multiple of 4, <= 4092 (pages: 2048) */
   int32_t n_q_heads;      /* attention query heads Hq                                   */
   int32_t n_kv_heads;     /* attention KV heads Hkv; Hq / Hkv in {1, 2, 4, 8}          */
   int32_t head_dim;       /* attention head dimension D: 64 or 128                      */
@@ -176,8 +176,10 @@ qsa_status qsa_index_topk(qsa_ctx* ctx, int32_t layer, const void* q_idx, const 
 
 /* The two halves of qsa_index_topk, for callers that want the scores alone or want to
  * select from scores they computed. qsa_index_scores writes scores [n_ctx/4] f32 (same
- * definition and requirements as above); qsa_select_topk selects from scores [n_ctx/4]
- * f32 with the same rule and outputs (NaN ranks lowest; -0 equals +0). */
+ * definition and requirements as above); qsa_select_topk selects from the first n_ctx/4
+ * entries of scores with the same rule and outputs (NaN ranks lowest; -0 equals +0).
+ * Both take a scores buffer of max_ctx/4 f32: qsa_select_topk may read all of it (the
+ * entries past n_ctx/4 are ignored). */
 qsa_status qsa_index_scores(qsa_ctx* ctx, int32_t layer, const void* q_idx, const float* w,
                             float* scores, qsa_stream_t stream);
 qsa_status qsa_select_topk(qsa_ctx* ctx, int32_t layer, const float* scores, int32_t* sel_blocks,

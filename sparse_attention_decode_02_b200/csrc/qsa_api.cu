@@ -35,7 +35,8 @@ const char* config_problem(const qsa_config& c) {
   if (c.d_idx != 64 && c.d_idx != 128) return "d_idx must be 64 or 128";
   if (!is_pow2_upto(c.n_idx_heads, 16)) return "n_idx_heads must be 1, 2, 4, 8 or 16";
   if (c.top_k_tokens < kBlock || c.top_k_tokens % kBlock) return "top_k_tokens must be a positive multiple of 4";
-  if (c.top_k_tokens / kBlock > kTopkMaxK) return "top_k_tokens above 4096";
+  // the attention cluster stages at most 16 x 256 cells: K blocks plus the 3-token tail
+  if (c.top_k_tokens > 4092 || c.top_k_tokens / kBlock > kTopkMaxK) return "top_k_tokens above 4092";
   if (c.head_dim != 64 && c.head_dim != 128) return "head_dim must be 64 or 128";
   if (c.n_kv_heads < 1 || c.n_q_heads < 1 || c.n_q_heads % c.n_kv_heads) return "n_q_heads must be a multiple of n_kv_heads";
   if (!is_pow2_upto(c.n_q_heads / c.n_kv_heads, 8)) return "n_q_heads / n_kv_heads must be 1, 2, 4 or 8";

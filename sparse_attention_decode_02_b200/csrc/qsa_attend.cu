@@ -407,23 +407,32 @@ attn_cluster_kernel(DevState* st, const __half* __restrict__ q, const int32_t* _
   pdl_launch_dependents();
   pdl_wait();
   const int n = ld_volatile(&st->n_ctx);
+  const int c0 = rank * Lc;
+  // this thread's id, loaded in the same round trip as the counts (clamped into the id
+  // buffer, checked against the counts below)
+  int id_spec = 0;
+  if (tid < Lc) {
+    const int ci = c0 + tid;
+    id_spec = FROM_BLOCKS ? ids[min(ci / kBlock, k_blocks - 1)] : ids[min(ci, max_cells - 1)];
+  }
+  const int n_ids_v = *n_ids;
+  asm volatile("" ::"r"(id_spec), "r"(n_ids_v), "r"(n));  // keep the loads ahead of the branches
   const int n_blocks = n / kBlock;
   int total, ns = 0;
   if constexpr (FROM_BLOCKS) {
-    ns = *n_ids;
+    ns = n_ids_v;
     if (ns < 0 || ns > k_blocks) {
       if (blockIdx.x == 0 && tid == 0) record_status(st, QSA_ERR_BAD_INDEX);
       ns = ns < 0 ? 0 : k_blocks;
     }
     total = kBlock * ns + (n - kBlock * n_blocks);
   } else {
-    total = *n_ids;
+    total = n_ids_v;
     if (total < 0 || total > max_cells) {
       if (blockIdx.x == 0 && tid == 0) record_status(st, QSA_ERR_BAD_INDEX);
       total = total < 0 ? 0 : max_cells;
     }
   }
-  const int c0 = rank * Lc;
   const int cnt = max(0, min(Lc, total - c0));
 
   for (int i = tid; i < LP; i += kAcThreads) {
@@ -432,13 +441,13 @@ attn_cluster_kernel(DevState* st, const __half* __restrict__ q, const int32_t* _
       const int ci = c0 + i;
       if constexpr (FROM_BLOCKS) {
         if (ci < kBlock * ns) {
-          const int b = ids[ci / kBlock];
+          const int b = i == tid ? id_spec : ids[ci / kBlock];
           cell = (b >= 0 && b < n_blocks) ? kBlock * b + ci % kBlock : -1;
         } else {
           cell = kBlock * n_blocks + (ci - kBlock * ns);
         }
       } else {
-        cell = ids[ci];
+        cell = i == tid ? id_spec : ids[ci];
       }
       if (cell < 0 || cell >= n) {
         record_status(st, QSA_ERR_BAD_INDEX);

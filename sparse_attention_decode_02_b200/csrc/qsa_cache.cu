@@ -196,18 +196,32 @@ __global__ void __launch_bounds__(256) decode_append_kernel(DevState* st, uint4*
   pdl_launch_dependents();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   pdl_wait();
+  // the token's first K/V/key units, loaded in the same round trip as the state
+  const int t0 = threadIdx.x;
+  uint4 k0 = make_uint4(0u, 0u, 0u, 0u), v0 = k0, i0 = k0;
+  if (t0 < kv_units) {
+    k0 = k[t0];
+    v0 = v[t0];
+  }
+  if (t0 < IDX_UNITS) i0 = idx[t0];
   const PoolLane<D> c = pool_lane_consts<D>(lane, gain, rope_base);
   const int n = ld_volatile(&st->n_ctx);
   const int b_first = ld_volatile(&st->n_pooled);
+  asm volatile("" ::"r"(k0.x), "r"(k0.y), "r"(k0.z), "r"(k0.w), "r"(v0.x), "r"(v0.y), "r"(v0.z), "r"(v0.w));
+  asm volatile("" ::"r"(i0.x), "r"(i0.y), "r"(i0.z), "r"(i0.w));
   if (n < 0 || n >= max_ctx) {
     if (threadIdx.x == 0) record_status(st, QSA_ERR_CAPACITY);
     return;
   }
-  for (int i = threadIdx.x; i < kv_units; i += blockDim.x) {
+  if (t0 < kv_units) {
+    kc[size_t(n) * kv_units + t0] = k0;
+    vc[size_t(n) * kv_units + t0] = v0;
+  }
+  for (int i = t0 + blockDim.x; i < kv_units; i += blockDim.x) {  // heads beyond one pass
     kc[size_t(n) * kv_units + i] = k[i];
     vc[size_t(n) * kv_units + i] = v[i];
   }
-  if (threadIdx.x < IDX_UNITS) ic[size_t(n) * IDX_UNITS + threadIdx.x] = idx[threadIdx.x];
+  if (t0 < IDX_UNITS) ic[size_t(n) * IDX_UNITS + t0] = i0;
   __syncthreads();  // the new indexer key is visible to every warp of the CTA
   const int b_end = (n + 1) / kBlock;
   const __half* ich = reinterpret_cast<const __half*>(ic);

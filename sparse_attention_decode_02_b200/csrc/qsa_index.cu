@@ -72,7 +72,7 @@ __device__ __forceinline__ uint32_t cta_exclusive_scan(uint32_t v, uint32_t* s_w
 template <int V>
 __global__ void __launch_bounds__(kThreads, 1)
 block_topk_kernel(DevState* st, const float* __restrict__ scores, int32_t* __restrict__ sel,
-                  int32_t* __restrict__ n_sel, int k_blocks) {
+                  int32_t* __restrict__ n_sel, int k_blocks, int max_blocks) {
   __shared__ uint32_t s_hist[2][256];
   __shared__ uint32_t s_warp[32];
   __shared__ uint32_t s_ctl[4];   // digit, count above the digit, count at the digit
@@ -85,9 +85,29 @@ block_topk_kernel(DevState* st, const float* __restrict__ scores, int32_t* __res
 
   pdl_launch_dependents();
   pdl_wait();
+  // this thread's V scores, read up to the buffer's capacity (max_ctx/4) in the same round
+  // trip as the state; blocks at or past n_ctx/4 are masked once the state is known
+  const int base = rank * kThreads * V + tid * V;
+  float f[V];
+  if (base + V <= max_blocks) {
+#pragma unroll
+    for (int j = 0; j < V; j += 4) {
+      const float4 x = *reinterpret_cast<const float4*>(scores + base + j);
+      f[j] = x.x;
+      f[j + 1] = x.y;
+      f[j + 2] = x.z;
+      f[j + 3] = x.w;
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < V; ++j) f[j] = base + j < max_blocks ? scores[base + j] : 0.0f;
+  }
   const int n = ld_volatile(&st->n_ctx);
+  const int n_pooled = ld_volatile(&st->n_pooled);
+#pragma unroll
+  for (int j = 0; j < V; ++j) asm volatile("" ::"f"(f[j]));  // keep the loads ahead of the branches
   const int n_blocks = n / kBlock;
-  if (ld_volatile(&st->n_pooled) != n_blocks) {
+  if (n_pooled != n_blocks) {
     if (rank == 0 && tid == 0) {
       record_status(st, QSA_ERR_STATE);
       *n_sel = 0;
@@ -100,28 +120,12 @@ block_topk_kernel(DevState* st, const float* __restrict__ scores, int32_t* __res
     return;
   }
 
-  const int base = rank * kThreads * V + tid * V;
   uint32_t key[V];
   uint32_t valid = 0;  // bit j: block base + j exists
-  if (base + V <= n_blocks) {
 #pragma unroll
-    for (int j = 0; j < V; j += 4) {
-      const float4 f = *reinterpret_cast<const float4*>(scores + base + j);
-      key[j] = score_key(f.x);
-      key[j + 1] = score_key(f.y);
-      key[j + 2] = score_key(f.z);
-      key[j + 3] = score_key(f.w);
-    }
-    valid = V == 32 ? 0xffffffffu : ((1u << V) - 1u);
-  } else {
-#pragma unroll
-    for (int j = 0; j < V; ++j) {
-      key[j] = 0u;
-      if (base + j < n_blocks) {
-        key[j] = score_key(scores[base + j]);
-        valid |= 1u << j;
-      }
-    }
+  for (int j = 0; j < V; ++j) {
+    key[j] = score_key(f[j]);
+    if (base + j < n_blocks) valid |= 1u << j;
   }
   if (tid < 256) s_hist[0][tid] = 0;
 
@@ -245,10 +249,10 @@ cudaError_t launch_topk(const LayerView& L, const float* scores, int32_t* sel, i
   const int kb = L.cfg.top_k_tokens / kBlock;
   const dim3 grid(kCS), block(kThreads);
   if (max_blocks <= kCS * kThreads * 8)
-    return launch_pdl(block_topk_kernel<8>, grid, block, 0, s, kCS, L.state, scores, sel, n_sel, kb);
+    return launch_pdl(block_topk_kernel<8>, grid, block, 0, s, kCS, L.state, scores, sel, n_sel, kb, max_blocks);
   if (max_blocks <= kCS * kThreads * 16)
-    return launch_pdl(block_topk_kernel<16>, grid, block, 0, s, kCS, L.state, scores, sel, n_sel, kb);
-  return launch_pdl(block_topk_kernel<32>, grid, block, 0, s, kCS, L.state, scores, sel, n_sel, kb);
+    return launch_pdl(block_topk_kernel<16>, grid, block, 0, s, kCS, L.state, scores, sel, n_sel, kb, max_blocks);
+  return launch_pdl(block_topk_kernel<32>, grid, block, 0, s, kCS, L.state, scores, sel, n_sel, kb, max_blocks);
 }
 
 }  // namespace qsa

@@ -51,6 +51,7 @@ def test_buffer_sizes(lib):
 @pytest.mark.parametrize("bad", [
     dict(d_idx=96), dict(n_idx_heads=3), dict(n_idx_heads=32), dict(top_k_tokens=2046),
     dict(head_dim=256), dict(n_q_heads=32, n_kv_heads=2), dict(max_ctx=1026), dict(max_ctx=4 << 20),
+    dict(top_k_tokens=4096), dict(top_k_tokens=0),
     dict(n_layers=0),
 ])
 def test_unsupported_configs_are_rejected(lib, bad):
