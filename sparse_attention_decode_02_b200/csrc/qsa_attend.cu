@@ -311,8 +311,9 @@ cudaError_t launch_attend_split(const LayerView& L, const void* q, const int32_t
 // One cluster of CS CTAs per KV head g covers the whole cell set: CTA r stages the K
 // and V rows of cells [r*Lc, (r+1)*Lc) in shared memory (16-byte cp.async, straight
 // from the cache: the gather is fused), computes the f32 logits, softmax statistics and
-// unnormalised P.V of the G query heads that share g, then the CTAs merge their
-// (max, sum, output) partials through DSMEM and write the final output. In the
+// unnormalised P.V of the G query heads that share g, then pushes its (max, sum, output)
+// partials through DSMEM to the CTAs that own each output slice, which merge them after
+// a single cluster barrier and write the final output. In the
 // FROM_BLOCKS form the cell ids are expanded on the fly from the selected blocks and
 // the open tail (cell expansion fused in as well).
 // ---------------------------------------------------------------------------------
@@ -371,7 +372,11 @@ struct AcSmem {
   __host__ __device__ static size_t ml_off(int lc) { return red_off(lc) + 2 * 16 * 8 * 4; }        // 2G f32
   __host__ __device__ static size_t cell_off(int lc) { return ml_off(lc) + 16 * 4; }
   __host__ __device__ static size_t stage_off(int lc) { return (cell_off(lc) + size_t(lp(lc)) * 4 + 15) / 16 * 16; }
-  __host__ __device__ static size_t bytes(int lc, int cs) { return stage_off(lc) + size_t(cs) * G * 2 * 4; }
+  // output pairs (2 dims of one head) each CTA of a cluster of cs merges
+  __host__ __device__ static int per(int cs) { return (G * (D / 2) + cs - 1) / cs; }
+  // inbox of this CTA's output slice: [cs source CTAs][per] float2
+  __host__ __device__ static size_t in_off(int lc, int cs) { return (stage_off(lc) + size_t(cs) * G * 2 * 4 + 15) / 16 * 16; }
+  __host__ __device__ static size_t bytes(int lc, int cs) { return in_off(lc, cs) + size_t(cs) * per(cs) * 8; }
 };
 
 template <int D, int G, int CS, bool FROM_BLOCKS>
@@ -552,17 +557,27 @@ attn_cluster_kernel(DevState* st, const __half* __restrict__ q, const int32_t* _
     }
     if (gq < G) *reinterpret_cast<float2*>(s_o + gq * D + warp * 8 + 2 * tq) = make_float2(acc[0], acc[1]);
   }
-  cluster.sync();
-  // merge the CS partials: (max, sum) of every CTA first, then this CTA's output slice
-  for (int t = tid; t < CS * G; t += kAcThreads) {
-    const int r = t / G, h = t % G;
-    const float* rm = cluster.map_shared_rank(s_m, r);
-    s_stage[(r * G + h) * 2] = rm[h];
-    s_stage[(r * G + h) * 2 + 1] = rm[G + h];
-  }
-  __syncthreads();
+  // ---- merge: CTA r owns output pairs [r*PER, (r+1)*PER) (2 dims of one head each).
+  //      Every CTA pushes its (max, sum) per head and its partial of each slice into the
+  //      owner's shared memory with DSMEM stores; after one cluster barrier each owner
+  //      merges its slice from local memory. Nothing reads another CTA's shared memory
+  //      after the barrier, so no second barrier is needed before exiting. ----
   constexpr int PAIRS = G * (D / 2);
   constexpr int PER = (PAIRS + CS - 1) / CS;
+  float2* s_in = reinterpret_cast<float2*>(smem + SM::in_off(Lc, CS));  // [CS][PER]
+  __syncthreads();  // s_o, s_m and s_l are complete
+  for (int pidx = tid; pidx < PAIRS; pidx += kAcThreads) {
+    const int h = pidx / (D / 2), d2 = pidx % (D / 2);
+    const float2 v = *reinterpret_cast<const float2*>(s_o + h * D + 2 * d2);
+    *(cluster.map_shared_rank(s_in, pidx / PER) + rank * PER + pidx % PER) = v;
+  }
+  for (int t = tid; t < CS * G; t += kAcThreads) {
+    const int owner = t / G, h = t % G;
+    float* dst = cluster.map_shared_rank(s_stage, owner) + (rank * G + h) * 2;
+    dst[0] = s_m[h];
+    dst[1] = s_l[h];
+  }
+  cluster.sync();  // release the pushes above, acquire every other CTA's
   for (int t = tid; t < PER; t += kAcThreads) {
     const int pidx = rank * PER + t;
     if (pidx >= PAIRS) break;
@@ -570,17 +585,15 @@ attn_cluster_kernel(DevState* st, const __half* __restrict__ q, const int32_t* _
     float M = -INFINITY;
 #pragma unroll
     for (int r = 0; r < CS; ++r) M = fmaxf(M, s_stage[(r * G + h) * 2]);
-    float2 o[CS];
-#pragma unroll
-    for (int r = 0; r < CS; ++r) o[r] = *reinterpret_cast<const float2*>(cluster.map_shared_rank(s_o, r) + h * D + 2 * d2);
     float a0 = 0.0f, a1 = 0.0f, den = 0.0f;
     if (M != -INFINITY) {
 #pragma unroll
       for (int r = 0; r < CS; ++r) {
         const float mr = s_stage[(r * G + h) * 2];
         const float e = mr == -INFINITY ? 0.0f : expf(mr - M);
-        a0 = fmaf(e, o[r].x, a0);
-        a1 = fmaf(e, o[r].y, a1);
+        const float2 o = s_in[r * PER + t];
+        a0 = fmaf(e, o.x, a0);
+        a1 = fmaf(e, o.y, a1);
         den = fmaf(e, s_stage[(r * G + h) * 2 + 1], den);
       }
     }
@@ -588,7 +601,6 @@ attn_cluster_kernel(DevState* st, const __half* __restrict__ q, const int32_t* _
     if (den > 0.0f) res = make_float2(a0 / den, a1 / den);
     *reinterpret_cast<float2*>(out + (size_t(g) * G + h) * D + 2 * d2) = res;
   }
-  cluster.sync();  // keep this CTA's shared memory alive until every remote read is done
 }
 
 template <int D, int G, int CS, bool FB>
