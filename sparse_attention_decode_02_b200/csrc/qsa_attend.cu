@@ -410,6 +410,7 @@ attn_cluster_kernel(DevState* st, const __half* __restrict__ q, const int32_t* _
   const int gq = lane >> 2, tq = lane & 3;  // MMA fragment row (query head) and column pair
 
   pdl_launch_dependents();
+  cluster_arrive_relaxed();  // paired with cluster_wait() before the partials are pushed
   pdl_wait();
   const int n = ld_volatile(&st->n_ctx);
   const int c0 = rank * Lc;
@@ -566,6 +567,7 @@ attn_cluster_kernel(DevState* st, const __half* __restrict__ q, const int32_t* _
   constexpr int PER = (PAIRS + CS - 1) / CS;
   float2* s_in = reinterpret_cast<float2*>(smem + SM::in_off(Lc, CS));  // [CS][PER]
   __syncthreads();  // s_o, s_m and s_l are complete
+  cluster_wait();   // every CTA of the cluster has started: its shared memory may be written
   for (int pidx = tid; pidx < PAIRS; pidx += kAcThreads) {
     const int h = pidx / (D / 2), d2 = pidx % (D / 2);
     const float2 v = *reinterpret_cast<const float2*>(s_o + h * D + 2 * d2);

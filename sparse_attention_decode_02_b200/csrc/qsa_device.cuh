@@ -23,6 +23,14 @@ __device__ __forceinline__ void pdl_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// Split cluster barrier: every thread arrives early (no memory ordering) and waits
+// right before its CTA first writes another CTA's shared memory, which is then known
+// to have started. Each thread alternates arrive and wait, like any cluster barrier.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
+
 __device__ __forceinline__ void record_status(DevState* st, int code) {
   atomicCAS(&st->status, 0, code);
 }

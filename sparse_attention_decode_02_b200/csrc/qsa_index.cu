@@ -63,27 +63,29 @@ __device__ __forceinline__ uint32_t cta_exclusive_scan(uint32_t v, uint32_t* s_w
 // from the top, stopping as soon as every key with the current prefix is needed.
 // CTA r owns blocks [r*kThreads*V, (r+1)*kThreads*V), thread t the V consecutive blocks
 // starting at t*V, held in registers (vector loads). Per pass, each CTA histograms its
-// keys in shared memory and every CTA adds the kCS histograms through distributed
-// shared memory (all remote loads in flight together). The output position of a
-// selected block is the number of keys above the threshold before it plus
-// min(need, ties before it), so one packed prefix scan and one exchange of per-CTA
-// totals give every position; ties are taken in block order.
+// keys in shared memory and pushes it into every CTA's inbox with distributed-shared-
+// memory stores; after one cluster barrier each CTA adds the kCS histograms from its
+// own memory. The output position of a selected block is the number of keys above the
+// threshold before it plus min(need, ties before it), so one packed prefix scan and one
+// pushed exchange of per-CTA totals give every position; ties are taken in block order.
+// Nothing reads another CTA's shared memory, so no barrier is needed before exiting.
 // ---------------------------------------------------------------------------------
 template <int V>
 __global__ void __launch_bounds__(kThreads, 1)
 block_topk_kernel(DevState* st, const float* __restrict__ scores, int32_t* __restrict__ sel,
                   int32_t* __restrict__ n_sel, int k_blocks, int max_blocks) {
-  __shared__ uint32_t s_hist[2][256];
+  __shared__ uint32_t s_hist[256];          // this CTA's histogram of the pass
+  __shared__ uint32_t s_in[2][kCS][256];    // every CTA's histogram, double-buffered by pass
   __shared__ uint32_t s_warp[32];
   __shared__ uint32_t s_ctl[4];   // digit, count above the digit, count at the digit
-  __shared__ uint32_t s_cta[2];   // this CTA's (greater, equal) totals, read by the cluster
-  __shared__ uint32_t s_all[2 * kCS];
+  __shared__ uint32_t s_all[2 * kCS];       // every CTA's (greater, equal) totals
 
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = int(cluster.block_rank());
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
   pdl_launch_dependents();
+  cluster_arrive_relaxed();  // paired with cluster_wait() before the first push
   pdl_wait();
   // this thread's V scores, read up to the buffer's capacity (max_ctx/4) in the same round
   // trip as the state; blocks at or past n_ctx/4 are masked once the state is known
@@ -112,11 +114,13 @@ block_topk_kernel(DevState* st, const float* __restrict__ scores, int32_t* __res
       record_status(st, QSA_ERR_STATE);
       *n_sel = 0;
     }
-    return;  // uniform over the cluster; no shared memory of another CTA is touched
+    cluster_wait();  // uniform over the cluster; no shared memory of another CTA is touched
+    return;
   }
-  if (n_blocks <= k_blocks) {  // every block is selected
+  if (n_blocks <= k_blocks) {  // every block is selected (uniform over the cluster)
     for (int i = rank * kThreads + tid; i < n_blocks; i += kCS * kThreads) sel[i] = i;
     if (rank == 0 && tid == 0) *n_sel = n_blocks;
+    cluster_wait();
     return;
   }
 
@@ -127,29 +131,33 @@ block_topk_kernel(DevState* st, const float* __restrict__ scores, int32_t* __res
     key[j] = score_key(f[j]);
     if (base + j < n_blocks) valid |= 1u << j;
   }
-  if (tid < 256) s_hist[0][tid] = 0;
+  if (tid < 256) s_hist[tid] = 0;
+  cluster_wait();  // every CTA of the cluster has started: its shared memory may be written
 
   uint32_t prefix = 0, mask = 0, need = uint32_t(k_blocks);
   for (int pass = 0; pass < 4; ++pass) {
     const int shift = 24 - 8 * pass;
-    uint32_t* hist = s_hist[pass & 1];
-    __syncthreads();  // this pass's buffer is zeroed
+    __syncthreads();  // the local histogram is zeroed
 #pragma unroll
     for (int j = 0; j < V; ++j)
-      if (((valid >> j) & 1u) && (key[j] & mask) == prefix) atomicAdd(&hist[(key[j] >> shift) & 255u], 1u);
-    // after this barrier every CTA has finished the previous pass, including its remote
-    // reads of the other buffer, which can therefore be cleared for the next pass
-    cluster.sync();
-    if (tid < 256) s_hist[(pass + 1) & 1][tid] = 0;
+      if (((valid >> j) & 1u) && (key[j] & mask) == prefix) atomicAdd(&s_hist[(key[j] >> shift) & 255u], 1u);
+    __syncthreads();
+    // push bin t into slot [rank][t] of every CTA's inbox for this pass, and clear it for
+    // the next pass. A CTA reuses an inbox buffer two passes later, after a barrier that
+    // every CTA passes only once all have finished reading it.
+    if (tid < 256) {
+      const uint32_t mine = s_hist[tid];
+      s_hist[tid] = 0;
+#pragma unroll
+      for (int r = 0; r < kCS; ++r) cluster.map_shared_rank(&s_in[pass & 1][0][0], r)[rank * 256 + tid] = mine;
+    }
+    cluster.sync();  // release the pushes, acquire every other CTA's
     // thread t < 256 takes digit (255 - t): an inclusive prefix over t counts keys >= digit
     uint32_t v = 0;
     if (tid < 256) {
       const int bin = 255 - tid;
-      uint32_t part[kCS];
 #pragma unroll
-      for (int r = 0; r < kCS; ++r) part[r] = cluster.map_shared_rank(hist, r)[bin];
-#pragma unroll
-      for (int r = 0; r < kCS; ++r) v += part[r];
+      for (int r = 0; r < kCS; ++r) v += s_in[pass & 1][r][bin];
     }
     uint32_t x = v;
 #pragma unroll
@@ -187,13 +195,12 @@ block_topk_kernel(DevState* st, const float* __restrict__ scores, int32_t* __res
   }
   uint32_t tot;
   const uint32_t before = cta_exclusive_scan((c_gt << 16) | c_eq, s_warp, &tot);
-  if (tid == 0) {
-    s_cta[0] = tot >> 16;
-    s_cta[1] = tot & 0xffffu;
+  if (tid < kCS) {  // push this CTA's totals to every CTA
+    uint32_t* dst = cluster.map_shared_rank(s_all, tid);
+    dst[2 * rank] = tot >> 16;
+    dst[2 * rank + 1] = tot & 0xffffu;
   }
   cluster.sync();
-  if (tid < 2 * kCS) s_all[tid] = cluster.map_shared_rank(s_cta, tid >> 1)[tid & 1];
-  __syncthreads();
   uint32_t gt_before = before >> 16, eq_before = before & 0xffffu;
 #pragma unroll
   for (int r = 0; r < kCS; ++r) {
@@ -213,7 +220,6 @@ block_topk_kernel(DevState* st, const float* __restrict__ scores, int32_t* __res
     }
   }
   if (rank == 0 && tid == 0) *n_sel = k_blocks;
-  cluster.sync();  // keep this CTA's shared memory alive until every remote read is done
 }
 
 namespace {
