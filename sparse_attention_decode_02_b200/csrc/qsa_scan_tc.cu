@@ -69,7 +69,7 @@ template <int D, int H>
 __global__ void __launch_bounds__(kThreads, 1)
 index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_constant__ CUtensorMap map_box,
                      DevState* st, const __half* __restrict__ q_idx, const float* __restrict__ w,
-                     float* __restrict__ scores, float rope_base) {
+                     float* __restrict__ scores, float rope_base, int max_blocks) {
   using S = ScanShape<D, H>;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -105,6 +105,16 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_
   if (warp == 4 && lane == 0) {
     tma_prefetch_desc(&map_tile);
     tma_prefetch_desc(&map_box);
+    // Start HBM -> L2 streaming of this CTA's rows while the previous kernels still run:
+    // the context length read here, before the dependency wait, may be one token stale,
+    // which only shifts the prefetched range slightly. Prefetches change nothing that
+    // later loads observe; the real loads below use the current length.
+    const int nb_hint = min(max(ld_volatile(&st->n_ctx), 0) / kBlock, max_blocks);
+    const int p0 = int((long long)blockIdx.x * nb_hint / gridDim.x);
+    const int p1 = int((long long)(blockIdx.x + 1) * nb_hint / gridDim.x);
+    for (int r = p0; r < p1; r += 128)
+#pragma unroll
+      for (int j = 0; j < S::HALVES; ++j) tma_prefetch_l2_2d(&map_tile, j * 64, r);
   }
   // RoPE frequencies do not depend on the previous kernel: compute them before waiting on it
   for (int i = threadIdx.x; i < D / 2; i += blockDim.x) s_theta[i] = pow((double)rope_base, -2.0 * (double)i / (double)D);
@@ -326,7 +336,7 @@ static cudaError_t launch_scan_tc_d(const LayerView& L, const void* q_idx, const
 #define QSA_SCAN_CASE(HH)                                                                                  \
   case HH:                                                                                                 \
     return launch_pdl(index_scan_tc_kernel<D, HH>, grid, block, ScanShape<D, HH>::SMEM, s, 1, L.pooled_tile_map, \
-                      L.pooled_box_map, L.state, (const __half*)q_idx, w, scores, base);
+                      L.pooled_box_map, L.state, (const __half*)q_idx, w, scores, base, L.cfg.max_ctx / kBlock);
   switch (L.cfg.n_idx_heads) {
     QSA_SCAN_CASE(1)
     QSA_SCAN_CASE(2)
