@@ -114,3 +114,39 @@ def test_select_extremes_of_float_range():
     got = _select(s, 4092)
     np.testing.assert_array_equal(got, O.topk_blocks(want, 1023))
 
+
+
+# pairs of score sets of 63,795 blocks selected one after the other on the same layer:
+# nothing of the first selection may leak into the second (same scale, another scale,
+# another sign)
+PAIRS = [("normal_63795", "normal_63795x1.01"), ("uniform_positive_63795", "uniform_positive_63795x1000"),
+         ("uniform_positive_63795", "normal_63795"), ("clustered_desc_63795", "sparse_spikes_63795"),
+         ("quantised_63795", "quantised_63795x0.5"), ("normal_63795", "negative_63795")]
+
+
+def _scores_of(name):
+    base, _, scale = name.partition("x")
+    if base == "negative_63795":
+        return (-_rng(3).random(63795) - 1.0).astype(np.float32)
+    s = CASES[base](_rng(zlib.crc32(base.encode())))
+    return (s * float(scale or 1.0)).astype(np.float32)
+
+
+@pytest.mark.parametrize("first,second", PAIRS)
+def test_select_after_a_previous_selection(first, second):
+    import sparse_attention_decode_02_b200 as Q
+    wl = synth.workload("ctx64k")
+    n = 4 * 63795 + 2
+    qsa = Q.Qsa(H.config_of(wl, max_ctx=n + 2))
+    g = H.GpuLayer(qsa)
+    qsa.restore_layer(0, n, n // 4)
+    sc = torch.zeros(qsa.cfg.max_ctx // 4, dtype=torch.float32, device="cuda")
+    o = g.outs
+    for name in (first, second):
+        s = _scores_of(name)
+        sc[: len(s)] = torch.from_numpy(s).cuda()
+        qsa.select_topk(0, sc, o["sel"], o["n_sel"])
+        torch.cuda.synchronize()
+        got = o["sel"][: int(o["n_sel"][0])].cpu().numpy().astype(np.int64)
+        np.testing.assert_array_equal(got, _expected(s, wl.k_blocks), err_msg=name)
+    assert g.state()[2] == 0
