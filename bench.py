@@ -283,6 +283,26 @@ def run_ours(wl, n_layers, K, W, rank, world, e2e_steps, sample_clocks, local):
     for layer in range(n_layers):
         assert wb.qsa.read_layer_state(layer)[2] == 0
 
+    # bulk pooled build (the prefill / rebuild path): invalidate layer 0's pooled cache and
+    # pool every block again (bit-identical to the live cache); bytes = 4 raw keys in and one
+    # pooled row out per block
+    reps = 5
+    b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    wb.qsa.invalidate_pooled_cache(0, 0)
+    wb.qsa.update_pooled_cache(0)
+    torch.cuda.synchronize()
+    b0.record(stream)
+    for _ in range(reps):
+        wb.qsa.invalidate_pooled_cache(0, 0)
+        wb.qsa.update_pooled_cache(0)
+    b1.record(stream)
+    torch.cuda.synchronize()
+    n_now, p_now, st_now = wb.qsa.read_layer_state(0)
+    assert p_now == n_now // 4 and st_now == 0, (n_now, p_now, st_now)
+    us = 1e3 * b0.elapsed_time(b1) / reps
+    nbytes = (n_now // 4) * (4 * wl.d_idx * 2 + wl.d_idx * 2)
+    bulk = {"blocks": n_now // 4, "us": round(us, 2), "bytes": int(nbytes), "gbs": round(nbytes / (us * 1e-6) / 1e9, 1)}
+
     # per-stage breakdown from an instrumented graph (events break the launch overlap,
     # so these are serialised per-kernel durations, used for the roofline)
     ig, start, evs = wb.capture_instrumented()
@@ -382,6 +402,7 @@ def run_ours(wl, n_layers, K, W, rank, world, e2e_steps, sample_clocks, local):
                "h2d_bytes_per_step": int(host_in[0].numel()), "d2h_bytes_per_step": int(host_out[0].numel() * 4),
                "steps": e2e_steps}
     return {"ms": ms, "clocks": clk, "per_launch_us": per_launch_us, "iso_us": iso, "n_ctx_instr": n_ctx_instr,
+            "bulk_pool": bulk,
             "n_layers": n_layers, "launches_per_step": n_layers * wb.launches_per_layer, "e2e": e2e,
             "graph_steps": G}
 
@@ -535,6 +556,7 @@ def main_ours(args):
             "e2e": main["e2e"],
             "gpu_launches": main["launches_per_step"] * K,
             "by_ctx": by_ctx,
+            "bulk_pool": dict(main["bulk_pool"], frac=round(main["bulk_pool"]["gbs"] / peak, 4)) if main["bulk_pool"] else None,
             "hbm_gbs_step": round(world * wl.n_layers * K * sum(sb.values()) / (main["ms"] / 1e3) / 1e9, 1),
         }
         print(json.dumps(line))
