@@ -258,10 +258,10 @@ qsa_status qsa_update_pooled_cache(qsa_ctx* ctx, int32_t layer, qsa_stream_t str
   if (!ctx) return QSA_ERR_INVALID_ARG;
   if (qsa_status st = ctx->layer_ok(layer)) return st;
   Layer& l = ctx->layers[layer];
-  // 8 warps per CTA, one block per warp per iteration
-  long long grid = (l.pending_blocks + 7) / 8;
+  // 8 warps per CTA, 4 blocks per warp per round; at most ~4 resident CTAs per SM
+  long long grid = (l.pending_blocks + 31) / 32;
   if (grid < 1) grid = 1;
-  if (grid > ctx->n_sms * 8) grid = ctx->n_sms * 8;
+  if (grid > ctx->n_sms * 4) grid = ctx->n_sms * 4;
   l.pending_blocks = 0;
   return ctx->cuda(launch_pool_update(ctx->view(layer), (int)grid, (cudaStream_t)stream), "update_pooled_cache");
 }

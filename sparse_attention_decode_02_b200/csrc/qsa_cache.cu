@@ -111,24 +111,62 @@ __device__ __forceinline__ PoolLane<D> pool_lane_consts(int lane, const float* _
   return c;
 }
 
+// cos and sin of the RoPE angle pos * theta. The angle is formed and reduced modulo 2*pi
+// in double (|angle| <= ~2.6e5 rad: the reduced angle is exact to ~1e-11 rad), then
+// evaluated in float: the positions reach 2^18, where a float angle would already be off by
+// ~0.016 rad, while the reduced argument keeps the result within a few float ulps.
+__device__ __forceinline__ void rope_cos_sin(double pos, double theta, float* cs, float* sn) {
+  constexpr double kTwoPi = 6.283185307179586;
+  const double angle = pos * theta;
+  const double r = fma(-rint(angle * (1.0 / kTwoPi)), kTwoPi, angle);
+  sincosf(float(r), sn, cs);
+}
+
+// The 4 raw indexer keys of one block as one lane of a warp holds them (f16, packed):
+// rotation pairs i = lane*P + j (j < P) and their partners i + D/2.
 template <int D>
+struct PoolRaw {
+  __half2 x1[kBlock], x2[kBlock];  // P == 1 uses the low half only
+};
+
 // `ic` is deliberately not __restrict__: the fused decode kernel reads back a row it has
 // just written, which must not go through the non-coherent load path.
-__device__ __forceinline__ void pool_one_block(int b, int lane, const PoolLane<D>& c, const __half* ic,
-                                               __half* __restrict__ pc, float eps) {
+template <int D>
+__device__ __forceinline__ void pool_load(int b, int lane, const __half* ic, PoolRaw<D>& raw) {
+  constexpr int P = PoolLane<D>::P;
+  constexpr int HALF = D / 2;
+  static_assert(P == 1 || P == 2, "one or two rotation pairs per lane");
+#pragma unroll
+  for (int t = 0; t < kBlock; ++t) {
+    const __half* row = ic + (size_t(b) * kBlock + t) * D;
+    if constexpr (P == 2) {
+      raw.x1[t] = *reinterpret_cast<const __half2*>(row + lane * 2);
+      raw.x2[t] = *reinterpret_cast<const __half2*>(row + lane * 2 + HALF);
+    } else {
+      raw.x1[t] = __halves2half2(row[lane], __float2half_rn(0.0f));
+      raw.x2[t] = __halves2half2(row[lane + HALF], __float2half_rn(0.0f));
+    }
+  }
+}
+
+// Summary of block b from its raw keys: mean (summed in token order), RMSNorm, RoPE at
+// the block position 4b, f16 store.
+template <int D>
+__device__ __forceinline__ void pool_finish(int b, int lane, const PoolLane<D>& c, const PoolRaw<D>& raw,
+                                            __half* __restrict__ pc, float eps) {
   constexpr int P = PoolLane<D>::P;
   constexpr int HALF = D / 2;
   float m1[P], m2[P];
 #pragma unroll
   for (int j = 0; j < P; ++j) m1[j] = m2[j] = 0.0f;
-  // mean of the 4 raw indexer keys, summed in token order
 #pragma unroll
   for (int t = 0; t < kBlock; ++t) {
-    const __half* row = ic + (size_t(b) * kBlock + t) * D;
-#pragma unroll
-    for (int j = 0; j < P; ++j) {
-      m1[j] += __half2float(row[lane * P + j]);
-      m2[j] += __half2float(row[lane * P + j + HALF]);
+    const float2 a = __half22float2(raw.x1[t]), z = __half22float2(raw.x2[t]);
+    m1[0] += a.x;
+    m2[0] += z.x;
+    if constexpr (P == 2) {
+      m1[P - 1] += a.y;
+      m2[P - 1] += z.y;
     }
   }
   float ss = 0.0f;
@@ -141,17 +179,31 @@ __device__ __forceinline__ void pool_one_block(int b, int lane, const PoolLane<D
   ss = warp_sum(ss);
   const float inv_rms = 1.0f / sqrtf(ss / (float)D + eps);
   const double pos = (double)(b * kBlock);
+  __half o1[P], o2[P];
 #pragma unroll
   for (int j = 0; j < P; ++j) {
     const float r1 = m1[j] * inv_rms * c.g1[j];
     const float r2 = m2[j] * inv_rms * c.g2[j];
-    double sd, cd;
-    sincos(pos * c.theta[j], &sd, &cd);
-    const float cs = (float)cd, sn = (float)sd;
-    const int i = lane * P + j;
-    pc[size_t(b) * D + i] = __float2half_rn(r1 * cs - r2 * sn);
-    pc[size_t(b) * D + i + HALF] = __float2half_rn(r1 * sn + r2 * cs);
+    float cs, sn;
+    rope_cos_sin(pos, c.theta[j], &cs, &sn);
+    o1[j] = __float2half_rn(r1 * cs - r2 * sn);
+    o2[j] = __float2half_rn(r1 * sn + r2 * cs);
   }
+  if constexpr (P == 2) {
+    *reinterpret_cast<__half2*>(pc + size_t(b) * D + lane * 2) = __halves2half2(o1[0], o1[1]);
+    *reinterpret_cast<__half2*>(pc + size_t(b) * D + lane * 2 + HALF) = __halves2half2(o2[0], o2[1]);
+  } else {
+    pc[size_t(b) * D + lane] = o1[0];
+    pc[size_t(b) * D + lane + HALF] = o2[0];
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void pool_one_block(int b, int lane, const PoolLane<D>& c, const __half* ic,
+                                               __half* __restrict__ pc, float eps) {
+  PoolRaw<D> raw;
+  pool_load<D>(b, lane, ic, raw);
+  pool_finish<D>(b, lane, c, raw, pc, eps);
 }
 
 // Pools blocks [n_pooled, n_ctx/4), one warp per block, grid-stride.
@@ -169,7 +221,19 @@ __global__ void __launch_bounds__(256) pool_update_kernel(DevState* st, const __
   const int warps = blockDim.x >> 5;
   const int gw = blockIdx.x * warps + (threadIdx.x >> 5);
   const PoolLane<D> c = pool_lane_consts<D>(lane, gain, rope_base);
-  for (int b = b_first + gw; b < b_end; b += gridDim.x * warps) pool_one_block<D>(b, lane, c, ic, pc, eps);
+  // warp gw takes blocks b_first + gw + u*W (W = all warps), kBatch of them per round with
+  // every raw-key load of the round in flight before the first block is finished
+  constexpr int kBatch = 4;
+  const int W = gridDim.x * warps;
+  for (int b0 = b_first + gw; b0 < b_end; b0 += kBatch * W) {
+    PoolRaw<D> raw[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u)
+      if (b0 + u * W < b_end) pool_load<D>(b0 + u * W, lane, ic, raw[u]);
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u)
+      if (b0 + u * W < b_end) pool_finish<D>(b0 + u * W, lane, c, raw[u], pc, eps);
+  }
   __syncthreads();
   if (threadIdx.x == 0) {
     __threadfence();
