@@ -34,9 +34,13 @@ Readings taken where the pages are silent (each one is listed in the design note
      one pooled key per block is shared by all indexer heads.
   R2 RoPE is the NeoX half-split rotation over all d dims: pair (i, i + d/2),
      theta_i = base^(-2i/d), base 10000; z_i = x_i + j*x_{i+d/2} is multiplied by
-     exp(j * pos * theta_i).
+     exp(j * pos * theta_i). Switches for the other readings: rope_dims = R < d rotates
+     only the first R dims (pairs (i, i + R/2), theta_i = base^(-2i/R)) and passes the
+     rest through; rope_interleaved pairs (2i, 2i + 1) instead (GPT-J style).
   R3 the position of block b is its first token, pos(b) = 4b; the query sits at
-     position n-1 (n = context length including the current token).
+     position n-1 (n = context length including the current token). Switches:
+     pos(b) = stride*b + offset, query position floor(stride*(n-1)/4); stride 1 puts
+     both in the block domain (pos(b) = b, query at the index of its own block).
   R4 RMS norm r = m / sqrt(mean(m^2) + eps) * g with eps 1e-6, unit gain unless a
      gain vector is given.
   R5 pooled summaries are stored as f16 (round to nearest even), like the cache.
@@ -68,16 +72,24 @@ class QsaShape:
     head_dim: int
     rope_base: float = 10000.0
     rms_eps: float = 1e-6
+    rope_dims: int = 0             # rotary dims R; 0 = all d_idx (reading R2)
+    rope_interleaved: bool = False  # pairs (2i, 2i+1) instead of (i, i+R/2) (reading R2)
+    rope_pos_stride: int = 4       # pos(b) = stride*b + offset (reading R3)
+    rope_pos_offset: int = 0
 
     @property
     def k_blocks(self) -> int:
         # indexer_top_k tokens / compression ratio 4 (Part 10 §FA-scaling)
         return self.top_k_tokens // BLOCK
 
+    @property
+    def rotary_dims(self) -> int:
+        return self.rope_dims or self.d_idx
+
     @classmethod
-    def of(cls, wl) -> "QsaShape":
+    def of(cls, wl, **rope) -> "QsaShape":
         return cls(wl.d_idx, wl.n_idx_heads, wl.top_k_tokens, wl.n_q_heads, wl.n_kv_heads,
-                   wl.head_dim, wl.rope_base, wl.rms_eps)
+                   wl.head_dim, wl.rope_base, wl.rms_eps, **rope)
 
 
 def to_f16(x) -> np.ndarray:
@@ -90,23 +102,45 @@ def to_f16(x) -> np.ndarray:
 # ---------------------------------------------------------------------------
 
 def rope_frequencies(dim: int, base: float) -> np.ndarray:
-    """theta_i = base^(-2i/dim), i < dim/2 (reading R2)."""
+    """theta_i = base^(-2i/dim), i < dim/2, dim = the rotary dims (reading R2)."""
     i = np.arange(dim // 2, dtype=np.float64)
     return base ** (-2.0 * i / dim)
 
 
-def rope(x, pos, base: float) -> np.ndarray:
-    """NeoX half-split RoPE of the last axis of x at position(s) pos (reading R2).
+def rope_pairs(d: int, rope_dims: int = 0, interleaved: bool = False):
+    """The rotation pairs (a_i, b_i), i < R/2, of a d-wide vector (reading R2).
 
-    x has shape [..., d]; pos is a scalar or broadcasts against x[..., 0].
-    Pair (x_i, x_{i+d/2}) is rotated by the angle pos * theta_i.
+    NeoX half-split: (i, i + R/2); interleaved (GPT-J): (2i, 2i + 1). Dims >= R are
+    in no pair. R = rope_dims, or d when rope_dims is 0.
+    """
+    r = rope_dims or d
+    if r % 2 or not 0 < r <= d:
+        raise ValueError("rotary dims must be even and within the vector")
+    i = np.arange(r // 2)
+    return (2 * i, 2 * i + 1) if interleaved else (i, i + r // 2)
+
+
+def rope(x, pos, base: float, rope_dims: int = 0, interleaved: bool = False) -> np.ndarray:
+    """RoPE of the last axis of x at position(s) pos (reading R2).
+
+    x has shape [..., d]; pos is a scalar or broadcasts against x[..., 0]. Pair i,
+    (x_a, x_b) = (x[a_i], x[b_i]), is read as the complex number x_a + j*x_b and
+    multiplied by exp(j * pos * theta_i); dims in no pair are copied unchanged.
     """
     x = np.asarray(x, dtype=np.float64)
-    half = x.shape[-1] // 2
-    angle = np.multiply.outer(np.asarray(pos, dtype=np.float64), rope_frequencies(2 * half, base))
+    a, b = rope_pairs(x.shape[-1], rope_dims, interleaved)
+    angle = np.multiply.outer(np.asarray(pos, dtype=np.float64), rope_frequencies(2 * a.size, base))
     c, s = np.cos(angle), np.sin(angle)
-    x1, x2 = x[..., :half], x[..., half:]
-    return np.concatenate([x1 * c - x2 * s, x1 * s + x2 * c], axis=-1)
+    xa, xb = x[..., a], x[..., b]
+    out = x.copy()
+    out[..., a] = xa * c - xb * s
+    out[..., b] = xa * s + xb * c
+    return out
+
+
+def shape_rope(x, pos, shape: "QsaShape") -> np.ndarray:
+    """rope() with the layer's rotary switches."""
+    return rope(x, pos, shape.rope_base, shape.rope_dims, shape.rope_interleaved)
 
 
 def mean_pool(raw_block) -> np.ndarray:
@@ -122,9 +156,14 @@ def rms_normalize(m, eps: float, gain=None) -> np.ndarray:
     return r if gain is None else r * np.asarray(gain, dtype=np.float64)
 
 
-def block_position(b):
-    """Position of micro-block b = its first token (reading R3)."""
-    return BLOCK * np.asarray(b)
+def block_position(b, stride: int = BLOCK, offset: int = 0):
+    """Position of micro-block b: stride*b + offset; by default its first token 4b (reading R3)."""
+    return stride * np.asarray(b) + offset
+
+
+def query_position(n: int, stride: int = BLOCK) -> int:
+    """Position of the current token n-1 on the block-position scale: floor(stride*(n-1)/4) (R3)."""
+    return (stride * (n - 1)) // BLOCK
 
 
 def pooled_summaries(raw_idx, first_block: int, last_block: int, shape: QsaShape,
@@ -135,7 +174,7 @@ def pooled_summaries(raw_idx, first_block: int, last_block: int, shape: QsaShape
     raw = np.asarray(raw_idx[BLOCK * first_block:BLOCK * last_block]).reshape(-1, BLOCK, d)
     m = mean_pool(raw)
     r = rms_normalize(m, shape.rms_eps, gain)
-    p = rope(r, block_position(blocks), shape.rope_base)
+    p = shape_rope(r, block_position(blocks, shape.rope_pos_stride, shape.rope_pos_offset), shape)
     return to_f16(p)
 
 
@@ -175,7 +214,7 @@ class PooledKeyCache:
 
 def indexer_query(q_idx, n: int, shape: QsaShape) -> np.ndarray:
     """q~_h = RoPE(q_h, n-1): the current token's indexer query (readings R2, R3)."""
-    return rope(np.asarray(q_idx, dtype=np.float64), n - 1, shape.rope_base)
+    return shape_rope(np.asarray(q_idx, dtype=np.float64), query_position(n, shape.rope_pos_stride), shape)
 
 
 def block_scores(pooled, q_idx, w, n: int, shape: QsaShape) -> np.ndarray:

@@ -75,6 +75,82 @@ def test_rope_identity_norms_and_relative_position():
         assert abs(lhs - rhs) <= 1e-9 * (np.abs(a).sum() * np.abs(b).sum())
 
 
+def test_rope_interleaved_equals_complex_exponential_per_adjacent_pair():
+    """GPT-J pairs: z_i = x[2i] + j*x[2i+1] times exp(j*pos*base^(-2i/d)), written out pair by pair."""
+    rng = np.random.default_rng(31)
+    d, base, pos = 12, 500.0, 37
+    x = rng.standard_normal(d)
+    want = np.empty(d)
+    for i in range(d // 2):
+        z = complex(x[2 * i], x[2 * i + 1]) * np.exp(1j * pos * base ** (-2.0 * i / d))
+        want[2 * i], want[2 * i + 1] = z.real, z.imag
+    np.testing.assert_allclose(O.rope(x, pos, base, interleaved=True), want, rtol=0, atol=1e-13)
+
+
+def test_rope_partial_rotates_leading_dims_only():
+    """rope_dims R < d: the first R dims turn like a full R-wide RoPE, the rest are copied."""
+    rng = np.random.default_rng(32)
+    x = rng.standard_normal((3, 64))
+    pos = np.array([1, 999, 262143])
+    for inter in (False, True):
+        got = O.rope(x, pos, 1e4, rope_dims=16, interleaved=inter)
+        np.testing.assert_array_equal(got[:, 16:], x[:, 16:])
+        np.testing.assert_array_equal(got[:, :16], O.rope(x[:, :16], pos, 1e4, interleaved=inter))
+    # written out: pair (i, i+8) of the 16 rotary dims turns by pos * base^(-2i/16)
+    i = 5
+    z = complex(x[1, i], x[1, i + 8]) * np.exp(1j * 999 * 1e4 ** (-2.0 * i / 16))
+    got = O.rope(x[1], 999, 1e4, rope_dims=16)
+    assert abs(got[i] - z.real) < 1e-12 and abs(got[i + 8] - z.imag) < 1e-12
+    with pytest.raises(ValueError):
+        O.rope(x, 1, 1e4, rope_dims=15)
+
+
+def test_rope_switches_keep_identity_norms_and_relative_position():
+    rng = np.random.default_rng(33)
+    a, b = rng.standard_normal(64), rng.standard_normal(64)
+    for dims, inter in [(0, True), (32, False), (32, True), (2, False)]:
+        f = lambda v, p: O.rope(v, p, 1e4, rope_dims=dims, interleaved=inter)
+        np.testing.assert_array_equal(f(a, 0), a)
+        assert abs(np.linalg.norm(f(a, 4321)) - np.linalg.norm(a)) < 1e-12
+        for m, n in [(7, 7), (100, 3), (4 * 63000, 255180)]:
+            assert abs(f(a, m) @ f(b, n) - a @ f(b, n - m)) <= 1e-9 * (np.abs(a).sum() * np.abs(b).sum())
+
+
+def test_query_position_table():
+    """Query position floor(stride*(n-1)/4), by hand: token n-1, or the index of its block."""
+    assert [O.query_position(n) for n in range(1, 10)] == [0, 1, 2, 3, 4, 5, 6, 7, 8]
+    assert [O.query_position(n, 1) for n in range(1, 10)] == [0, 0, 0, 0, 1, 1, 1, 1, 2]
+    assert [O.query_position(n, 2) for n in range(1, 10)] == [0, 0, 1, 1, 2, 2, 3, 3, 4]
+    assert O.block_position(np.array([0, 1, 5])).tolist() == [0, 4, 20]
+    assert O.block_position(np.array([0, 1, 5]), 1, 3).tolist() == [3, 4, 8]
+
+
+def test_block_position_switches_on_periodic_keys():
+    """With every block holding the same 4 raw keys, summaries differ only by position:
+    offset 4 at block b is the default summary of block b+1; stride 8 at b is the default of 2b."""
+    rng = np.random.default_rng(34)
+    d = 32
+    one = rng.standard_normal((4, d)).astype(np.float16)
+    raw = np.tile(one, (40, 1))
+    base = O.QsaShape(d, 1, 8, 1, 1, 8)
+    dflt = O.pooled_cache_full(raw, 160, base)
+    off4 = O.pooled_cache_full(raw, 160, O.QsaShape(d, 1, 8, 1, 1, 8, rope_pos_offset=4))
+    st8 = O.pooled_cache_full(raw, 80, O.QsaShape(d, 1, 8, 1, 1, 8, rope_pos_stride=8))
+    np.testing.assert_array_equal(off4[:39], dflt[1:40])
+    np.testing.assert_array_equal(st8[:20], dflt[0:40:2])
+    # block domain (stride 1): the query's own block is at relative distance 0, so its dot
+    # is the un-rotated q . r (up to the f16 rounding of the stored row)
+    shape = O.QsaShape(d, 1, 8, 1, 1, 8, rope_pos_stride=1)
+    raw2 = rng.standard_normal((4 * 30, d)).astype(np.float16)
+    q = rng.standard_normal((1, d)).astype(np.float16)
+    n = 4 * 30                                    # query token 119 sits in block 29
+    pooled = O.pooled_cache_full(raw2, n, shape)
+    r = O.rms_normalize(O.mean_pool(raw2[116:120]), shape.rms_eps)
+    qr = float(q[0].astype(np.float64) @ r)
+    dot29 = float(pooled[29].astype(np.float64) @ O.indexer_query(q, n, shape)[0])
+    assert abs(dot29 - qr) <= 2e-3 * np.abs(q[0].astype(np.float64)).sum() * np.abs(r).max()
+
+
 # ---------------------------------------------------------------- pool + RMS norm
 
 def test_mean_pool_is_exact_mean():
