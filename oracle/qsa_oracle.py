@@ -308,6 +308,30 @@ class OracleLayer:
     def attend(self, q, cells) -> np.ndarray:
         return sparse_attention(q, self.k, self.v, cells, self.shape)
 
+    def rollback(self, n_keep: int) -> None:
+        """Drop the tokens at positions >= n_keep (rejected speculative tokens). Summaries of
+        blocks those tokens completed are no longer trusted (Part 10 §COMMON-004: dirty
+        speculative writes must not corrupt the cached range)."""
+        self.n = min(self.n, max(0, n_keep))
+        self.pooled.invalidate(self.n // BLOCK)
+
+    def multi_query_step(self, k, v, idx, q_idx, w, q):
+        """Verify T tokens at once (speculative / multi-token decode): append all T, bring the
+        pooled cache up to date, then query t (token n-T+t) selects and attends over the
+        context it can see, n_t = n-T+t+1 tokens: the blocks completed within n_t and its own
+        open tail. k, v: [T, Hkv, D]; idx: [T, d]; q_idx: [T, H, d]; w: [T, H]; q: [T, Hq, D]."""
+        T = len(k)
+        self.append_tokens(k, v, idx)
+        self.update_pooled_cache()
+        outs = []
+        for t in range(T):
+            n_t = self.n - T + t + 1
+            s = block_scores(self.pooled.rows, q_idx[t], w[t], n_t, self.shape)
+            sel = topk_blocks(s, self.shape.k_blocks)
+            cells = expand_cells(sel, n_t)
+            outs.append({"sel": sel, "scores": s, "cells": cells, "out": self.attend(q[t], cells)})
+        return outs
+
     def decode_step(self, k, v, idx, q_idx, w, q):
         """append -> incremental pooled update -> scores + top-k -> cells -> attention."""
         self.append_tokens(k[None], v[None], idx[None])

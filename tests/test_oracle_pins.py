@@ -416,3 +416,64 @@ def test_golden_tiny_chain_regression():
     assert sorted(want.files) == sorted(got)
     for key in want.files:
         np.testing.assert_allclose(got[key], want[key], rtol=1e-12, atol=0, err_msg=key)
+
+
+# ---------------------------------------------------------------- multi-query step (speculative verify)
+
+def _tokens(rng, shape, T):
+    f16 = lambda *s: rng.standard_normal(s).astype(np.float16)
+    return dict(k=f16(T, shape.n_kv_heads, shape.head_dim), v=f16(T, shape.n_kv_heads, shape.head_dim),
+                idx=f16(T, shape.d_idx), q_idx=f16(T, shape.n_idx_heads, shape.d_idx),
+                w=rng.random((T, shape.n_idx_heads)), q=f16(T, shape.n_q_heads, shape.head_dim))
+
+
+@pytest.mark.parametrize("n0,T", [(97, 4), (98, 3), (100, 2), (101, 1), (4 * 9 + 2, 4)])
+def test_multi_query_step_equals_sequential_decode(n0, T):
+    """T queries verified in one step see exactly what T single-token steps would see."""
+    rng = np.random.default_rng(n0 * 10 + T)
+    shape = SMALL
+    pre = _tokens(rng, shape, n0)
+    a, b = O.OracleLayer(shape, 256), O.OracleLayer(shape, 256)
+    for L in (a, b):
+        L.append_tokens(pre["k"], pre["v"], pre["idx"])
+        L.update_pooled_cache()
+    x = _tokens(rng, shape, T)
+    multi = a.multi_query_step(x["k"], x["v"], x["idx"], x["q_idx"], x["w"], x["q"])
+    for t in range(T):
+        one = b.decode_step(x["k"][t], x["v"][t], x["idx"][t], x["q_idx"][t], x["w"][t], x["q"][t])
+        for key in ("sel", "cells", "scores", "out"):
+            np.testing.assert_array_equal(multi[t][key], one[key])
+        # causality: query t never sees a later token, and its own open tail is attended
+        n_t = n0 + t + 1
+        assert multi[t]["cells"].max() < n_t
+        assert set(range(4 * (n_t // 4), n_t)) <= set(multi[t]["cells"].tolist())
+    np.testing.assert_array_equal(a.pooled.rows, b.pooled.rows)
+
+
+def test_rollback_recomputes_blocks_completed_by_rejected_tokens():
+    """Tokens n0..n0+3 with n0 = 4m+2: token n0+1 completes block m. Rejecting it (keep n0+1
+    tokens) must drop that summary, so later steps equal a layer that never saw it."""
+    rng = np.random.default_rng(77)
+    shape = SMALL
+    n0 = 4 * 20 + 2
+    pre = _tokens(rng, shape, n0)
+    a, b = O.OracleLayer(shape, 256), O.OracleLayer(shape, 256)
+    for L in (a, b):
+        L.append_tokens(pre["k"], pre["v"], pre["idx"])
+        L.update_pooled_cache()
+    draft = _tokens(rng, shape, 4)
+    a.multi_query_step(draft["k"], draft["v"], draft["idx"], draft["q_idx"], draft["w"], draft["q"])
+    assert a.pooled.n_pooled == 21
+    a.rollback(n0 + 1)                                # keep the first draft token only
+    assert (a.n, a.pooled.n_pooled) == (n0 + 1, 20)
+    b.decode_step(draft["k"][0], draft["v"][0], draft["idx"][0], draft["q_idx"][0], draft["w"][0], draft["q"][0])
+    nxt = _tokens(rng, shape, 3)                      # different tokens at the rejected positions
+    ra = a.multi_query_step(nxt["k"], nxt["v"], nxt["idx"], nxt["q_idx"], nxt["w"], nxt["q"])
+    rb = b.multi_query_step(nxt["k"], nxt["v"], nxt["idx"], nxt["q_idx"], nxt["w"], nxt["q"])
+    np.testing.assert_array_equal(a.pooled.rows[:a.n // 4], b.pooled.rows[:b.n // 4])
+    for x, y in zip(ra, rb):
+        np.testing.assert_array_equal(x["out"], y["out"])
+        np.testing.assert_array_equal(x["sel"], y["sel"])
+    # without the invalidation the stale summary of block 20 would differ from the fresh one
+    stale = O.pooled_summaries(np.concatenate([pre["idx"], draft["idx"][:2]]), 20, 21, shape)
+    assert not np.array_equal(stale[0], a.pooled.rows[20])
