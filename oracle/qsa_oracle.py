@@ -50,6 +50,8 @@ Readings taken where the pages are silent (each one is listed in the design note
      completed is scored like any other, not force-included.
   R8 attention: scale 1/sqrt(D), query head i uses KV head floor(i / (Hq/Hkv)), no
      extra mask, sink, gate or softcap.
+  R12 FP8 K/V cache (optional): per (token, KV head) row, scale = amax/448 and e4m3 codes
+     of x * 448/amax (nearest-even, saturating); attention reads code * scale.
 """
 from __future__ import annotations
 
@@ -261,6 +263,76 @@ def sparse_attention(q, k_cache, v_cache, cells, shape: QsaShape) -> np.ndarray:
         e = np.exp(logits - logits.max())
         out[i] = (e @ vc) / e.sum()
     return out
+
+
+# ---------------------------------------------------------------------------
+# FP8 K/V cache (survey row f4; the pages measured a Q8_0 KV cache on their hardware).
+# Reading R12: one f32 scale per (token, KV head) row, scale = amax / 448, codes =
+# e4m3(x * (448 / amax)) with round-to-nearest-even and saturation to +-448; an all-zero
+# row gets scale 1 and zero codes. Attention runs over code * scale.
+# ---------------------------------------------------------------------------
+
+E4M3_MAX = 448.0
+
+
+def e4m3_value(code: int) -> float:
+    """Value of an e4m3 byte: 1 sign bit, 4 exponent bits (bias 7), 3 mantissa bits;
+    exponent 0 is subnormal (m * 2^-9); S.1111.111 is NaN (no infinities)."""
+    code = int(code)
+    sign = -1.0 if code & 0x80 else 1.0
+    e, m = (code >> 3) & 0xF, code & 0x7
+    if e == 0xF and m == 0x7:
+        return float("nan")
+    if e == 0:
+        return sign * m * 2.0 ** -9
+    return sign * (1.0 + m / 8.0) * 2.0 ** (e - 7)
+
+
+def e4m3_encode(x) -> np.ndarray:
+    """Round float32 values to e4m3 bytes: nearest representable value, ties to the even
+    mantissa, magnitudes above 448 saturate to 448, the sign bit kept for zero results
+    (the values here are finite)."""
+    x = np.asarray(x, dtype=np.float32).astype(np.float64)
+    mag = np.abs(x)
+    # quantum of the binade of |x| (2^(e-3)), with the subnormal quantum 2^-9 below 2^-6
+    e = np.floor(np.log2(np.where(mag > 0, mag, 1.0)))
+    e = np.maximum(e, -6.0)
+    quantum = 2.0 ** (e - 3)
+    k = np.round(mag / quantum)          # numpy rounds halves to even
+    r = np.minimum(k * quantum, E4M3_MAX)
+    # encode r (exactly representable) into sign/exponent/mantissa bits
+    out = np.zeros(x.shape, dtype=np.uint8)
+    nz = r > 0
+    er = np.floor(np.log2(np.where(nz, r, 1.0)))
+    sub = nz & (er < -6)
+    norm = nz & ~sub
+    m_sub = np.where(sub, r / 2.0 ** -9, 0).astype(np.int64)
+    exp_n = np.where(norm, er + 7, 0).astype(np.int64)
+    m_n = np.where(norm, (r / 2.0 ** np.where(norm, er, 0) - 1.0) * 8.0, 0).astype(np.int64)
+    bits = np.where(sub, m_sub, (exp_n << 3) | m_n)
+    out[...] = np.where(np.signbit(x), 0x80, 0) | bits   # -0 and negatives that round to 0 keep the sign
+    return out
+
+
+def quantize_kv_rows(rows):
+    """[..., D] f16 rows -> (e4m3 codes [..., D] uint8, scales [...] f32), reading R12.
+    The scale and the multiplier are single f32 operations, like the library's."""
+    x = np.asarray(rows, dtype=np.float16).astype(np.float32)
+    amax = np.max(np.abs(x), axis=-1)
+    zero = amax == 0
+    safe = np.where(zero, np.float32(1.0), amax).astype(np.float32)
+    scale = np.where(zero, np.float32(1.0), safe / np.float32(E4M3_MAX)).astype(np.float32)
+    mult = np.where(zero, np.float32(0.0), np.float32(E4M3_MAX) / safe).astype(np.float32)
+    codes = e4m3_encode((x * mult[..., None]).astype(np.float32))
+    return codes, scale
+
+
+_E4M3_TABLE = np.array([e4m3_value(c) for c in range(256)])
+
+
+def dequantize_kv_rows(codes, scales) -> np.ndarray:
+    """code * scale in float64."""
+    return _E4M3_TABLE[np.asarray(codes)] * np.asarray(scales, dtype=np.float64)[..., None]
 
 
 # ---------------------------------------------------------------------------

@@ -477,3 +477,57 @@ def test_rollback_recomputes_blocks_completed_by_rejected_tokens():
     # without the invalidation the stale summary of block 20 would differ from the fresh one
     stale = O.pooled_summaries(np.concatenate([pre["idx"], draft["idx"][:2]]), 20, 21, shape)
     assert not np.array_equal(stale[0], a.pooled.rows[20])
+
+
+# ---------------------------------------------------------------- FP8 (e4m3) K/V cache
+
+def test_e4m3_known_codes():
+    """Values fixed by the e4m3 layout (bias 7, 3 mantissa bits, subnormals, S.1111.111 = NaN)."""
+    known = {0x00: 0.0, 0x01: 2.0 ** -9, 0x07: 7 * 2.0 ** -9, 0x08: 2.0 ** -6, 0x38: 1.0, 0x39: 1.125,
+             0x40: 2.0, 0x7E: 448.0, 0xB8: -1.0, 0xFE: -448.0}
+    for c, v in known.items():
+        assert O.e4m3_value(c) == v, hex(c)
+    assert np.isnan(O.e4m3_value(0x7F)) and np.isnan(O.e4m3_value(0xFF))
+    assert np.signbit(O.e4m3_value(0x80))
+    finite = [c for c in range(256) if not np.isnan(O.e4m3_value(c))]
+    assert len(finite) == 254
+    np.testing.assert_array_equal(O.e4m3_encode(np.array([O.e4m3_value(c) for c in finite], np.float32)), finite)
+
+
+def test_e4m3_encode_is_nearest_even_by_brute_force():
+    rng = np.random.default_rng(41)
+    x = np.concatenate([rng.standard_normal(3000) * s for s in (1e-3, 0.05, 1, 30, 300)]).astype(np.float32)
+    vals = np.array([O.e4m3_value(c) for c in range(256)])
+    codes = np.array([c for c in range(256) if not np.isnan(vals[c])])
+    # midpoints between neighbours and values past the largest finite one
+    grid = np.unique(np.abs(vals[codes]))
+    x = np.concatenate([x, ((grid[:-1] + grid[1:]) / 2).astype(np.float32), np.float32([449, 500, -1e4])])
+    got = O.e4m3_encode(x)
+    for xi, gi in zip(x.astype(np.float64), got):
+        if abs(xi) > 448:
+            assert O.e4m3_value(gi) == np.sign(xi) * 448.0
+            continue
+        d = np.abs(vals[codes] - xi)
+        best = codes[d == d.min()]
+        best = best[(best & 0x80) == (0x80 if np.signbit(xi) else 0)] if len(best) > 1 else best
+        if len(best) > 1:                       # a tie: the even mantissa wins
+            best = best[(best & 1) == 0]
+        assert O.e4m3_value(gi) == O.e4m3_value(best[0]), (xi, hex(gi), [hex(b) for b in best])
+
+
+def test_kv_row_quantization_closed_forms():
+    rng = np.random.default_rng(42)
+    rows = rng.standard_normal((64, 4, 128)).astype(np.float16)
+    rows[3, 1] = 0
+    codes, scales = O.quantize_kv_rows(rows)
+    assert codes.dtype == np.uint8 and scales.dtype == np.float32 and scales.shape == (64, 4)
+    amax = np.abs(rows.astype(np.float32)).max(axis=-1)
+    nz = amax > 0
+    np.testing.assert_array_equal(scales[nz], (amax / np.float32(448))[nz])
+    assert scales[3, 1] == 1.0 and not codes[3, 1].any()
+    deq = O.dequantize_kv_rows(codes, scales)
+    # the row maximum lands on +-448 exactly; every element within half a quantum
+    np.testing.assert_array_equal(np.abs(deq).max(axis=-1)[nz], 448.0 * scales[nz].astype(np.float64))
+    x = rows.astype(np.float64)
+    bound = np.maximum(np.abs(x) * 2.0 ** -4, 2.0 ** -10 * scales[..., None])
+    assert np.all(np.abs(deq - x) <= bound * (1 + 1e-6))
