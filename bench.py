@@ -48,6 +48,7 @@ def parse_args():
     ap.add_argument("--workload", default="ctx256k_12l")
     ap.add_argument("--no-by-ctx", action="store_true", help="skip the 64k/128k lines")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-fp8", action="store_true", help="skip the FP8 K/V cache line")
     ap.add_argument("--e2e-steps", type=int, default=300)
     ap.add_argument("--profile-case", action="store_true",
                     help="small case for ncu: 1 layer at 256k, few steps, no extras")
@@ -169,7 +170,7 @@ def max_over_ranks(x, world):
 class Workbench:
     """L bound layers prefilled with the workload's context and graph-captured steps."""
 
-    def __init__(self, wl, n_layers, n_graph_steps, extra_steps, rank):
+    def __init__(self, wl, n_layers, n_graph_steps, extra_steps, rank, kv_format=0):
         import torch
 
         import synth
@@ -177,7 +178,7 @@ class Workbench:
         self.torch, self.Q, self.wl, self.L = torch, Q, wl, n_layers
         max_ctx = int(math.ceil((wl.n_prefill + n_graph_steps + extra_steps + 8) / 4) * 4)
         self.cfg = Q.make_config(n_layers, max_ctx, wl.d_idx, wl.n_idx_heads, wl.top_k_tokens, wl.n_q_heads,
-                                 wl.n_kv_heads, wl.head_dim, wl.rope_base, wl.rms_eps)
+                                 wl.n_kv_heads, wl.head_dim, wl.rope_base, wl.rms_eps, kv_format=kv_format)
         self.qsa = Q.Qsa(self.cfg)
         self.bufs, self.outs = [], []
         for layer in range(n_layers):
@@ -257,10 +258,75 @@ class Workbench:
         return self.qsa.read_layer_state(0)[0]
 
 
-def run_ours(wl, n_layers, K, W, rank, world, e2e_steps, sample_clocks, local):
+def run_multi_query(wb, wl, n_layers, T=4, steps_per_graph=8, replays=4):
+    """Speculative verification of T drafted tokens per step, on every layer: append the T
+    tokens, pool, one T-query scan + selection, one T-query attention, then roll back the
+    T-1 rejected drafts (one token accepted per step). Captured as one graph of
+    `steps_per_graph` steps; the rollback targets are absolute, so each replay restarts
+    from the same length. Also times the T-query scan + selection alone."""
+    import torch
+    Q = wb.Q
+    mk = lambda *shape: torch.randn(*shape, device="cuda").to(torch.float16)
+    xs = [{"k": mk(T, wl.n_kv_heads, wl.head_dim), "v": mk(T, wl.n_kv_heads, wl.head_dim), "idx": mk(T, wl.d_idx),
+           "q_idx": mk(T, wl.n_idx_heads, wl.d_idx), "w": torch.rand(T, wl.n_idx_heads, device="cuda"),
+           "q": mk(T, wl.n_q_heads, wl.head_dim)} for _ in range(n_layers)]
+    mo = [Q.alloc_multi_outputs(wb.cfg, T) for _ in range(n_layers)]
+    n0 = wb.n_ctx()
+    q = wb.qsa
+
+    def verify(layer, n_keep):
+        x, o = xs[layer], mo[layer]
+        q.append_tokens(layer, x["k"], x["v"], x["idx"])
+        q.update_pooled_cache(layer)
+        q.index_topk_multi(layer, x["q_idx"], x["w"], o["sel"], o["n_sel"], o["scores"])
+        q.sparse_attend_selected_multi(layer, x["q"], o["sel"], o["n_sel"], o["out"])
+        q.rollback(layer, n_keep)
+
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for j in range(steps_per_graph):
+            for layer in range(n_layers):
+                verify(layer, n0 + 1 + j)
+    g.replay()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(replays):
+        g.replay()
+    b.record(stream)
+    torch.cuda.synchronize()
+    us = 1e3 * a.elapsed_time(b) / (replays * steps_per_graph * n_layers)
+    for layer in range(n_layers):
+        n, p, st = q.read_layer_state(layer)
+        assert (n, p, st) == (n0 + steps_per_graph, (n0 + steps_per_graph) // 4, 0), (layer, n, p, st)
+        assert int(mo[layer]["n_sel"].min()) == wl.k_blocks and torch.isfinite(mo[layer]["out"]).all()
+    del g
+    # the T-query scan + selection alone, back to back over the layers
+    g2 = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g2):
+        for _ in range(4):
+            for layer in range(n_layers):
+                x, o = xs[layer], mo[layer]
+                q.index_topk_multi(layer, x["q_idx"], x["w"], o["sel"], o["n_sel"], o["scores"])
+    g2.replay()
+    torch.cuda.synchronize()
+    a.record(stream)
+    for _ in range(5):
+        g2.replay()
+    b.record(stream)
+    torch.cuda.synchronize()
+    idx_us = 1e3 * a.elapsed_time(b) / (5 * 4 * n_layers)
+    del g2
+    return {"n_queries": T, "steps": replays * steps_per_graph, "us_per_layer_step": round(us, 3),
+            "value": round(T * n_layers * 1e6 / (us * n_layers), 1), "unit": "layer-queries/s",
+            "index_topk_us": round(idx_us, 3), "launches_per_layer_step": 5}
+
+
+def run_ours(wl, n_layers, K, W, rank, world, e2e_steps, sample_clocks, local, multi_query=False, kv_format=0):
     import torch
     G = max(d for d in range(1, 33) if K % d == 0)       # steps per timed graph
-    wb = Workbench(wl, n_layers, W + K, extra_steps=e2e_steps + 64, rank=rank)
+    wb = Workbench(wl, n_layers, W + K, extra_steps=e2e_steps + 128, rank=rank, kv_format=kv_format)
     warm = [wb.capture([s]) for s in range(W)]
     timed = [wb.capture(list(range(W + j * G, W + (j + 1) * G))) for j in range(K // G)]
     torch.cuda.synchronize()
@@ -409,8 +475,9 @@ def run_ours(wl, n_layers, K, W, rank, world, e2e_steps, sample_clocks, local):
         e2e = {"value": world * n_layers * e2e_steps / (e_ms / 1e3), "unit": UNIT,
                "h2d_bytes_per_step": int(host_in[0].numel()), "d2h_bytes_per_step": int(host_out[0].numel() * 4),
                "steps": e2e_steps}
+    mq = run_multi_query(wb, wl, n_layers) if multi_query else None
     return {"ms": ms, "clocks": clk, "per_launch_us": per_launch_us, "iso_us": iso, "n_ctx_instr": n_ctx_instr,
-            "bulk_pool": bulk,
+            "bulk_pool": bulk, "multi_query": mq,
             "n_layers": n_layers, "launches_per_step": n_layers * wb.launches_per_layer, "e2e": e2e,
             "graph_steps": G}
 
@@ -432,10 +499,11 @@ def ncu_traffic(stage):
         return None
 
 
-def stage_bytes(wl, n_ctx):
-    """Algorithmic HBM bytes per launch of each stage at context n_ctx (per layer)."""
+def stage_bytes(wl, n_ctx, kv_fp8=False):
+    """Algorithmic HBM bytes per launch of each stage at context n_ctx (per layer). With an
+    FP8 K/V cache a row is head_dim code bytes plus its 4-byte scale."""
     B = n_ctx // 4
-    kv_row = wl.n_kv_heads * wl.head_dim * 2
+    kv_row = wl.n_kv_heads * (wl.head_dim + 4 if kv_fp8 else wl.head_dim * 2)
     n_cells = 4 * min(wl.k_blocks, B) + n_ctx % 4
     return {
         # read the token's inputs, write the caches; one pooled block (4 raw keys in, 1 row out)
@@ -496,7 +564,7 @@ def main_ours(args):
     peak, peak_src = measured_peaks()
 
     main = run_ours(wl, wl.n_layers, K, W, rank, world, 0 if args.profile_case else args.e2e_steps,
-                    sample_clocks=not args.profile_case, local=local)
+                    sample_clocks=not args.profile_case, local=local, multi_query=not args.profile_case)
     layer_steps = world * wl.n_layers * K
     value = layer_steps / (main["ms"] / 1e3)
 
@@ -543,6 +611,23 @@ def main_ours(args):
                             "scan_attn_gbs": round(hb / (hu * 1e-6) / 1e9, 1)}
             torch.cuda.empty_cache()
 
+    # the same step with the FP8 (e4m3 + per-row scale) K/V cache: attention reads half the bytes
+    kv_fp8 = None
+    if not args.profile_case and not args.no_fp8:
+        torch.cuda.empty_cache()
+        k8 = max(500, min(K // 5, 1000))
+        k8 -= k8 % 25
+        r8 = run_ours(wl, wl.n_layers, k8, 5, rank, world, 0, sample_clocks=False, local=local, kv_format=1)
+        b8 = stage_bytes(wl, r8["n_ctx_instr"], kv_fp8=True)
+        a8 = r8["iso_us"]["sparse_attend"]
+        kv_fp8 = {"value": round(world * wl.n_layers * k8 / (r8["ms"] / 1e3), 1), "unit": UNIT, "steps": k8,
+                  "ms_per_step": round(r8["ms"] / k8, 5), "attend_us": round(a8, 3),
+                  "attend_bytes": int(b8["sparse_attend"]),
+                  "attend_gbs": round(b8["sparse_attend"] / (a8 * 1e-6) / 1e9, 1),
+                  "attend_us_f16": round(per["sparse_attend"], 3)}
+        del r8
+        torch.cuda.empty_cache()
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(wl)
@@ -565,6 +650,8 @@ def main_ours(args):
             "gpu_launches": main["launches_per_step"] * K,
             "by_ctx": by_ctx,
             "bulk_pool": dict(main["bulk_pool"], frac=round(main["bulk_pool"]["gbs"] / peak, 4)) if main["bulk_pool"] else None,
+            "multi_query": main["multi_query"],
+            "kv_fp8": kv_fp8,
             "hbm_gbs_step": round(world * wl.n_layers * K * sum(sb.values()) / (main["ms"] / 1e3) / 1e9, 1),
         }
         print(json.dumps(line))

@@ -72,16 +72,38 @@ typedef struct {
   int32_t head_dim;       /* attention head dimension D: 64 or 128                      */
   float rope_base;        /* RoPE base (10000)                                          */
   float rms_eps;          /* RMS-norm epsilon inside the square root (1e-6)             */
+  /* RoPE of the indexer keys and query (Part 10, section "QSA indexer": RoPE at the block
+   * position). The pages fix neither the pairing, the rotary width nor the position scale;
+   * zero-initialised fields give the defaults below. */
+  int32_t rope_dims;        /* rotary dims R: even, 2..d_idx; the rest pass through. 0 = d_idx */
+  int32_t rope_interleaved; /* 0: NeoX pairs (i, i+R/2); 1: GPT-J pairs (2i, 2i+1). Pair i
+                               turns by pos * rope_base^(-2i/R)                          */
+  int32_t rope_pos_stride;  /* block b sits at position stride*b + offset and the query at
+                               floor(stride*(n-1)/4): 4 = token positions (block = its first
+                               token, query = token n-1), 1 = block indices. 1..16; 0 = 4 */
+  int32_t rope_pos_offset;  /* 0..1,048,576 (0)                                          */
+  /* Storage of the attention K/V cache (the Qwen3.8-Flash-Next parameter-tuning post on
+   * EVO-X2, section "KV cacheをQ8_0にしてみる", tried an 8-bit K/V cache).
+   * QSA_KV_F16 (0): f16 rows. QSA_KV_FP8 (1): e4m3 codes with one f32 scale per
+   * (token, KV head) row, scale = amax/448, code = e4m3(x * 448/amax) rounded to
+   * nearest-even and saturated (an all-zero row: scale 1, zero codes); attention reads
+   * code * scale. The indexer caches stay f16 either way. */
+  int32_t kv_format;
 } qsa_config;
+
+enum { QSA_KV_F16 = 0, QSA_KV_FP8 = 1 };
 
 /* Caller-owned device buffers of one layer. Sizes come from qsa_buffer_bytes(). */
 typedef struct {
-  void* k_cache;          /* [max_ctx][n_kv_heads][head_dim] f16, token-major           */
-  void* v_cache;          /* [max_ctx][n_kv_heads][head_dim] f16, token-major           */
+  void* k_cache;          /* [max_ctx][n_kv_heads][head_dim] f16 (e4m3 bytes with
+                             QSA_KV_FP8), token-major                                   */
+  void* v_cache;          /* same layout as k_cache                                     */
   void* idx_cache;        /* [max_ctx][d_idx] f16: raw per-token indexer keys           */
   void* pooled_cache;     /* [max_ctx/4][d_idx] f16: pooled summaries p_b               */
   const float* rms_gain;  /* [d_idx] f32 RMS-norm gain, or NULL for unit gain           */
   void* workspace;        /* device state + scratch; QSA_BUF_WORKSPACE bytes            */
+  void* kv_scales;        /* QSA_KV_FP8 only: [max_ctx][n_kv_heads][2] f32, the K and V
+                             scales of each row; NULL with QSA_KV_F16                   */
 } qsa_layer_buffers;
 
 enum {
@@ -89,7 +111,10 @@ enum {
   QSA_BUF_IDX = 1,        /* bytes of idx_cache                           */
   QSA_BUF_POOLED = 2,     /* bytes of pooled_cache                        */
   QSA_BUF_WORKSPACE = 3,  /* bytes of workspace                           */
-  QSA_BUF_MAX_CELLS = 4   /* not bytes: max cells per step = 4*(top_k_tokens/4) + 3 */
+  QSA_BUF_MAX_CELLS = 4,  /* not bytes: max cells per step = 4*(top_k_tokens/4) + 3 */
+  QSA_BUF_SCORE_STRIDE = 5, /* not bytes: floats per row of a multi-query score table
+                               (max_ctx/4 rounded up to a multiple of 64) */
+  QSA_BUF_KV_SCALES = 6   /* bytes of kv_scales (0 with QSA_KV_F16)      */
 };
 
 typedef struct qsa_ctx qsa_ctx;
@@ -190,7 +215,8 @@ qsa_status qsa_select_topk(qsa_ctx* ctx, int32_t layer, const float* scores, int
  *   cells [4*(top_k_tokens/4)+3] i32 (ascending when sel_blocks is ascending),
  *   n_cells device i32 scalar = 4*n_sel + n_ctx mod 4.
  * If k_compact / v_compact are non-NULL, also copies the selected rows into them:
- * [max_cells][n_kv_heads][head_dim] f16 each (the literal compact K/V). Block ids out
+ * [max_cells][n_kv_heads][head_dim] f16 each (the literal compact K/V; f16 caches only,
+ * QSA_ERR_UNSUPPORTED with QSA_KV_FP8). Block ids out
  * of range are reported as device status QSA_ERR_BAD_INDEX and their cells written as
  * -1, which qsa_sparse_attend skips. */
 qsa_status qsa_gather_kv(qsa_ctx* ctx, int32_t layer, const int32_t* sel_blocks,
@@ -218,6 +244,45 @@ qsa_status qsa_sparse_attend(qsa_ctx* ctx, int32_t layer, const void* q, const i
 qsa_status qsa_sparse_attend_selected(qsa_ctx* ctx, int32_t layer, const void* q,
                                       const int32_t* sel_blocks, const int32_t* n_sel, float* out,
                                       qsa_stream_t stream);
+
+/* ---- Multi-query step: speculative / multi-token verification ----
+ * Part 10 (section COMMON-004) requires that speculative decoding's dirty writes never
+ * corrupt the cached pooled range. A verification step appends T drafted tokens
+ * (qsa_append_tokens, then qsa_update_pooled_cache), scores, selects and attends for
+ * all T queries at once, then drops the rejected tokens with qsa_rollback. Query u
+ * (u < T) belongs to token n_ctx - T + u and sees exactly what a single-token step at
+ * that token would: the blocks completed within its first n_ctx - T + u + 1 tokens and
+ * its own open tail. T ranges over 1..4. */
+#define QSA_MAX_QUERIES 4
+
+/* qsa_index_topk for T queries in one pass over the pooled cache (one launch of the
+ * scan, one of the selection):
+ *   q_idx [T][n_idx_heads][d_idx] f16 (un-rotated; query u is rotated at its own
+ *         token's position), w [T][n_idx_heads] f32;
+ *   sel_blocks [T][top_k_tokens/4] i32 (row u ascending), n_sel [T] device i32;
+ *   scores: NULL (the layer workspace holds them) or [T][S] f32 with S =
+ *         qsa_buffer_bytes(cfg, QSA_BUF_SCORE_STRIDE); row u is meaningful for blocks
+ *         < (n_ctx - T + u + 1)/4, later entries are not part of the result.
+ * Requires the pooled cache to be current for the whole context (n_pooled == n_ctx/4)
+ * and n_ctx >= T - 1; otherwise device status QSA_ERR_STATE and n_sel = 0. */
+qsa_status qsa_index_topk_multi(qsa_ctx* ctx, int32_t layer, int32_t n_queries, const void* q_idx,
+                                const float* w, int32_t* sel_blocks, int32_t* n_sel, float* scores,
+                                qsa_stream_t stream);
+
+/* qsa_sparse_attend_selected for T queries in one launch: q [T][n_q_heads][head_dim]
+ * f16, sel_blocks [T][top_k_tokens/4] and n_sel [T] as qsa_index_topk_multi writes
+ * them, out [T][n_q_heads][head_dim] f32. Query u attends over its selected blocks and
+ * the tail [4*(n_u/4), n_u), n_u = n_ctx - T + u + 1. */
+qsa_status qsa_sparse_attend_selected_multi(qsa_ctx* ctx, int32_t layer, int32_t n_queries, const void* q,
+                                            const int32_t* sel_blocks, const int32_t* n_sel, float* out,
+                                            qsa_stream_t stream);
+
+/* Drop the tokens at positions >= n_keep (the rejected drafts): n_ctx = min(n_ctx,
+ * n_keep) and n_pooled = min(n_pooled, n_ctx/4) on the device, so summaries of blocks
+ * that rejected tokens completed are recomputed by the next pooled update (or
+ * qsa_decode_append). The cache rows past n_keep are left as they are and overwritten
+ * by later appends. n_keep >= 0; a larger n_keep than n_ctx changes nothing. */
+qsa_status qsa_rollback(qsa_ctx* ctx, int32_t layer, int32_t n_keep, qsa_stream_t stream);
 
 /* Size of the fixed scratch array behind qsa_sparse_attend_noalloc (1 MiB). */
 #define QSA_NOALLOC_SCRATCH_BYTES (1u << 20)

@@ -266,7 +266,8 @@ def sparse_attention(q, k_cache, v_cache, cells, shape: QsaShape) -> np.ndarray:
 
 
 # ---------------------------------------------------------------------------
-# FP8 K/V cache (survey row f4; the pages measured a Q8_0 KV cache on their hardware).
+# FP8 K/V cache. The Qwen3.8-Flash-Next parameter-tuning post on EVO-X2 (section
+# "KV cacheをQ8_0にしてみる") tried an 8-bit K/V cache and gives no layout.
 # Reading R12: one f32 scale per (token, KV head) row, scale = amax / 448, codes =
 # e4m3(x * (448 / amax)) with round-to-nearest-even and saturation to +-448; an all-zero
 # row gets scale 1 and zero codes. Attention runs over code * scale.
@@ -342,12 +343,19 @@ def dequantize_kv_rows(codes, scales) -> np.ndarray:
 class OracleLayer:
     """One QSA layer's caches and the decode-step calls, in plain numpy."""
 
-    def __init__(self, shape: QsaShape, max_ctx: int, gain=None):
+    def __init__(self, shape: QsaShape, max_ctx: int, gain=None, kv_fp8: bool = False):
         self.shape = shape
         self.max_ctx = max_ctx
         self.gain = gain
-        self.k = np.zeros((max_ctx, shape.n_kv_heads, shape.head_dim), dtype=np.float16)
+        self.kv_fp8 = kv_fp8
+        kv_shape = (max_ctx, shape.n_kv_heads, shape.head_dim)
+        # attention reads self.k / self.v: the f16 rows, or code * scale (reading R12)
+        self.k = np.zeros(kv_shape, dtype=np.float64 if kv_fp8 else np.float16)
         self.v = np.zeros_like(self.k)
+        if kv_fp8:
+            self.k_codes = np.zeros(kv_shape, dtype=np.uint8)
+            self.v_codes = np.zeros(kv_shape, dtype=np.uint8)
+            self.kv_scales = np.zeros((max_ctx, shape.n_kv_heads, 2), dtype=np.float32)
         self.idx = np.zeros((max_ctx, shape.d_idx), dtype=np.float16)
         self.pooled = PooledKeyCache(max_ctx // BLOCK, shape.d_idx)
         self.n = 0
@@ -357,8 +365,16 @@ class OracleLayer:
         m = k.shape[0]
         if self.n + m > self.max_ctx:
             raise ValueError("context capacity exceeded")
-        self.k[self.n:self.n + m] = k
-        self.v[self.n:self.n + m] = np.asarray(v, np.float16).reshape(k.shape)
+        v = np.asarray(v, np.float16).reshape(k.shape)
+        if self.kv_fp8:
+            for rows, codes, which, deq in ((k, self.k_codes, 0, self.k), (v, self.v_codes, 1, self.v)):
+                c, sc = quantize_kv_rows(rows)
+                codes[self.n:self.n + m] = c
+                self.kv_scales[self.n:self.n + m, :, which] = sc
+                deq[self.n:self.n + m] = dequantize_kv_rows(c, sc)
+        else:
+            self.k[self.n:self.n + m] = k
+            self.v[self.n:self.n + m] = v
         self.idx[self.n:self.n + m] = np.asarray(idx, np.float16).reshape(m, self.shape.d_idx)
         self.n += m
 

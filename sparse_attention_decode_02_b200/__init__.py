@@ -3,5 +3,6 @@
 The compute lives in csrc/ (hand-written CUDA for sm_100a behind the C ABI declared in
 include/qsa.h); qsa.py only marshals torch device tensors and streams into that ABI.
 """
-from .qsa import (Qsa, QsaConfig, QsaError, alloc_layer, alloc_step_outputs, buffer_bytes,  # noqa: F401
-                  load_library, make_config, sparse_attend_noalloc)
+from .qsa import (QSA_KV_F16, QSA_KV_FP8, QSA_MAX_QUERIES, Qsa, QsaConfig, QsaError, alloc_layer,  # noqa: F401
+                  alloc_multi_outputs, alloc_step_outputs, buffer_bytes, load_library, make_config,
+                  sparse_attend_noalloc)

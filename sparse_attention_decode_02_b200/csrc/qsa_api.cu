@@ -15,6 +15,8 @@
 
 using namespace qsa;
 
+static_assert(QSA_MAX_QUERIES == kMaxQueries, "header and kernels agree on the multi-query limit");
+
 namespace {
 
 struct Layer {
@@ -42,6 +44,11 @@ const char* config_problem(const qsa_config& c) {
   if (!is_pow2_upto(c.n_q_heads / c.n_kv_heads, 8)) return "n_q_heads / n_kv_heads must be 1, 2, 4 or 8";
   if (!(c.rope_base > 1.0f)) return "rope_base must be > 1";
   if (!(c.rms_eps >= 0.0f)) return "rms_eps must be >= 0";
+  if (c.rope_dims < 0 || c.rope_dims > c.d_idx || c.rope_dims % 2) return "rope_dims must be even and <= d_idx";
+  if (c.rope_interleaved != 0 && c.rope_interleaved != 1) return "rope_interleaved must be 0 or 1";
+  if (c.rope_pos_stride < 0 || c.rope_pos_stride > 16) return "rope_pos_stride must be 0..16";
+  if (c.rope_pos_offset < 0 || c.rope_pos_offset > (1 << 20)) return "rope_pos_offset must be 0..1048576";
+  if (c.kv_format != QSA_KV_F16 && c.kv_format != QSA_KV_FP8) return "kv_format must be QSA_KV_F16 or QSA_KV_FP8";
   return nullptr;
 }
 
@@ -87,6 +94,7 @@ struct qsa_ctx {
     v.idx_cache = l.buf.idx_cache;
     v.pooled_cache = l.buf.pooled_cache;
     v.rms_gain = l.buf.rms_gain;
+    v.kv_scales = static_cast<float*>(l.buf.kv_scales);
     v.state = reinterpret_cast<DevState*>(wsp + ws.state);
     v.scores = reinterpret_cast<float*>(wsp + ws.scores);
     v.part_o = reinterpret_cast<float*>(wsp + ws.part_o);
@@ -114,7 +122,8 @@ size_t qsa_buffer_bytes(const qsa_config* cfg, int32_t which) {
   if (!cfg || config_problem(*cfg)) return 0;
   const qsa_config& c = *cfg;
   switch (which) {
-    case QSA_BUF_KV: return size_t(c.max_ctx) * c.n_kv_heads * c.head_dim * 2;
+    case QSA_BUF_KV: return size_t(c.max_ctx) * c.n_kv_heads * c.head_dim * (c.kv_format == QSA_KV_FP8 ? 1 : 2);
+    case QSA_BUF_KV_SCALES: return c.kv_format == QSA_KV_FP8 ? size_t(c.max_ctx) * c.n_kv_heads * 2 * 4 : 0;
     case QSA_BUF_IDX: return size_t(c.max_ctx) * c.d_idx * 2;
     case QSA_BUF_POOLED: return size_t(c.max_ctx / kBlock) * c.d_idx * 2;
     case QSA_BUF_WORKSPACE: {
@@ -129,6 +138,7 @@ size_t qsa_buffer_bytes(const qsa_config* cfg, int32_t which) {
       return workspace_layout(c, n_splits).total;
     }
     case QSA_BUF_MAX_CELLS: return size_t(max_cells_of(c));
+    case QSA_BUF_SCORE_STRIDE: return size_t(score_stride_of(c));
     default: return 0;
   }
 }
@@ -140,6 +150,8 @@ qsa_status qsa_create(const qsa_config* cfg, qsa_ctx** out) {
   qsa_ctx* ctx = new (std::nothrow) qsa_ctx();
   if (!ctx) return QSA_ERR_INVALID_ARG;
   ctx->cfg = *cfg;
+  if (ctx->cfg.rope_dims == 0) ctx->cfg.rope_dims = ctx->cfg.d_idx;  // zero fields take the defaults
+  if (ctx->cfg.rope_pos_stride == 0) ctx->cfg.rope_pos_stride = kBlock;
   if (cudaGetDevice(&ctx->device) != cudaSuccess ||
       cudaDeviceGetAttribute(&ctx->n_sms, cudaDevAttrMultiProcessorCount, ctx->device) != cudaSuccess) {
     delete ctx;
@@ -176,6 +188,7 @@ qsa_status qsa_bind_layer(qsa_ctx* ctx, int32_t layer, const qsa_layer_buffers* 
   QSA_CHECK_PTR(buf->workspace, 256, "workspace");
   if (buf->rms_gain && !aligned(buf->rms_gain, 16))
     return ctx->fail(QSA_ERR_INVALID_ARG, "rms_gain must be 16-byte aligned");
+  if (ctx->cfg.kv_format == QSA_KV_FP8) QSA_CHECK_PTR(buf->kv_scales, 16, "kv_scales");
   Layer& l = ctx->layers[layer];
   CUtensorMap tile_map, box_map;
   if (qsa_status st = ctx->cuda(encode_pooled_map(ctx->cfg, buf->pooled_cache, 128, &tile_map), "bind_layer: pooled TMA map"))
@@ -321,6 +334,8 @@ qsa_status qsa_gather_kv(qsa_ctx* ctx, int32_t layer, const int32_t* sel_blocks,
   QSA_CHECK_PTR(n_cells, 4, "n_cells");
   if ((k_compact && !aligned(k_compact, 16)) || (v_compact && !aligned(v_compact, 16)))
     return ctx->fail(QSA_ERR_INVALID_ARG, "compact K/V must be 16-byte aligned");
+  if ((k_compact || v_compact) && ctx->cfg.kv_format == QSA_KV_FP8)
+    return ctx->fail(QSA_ERR_UNSUPPORTED, "compact K/V copies need an f16 K/V cache");
   return ctx->cuda(launch_gather(ctx->view(layer), sel_blocks, n_sel, cells, n_cells, k_compact, v_compact,
                                  (cudaStream_t)stream),
                    "gather_kv");
@@ -335,6 +350,52 @@ qsa_status qsa_sparse_attend(qsa_ctx* ctx, int32_t layer, const void* q, const i
   QSA_CHECK_PTR(n_cells, 4, "n_cells");
   QSA_CHECK_PTR(out, 16, "out");
   return ctx->cuda(launch_attend(ctx->view(layer), q, cells, n_cells, out, (cudaStream_t)stream), "sparse_attend");
+}
+
+qsa_status qsa_index_topk_multi(qsa_ctx* ctx, int32_t layer, int32_t n_queries, const void* q_idx, const float* w,
+                                int32_t* sel_blocks, int32_t* n_sel, float* scores, qsa_stream_t stream) {
+  if (!ctx) return QSA_ERR_INVALID_ARG;
+  if (qsa_status st = ctx->layer_ok(layer)) return st;
+  if (n_queries < 1 || n_queries > kMaxQueries)
+    return ctx->fail(QSA_ERR_INVALID_ARG, "n_queries %d outside [1, %d]", n_queries, kMaxQueries);
+  QSA_CHECK_PTR(q_idx, 16, "q_idx");
+  QSA_CHECK_PTR(w, 4, "w");
+  QSA_CHECK_PTR(sel_blocks, 16, "sel_blocks");
+  QSA_CHECK_PTR(n_sel, 4, "n_sel");
+  if (scores && !aligned(scores, 16)) return ctx->fail(QSA_ERR_INVALID_ARG, "scores must be 16-byte aligned");
+  LayerView v = ctx->view(layer);
+  const int stride = score_stride_of(ctx->cfg);
+  float* s = scores ? scores : v.scores;
+  if (qsa_status st = ctx->cuda(launch_index_scan(v, q_idx, w, s, (cudaStream_t)stream, n_queries, stride),
+                                "index scan (multi-query)"))
+    return st;
+  return ctx->cuda(launch_topk(v, s, sel_blocks, n_sel, (cudaStream_t)stream, n_queries, stride),
+                   "block top-k (multi-query)");
+}
+
+qsa_status qsa_sparse_attend_selected_multi(qsa_ctx* ctx, int32_t layer, int32_t n_queries, const void* q,
+                                            const int32_t* sel_blocks, const int32_t* n_sel, float* out,
+                                            qsa_stream_t stream) {
+  if (!ctx) return QSA_ERR_INVALID_ARG;
+  if (qsa_status st = ctx->layer_ok(layer)) return st;
+  if (n_queries < 1 || n_queries > kMaxQueries)
+    return ctx->fail(QSA_ERR_INVALID_ARG, "n_queries %d outside [1, %d]", n_queries, kMaxQueries);
+  QSA_CHECK_PTR(q, 16, "q");
+  QSA_CHECK_PTR(sel_blocks, 16, "sel_blocks");
+  QSA_CHECK_PTR(n_sel, 4, "n_sel");
+  QSA_CHECK_PTR(out, 16, "out");
+  return ctx->cuda(launch_attend_selected(ctx->view(layer), q, sel_blocks, n_sel, out, (cudaStream_t)stream,
+                                          n_queries),
+                   "sparse_attend_selected (multi-query)");
+}
+
+qsa_status qsa_rollback(qsa_ctx* ctx, int32_t layer, int32_t n_keep, qsa_stream_t stream) {
+  if (!ctx) return QSA_ERR_INVALID_ARG;
+  if (qsa_status st = ctx->layer_ok(layer)) return st;
+  if (n_keep < 0) return ctx->fail(QSA_ERR_INVALID_ARG, "n_keep must be >= 0");
+  Layer& l = ctx->layers[layer];
+  l.pending_blocks += 2;  // the invalidated tail blocks (sizes the next update's grid only)
+  return ctx->cuda(launch_set_state(ctx->view(layer), n_keep, 0, kSetRollback, (cudaStream_t)stream), "rollback");
 }
 
 qsa_status qsa_sparse_attend_selected(qsa_ctx* ctx, int32_t layer, const void* q, const int32_t* sel_blocks,

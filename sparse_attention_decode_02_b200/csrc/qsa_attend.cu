@@ -10,6 +10,7 @@
 //    the selected rows straight from the f16 cache; qsa_gather_kv can still materialise
 //    the compact K/V.
 #include <cuda_fp16.h>
+#include <cuda_fp8.h>
 
 #include <cooperative_groups.h>
 
@@ -315,7 +316,9 @@ cudaError_t launch_attend_split(const LayerView& L, const void* q, const int32_t
 // partials through DSMEM to the CTAs that own each output slice, which merge them after
 // a single cluster barrier and write the final output. In the
 // FROM_BLOCKS form the cell ids are expanded on the fly from the selected blocks and
-// the open tail (cell expansion fused in as well).
+// the open tail (cell expansion fused in as well). With gridDim.y = T > 1 (multi-query
+// step), the clusters of row u serve the query of token n_ctx - T + u: its q, id and
+// output rows, and only the first n_ctx - T + u + 1 tokens (its own open tail).
 // ---------------------------------------------------------------------------------
 constexpr int kAcThreads = 512;
 constexpr int kAcWarps = kAcThreads / 32;
@@ -379,11 +382,32 @@ struct AcSmem {
   __host__ __device__ static size_t bytes(int lc, int cs) { return in_off(lc, cs) + size_t(cs) * per(cs) * 8; }
 };
 
-template <int D, int G, int CS, bool FROM_BLOCKS>
+// FP8 (K/V cache in e4m3 with a per-row scale): each staged row is converted to f16 as
+// code * scale (one rounding) on its way into shared memory; everything after the
+// staging is the f16 path.
+__device__ __forceinline__ uint4 fp8x16_to_half(uint4 codes, float scale, int half_index) {
+  // codes holds 16 e4m3 bytes; returns the 8 halves of bytes [8*half_index, 8*half_index+8)
+  const uint32_t w0 = half_index ? codes.z : codes.x, w1 = half_index ? codes.w : codes.y;
+  uint32_t r[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t w = j < 2 ? w0 : w1;
+    const __nv_fp8x2_storage_t pair = (__nv_fp8x2_storage_t)((w >> (16 * (j & 1))) & 0xffffu);
+    const float2 f = __half22float2(__half2(__nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3)));
+    const __half2 h = __floats2half2_rn(f.x * scale, f.y * scale);
+    r[j] = *reinterpret_cast<const uint32_t*>(&h);
+  }
+  return make_uint4(r[0], r[1], r[2], r[3]);
+}
+
+template <int D, int G, int CS, bool FROM_BLOCKS, bool FP8>
 __global__ void __launch_bounds__(kAcThreads, 1)
 attn_cluster_kernel(DevState* st, const __half* __restrict__ q, const int32_t* __restrict__ ids,
-                    const int32_t* __restrict__ n_ids, const __half* __restrict__ kc, const __half* __restrict__ vc,
-                    float* __restrict__ out, int n_kv_heads, int cells_per_cta, int max_cells, int k_blocks) {
+                    const int32_t* __restrict__ n_ids, const void* __restrict__ kc_raw,
+                    const void* __restrict__ vc_raw, float* __restrict__ out, int n_kv_heads, int cells_per_cta,
+                    int max_cells, int k_blocks, const float* __restrict__ kv_scales) {
+  const __half* __restrict__ kc = static_cast<const __half*>(kc_raw);
+  const __half* __restrict__ vc = static_cast<const __half*>(vc_raw);
   using SM = AcSmem<D, G>;
   constexpr int RS = SM::RS;
   constexpr int KSTEPS = D / 16;
@@ -408,11 +432,16 @@ attn_cluster_kernel(DevState* st, const __half* __restrict__ q, const int32_t* _
   const int g = blockIdx.x / CS;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int gq = lane >> 2, tq = lane & 3;  // MMA fragment row (query head) and column pair
+  const int u = blockIdx.y, n_back = gridDim.y - 1 - blockIdx.y;
+  q += size_t(u) * n_kv_heads * G * D;
+  out += size_t(u) * n_kv_heads * G * D;
+  ids += size_t(u) * (FROM_BLOCKS ? k_blocks : max_cells);
+  n_ids += u;
 
   pdl_launch_dependents();
   cluster_arrive_relaxed();  // paired with cluster_wait() before the partials are pushed
   pdl_wait();
-  const int n = ld_volatile(&st->n_ctx);
+  const int n_full = ld_volatile(&st->n_ctx);
   const int c0 = rank * Lc;
   // this thread's id, loaded in the same round trip as the counts (clamped into the id
   // buffer, checked against the counts below)
@@ -422,7 +451,12 @@ attn_cluster_kernel(DevState* st, const __half* __restrict__ q, const int32_t* _
     id_spec = FROM_BLOCKS ? ids[min(ci / kBlock, k_blocks - 1)] : ids[min(ci, max_cells - 1)];
   }
   const int n_ids_v = *n_ids;
-  asm volatile("" ::"r"(id_spec), "r"(n_ids_v), "r"(n));  // keep the loads ahead of the branches
+  asm volatile("" ::"r"(id_spec), "r"(n_ids_v), "r"(n_full));  // keep the loads ahead of the branches
+  int n = n_full - n_back;  // tokens this query sees
+  if (n < 0) {
+    if (rank == 0 && tid == 0) record_status(st, QSA_ERR_STATE);
+    n = 0;
+  }
   const int n_blocks = n / kBlock;
   int total, ns = 0;
   if constexpr (FROM_BLOCKS) {
@@ -464,12 +498,38 @@ attn_cluster_kernel(DevState* st, const __half* __restrict__ q, const int32_t* _
   }
   __syncthreads();
   // stage the selected K and V rows (rows of invalid or padding cells are zero-filled)
-  for (int e = tid; e < LP * CH; e += kAcThreads) {
-    const int i = e / CH, ch = e % CH;
-    const int cell = s_cell[i];
-    const size_t off = cell >= 0 ? ((size_t(cell) * n_kv_heads + g) * D + ch * 8) : 0;
-    cp_async_16(sK + size_t(i) * RS + ch * 8, kc + off, cell >= 0 ? 16 : 0);
-    cp_async_16(sV + size_t(i) * RS + ch * 8, vc + off, cell >= 0 ? 16 : 0);
+  if constexpr (!FP8) {
+    for (int e = tid; e < LP * CH; e += kAcThreads) {
+      const int i = e / CH, ch = e % CH;
+      const int cell = s_cell[i];
+      const size_t off = cell >= 0 ? ((size_t(cell) * n_kv_heads + g) * D + ch * 8) : 0;
+      cp_async_16(sK + size_t(i) * RS + ch * 8, kc + off, cell >= 0 ? 16 : 0);
+      cp_async_16(sV + size_t(i) * RS + ch * 8, vc + off, cell >= 0 ? 16 : 0);
+    }
+  } else {
+    // 16 e4m3 codes per 16-byte load; a row is D/16 of them
+    constexpr int CH8 = D / 16;
+    const unsigned char* kc8 = static_cast<const unsigned char*>(kc_raw);
+    const unsigned char* vc8 = static_cast<const unsigned char*>(vc_raw);
+#pragma unroll 2
+    for (int e = tid; e < LP * CH8; e += kAcThreads) {
+      const int i = e / CH8, ch = e % CH8;
+      const int cell = s_cell[i];
+      uint4 kq = make_uint4(0u, 0u, 0u, 0u), vq = kq;
+      float2 sc = make_float2(0.0f, 0.0f);
+      if (cell >= 0) {
+        const size_t row = size_t(cell) * n_kv_heads + g;
+        kq = *reinterpret_cast<const uint4*>(kc8 + row * D + ch * 16);
+        vq = *reinterpret_cast<const uint4*>(vc8 + row * D + ch * 16);
+        sc = *reinterpret_cast<const float2*>(kv_scales + row * 2);
+      }
+      __half* kd = sK + size_t(i) * RS + ch * 16;
+      __half* vd = sV + size_t(i) * RS + ch * 16;
+      *reinterpret_cast<uint4*>(kd) = fp8x16_to_half(kq, sc.x, 0);
+      *reinterpret_cast<uint4*>(kd + 8) = fp8x16_to_half(kq, sc.x, 1);
+      *reinterpret_cast<uint4*>(vd) = fp8x16_to_half(vq, sc.y, 0);
+      *reinterpret_cast<uint4*>(vd + 8) = fp8x16_to_half(vq, sc.y, 1);
+    }
   }
   // query fragments (A operand, rows = the G heads of KV head g, rows >= G zero)
   uint32_t qa[KSTEPS][2];
@@ -605,58 +665,68 @@ attn_cluster_kernel(DevState* st, const __half* __restrict__ q, const int32_t* _
   }
 }
 
+template <int D, int G, int CS, bool FB, bool FP8>
+static cudaError_t set_ac_attr1(size_t smem) {
+  cudaError_t e = cudaFuncSetAttribute(attn_cluster_kernel<D, G, CS, FB, FP8>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e == cudaSuccess && CS > 8)
+    e = cudaFuncSetAttribute(attn_cluster_kernel<D, G, CS, FB, FP8>, cudaFuncAttributeNonPortableClusterSizeAllowed,
+                             1);
+  return e;
+}
+
 template <int D, int G, int CS, bool FB>
 static cudaError_t set_ac_attr(size_t smem) {
-  cudaError_t e = cudaFuncSetAttribute(attn_cluster_kernel<D, G, CS, FB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
-  if (e == cudaSuccess && CS > 8)
-    e = cudaFuncSetAttribute(attn_cluster_kernel<D, G, CS, FB>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-  return e;
+  cudaError_t e = set_ac_attr1<D, G, CS, FB, false>(smem);
+  return e == cudaSuccess ? set_ac_attr1<D, G, CS, FB, true>(smem) : e;
 }
 
 template <int D, int G, int CS>
 static cudaError_t launch_ac(const LayerView& L, bool from_blocks, const void* q, const int32_t* ids,
-                             const int32_t* n_ids, float* out, cudaStream_t s) {
+                             const int32_t* n_ids, float* out, cudaStream_t s, int n_queries) {
   const int lc = L.attn_cells_per_cta;
   const size_t smem = AcSmem<D, G>::bytes(lc, CS);
-  const dim3 grid(L.cfg.n_kv_heads * CS), block(kAcThreads);
+  const dim3 grid(L.cfg.n_kv_heads * CS, n_queries), block(kAcThreads);
   const int mc = max_cells_of(L.cfg), kb = L.cfg.top_k_tokens / kBlock;
-  if (from_blocks)
-    return launch_pdl(attn_cluster_kernel<D, G, CS, true>, grid, block, smem, s, CS, L.state, (const __half*)q, ids,
-                      n_ids, (const __half*)L.k_cache, (const __half*)L.v_cache, out, L.cfg.n_kv_heads, lc, mc, kb);
-  return launch_pdl(attn_cluster_kernel<D, G, CS, false>, grid, block, smem, s, CS, L.state, (const __half*)q, ids,
-                    n_ids, (const __half*)L.k_cache, (const __half*)L.v_cache, out, L.cfg.n_kv_heads, lc, mc, kb);
+  const bool fp8 = L.cfg.kv_format == QSA_KV_FP8;
+  const float* scl = L.kv_scales;
+#define QSA_AC_LAUNCH(FB, F8)                                                                                    \
+  launch_pdl(attn_cluster_kernel<D, G, CS, FB, F8>, grid, block, smem, s, CS, L.state, (const __half*)q, ids, n_ids, \
+             (const void*)L.k_cache, (const void*)L.v_cache, out, L.cfg.n_kv_heads, lc, mc, kb, scl)
+  if (from_blocks) return fp8 ? QSA_AC_LAUNCH(true, true) : QSA_AC_LAUNCH(true, false);
+  return fp8 ? QSA_AC_LAUNCH(false, true) : QSA_AC_LAUNCH(false, false);
+#undef QSA_AC_LAUNCH
 }
 
 template <int D, int G>
 static cudaError_t launch_ac_g(const LayerView& L, bool fb, const void* q, const int32_t* ids, const int32_t* n_ids,
-                               float* out, cudaStream_t s) {
-  return L.attn_cluster == 16 ? launch_ac<D, G, 16>(L, fb, q, ids, n_ids, out, s)
-                              : launch_ac<D, G, 8>(L, fb, q, ids, n_ids, out, s);
+                               float* out, cudaStream_t s, int nq) {
+  return L.attn_cluster == 16 ? launch_ac<D, G, 16>(L, fb, q, ids, n_ids, out, s, nq)
+                              : launch_ac<D, G, 8>(L, fb, q, ids, n_ids, out, s, nq);
 }
 
 template <int D>
 static cudaError_t launch_ac_d(const LayerView& L, bool fb, const void* q, const int32_t* ids, const int32_t* n_ids,
-                               float* out, cudaStream_t s) {
+                               float* out, cudaStream_t s, int nq) {
   switch (L.cfg.n_q_heads / L.cfg.n_kv_heads) {
-    case 1: return launch_ac_g<D, 1>(L, fb, q, ids, n_ids, out, s);
-    case 2: return launch_ac_g<D, 2>(L, fb, q, ids, n_ids, out, s);
-    case 4: return launch_ac_g<D, 4>(L, fb, q, ids, n_ids, out, s);
-    case 8: return launch_ac_g<D, 8>(L, fb, q, ids, n_ids, out, s);
+    case 1: return launch_ac_g<D, 1>(L, fb, q, ids, n_ids, out, s, nq);
+    case 2: return launch_ac_g<D, 2>(L, fb, q, ids, n_ids, out, s, nq);
+    case 4: return launch_ac_g<D, 4>(L, fb, q, ids, n_ids, out, s, nq);
+    case 8: return launch_ac_g<D, 8>(L, fb, q, ids, n_ids, out, s, nq);
     default: return cudaErrorInvalidValue;
   }
 }
 
 cudaError_t launch_attend(const LayerView& L, const void* q, const int32_t* cells, const int32_t* n_cells, float* out,
                           cudaStream_t s) {
-  return L.cfg.head_dim == 128 ? launch_ac_d<128>(L, false, q, cells, n_cells, out, s)
-                               : launch_ac_d<64>(L, false, q, cells, n_cells, out, s);
+  return L.cfg.head_dim == 128 ? launch_ac_d<128>(L, false, q, cells, n_cells, out, s, 1)
+                               : launch_ac_d<64>(L, false, q, cells, n_cells, out, s, 1);
 }
 
 cudaError_t launch_attend_selected(const LayerView& L, const void* q, const int32_t* sel, const int32_t* n_sel,
-                                   float* out, cudaStream_t s) {
-  return L.cfg.head_dim == 128 ? launch_ac_d<128>(L, true, q, sel, n_sel, out, s)
-                               : launch_ac_d<64>(L, true, q, sel, n_sel, out, s);
+                                   float* out, cudaStream_t s, int n_queries) {
+  return L.cfg.head_dim == 128 ? launch_ac_d<128>(L, true, q, sel, n_sel, out, s, n_queries)
+                               : launch_ac_d<64>(L, true, q, sel, n_sel, out, s, n_queries);
 }
 
 // Cluster size and cells per CTA for a configuration, plus the kernel attributes they
@@ -687,8 +757,8 @@ static cudaError_t plan_ac_g(const qsa_config& c, int* cluster, int* lc) {
     cfg.attrs = &attr;
     cfg.numAttrs = 1;
     int active = 0;
-    e = cs == 16 ? cudaOccupancyMaxActiveClusters(&active, attn_cluster_kernel<D, G, 16, true>, &cfg)
-                 : cudaOccupancyMaxActiveClusters(&active, attn_cluster_kernel<D, G, 8, true>, &cfg);
+    e = cs == 16 ? cudaOccupancyMaxActiveClusters(&active, attn_cluster_kernel<D, G, 16, true, false>, &cfg)
+                 : cudaOccupancyMaxActiveClusters(&active, attn_cluster_kernel<D, G, 8, true, false>, &cfg);
     if (e != cudaSuccess) {
       cudaGetLastError();
       continue;

@@ -31,6 +31,24 @@ __device__ __forceinline__ void cluster_arrive_relaxed() {
 }
 __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
 
+// Rotation pair of element e of an indexer key or query whose first R dims are rotary
+// (Part 10, section "QSA indexer": RoPE at the block position). NeoX style pairs
+// (i, i + R/2), interleaved (GPT-J) style pairs (2i, 2i + 1); pair i turns by the angle
+// pos * base^(-2i/R). Output e = x[e] * cos + sign * x[partner] * sin, so the first element
+// of a pair takes sign -1 and the second +1. Elements e >= R are not rotated (freq < 0).
+struct RopeSlot {
+  int partner;
+  float sign;
+  int freq;
+};
+
+__host__ __device__ __forceinline__ RopeSlot rope_slot(int e, int R, bool interleaved) {
+  if (e >= R) return RopeSlot{e, 0.0f, -1};
+  if (interleaved) return RopeSlot{e ^ 1, (e & 1) ? 1.0f : -1.0f, e >> 1};
+  const int half = R / 2;
+  return e < half ? RopeSlot{e + half, -1.0f, e} : RopeSlot{e - half, 1.0f, e - half};
+}
+
 __device__ __forceinline__ void record_status(DevState* st, int code) {
   atomicCAS(&st->status, 0, code);
 }

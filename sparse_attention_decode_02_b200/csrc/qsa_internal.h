@@ -16,6 +16,7 @@ constexpr int kTopkCluster = 16;      // CTAs in the top-k cluster
 constexpr int kTopkThreads = 512;
 constexpr int kTopkMaxPerCta = kTopkThreads * 32;  // keys held in registers per top-k CTA
 constexpr int kTopkMaxK = kTopkThreads * 32 / kTopkCluster;  // largest top_k_tokens / 4 (1024)
+constexpr int kMaxQueries = 4;        // queries verified together by the multi-query calls
 constexpr int kAttnWarps = 8;         // warps per attention CTA
 constexpr int kAttnMaxCells = 64;     // cells per attention CTA (split size cap)
 
@@ -57,13 +58,16 @@ inline AttnSplit attn_split(const qsa_config& c, int n_sms) {
   return AttnSplit{l, (max_cells + l - 1) / l};
 }
 
+// Row stride (floats) of a multi-query score table: one row per query, 256-byte aligned.
+inline int score_stride_of(const qsa_config& c) { return (c.max_ctx / kBlock + 63) / 64 * 64; }
+
 inline WorkspaceLayout workspace_layout(const qsa_config& c, int n_splits) {
   WorkspaceLayout w{};
   size_t off = 0;
   w.state = off;
   off += align256(sizeof(DevState));
-  w.scores = off;
-  off += align256(size_t(c.max_ctx / kBlock) * sizeof(float));
+  w.scores = off;  // kMaxQueries rows of score_stride_of(c) floats
+  off += align256(size_t(kMaxQueries) * score_stride_of(c) * sizeof(float));
   w.part_o = off;
   off += align256(size_t(n_splits) * c.n_q_heads * c.head_dim * sizeof(float));
   w.part_ml = off;
@@ -80,6 +84,7 @@ struct LayerView {
   void* idx_cache;
   void* pooled_cache;
   const float* rms_gain;
+  float* kv_scales;       // [max_ctx][n_kv_heads][2] f32 with QSA_KV_FP8, else null
   DevState* state;
   float* scores;          // workspace scores
   float* part_o;
@@ -101,22 +106,25 @@ cudaError_t launch_append(const LayerView& L, int n, const void* k, const void* 
                           const void* idx, int grid_hint, cudaStream_t s);
 cudaError_t launch_pool_update(const LayerView& L, int grid_hint, cudaStream_t s);
 cudaError_t launch_decode_append(const LayerView& L, const void* k, const void* v, const void* idx, cudaStream_t s);
+// The index/top-k/attention launchers take n_queries T >= 1: query t (t < T) belongs to
+// token n_ctx - T + t and sees only the first n_ctx - T + t + 1 tokens. Per-query inputs
+// and outputs are consecutive rows (scores: rows of score_stride floats).
 cudaError_t launch_index_scan(const LayerView& L, const void* q_idx, const float* w,
-                              float* scores, cudaStream_t s);
+                              float* scores, cudaStream_t s, int n_queries = 1, int score_stride = 0);
 cudaError_t launch_topk(const LayerView& L, const float* scores, int32_t* sel, int32_t* n_sel,
-                        cudaStream_t s);
+                        cudaStream_t s, int n_queries = 1, int score_stride = 0);
 cudaError_t launch_gather(const LayerView& L, const int32_t* sel, const int32_t* n_sel,
                           int32_t* cells, int32_t* n_cells, void* k_compact, void* v_compact,
                           cudaStream_t s);
 cudaError_t launch_attend(const LayerView& L, const void* q, const int32_t* cells,
                           const int32_t* n_cells, float* out, cudaStream_t s);
 cudaError_t launch_attend_selected(const LayerView& L, const void* q, const int32_t* sel,
-                                   const int32_t* n_sel, float* out, cudaStream_t s);
+                                   const int32_t* n_sel, float* out, cudaStream_t s, int n_queries = 1);
 cudaError_t launch_attend_split(const LayerView& L, const void* q, const int32_t* cells,
                                 const int32_t* n_cells, float* out, cudaStream_t s);
 cudaError_t plan_attention(const qsa_config& c, int* cluster, int* cells_per_cta);
 
 // set_state modes
-enum { kSetReset = 0, kSetRestore = 1, kSetInvalidate = 2, kSetClearStatus = 3 };
+enum { kSetReset = 0, kSetRestore = 1, kSetInvalidate = 2, kSetClearStatus = 3, kSetRollback = 4 };
 
 }  // namespace qsa

@@ -3,7 +3,8 @@
 // Web page "Part 10" (第10回 EVO-X2 ... 長コンテキストのTGを高速化した話), section
 // "QSA indexer": the current indexer query is scored against every completed block's
 // pooled summary. This library's score (the pages give no formula):
-//    score_b = sum_h w_h * max(0, q~_h . p_b) / sqrt(d),   q~_h = RoPE(q_h, n-1).
+//    score_b = sum_h w_h * max(0, q~_h . p_b) / sqrt(d),   q~_h = RoPE(q_h, n-1)
+// (the query's RoPE follows the layer's rotary settings, like the pooled keys).
 //
 // The dots q~_h . p_b for all B blocks and H heads form a dense [B x d] . [d x H]
 // contraction over f16 pooled rows, which at d = 128, H = 16 needs 8 FMA per byte read:
@@ -30,28 +31,38 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kStages = 6;       // shared-memory ring of 128-row tiles
 constexpr int kAcc = 4;          // TMEM accumulators
 constexpr int kBoxRows = 16;     // TMA box height
 constexpr int kThreads = 192;    // warps 0-3 epilogue, warp 4 TMA, warp 5 MMA + TMEM owner
 constexpr float kLoScale = 4096.0f;
 
-template <int D, int H>
+constexpr size_t kSmemMax = 227 * 1024;  // dynamic shared memory per CTA
+
+// Shapes of the scan for d = D, H indexer heads and T queries scored in one pass.
+template <int D, int H, int T>
 struct ScanShape {
   static constexpr int HALVES = D / 64;                  // one 128-byte swizzle span = 64 f16
-  static constexpr int N = 2 * H < 16 ? 16 : 2 * H;      // MMA N: hi rows, lo rows, zero pad
+  static constexpr int NQ = 2 * H < 16 ? 16 : 2 * H;     // B rows per query: hi rows, lo rows, zero pad
+  static constexpr int N = T * NQ;                       // MMA N
   static constexpr int TILE_BYTES = 128 * D * 2;         // A tile: 128 rows
   static constexpr int HALF_BYTES = 128 * 128;           // 128 rows x 128 bytes
   static constexpr int B_HALF_BYTES = N * 128;
   static constexpr int B_BYTES = N * D * 2;
   static constexpr int ACC_COLS = kAcc * N;
-  static constexpr int TMEM_COLS = ACC_COLS <= 32 ? 32 : ACC_COLS <= 64 ? 64 : ACC_COLS <= 128 ? 128 : 256;
+  static constexpr int TMEM_COLS =
+      ACC_COLS <= 32 ? 32 : ACC_COLS <= 64 ? 64 : ACC_COLS <= 128 ? 128 : ACC_COLS <= 256 ? 256 : 512;
   static constexpr uint32_t IDESC = idesc_f16_f32(128, N);
-  // barriers and TMEM address (256 B), sin/cos (D floats), RoPE frequencies (D/2 doubles),
-  // raw query (H*D f16)
-  static constexpr int CTRL_BYTES = 256 + D * 4 + D / 2 * 8 + H * D * 2;
-  static constexpr size_t SMEM = 1024 + size_t(kStages) * TILE_BYTES + B_BYTES + CTRL_BYTES;
-  static_assert(N <= 32, "the epilogue reads at most 32 accumulator columns");
+  // barriers and TMEM address (256 B), sin/cos (T*D floats), RoPE frequencies (D/2
+  // doubles), raw queries (T*H*D f16)
+  static constexpr int CTRL_BYTES = 256 + T * D * 4 + D / 2 * 8 + T * H * D * 2;
+  static constexpr size_t FIXED = 1024 + size_t(B_BYTES) + CTRL_BYTES;
+  // ring depth: 6 tiles where they fit (all single-query shapes), fewer for wide B operands
+  static constexpr int STAGES = FIXED + 6 * size_t(TILE_BYTES) <= kSmemMax ? 6
+                                : FIXED + 5 * size_t(TILE_BYTES) <= kSmemMax ? 5 : 4;
+  static constexpr size_t SMEM = FIXED + size_t(STAGES) * TILE_BYTES;
+  static_assert(NQ <= 32, "the epilogue reads at most 32 accumulator columns per query");
+  static_assert(N <= 256 && ACC_COLS <= 512, "MMA N and TMEM columns");
+  static_assert(SMEM <= kSmemMax, "shared memory");
   static_assert(TILE_BYTES % 1024 == 0 && B_HALF_BYTES % 1024 == 0, "1024-byte swizzle atoms");
 };
 
@@ -65,12 +76,14 @@ __device__ __forceinline__ uint32_t sw128_offset(int n, int k, int half_bytes) {
 
 }  // namespace
 
-template <int D, int H>
+template <int D, int H, int T>
 __global__ void __launch_bounds__(kThreads, 1)
 index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_constant__ CUtensorMap map_box,
                      DevState* st, const __half* __restrict__ q_idx, const float* __restrict__ w,
-                     float* __restrict__ scores, float rope_base, int max_blocks) {
-  using S = ScanShape<D, H>;
+                     float* __restrict__ scores, float rope_base, int max_blocks, int rope_dims,
+                     int rope_interleaved, int rope_pos_stride, int score_stride) {
+  using S = ScanShape<D, H, T>;
+  constexpr int kStages = S::STAGES;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   unsigned char* sA = smem;
@@ -81,9 +94,9 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_
   uint64_t* tempty = tfull + kAcc;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tempty + kAcc);
   float* s_cos = reinterpret_cast<float*>(tmem_holder + 4);
-  float* s_sin = s_cos + D / 2;
-  double* s_theta = reinterpret_cast<double*>(s_sin + D / 2);         // D/2 doubles
-  __half* s_q = reinterpret_cast<__half*>(s_theta + D / 2);           // raw query, H x D
+  float* s_sin = s_cos + T * (D / 2);                                 // [T][D/2] each
+  double* s_theta = reinterpret_cast<double*>(s_sin + T * (D / 2));   // D/2 doubles
+  __half* s_q = reinterpret_cast<__half*>(s_theta + D / 2);           // raw queries, T x H x D
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   pdl_launch_dependents();
@@ -117,7 +130,8 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_
       for (int j = 0; j < S::HALVES; ++j) tma_prefetch_l2_2d(&map_tile, j * 64, r);
   }
   // RoPE frequencies do not depend on the previous kernel: compute them before waiting on it
-  for (int i = threadIdx.x; i < D / 2; i += blockDim.x) s_theta[i] = pow((double)rope_base, -2.0 * (double)i / (double)D);
+  for (int i = threadIdx.x; i < rope_dims / 2; i += blockDim.x)
+    s_theta[i] = pow((double)rope_base, -2.0 * (double)i / (double)rope_dims);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -200,44 +214,76 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_
     } else {
       // ---------------- warps 0-3: rotated, split query -> B operand; then epilogue ----------------
       const int tid = threadIdx.x;  // 0..127
-      // raw query: H*D f16 = H*D/8 16-byte vectors, all loads in flight at once
-      constexpr int QV = H * D / 8;
+      // raw queries: T*H*D f16 = T*H*D/8 16-byte vectors, all loads in flight at once
+      constexpr int QV = T * H * D / 8;
       uint4 qraw[(QV + 127) / 128];
 #pragma unroll
       for (int k = 0; k < (QV + 127) / 128; ++k)
         if (tid + k * 128 < QV) qraw[k] = reinterpret_cast<const uint4*>(q_idx)[tid + k * 128];
-      for (int i = tid; i < D / 2; i += 128) {
+      // query u belongs to token n - T + u: on the block-position scale it sits at
+      // floor(stride * (n_u - 1) / 4), n_u = n - T + u + 1 (token n_u - 1 when stride = 4)
+      const int half_r = rope_dims / 2;
+      for (int i = tid; i < T * half_r; i += 128) {
+        const int u = i / half_r, f = i % half_r;
+        const int n_u = n - (T - 1 - u);
+        const double qpos = n_u > 0 ? (double)(((long long)rope_pos_stride * (n_u - 1)) / kBlock) : 0.0;
         double sd, cd;
-        sincos((double)(n - 1) * s_theta[i], &sd, &cd);
-        s_cos[i] = (float)cd;
-        s_sin[i] = (float)sd;
+        sincos(qpos * s_theta[f], &sd, &cd);
+        s_cos[u * (D / 2) + f] = (float)cd;
+        s_sin[u * (D / 2) + f] = (float)sd;
       }
 #pragma unroll
       for (int k = 0; k < (QV + 127) / 128; ++k)
         if (tid + k * 128 < QV) reinterpret_cast<uint4*>(s_q)[tid + k * 128] = qraw[k];
       named_bar_sync(2, 128);
-      for (int e = tid; e < H * (D / 2); e += 128) {
-        const int h = e / (D / 2), i = e % (D / 2);
-        const float x1 = __half2float(s_q[h * D + i]);
-        const float x2 = __half2float(s_q[h * D + i + D / 2]);
-        const float r1 = x1 * s_cos[i] - x2 * s_sin[i];
-        const float r2 = x1 * s_sin[i] + x2 * s_cos[i];
-        const __half h1 = __float2half_rn(r1), h2 = __float2half_rn(r2);
-        const __half l1 = __float2half_rn((r1 - __half2float(h1)) * kLoScale);
-        const __half l2 = __float2half_rn((r2 - __half2float(h2)) * kLoScale);
-        *reinterpret_cast<__half*>(sB + sw128_offset(h, i, S::B_HALF_BYTES)) = h1;
-        *reinterpret_cast<__half*>(sB + sw128_offset(h, i + D / 2, S::B_HALF_BYTES)) = h2;
-        *reinterpret_cast<__half*>(sB + sw128_offset(H + h, i, S::B_HALF_BYTES)) = l1;
-        *reinterpret_cast<__half*>(sB + sw128_offset(H + h, i + D / 2, S::B_HALF_BYTES)) = l2;
+      // rotated element e of head h of query u -> high f16 part in B row u*NQ + h, scaled
+      // residual in row u*NQ + H + h
+      auto put = [&](int u, int h, int e, float r) {
+        const __half hi = __float2half_rn(r);
+        const __half lo = __float2half_rn((r - __half2float(hi)) * kLoScale);
+        *reinterpret_cast<__half*>(sB + sw128_offset(u * S::NQ + h, e, S::B_HALF_BYTES)) = hi;
+        *reinterpret_cast<__half*>(sB + sw128_offset(u * S::NQ + H + h, e, S::B_HALF_BYTES)) = lo;
+      };
+      if (rope_dims == D && !rope_interleaved) {  // NeoX pairs (i, i + D/2) over all dims
+        for (int e = tid; e < T * H * (D / 2); e += 128) {
+          const int uh = e / (D / 2), i = e % (D / 2);
+          const int u = uh / H, h = uh % H;
+          const __half* x = s_q + uh * D;
+          const float c = s_cos[u * (D / 2) + i], sn = s_sin[u * (D / 2) + i];
+          const float x1 = __half2float(x[i]);
+          const float x2 = __half2float(x[i + D / 2]);
+          put(u, h, i, x1 * c - x2 * sn);
+          put(u, h, i + D / 2, x1 * sn + x2 * c);
+        }
+      } else {  // partial rotary or interleaved pairs: one element at a time
+        for (int e = tid; e < T * H * D; e += 128) {
+          const int uh = e / D, k = e % D;
+          const int u = uh / H, h = uh % H;
+          const __half* x = s_q + uh * D;
+          const RopeSlot sl = rope_slot(k, rope_dims, rope_interleaved != 0);
+          const float xk = __half2float(x[k]);
+          float r = xk;
+          if (sl.freq >= 0)
+            r = xk * s_cos[u * (D / 2) + sl.freq] + sl.sign * __half2float(x[sl.partner]) * s_sin[u * (D / 2) + sl.freq];
+          put(u, h, k, r);
+        }
       }
-      for (int e = tid; e < (S::N - 2 * H) * D; e += 128)
-        *reinterpret_cast<__half*>(sB + sw128_offset(2 * H + e / D, e % D, S::B_HALF_BYTES)) = __float2half_rn(0.0f);
+      constexpr int PAD = S::NQ - 2 * H;  // zero rows after each query's hi and lo rows
+      if constexpr (PAD > 0) {
+        for (int e = tid; e < T * PAD * D; e += 128) {
+          const int u = e / (PAD * D), rem = e % (PAD * D);
+          *reinterpret_cast<__half*>(sB + sw128_offset(u * S::NQ + 2 * H + rem / D, rem % D, S::B_HALF_BYTES)) =
+              __float2half_rn(0.0f);
+        }
+      }
       fence_proxy_async_smem();
       named_bar_sync(1, 160);
 
-      float wr[H];
+      float wr[T][H];
 #pragma unroll
-      for (int h = 0; h < H; ++h) wr[h] = w[h];
+      for (int u = 0; u < T; ++u)
+#pragma unroll
+        for (int h = 0; h < H; ++h) wr[u][h] = w[u * H + h];
       const float sqrt_d = sqrtf((float)D);
       bool ok = true;
       for (int t = 0; t < n_tiles; ++t) {
@@ -245,28 +291,25 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_
         if (!mbar_wait(&tfull[a], (t / kAcc) & 1)) { ok = false; break; }
         tc_fence_after();
         const uint32_t taddr = tmem_base + (uint32_t(32 * warp) << 16) + uint32_t(a * S::N);
-        float acc[32];
-        if constexpr (S::N == 32) {
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(taddr, r);
-          tmem_ld_wait();
+        uint32_t r[T][S::NQ];  // query u's columns [u*NQ, (u+1)*NQ) of this row
 #pragma unroll
-          for (int c = 0; c < 32; ++c) acc[c] = __uint_as_float(r[c]);
-        } else {
-          uint32_t r[16];
-          tmem_ld_32x32b_x16(taddr, r);
-          tmem_ld_wait();
-#pragma unroll
-          for (int c = 0; c < 16; ++c) acc[c] = __uint_as_float(r[c]);
+        for (int u = 0; u < T; ++u) {
+          if constexpr (S::NQ == 32) tmem_ld_32x32b_x32(taddr + uint32_t(u * S::NQ), r[u]);
+          else tmem_ld_32x32b_x16(taddr + uint32_t(u * S::NQ), r[u]);
         }
+        tmem_ld_wait();
         tc_fence_before();
         mbar_arrive(&tempty[a]);
         const int row = r0 + t * 128 + tid;
         if (row < r1) {
-          float s = 0.0f;
 #pragma unroll
-          for (int h = 0; h < H; ++h) s += wr[h] * fmaxf(acc[h] + acc[H + h] * (1.0f / kLoScale), 0.0f);
-          scores[row] = s / sqrt_d;
+          for (int u = 0; u < T; ++u) {
+            float s = 0.0f;
+#pragma unroll
+            for (int h = 0; h < H; ++h)
+              s += wr[u][h] * fmaxf(__uint_as_float(r[u][h]) + __uint_as_float(r[u][H + h]) * (1.0f / kLoScale), 0.0f);
+            scores[size_t(u) * score_stride + row] = s / sqrt_d;
+          }
         }
       }
       if (!ok && tid == 0) record_status(st, QSA_ERR_TIMEOUT);
@@ -283,18 +326,28 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_
 // ---------------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------------
-template <int D, int H>
+template <int D, int H, int T>
 static cudaError_t set_scan_attr() {
-  return cudaFuncSetAttribute(index_scan_tc_kernel<D, H>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              (int)ScanShape<D, H>::SMEM);
+  return cudaFuncSetAttribute(index_scan_tc_kernel<D, H, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)ScanShape<D, H, T>::SMEM);
+}
+
+template <int D, int H>
+static cudaError_t set_scan_attr_t() {
+  cudaError_t e;
+  if ((e = set_scan_attr<D, H, 1>()) != cudaSuccess || (e = set_scan_attr<D, H, 2>()) != cudaSuccess ||
+      (e = set_scan_attr<D, H, 3>()) != cudaSuccess || (e = set_scan_attr<D, H, 4>()) != cudaSuccess)
+    return e;
+  return cudaSuccess;
 }
 
 cudaError_t init_scan_attributes() {
+  static_assert(kMaxQueries == 4, "one scan instantiation per query count");
   cudaError_t e = cudaSuccess;
-#define QSA_SCAN_ATTR(DD)                                                                             \
-  if ((e = set_scan_attr<DD, 1>()) != cudaSuccess || (e = set_scan_attr<DD, 2>()) != cudaSuccess ||   \
-      (e = set_scan_attr<DD, 4>()) != cudaSuccess || (e = set_scan_attr<DD, 8>()) != cudaSuccess ||   \
-      (e = set_scan_attr<DD, 16>()) != cudaSuccess)                                                   \
+#define QSA_SCAN_ATTR(DD)                                                                                 \
+  if ((e = set_scan_attr_t<DD, 1>()) != cudaSuccess || (e = set_scan_attr_t<DD, 2>()) != cudaSuccess ||   \
+      (e = set_scan_attr_t<DD, 4>()) != cudaSuccess || (e = set_scan_attr_t<DD, 8>()) != cudaSuccess ||   \
+      (e = set_scan_attr_t<DD, 16>()) != cudaSuccess)                                                     \
     return e;
   QSA_SCAN_ATTR(64)
   QSA_SCAN_ATTR(128)
@@ -328,30 +381,44 @@ cudaError_t encode_pooled_map(const qsa_config& c, void* pooled, int box_rows, C
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-template <int D>
-static cudaError_t launch_scan_tc_d(const LayerView& L, const void* q_idx, const float* w, float* scores,
-                                    cudaStream_t s) {
-  const dim3 grid(L.n_sms), block(kThreads);
-  const float base = L.cfg.rope_base;
-#define QSA_SCAN_CASE(HH)                                                                                  \
-  case HH:                                                                                                 \
-    return launch_pdl(index_scan_tc_kernel<D, HH>, grid, block, ScanShape<D, HH>::SMEM, s, 1, L.pooled_tile_map, \
-                      L.pooled_box_map, L.state, (const __half*)q_idx, w, scores, base, L.cfg.max_ctx / kBlock);
-  switch (L.cfg.n_idx_heads) {
-    QSA_SCAN_CASE(1)
-    QSA_SCAN_CASE(2)
-    QSA_SCAN_CASE(4)
-    QSA_SCAN_CASE(8)
-    QSA_SCAN_CASE(16)
+template <int D, int H, int T>
+static cudaError_t launch_scan_tc(const LayerView& L, const void* q_idx, const float* w, float* scores,
+                                  cudaStream_t s, int score_stride) {
+  return launch_pdl(index_scan_tc_kernel<D, H, T>, dim3(L.n_sms), dim3(kThreads), ScanShape<D, H, T>::SMEM, s, 1,
+                    L.pooled_tile_map, L.pooled_box_map, L.state, (const __half*)q_idx, w, scores, L.cfg.rope_base,
+                    L.cfg.max_ctx / kBlock, L.cfg.rope_dims, L.cfg.rope_interleaved, L.cfg.rope_pos_stride,
+                    score_stride);
+}
+
+template <int D, int H>
+static cudaError_t launch_scan_tc_t(const LayerView& L, const void* q_idx, const float* w, float* scores,
+                                    cudaStream_t s, int n_queries, int score_stride) {
+  switch (n_queries) {
+    case 1: return launch_scan_tc<D, H, 1>(L, q_idx, w, scores, s, score_stride);
+    case 2: return launch_scan_tc<D, H, 2>(L, q_idx, w, scores, s, score_stride);
+    case 3: return launch_scan_tc<D, H, 3>(L, q_idx, w, scores, s, score_stride);
+    case 4: return launch_scan_tc<D, H, 4>(L, q_idx, w, scores, s, score_stride);
     default: return cudaErrorInvalidValue;
   }
-#undef QSA_SCAN_CASE
+}
+
+template <int D>
+static cudaError_t launch_scan_tc_d(const LayerView& L, const void* q_idx, const float* w, float* scores,
+                                    cudaStream_t s, int n_queries, int score_stride) {
+  switch (L.cfg.n_idx_heads) {
+    case 1: return launch_scan_tc_t<D, 1>(L, q_idx, w, scores, s, n_queries, score_stride);
+    case 2: return launch_scan_tc_t<D, 2>(L, q_idx, w, scores, s, n_queries, score_stride);
+    case 4: return launch_scan_tc_t<D, 4>(L, q_idx, w, scores, s, n_queries, score_stride);
+    case 8: return launch_scan_tc_t<D, 8>(L, q_idx, w, scores, s, n_queries, score_stride);
+    case 16: return launch_scan_tc_t<D, 16>(L, q_idx, w, scores, s, n_queries, score_stride);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 cudaError_t launch_index_scan(const LayerView& L, const void* q_idx, const float* w, float* scores,
-                              cudaStream_t s) {
-  return L.cfg.d_idx == 128 ? launch_scan_tc_d<128>(L, q_idx, w, scores, s)
-                            : launch_scan_tc_d<64>(L, q_idx, w, scores, s);
+                              cudaStream_t s, int n_queries, int score_stride) {
+  return L.cfg.d_idx == 128 ? launch_scan_tc_d<128>(L, q_idx, w, scores, s, n_queries, score_stride)
+                            : launch_scan_tc_d<64>(L, q_idx, w, scores, s, n_queries, score_stride);
 }
 
 }  // namespace qsa

@@ -1,6 +1,5 @@
 // Block-domain top-k as a device routine run by one cluster of kTopkCluster CTAs of
-// kTopkThreads threads. Used by the stand-alone selection kernel (qsa_index.cu) and by
-// the attention kernel that selects and attends in one launch (qsa_attend.cu).
+// kTopkThreads threads (used by the selection kernel in qsa_index.cu).
 //
 // Web page "Part 10" (第10回 EVO-X2 ... 長コンテキストのTGを高速化した話):
 //  - section "QSA indexer": the high-scoring blocks are chosen by top-k;
@@ -83,12 +82,14 @@ struct Result {
 };
 
 // Preconditions: every thread of the cluster executed cluster_arrive_relaxed() and then
-// pdl_wait(). Calls emit(position, block) once per selected block (kTopK only) and
-// returns the same result in every thread of the cluster. Cluster-barrier pairing is
-// complete on return on every path.
+// pdl_wait(). Selects among the blocks completed within the first n_ctx - n_back tokens
+// (n_back > 0: a query of an earlier token of a multi-query step). Calls
+// emit(position, block) once per selected block (kTopK only) and returns the same result
+// in every thread of the cluster. Cluster-barrier pairing is complete on return on every
+// path.
 template <int V, class Emit>
 __device__ __forceinline__ Result cluster_select(DevState* st, const float* __restrict__ scores, int k_blocks,
-                                                 int max_blocks, Emit&& emit) {
+                                                 int max_blocks, int n_back, Emit&& emit) {
   __shared__ uint32_t s_hist[256];          // this CTA's histogram of the pass
   __shared__ uint32_t s_in[2][kCS][256];    // every CTA's histogram, double-buffered by pass
   __shared__ uint32_t s_warp[32];
@@ -116,15 +117,16 @@ __device__ __forceinline__ Result cluster_select(DevState* st, const float* __re
 #pragma unroll
     for (int j = 0; j < V; ++j) f[j] = base + j < max_blocks ? scores[base + j] : 0.0f;
   }
-  const int n = ld_volatile(&st->n_ctx);
+  const int n_full = ld_volatile(&st->n_ctx);
   const int n_pooled = ld_volatile(&st->n_pooled);
 #pragma unroll
   for (int j = 0; j < V; ++j) asm volatile("" ::"f"(f[j]));  // keep the loads ahead of the branches
+  const int n = n_full - n_back;
   const int n_blocks = n / kBlock;
-  if (n_pooled != n_blocks) {  // uniform over the cluster
+  if (n_pooled != n_full / kBlock || n < 0) {  // uniform over the cluster
     if (rank == 0 && tid == 0) record_status(st, QSA_ERR_STATE);
     cluster_wait();
-    return Result{kStale, n, n_blocks};
+    return Result{kStale, n, 0};
   }
   if (n_blocks <= k_blocks) {  // uniform over the cluster
     cluster_wait();

@@ -18,7 +18,10 @@ QSA_OK = 0
 STATUS_NAMES = {0: "QSA_OK", 1: "QSA_ERR_INVALID_ARG", 2: "QSA_ERR_CAPACITY", 3: "QSA_ERR_STATE",
                 4: "QSA_ERR_CUDA", 5: "QSA_ERR_UNSUPPORTED", 6: "QSA_ERR_BAD_INDEX",
                 7: "QSA_ERR_TIMEOUT"}
-QSA_BUF_KV, QSA_BUF_IDX, QSA_BUF_POOLED, QSA_BUF_WORKSPACE, QSA_BUF_MAX_CELLS = range(5)
+(QSA_BUF_KV, QSA_BUF_IDX, QSA_BUF_POOLED, QSA_BUF_WORKSPACE, QSA_BUF_MAX_CELLS, QSA_BUF_SCORE_STRIDE,
+ QSA_BUF_KV_SCALES) = range(7)
+QSA_KV_F16, QSA_KV_FP8 = 0, 1
+QSA_MAX_QUERIES = 4
 
 
 class QsaError(RuntimeError):
@@ -31,12 +34,14 @@ class QsaConfig(ctypes.Structure):
     _fields_ = [("n_layers", c_int32), ("max_ctx", c_int32), ("d_idx", c_int32),
                 ("n_idx_heads", c_int32), ("top_k_tokens", c_int32), ("n_q_heads", c_int32),
                 ("n_kv_heads", c_int32), ("head_dim", c_int32), ("rope_base", c_float),
-                ("rms_eps", c_float)]
+                ("rms_eps", c_float), ("rope_dims", c_int32), ("rope_interleaved", c_int32),
+                ("rope_pos_stride", c_int32), ("rope_pos_offset", c_int32), ("kv_format", c_int32)]
 
 
 class QsaLayerBuffers(ctypes.Structure):
     _fields_ = [("k_cache", c_void_p), ("v_cache", c_void_p), ("idx_cache", c_void_p),
-                ("pooled_cache", c_void_p), ("rms_gain", c_void_p), ("workspace", c_void_p)]
+                ("pooled_cache", c_void_p), ("rms_gain", c_void_p), ("workspace", c_void_p),
+                ("kv_scales", c_void_p)]
 
 
 _P = c_void_p
@@ -62,6 +67,9 @@ SIGNATURES = {
     "qsa_sparse_attend": (_I, [_P, _I, _P, _P, _P, _P, _P]),
     "qsa_sparse_attend_selected": (_I, [_P, _I, _P, _P, _P, _P, _P]),
     "qsa_sparse_attend_noalloc": (_I, [_P, _P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _P]),
+    "qsa_index_topk_multi": (_I, [_P, _I, _I, _P, _P, _P, _P, _P, _P]),
+    "qsa_sparse_attend_selected_multi": (_I, [_P, _I, _I, _P, _P, _P, _P, _P]),
+    "qsa_rollback": (_I, [_P, _I, _I, _P]),
 }
 
 _lib = None
@@ -104,9 +112,11 @@ def _stream(stream):
 
 
 def make_config(n_layers, max_ctx, d_idx, n_idx_heads, top_k_tokens, n_q_heads, n_kv_heads, head_dim,
-                rope_base=10000.0, rms_eps=1e-6) -> QsaConfig:
+                rope_base=10000.0, rms_eps=1e-6, rope_dims=0, rope_interleaved=False, rope_pos_stride=4,
+                rope_pos_offset=0, kv_format=QSA_KV_F16) -> QsaConfig:
     return QsaConfig(n_layers, max_ctx, d_idx, n_idx_heads, top_k_tokens, n_q_heads, n_kv_heads, head_dim,
-                     rope_base, rms_eps)
+                     rope_base, rms_eps, rope_dims, int(bool(rope_interleaved)), rope_pos_stride, rope_pos_offset,
+                     kv_format)
 
 
 def buffer_bytes(cfg: QsaConfig, which: int) -> int:
@@ -145,9 +155,9 @@ class Qsa:
         return buffer_bytes(self.cfg, which)
 
     def bind_layer(self, layer, k_cache, v_cache, idx_cache, pooled_cache, workspace, rms_gain=None,
-                   stream=None):
+                   kv_scales=None, stream=None):
         b = QsaLayerBuffers(_ptr(k_cache), _ptr(v_cache), _ptr(idx_cache), _ptr(pooled_cache),
-                            _ptr(rms_gain), _ptr(workspace))
+                            _ptr(rms_gain), _ptr(workspace), _ptr(kv_scales))
         self._check(self.lib.qsa_bind_layer(self.handle, layer, ctypes.byref(b), _stream(stream)))
 
     def restore_layer(self, layer, n_ctx, n_pooled, stream=None):
@@ -201,6 +211,19 @@ class Qsa:
         self._check(self.lib.qsa_sparse_attend(self.handle, layer, _ptr(q), _ptr(cells), _ptr(n_cells),
                                                _ptr(out), _stream(stream)))
 
+    def index_topk_multi(self, layer, q_idx, w, sel_blocks, n_sel, scores=None, stream=None):
+        """T = q_idx.shape[0] queries (the last T tokens) in one scan and one selection."""
+        self._check(self.lib.qsa_index_topk_multi(self.handle, layer, int(q_idx.shape[0]), _ptr(q_idx), _ptr(w),
+                                                  _ptr(sel_blocks), _ptr(n_sel), _ptr(scores), _stream(stream)))
+
+    def sparse_attend_selected_multi(self, layer, q, sel_blocks, n_sel, out, stream=None):
+        self._check(self.lib.qsa_sparse_attend_selected_multi(self.handle, layer, int(q.shape[0]), _ptr(q),
+                                                              _ptr(sel_blocks), _ptr(n_sel), _ptr(out),
+                                                              _stream(stream)))
+
+    def rollback(self, layer, n_keep, stream=None):
+        self._check(self.lib.qsa_rollback(self.handle, layer, int(n_keep), _stream(stream)))
+
 
 def sparse_attend_noalloc(q, k_cache, v_cache, n_ctx, cells, n_cells, out, n_q_heads, n_kv_heads, head_dim,
                           top_k_tokens, stream=None):
@@ -214,17 +237,35 @@ def sparse_attend_noalloc(q, k_cache, v_cache, n_ctx, cells, n_cells, out, n_q_h
 
 
 def alloc_layer(cfg: QsaConfig, device="cuda"):
-    """Allocate one layer's buffers with torch (the caller owns them)."""
+    """Allocate one layer's buffers with torch (the caller owns them). With QSA_KV_FP8 the
+    K/V caches are uint8 e4m3 codes and `kv_scales` holds the per-row K and V scales."""
     import torch
-    kv_elems = buffer_bytes(cfg, QSA_BUF_KV) // 2
-    return {
-        "k_cache": torch.zeros(kv_elems, dtype=torch.float16, device=device).view(
-            cfg.max_ctx, cfg.n_kv_heads, cfg.head_dim),
-        "v_cache": torch.zeros(kv_elems, dtype=torch.float16, device=device).view(
-            cfg.max_ctx, cfg.n_kv_heads, cfg.head_dim),
+    fp8 = cfg.kv_format == QSA_KV_FP8
+    kv_dtype = torch.uint8 if fp8 else torch.float16
+    shape = (cfg.max_ctx, cfg.n_kv_heads, cfg.head_dim)
+    bufs = {
+        "k_cache": torch.zeros(shape, dtype=kv_dtype, device=device),
+        "v_cache": torch.zeros(shape, dtype=kv_dtype, device=device),
         "idx_cache": torch.zeros(cfg.max_ctx, cfg.d_idx, dtype=torch.float16, device=device),
         "pooled_cache": torch.zeros(cfg.max_ctx // 4, cfg.d_idx, dtype=torch.float16, device=device),
         "workspace": torch.zeros(buffer_bytes(cfg, QSA_BUF_WORKSPACE), dtype=torch.uint8, device=device),
+    }
+    assert bufs["k_cache"].numel() * bufs["k_cache"].element_size() == buffer_bytes(cfg, QSA_BUF_KV)
+    if fp8:
+        bufs["kv_scales"] = torch.zeros(cfg.max_ctx, cfg.n_kv_heads, 2, dtype=torch.float32, device=device)
+    return bufs
+
+
+def alloc_multi_outputs(cfg: QsaConfig, n_queries: int, device="cuda"):
+    """Outputs of a multi-query step: per-query selections, counts, scores and attention."""
+    import torch
+    k_blocks = cfg.top_k_tokens // 4
+    return {
+        "sel": torch.zeros(n_queries, k_blocks, dtype=torch.int32, device=device),
+        "n_sel": torch.zeros(n_queries, dtype=torch.int32, device=device),
+        "scores": torch.zeros(n_queries, buffer_bytes(cfg, QSA_BUF_SCORE_STRIDE), dtype=torch.float32,
+                              device=device),
+        "out": torch.zeros(n_queries, cfg.n_q_heads, cfg.head_dim, dtype=torch.float32, device=device),
     }
 
 

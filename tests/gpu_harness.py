@@ -23,10 +23,11 @@ def ensure_library():
     return Q.load_library()
 
 
-def config_of(wl: synth.Workload, max_ctx=None, n_layers=1, top_k_tokens=None) -> Q.QsaConfig:
+def config_of(wl: synth.Workload, max_ctx=None, n_layers=1, top_k_tokens=None, **rope) -> Q.QsaConfig:
+    """Library config of a workload; `rope` takes the rope_* switches of make_config."""
     return Q.make_config(n_layers, max_ctx or wl.max_ctx, wl.d_idx, wl.n_idx_heads,
                          top_k_tokens or wl.top_k_tokens, wl.n_q_heads, wl.n_kv_heads, wl.head_dim,
-                         wl.rope_base, wl.rms_eps)
+                         wl.rope_base, wl.rms_eps, **rope)
 
 
 def to_dev(a, dtype=None):

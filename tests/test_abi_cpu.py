@@ -53,16 +53,55 @@ def test_buffer_sizes(lib):
     dict(head_dim=256), dict(n_q_heads=32, n_kv_heads=2), dict(max_ctx=1026), dict(max_ctx=4 << 20),
     dict(top_k_tokens=4096), dict(top_k_tokens=0),
     dict(n_layers=0),
+    dict(rope_dims=33), dict(rope_dims=130), dict(rope_dims=-2), dict(rope_interleaved=2),
+    dict(rope_pos_stride=17), dict(rope_pos_stride=-1), dict(rope_pos_offset=-1),
+    dict(rope_pos_offset=(1 << 20) + 1),
 ])
 def test_unsupported_configs_are_rejected(lib, bad):
     base = dict(n_layers=1, max_ctx=4096, d_idx=128, n_idx_heads=16, top_k_tokens=2048, n_q_heads=32,
                 n_kv_heads=4, head_dim=128)
-    base.update(bad)
-    cfg = Q.make_config(**base)
+    cfg = Q.make_config(**{**base, **{k: v for k, v in bad.items() if k in base}})
+    for k, v in bad.items():  # raw struct fields, past the binding's own conversions
+        setattr(cfg, k, v)
     assert Q.buffer_bytes(cfg, Q.QSA_BUF_KV) == 0
     h = ctypes.c_void_p()
     assert lib.qsa_create(ctypes.byref(cfg), ctypes.byref(h)) == 5  # QSA_ERR_UNSUPPORTED
     assert not h.value
+
+
+def test_config_struct_matches_header():
+    import re
+    with open(os.path.join(ROOT, "include", "qsa.h")) as f:
+        text = f.read()
+    body = re.search(r"typedef struct \{(.*?)\} qsa_config;", text, re.S).group(1)
+    body = re.sub(r"/\*.*?\*/", "", body, flags=re.S)
+    fields = re.findall(r"(int32_t|float)\s+(\w+);", body)
+    ctype = {"int32_t": ctypes.c_int32, "float": ctypes.c_float}
+    assert [(n, ctype[t]) for t, n in fields] == list(Q.QsaConfig._fields_)
+
+
+def test_buffers_struct_matches_header():
+    import re
+    with open(os.path.join(ROOT, "include", "qsa.h")) as f:
+        text = f.read()
+    body = re.search(r"typedef struct \{([^{}]*?)\} qsa_layer_buffers;", text, re.S).group(1)
+    body = re.sub(r"/\*.*?\*/", "", body, flags=re.S)
+    names = re.findall(r"\*\s*(\w+);", body)
+    assert names == [n for n, _ in Q.QsaLayerBuffers._fields_]
+    assert all(t is ctypes.c_void_p for _, t in Q.QsaLayerBuffers._fields_)
+
+
+def test_fp8_buffer_sizes(lib):
+    cfg = Q.make_config(1, 4096, 128, 16, 2048, 32, 4, 128, kv_format=Q.QSA_KV_FP8)
+    assert Q.buffer_bytes(cfg, Q.QSA_BUF_KV) == 4096 * 4 * 128
+    assert Q.buffer_bytes(cfg, Q.QSA_BUF_KV_SCALES) == 4096 * 4 * 2 * 4
+    f16 = Q.make_config(1, 4096, 128, 16, 2048, 32, 4, 128)
+    assert Q.buffer_bytes(f16, Q.QSA_BUF_KV) == 2 * Q.buffer_bytes(cfg, Q.QSA_BUF_KV)
+    assert Q.buffer_bytes(f16, Q.QSA_BUF_KV_SCALES) == 0
+    assert Q.buffer_bytes(cfg, Q.QSA_BUF_SCORE_STRIDE) == 1024
+    bad = Q.make_config(1, 4096, 128, 16, 2048, 32, 4, 128)
+    bad.kv_format = 2
+    assert Q.buffer_bytes(bad, Q.QSA_BUF_KV) == 0
 
 
 def test_null_arguments_are_rejected(lib):

@@ -531,3 +531,25 @@ def test_kv_row_quantization_closed_forms():
     x = rows.astype(np.float64)
     bound = np.maximum(np.abs(x) * 2.0 ** -4, 2.0 ** -10 * scales[..., None])
     assert np.all(np.abs(deq - x) <= bound * (1 + 1e-6))
+
+
+def test_fp8_layer_is_exact_on_e4m3_grid_rows():
+    """Rows whose values lie on the e4m3 grid and whose largest magnitude is 448 quantise
+    with scale 1 and no rounding, so the FP8 layer attends exactly like the f16 layer."""
+    rng = np.random.default_rng(43)
+    shape = SMALL
+    grid = np.array([O.e4m3_value(c) for c in range(256) if not np.isnan(O.e4m3_value(c))])
+    grid = grid[np.abs(grid) <= 8]
+    n = 37
+    k = rng.choice(grid, (n, shape.n_kv_heads, shape.head_dim)).astype(np.float16)
+    v = rng.choice(grid, (n, shape.n_kv_heads, shape.head_dim)).astype(np.float16)
+    k[:, :, 0] = 448.0
+    v[:, :, 3] = -448.0
+    idx = rng.standard_normal((n, shape.d_idx)).astype(np.float16)
+    a, b = O.OracleLayer(shape, 64), O.OracleLayer(shape, 64, kv_fp8=True)
+    for L in (a, b):
+        L.append_tokens(k, v, idx)
+    assert np.all(b.kv_scales[:n] == 1.0)
+    q = rng.standard_normal((shape.n_q_heads, shape.head_dim)).astype(np.float16) * 0.01
+    cells = np.arange(n)
+    np.testing.assert_array_equal(a.attend(q, cells), b.attend(q, cells))
