@@ -425,3 +425,49 @@ def test_decode_append_equals_append_then_update():
     assert ga.state() == gb.state() and ga.state()[1] == ga.state()[0] // 4
     n = ga.state()[0]
     np.testing.assert_array_equal(ga.pooled_rows(0, n // 4), gb.pooled_rows(0, n // 4))
+
+
+@pytest.mark.slow
+def test_streaming_512_steps_12_layers():
+    """The streaming workload: from the 256k prefill, 512 fused decode steps on each of the 12
+    layers (128 block completions per layer). Every 128 steps the live pooled cache equals a
+    full rebuild bit for bit; at steps 0, 127, 255, 383 and 511 the step's selection and
+    attention match the oracle, whose pooled cache evolves incrementally every step."""
+    wl = synth.workload("stream256k_12l")
+    shape = O.QsaShape.of(wl)
+    checks = {0, 127, 255, 383, 511}
+    for layer in range(wl.n_layers):
+        qsa = _qsa(wl)
+        g = H.GpuLayer(qsa)
+        ref = O.OracleLayer(shape, max_ctx=g.cfg.max_ctx)
+        pre = synth.prefill_tokens(wl, layer)
+        g.append(pre["k"], pre["v"], pre["idx"])
+        g.update()
+        ref.append_tokens(pre["k"], pre["v"], pre["idx"])
+        ref.update_pooled_cache()
+        del pre
+        for step in range(wl.n_steps):
+            st = synth.step_inputs(wl, layer, step)
+            qsa.decode_append(0, H.to_dev(st["k"]), H.to_dev(st["v"]), H.to_dev(st["idx"]))
+            g.index_topk(st["q_idx"], st["w"])
+            g.attend_selected(st["q"])
+            ref.append_tokens(st["k"][None], st["v"][None], st["idx"][None])
+            ref.update_pooled_cache()
+            n = ref.n
+            if step in checks:
+                got = g.fetch()
+                ref_scores = O.block_scores(ref.pooled.rows, st["q_idx"], st["w"], n, shape)
+                H.selection_mismatch(got["sel"], ref_scores, shape.k_blocks, H.CHAIN_GAP_REL)
+                cells = O.expand_cells(got["sel"], n)
+                H.assert_attention_close(got["out"], O.sparse_attention(st["q"], ref.k, ref.v, cells, shape))
+                rows = np.arange(max(0, n // 4 - 64), n // 4)
+                H.assert_pooled_close(g.pooled_rows(0, n // 4)[rows], ref.pooled.rows[rows])
+            if (step + 1) % 128 == 0:
+                live = g.pooled_rows(0, n // 4)
+                qsa.invalidate_pooled_cache(0, 0)
+                g.buf["pooled_cache"].zero_()
+                g.update()
+                np.testing.assert_array_equal(g.pooled_rows(0, n // 4), live)
+        assert g.state() == (wl.n_prefill + wl.n_steps, (wl.n_prefill + wl.n_steps) // 4, 0)
+        del g, qsa, ref
+        torch.cuda.empty_cache()
