@@ -284,6 +284,30 @@ qsa_status qsa_sparse_attend_selected_multi(qsa_ctx* ctx, int32_t layer, int32_t
  * by later appends. n_keep >= 0; a larger n_keep than n_ctx changes nothing. */
 qsa_status qsa_rollback(qsa_ctx* ctx, int32_t layer, int32_t n_keep, qsa_stream_t stream);
 
+/* ---- Conveniences ---- */
+
+/* Same as qsa_buffer_bytes (the sizing helper under its other name). */
+size_t qsa_layer_bytes(const qsa_config* cfg, int32_t which);
+
+/* Tokens in the layer's caches. The sequence state lives on the device (so that captured
+ * steps replay without the host), so this synchronises the device and reads it. Returns
+ * -1 if ctx or layer is invalid or the read fails. */
+int32_t qsa_n_ctx(const qsa_ctx* ctx, int32_t layer);
+
+/* Synchronise the device and report device-side errors: *status_out = the first non-zero
+ * status word over the bound layers in layer order (QSA_OK if none). The status words are
+ * left as they are (qsa_read_layer_state clears one). Returns QSA_ERR_CUDA if the device
+ * reports a CUDA error. */
+qsa_status qsa_get_device_status(qsa_ctx* ctx, int32_t* status_out);
+
+/* One decode step of one layer, the whole hot path in four launches on `stream`:
+ * qsa_decode_append(k, v, idx_key), the indexer scan of q_idx / w into the layer
+ * workspace, the block top-k into sel_blocks / n_sel, and qsa_sparse_attend_selected(q)
+ * into out. Arguments as in those calls; the same results as making them one by one. */
+qsa_status qsa_decode_step(qsa_ctx* ctx, int32_t layer, const void* k, const void* v, const void* idx_key,
+                           const void* q_idx, const float* w, const void* q, int32_t* sel_blocks,
+                           int32_t* n_sel, float* out, qsa_stream_t stream);
+
 /* Size of the fixed scratch array behind qsa_sparse_attend_noalloc (1 MiB). */
 #define QSA_NOALLOC_SCRATCH_BYTES (1u << 20)
 

@@ -389,6 +389,57 @@ qsa_status qsa_sparse_attend_selected_multi(qsa_ctx* ctx, int32_t layer, int32_t
                    "sparse_attend_selected (multi-query)");
 }
 
+size_t qsa_layer_bytes(const qsa_config* cfg, int32_t which) { return qsa_buffer_bytes(cfg, which); }
+
+int32_t qsa_n_ctx(const qsa_ctx* ctx, int32_t layer) {
+  if (!ctx || layer < 0 || layer >= ctx->cfg.n_layers || !ctx->layers[layer].bound) return -1;
+  if (cudaDeviceSynchronize() != cudaSuccess) return -1;
+  DevState h;
+  if (cudaMemcpy(&h, ctx->view(layer).state, sizeof h, cudaMemcpyDeviceToHost) != cudaSuccess) return -1;
+  return h.n_ctx;
+}
+
+qsa_status qsa_get_device_status(qsa_ctx* ctx, int32_t* status_out) {
+  if (!ctx || !status_out) return QSA_ERR_INVALID_ARG;
+  *status_out = QSA_OK;
+  if (qsa_status st = ctx->cuda(cudaDeviceSynchronize(), "get_device_status: sync")) return st;
+  for (int32_t layer = 0; layer < ctx->cfg.n_layers; ++layer) {
+    if (!ctx->layers[layer].bound) continue;
+    DevState h;
+    if (qsa_status st = ctx->cuda(cudaMemcpy(&h, ctx->view(layer).state, sizeof h, cudaMemcpyDeviceToHost),
+                                  "get_device_status: copy"))
+      return st;
+    if (h.status != 0) {
+      *status_out = h.status;
+      break;
+    }
+  }
+  return QSA_OK;
+}
+
+qsa_status qsa_decode_step(qsa_ctx* ctx, int32_t layer, const void* k, const void* v, const void* idx_key,
+                           const void* q_idx, const float* w, const void* q, int32_t* sel_blocks, int32_t* n_sel,
+                           float* out, qsa_stream_t stream) {
+  if (!ctx) return QSA_ERR_INVALID_ARG;
+  if (qsa_status st = ctx->layer_ok(layer)) return st;
+  QSA_CHECK_PTR(k, 16, "k");
+  QSA_CHECK_PTR(v, 16, "v");
+  QSA_CHECK_PTR(idx_key, 16, "idx_key");
+  QSA_CHECK_PTR(q_idx, 16, "q_idx");
+  QSA_CHECK_PTR(w, 4, "w");
+  QSA_CHECK_PTR(q, 16, "q");
+  QSA_CHECK_PTR(sel_blocks, 16, "sel_blocks");
+  QSA_CHECK_PTR(n_sel, 4, "n_sel");
+  QSA_CHECK_PTR(out, 16, "out");
+  const LayerView lv = ctx->view(layer);
+  const cudaStream_t s = (cudaStream_t)stream;
+  if (qsa_status st = ctx->cuda(launch_decode_append(lv, k, v, idx_key, s), "decode_step: append")) return st;
+  if (qsa_status st = ctx->cuda(launch_index_scan(lv, q_idx, w, lv.scores, s), "decode_step: index scan")) return st;
+  if (qsa_status st = ctx->cuda(launch_topk(lv, lv.scores, sel_blocks, n_sel, s), "decode_step: block top-k"))
+    return st;
+  return ctx->cuda(launch_attend_selected(lv, q, sel_blocks, n_sel, out, s), "decode_step: sparse attend");
+}
+
 qsa_status qsa_rollback(qsa_ctx* ctx, int32_t layer, int32_t n_keep, qsa_stream_t stream) {
   if (!ctx) return QSA_ERR_INVALID_ARG;
   if (qsa_status st = ctx->layer_ok(layer)) return st;

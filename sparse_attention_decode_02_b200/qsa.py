@@ -70,6 +70,10 @@ SIGNATURES = {
     "qsa_index_topk_multi": (_I, [_P, _I, _I, _P, _P, _P, _P, _P, _P]),
     "qsa_sparse_attend_selected_multi": (_I, [_P, _I, _I, _P, _P, _P, _P, _P]),
     "qsa_rollback": (_I, [_P, _I, _I, _P]),
+    "qsa_layer_bytes": (c_size_t, [ctypes.POINTER(QsaConfig), _I]),
+    "qsa_n_ctx": (_I, [_P, _I]),
+    "qsa_get_device_status": (_I, [_P, ctypes.POINTER(_I)]),
+    "qsa_decode_step": (_I, [_P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
 }
 
 _lib = None
@@ -223,6 +227,25 @@ class Qsa:
 
     def rollback(self, layer, n_keep, stream=None):
         self._check(self.lib.qsa_rollback(self.handle, layer, int(n_keep), _stream(stream)))
+
+    def decode_step(self, layer, k, v, idx_key, q_idx, w, q, sel_blocks, n_sel, out, stream=None):
+        """The whole hot path of one decode step of one layer in one ABI call."""
+        self._check(self.lib.qsa_decode_step(self.handle, layer, _ptr(k), _ptr(v), _ptr(idx_key), _ptr(q_idx),
+                                             _ptr(w), _ptr(q), _ptr(sel_blocks), _ptr(n_sel), _ptr(out),
+                                             _stream(stream)))
+
+    def n_ctx(self, layer) -> int:
+        """Tokens in the layer's caches (synchronises the device)."""
+        n = self.lib.qsa_n_ctx(self.handle, layer)
+        if n < 0:
+            raise QsaError(1, f"qsa_n_ctx failed for layer {layer}")
+        return n
+
+    def device_status(self) -> int:
+        """First non-zero device status word over the bound layers (synchronises the device)."""
+        st = c_int32()
+        self._check(self.lib.qsa_get_device_status(self.handle, ctypes.byref(st)))
+        return st.value
 
 
 def sparse_attend_noalloc(q, k_cache, v_cache, n_ctx, cells, n_cells, out, n_q_heads, n_kv_heads, head_dim,

@@ -108,6 +108,18 @@ def test_null_arguments_are_rejected(lib):
     assert lib.qsa_create(None, None) == 1
     lib.qsa_destroy(None)  # no-op
     assert lib.qsa_last_error(None) == b"null context"
+    assert lib.qsa_n_ctx(None, 0) == -1
+    st = ctypes.c_int32(7)
+    assert lib.qsa_get_device_status(None, ctypes.byref(st)) == 1
+    assert lib.qsa_decode_step(None, 0, *([None] * 9), None) == 1
+    assert lib.qsa_rollback(None, 0, 0, None) == 1
+    assert lib.qsa_index_topk_multi(None, 0, 1, *([None] * 5), None) == 1
+
+
+def test_layer_bytes_is_buffer_bytes(lib):
+    cfg = Q.make_config(12, 255184 + 512, 128, 16, 2048, 32, 4, 128)
+    for which in range(7):
+        assert lib.qsa_layer_bytes(ctypes.byref(cfg), which) == Q.buffer_bytes(cfg, which)
 
 
 def test_binding_has_no_fallback(tmp_path):

@@ -471,3 +471,38 @@ def test_streaming_512_steps_12_layers():
         assert g.state() == (wl.n_prefill + wl.n_steps, (wl.n_prefill + wl.n_steps) // 4, 0)
         del g, qsa, ref
         torch.cuda.empty_cache()
+
+
+def test_decode_step_call_equals_separate_calls():
+    """qsa_decode_step (the four launches in one ABI call) gives bit-identical results to
+    qsa_decode_append + qsa_index_topk + qsa_sparse_attend_selected; qsa_n_ctx and
+    qsa_get_device_status report the device state."""
+    wl = synth.workload("tiny")
+    layers = []
+    for _ in range(2):
+        qsa = _qsa(wl)
+        g = H.GpuLayer(qsa)
+        pre = synth.prefill_tokens(wl, 0, 1021)
+        g.append(pre["k"], pre["v"], pre["idx"])
+        g.update()
+        layers.append((qsa, g))
+    (qa, ga), (qb, gb) = layers
+    for step in range(6):
+        st = synth.step_inputs(wl, 0, step)
+        d = {k: H.to_dev(x) for k, x in st.items()}
+        qa.decode_step(0, d["k"], d["v"], d["idx"], d["q_idx"], d["w"], d["q"], ga.outs["sel"], ga.outs["n_sel"],
+                       ga.outs["out"])
+        qb.decode_append(0, d["k"], d["v"], d["idx"])
+        gb.index_topk(st["q_idx"], st["w"])
+        gb.attend_selected(st["q"])
+        torch.cuda.synchronize()
+        na, nb = int(ga.outs["n_sel"][0]), int(gb.outs["n_sel"][0])
+        assert na == nb
+        assert torch.equal(ga.outs["sel"][:na], gb.outs["sel"][:nb])
+        assert torch.equal(ga.outs["out"], gb.outs["out"])
+        assert qa.n_ctx(0) == 1021 + step + 1
+    assert qa.device_status() == 0
+    # a stale pooled cache is reported through the device status
+    qa.invalidate_pooled_cache(0, 10)
+    qa.index_topk(0, H.to_dev(st["q_idx"]), H.to_dev(st["w"]), ga.outs["sel"], ga.outs["n_sel"])
+    assert qa.device_status() == 3  # QSA_ERR_STATE
