@@ -149,6 +149,23 @@ def step_inputs(wl: Workload, layer: int, step: int):
     return {"k": tok["k"][0], "v": tok["v"][0], "idx": tok["idx"][0], "q_idx": q_idx, "w": w, "q": q}
 
 
+def step_inputs_range(wl: Workload, layer: int, first_step: int, count: int):
+    """step_inputs for steps [first_step, first_step + count), the same values, with the
+    appended tokens drawn in one pass (one chunk draw per 4,096 positions instead of one
+    per step)."""
+    tok = prefill_tokens(wl, layer, count, wl.n_prefill + first_step)
+    out = []
+    for i in range(count):
+        step = first_step + i
+        g = _rng(wl, layer, _T_QIDX, step)
+        q_idx = g.standard_normal((wl.n_idx_heads, wl.d_idx), dtype=np.float32).astype(np.float16)
+        w = _rng(wl, layer, _T_W, step).random(wl.n_idx_heads, dtype=np.float32)
+        q = _rng(wl, layer, _T_Q, step).standard_normal((wl.n_q_heads, wl.head_dim),
+                                                          dtype=np.float32).astype(np.float16)
+        out.append({"k": tok["k"][i], "v": tok["v"][i], "idx": tok["idx"][i], "q_idx": q_idx, "w": w, "q": q})
+    return out
+
+
 def random_cells(wl: Workload, layer: int, n_ctx: int, n_cells: int, salt: int = 0):
     """A sorted set of `n_cells` distinct cell ids in [0, n_ctx) (stage-isolated attention input)."""
     g = _rng(wl, layer, _T_CELLS, salt)

@@ -446,8 +446,7 @@ def test_streaming_512_steps_12_layers():
         ref.append_tokens(pre["k"], pre["v"], pre["idx"])
         ref.update_pooled_cache()
         del pre
-        for step in range(wl.n_steps):
-            st = synth.step_inputs(wl, layer, step)
+        for step, st in enumerate(synth.step_inputs_range(wl, layer, 0, wl.n_steps)):
             qsa.decode_append(0, H.to_dev(st["k"]), H.to_dev(st["v"]), H.to_dev(st["idx"]))
             g.index_topk(st["q_idx"], st["w"])
             g.attend_selected(st["q"])

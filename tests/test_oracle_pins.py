@@ -553,3 +553,17 @@ def test_fp8_layer_is_exact_on_e4m3_grid_rows():
     q = rng.standard_normal((shape.n_q_heads, shape.head_dim)).astype(np.float16) * 0.01
     cells = np.arange(n)
     np.testing.assert_array_equal(a.attend(q, cells), b.attend(q, cells))
+
+
+# ---------------------------------------------------------------- seeded inputs
+
+@pytest.mark.parametrize("first", [250, 258048 - 255181 - 5])   # the second range crosses a chunk boundary
+def test_step_inputs_range_equals_single_steps(first):
+    """The range draw returns exactly what one call per step returns (position-keyed chunks)."""
+    wl = synth.workload("stream256k_12l")
+    rng_steps = synth.step_inputs_range(wl, 3, first, 12)
+    for i, got in enumerate(rng_steps):
+        want = synth.step_inputs(wl, 3, first + i)
+        assert got.keys() == want.keys()
+        for k in want:
+            np.testing.assert_array_equal(got[k], want[k])
