@@ -266,6 +266,72 @@ def sparse_attention(q, k_cache, v_cache, cells, shape: QsaShape) -> np.ndarray:
 
 
 # ---------------------------------------------------------------------------
+# Context-parallel form of one decode step (survey row f3; the pages run one GPU).
+# The context of one layer is split into contiguous, block-aligned shards; the last
+# shard holds the open tail. Each shard scores its own completed blocks (the query at
+# the global position n-1, the blocks at their global positions), keeps its local top-K
+# as (score, global block) candidates, and after an exchange every shard takes the global
+# top-K of all candidates with the same rule. Each shard attends over its selected cells
+# and returns (o, lse) per head; the exact merge is o = sum_r exp(lse_r - LSE) o_r with
+# LSE = log sum_r exp(lse_r). Any block of the global top-K is in its shard's local top-K
+# (fewer than K blocks beat it anywhere), and candidates listed shard by shard in
+# ascending block order keep "ties to the lower block" intact, so the result equals the
+# single-device step.
+# ---------------------------------------------------------------------------
+
+def shard_candidates(pooled_shard, first_block: int, q_idx, w, n: int, shape: QsaShape):
+    """Local top-K of one shard: (scores, global block ids), ascending by block.
+    pooled_shard holds the summaries of global blocks first_block, first_block+1, ...
+    (completed ones only)."""
+    q = indexer_query(q_idx, n, shape)
+    p = np.asarray(pooled_shard, dtype=np.float64)
+    s = (np.maximum(p @ q.T, 0.0) @ np.asarray(w, dtype=np.float64)) / np.sqrt(shape.d_idx)
+    local = topk_blocks(s, shape.k_blocks) if len(s) else np.zeros(0, np.int64)
+    return s[local], local + first_block
+
+
+def merge_candidates(cand_scores, cand_blocks, k_blocks: int) -> np.ndarray:
+    """Global top-K from the shards' candidates listed shard by shard (block order)."""
+    scores = np.concatenate(cand_scores) if cand_scores else np.zeros(0)
+    blocks = np.concatenate(cand_blocks) if cand_blocks else np.zeros(0, np.int64)
+    pick = topk_blocks(scores, k_blocks) if len(scores) else np.zeros(0, np.int64)
+    return blocks[pick]
+
+
+def attention_partial(q, k_cache, v_cache, cells, shape: QsaShape):
+    """(o, lse) per query head over `cells`: o normalised, lse = log sum_c exp(logit_c);
+    an empty cell set gives o = 0 and lse = -inf."""
+    q = np.asarray(q, dtype=np.float64)
+    cells = np.asarray(cells, dtype=np.int64)
+    group = shape.n_q_heads // shape.n_kv_heads
+    o = np.zeros((shape.n_q_heads, shape.head_dim))
+    lse = np.full(shape.n_q_heads, -np.inf)
+    if len(cells) == 0:
+        return o, lse
+    for i in range(shape.n_q_heads):
+        g = i // group
+        kc = np.asarray(k_cache[cells, g], dtype=np.float64)
+        vc = np.asarray(v_cache[cells, g], dtype=np.float64)
+        logits = kc @ q[i] / np.sqrt(shape.head_dim)
+        m = logits.max()
+        e = np.exp(logits - m)
+        o[i] = (e @ vc) / e.sum()
+        lse[i] = m + np.log(e.sum())
+    return o, lse
+
+
+def merge_partials(partials):
+    """Exact merge of per-shard (o, lse) into the attention over the union of the cells."""
+    lse = np.stack([p[1] for p in partials])                   # [G, Hq]
+    top = lse.max(axis=0)
+    safe = np.where(np.isfinite(top), top, 0.0)
+    wts = np.where(np.isfinite(lse), np.exp(lse - safe), 0.0)  # [G, Hq]
+    den = wts.sum(axis=0)
+    o = sum(wts[r][:, None] * partials[r][0] for r in range(len(partials)))
+    return np.where(den[:, None] > 0, o / np.where(den > 0, den, 1.0)[:, None], 0.0)
+
+
+# ---------------------------------------------------------------------------
 # FP8 K/V cache. The Qwen3.8-Flash-Next parameter-tuning post on EVO-X2 (section
 # "KV cacheをQ8_0にしてみる") tried an 8-bit K/V cache and gives no layout.
 # Reading R12: one f32 scale per (token, KV head) row, scale = amax / 448, codes =

@@ -567,3 +567,73 @@ def test_step_inputs_range_equals_single_steps(first):
         assert got.keys() == want.keys()
         for k in want:
             np.testing.assert_array_equal(got[k], want[k])
+
+
+# ---------------------------------------------------------------- context-parallel decomposition
+
+def _cp_layer(seed, n, shape):
+    rng = np.random.default_rng(seed)
+    L = O.OracleLayer(shape, max_ctx=n + 4)
+    L.append_tokens(rng.standard_normal((n, shape.n_kv_heads, shape.head_dim)).astype(np.float16),
+                    rng.standard_normal((n, shape.n_kv_heads, shape.head_dim)).astype(np.float16),
+                    rng.standard_normal((n, shape.d_idx)).astype(np.float16))
+    L.update_pooled_cache()
+    q_idx = rng.standard_normal((shape.n_idx_heads, shape.d_idx)).astype(np.float16)
+    w = rng.random(shape.n_idx_heads)
+    q = rng.standard_normal((shape.n_q_heads, shape.head_dim)).astype(np.float16)
+    return L, q_idx, w, q
+
+
+def _cp_step(L, starts, q_idx, w, q):
+    """The sharded step over layer L's caches, shards starting at the given block-aligned tokens."""
+    n, shape = L.n, L.shape
+    bounds = list(starts) + [n]
+    cand_s, cand_b = [], []
+    for r in range(len(starts)):
+        b0, b1 = bounds[r] // 4, bounds[r + 1] // 4        # the last shard's open tail has no block
+        s, b = O.shard_candidates(L.pooled.rows[b0:b1], b0, q_idx, w, n, shape)
+        cand_s.append(s)
+        cand_b.append(b)
+    sel = O.merge_candidates(cand_s, cand_b, shape.k_blocks)
+    parts = []
+    for r in range(len(starts)):
+        mine = sel[(sel >= bounds[r] // 4) & (sel < bounds[r + 1] // 4)]
+        cells = O.expand_cells(mine, 4 * (bounds[r + 1] // 4))          # no tail ...
+        if r == len(starts) - 1:                                            # ... except on the last shard
+            cells = O.expand_cells(mine, n)
+        parts.append(O.attention_partial(q, L.k, L.v, cells, shape))
+    return sel, O.merge_partials(parts)
+
+
+@pytest.mark.parametrize("starts", [[0], [0, 400], [0, 128, 132], [0, 4, 200, 204, 500], [0, 700]])
+def test_context_parallel_step_equals_single_device(starts):
+    shape = O.QsaShape(d_idx=32, n_idx_heads=3, top_k_tokens=64, n_q_heads=4, n_kv_heads=2, head_dim=16)
+    n = 4 * 180 + 3
+    L, q_idx, w, q = _cp_layer(len(starts) * 7 + starts[-1], n, shape)
+    sel, out = _cp_step(L, starts, q_idx, w, q)
+    ref_sel = O.topk_blocks(O.block_scores(L.pooled.rows, q_idx, w, n, shape), shape.k_blocks)
+    np.testing.assert_array_equal(sel, ref_sel)
+    ref_out = O.sparse_attention(q, L.k, L.v, O.expand_cells(ref_sel, n), shape)
+    np.testing.assert_allclose(out, ref_out, rtol=0, atol=1e-12)
+
+
+def test_candidate_merge_keeps_ties_to_the_lower_block():
+    # equal scores across shards: the lower block wins, exactly as in one list
+    got = O.merge_candidates([np.array([5.0, 3.0]), np.array([5.0, 3.0]), np.array([], float)],
+                             [np.array([2, 7]), np.array([12, 20]), np.array([], np.int64)], 3)
+    assert got.tolist() == [2, 7, 12]
+    got = O.merge_candidates([np.array([1.0]), np.array([1.0, 1.0])], [np.array([9]), np.array([10, 11])], 2)
+    assert got.tolist() == [9, 10]
+
+
+def test_lse_merge_over_any_cell_partition():
+    shape = O.QsaShape(d_idx=32, n_idx_heads=3, top_k_tokens=64, n_q_heads=4, n_kv_heads=2, head_dim=16)
+    L, _, _, q = _cp_layer(99, 300, shape)
+    cells = np.arange(300)
+    rng = np.random.default_rng(3)
+    owner = rng.integers(0, 4, size=300)                  # shard 3 may own nothing
+    owner[owner == 3] = 2
+    parts = [O.attention_partial(q, L.k, L.v, cells[owner == r], shape) for r in range(4)]
+    assert np.all(np.isneginf(parts[3][1]))
+    np.testing.assert_allclose(O.merge_partials(parts), O.sparse_attention(q, L.k, L.v, cells, shape),
+                               rtol=0, atol=1e-12)
