@@ -266,7 +266,7 @@ def sparse_attention(q, k_cache, v_cache, cells, shape: QsaShape) -> np.ndarray:
 
 
 # ---------------------------------------------------------------------------
-# Context-parallel form of one decode step (survey row f3; the pages run one GPU).
+# Context-parallel form of one decode step (the pages run one GPU; this is the sharded form).
 # The context of one layer is split into contiguous, block-aligned shards; the last
 # shard holds the open tail. Each shard scores its own completed blocks (the query at
 # the global position n-1, the blocks at their global positions), keeps its local top-K
