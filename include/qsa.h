@@ -22,7 +22,10 @@
  *    default stream) and returns after HOST-side argument validation only; kernels are
  *    launched with programmatic dependent launch so that consecutive calls on one
  *    stream overlap their launch latency, and all of them are safe to capture in a
- *    CUDA graph.
+ *    CUDA graph. The exceptions synchronise and must stay outside a capture:
+ *    qsa_read_layer_state, qsa_n_ctx and qsa_get_device_status.
+ *  - A context is not internally locked: use it from one host thread at a time.
+ *    Separate contexts are independent.
  *  - The sequence state of each layer (context length n_ctx and number of pooled
  *    blocks n_pooled) lives in DEVICE memory inside the layer's workspace and is
  *    advanced by the kernels themselves, so a captured decode step can be replayed.
