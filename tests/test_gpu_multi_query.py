@@ -80,7 +80,8 @@ def _check_query(p, got, ref, n_u, x, u):
 
 @pytest.mark.parametrize("wl_name,n0,T", [("tiny", 1016, 1), ("tiny", 1017, 2), ("tiny", 1018, 3),
                                           ("tiny", 1019, 4), ("tiny", 1020, 4), ("tiny", 1021, 3),
-                                          ("ctx64k", 61789 - 4, 4), ("ctx64k", 61789 - 3, 2)])
+                                          ("ctx64k", 61789 - 4, 4), ("ctx64k", 61789 - 3, 2),
+                                          ("ctx64k", 61789 - 2, 3)])   # 3 queries x 16 heads: MMA N = 96
 def test_multi_query_step_matches_oracle(wl_name, n0, T):
     p = Pair(wl_name, n0)
     x = _drafts(p.wl, T)
