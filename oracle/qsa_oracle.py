@@ -50,8 +50,15 @@ Readings taken where the pages are silent (each one is listed in the design note
      completed is scored like any other, not force-included.
   R8 attention: scale 1/sqrt(D), query head i uses KV head floor(i / (Hq/Hkv)), no
      extra mask, sink, gate or softcap.
+  R11 verifying T drafted tokens at once is T single-token steps: query t (token n-T+t)
+     sees the blocks completed within its first n-T+t+1 tokens and its own open tail; a
+     rollback drops rejected tokens and the summaries of blocks they completed (Part 10
+     §COMMON-004: speculative writes must not corrupt the cached range).
   R12 FP8 K/V cache (optional): per (token, KV head) row, scale = amax/448 and e4m3 codes
      of x * 448/amax (nearest-even, saturating); attention reads code * scale.
+
+Also stated here: the sharded (context-parallel) form of one step, whose local top-K
+candidates, merged selection and (o, lse) partials reproduce the single-device step.
 """
 from __future__ import annotations
 
