@@ -11,6 +11,12 @@ ABI while capturing). The headline workload is all 12 QSA layers at the pages' 2
 input (255,181 tokens); 64k and 128k single-layer lines (rotated over enough layer
 replicas that the working set exceeds L2) are reported under "by_ctx".
 
+Beside the headline: "e2e" (the same steps with each step's inputs copied in from pinned
+host memory and its outputs copied back, overlapped on a second stream), "bulk_pool"
+(the whole pooled cache of one 256k layer rebuilt), "multi_query" (verification of 4
+drafted tokens per step with rollback, every layer) and "kv_fp8" (the step with the
+e4m3 K/V cache).
+
 Timing: W untimed warm-up steps, then exactly K steps bracketed by a barrier and
 torch.cuda.synchronize(), timed with CUDA events on the launching stream; the max over
 ranks is reported. Inputs are larger than L2 (12 layers x ~20.6 MB per step), so no
