@@ -367,13 +367,14 @@ template <int D, bool GEN>
 __global__ void __launch_bounds__(kPoolThreads) pool_update_kernel(DevState* st, const __half* __restrict__ ic,
                                                                    __half* __restrict__ pc,
                                                                    const float* __restrict__ gain, float eps,
-                                                                   PoolRope rope) {
+                                                                   PoolRope rope, int max_blocks) {
   __shared__ float s_rows[GEN ? kPoolThreads / 32 : 1][GEN ? D : 1];
   pdl_launch_dependents();
   pdl_wait();
   const int n = ld_volatile(&st->n_ctx);
   const int b_first = ld_volatile(&st->n_pooled);
-  const int b_end = n / kBlock;
+  int b_end = n / kBlock;
+  if (!QSA_GUARD(st, b_end <= max_blocks && b_first >= 0)) b_end = b_first;  // pool nothing
   const int lane = threadIdx.x & 31;
   const int warps = blockDim.x >> 5;
   const int gw = blockIdx.x * warps + (threadIdx.x >> 5);
@@ -510,7 +511,8 @@ cudaError_t launch_decode_append(const LayerView& L, const void* k, const void* 
 template <int D, bool GEN>
 static cudaError_t launch_pool_update_d(const LayerView& L, int grid, cudaStream_t s) {
   return launch_pdl(pool_update_kernel<D, GEN>, dim3(grid), dim3(kPoolThreads), 0, s, 1, L.state,
-                    (const __half*)L.idx_cache, (__half*)L.pooled_cache, L.rms_gain, L.cfg.rms_eps, pool_rope(L.cfg));
+                    (const __half*)L.idx_cache, (__half*)L.pooled_cache, L.rms_gain, L.cfg.rms_eps, pool_rope(L.cfg),
+                    L.cfg.max_ctx / kBlock);
 }
 
 cudaError_t launch_pool_update(const LayerView& L, int grid_hint, cudaStream_t s) {

@@ -30,7 +30,10 @@ block_topk_kernel(DevState* st, const float* __restrict__ scores, int32_t* __res
   cluster_arrive_relaxed();  // paired inside cluster_select
   pdl_wait();
   const sel::Result res = sel::cluster_select<V>(st, scores, k_blocks, max_blocks, n_back,
-                                                 [&](uint32_t pos, int block) { sel_out[pos] = block; });
+                                                 [&](uint32_t pos, int block) {
+                                                   if (QSA_GUARD(st, pos < uint32_t(k_blocks) && block < max_blocks))
+                                                     sel_out[pos] = block;
+                                                 });
   if (res.status == sel::kAll)
     for (int i = rank * sel::kThreads + threadIdx.x; i < res.n_blocks; i += sel::kCS * sel::kThreads) sel_out[i] = i;
   if (rank == 0 && threadIdx.x == 0)

@@ -80,11 +80,12 @@ _lib = None
 
 
 def load_library(path: str | None = None) -> ctypes.CDLL:
-    """Load libqsa.so and declare its signatures. Raises if it is missing."""
+    """Load libqsa.so (or the library QSA_LIBRARY names, e.g. the checked build) and
+    declare its signatures. Raises if it is missing."""
     global _lib
     if _lib is not None and path is None:
         return _lib
-    p = path or LIB_PATH
+    p = path or os.environ.get("QSA_LIBRARY") or LIB_PATH
     if not os.path.exists(p):
         raise ImportError(f"{p} is missing: build it with `python -m sparse_attention_decode_02_b200.build`")
     lib = ctypes.CDLL(p)

@@ -126,3 +126,15 @@ def test_binding_has_no_fallback(tmp_path):
     with pytest.raises(ImportError):
         Q.load_library(str(tmp_path / "missing.so"))
     assert qsa_pkg.Qsa is Q.Qsa
+
+
+@pytest.mark.slow
+def test_checked_build_compiles_and_exports(tmp_path):
+    """The checked build (-DQSA_CHECKED bounds guards) compiles, links and exports the ABI."""
+    lib_path = qbuild.build(checked=True)
+    assert lib_path.endswith("libqsa_checked.so") and os.path.exists(lib_path)
+    lib = Q.load_library(lib_path)
+    for name in _declared():
+        assert hasattr(lib, name), name
+    cfg = Q.make_config(1, 4096, 128, 16, 2048, 32, 4, 128)
+    assert lib.qsa_buffer_bytes(ctypes.byref(cfg), Q.QSA_BUF_MAX_CELLS) == 2051
