@@ -14,6 +14,7 @@
 #include <cuda_fp8.h>
 
 #include "qsa_device.cuh"
+#include "qsa_checked.cuh"
 
 namespace qsa {
 

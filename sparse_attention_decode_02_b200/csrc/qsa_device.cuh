@@ -53,15 +53,6 @@ __device__ __forceinline__ void record_status(DevState* st, int code) {
   atomicCAS(&st->status, 0, code);
 }
 
-// Bounds guard of the checked build (-DQSA_CHECKED, the stand-in for a memory sanitizer):
-// a false condition records QSA_ERR_BAD_INDEX in the layer status and the guarded access is
-// skipped; nothing traps. In the default build the guard is the constant true.
-#ifdef QSA_CHECKED
-#define QSA_GUARD(st, cond) ((cond) ? true : (record_status((st), QSA_ERR_BAD_INDEX), false))
-#else
-#define QSA_GUARD(st, cond) true
-#endif
-
 __device__ __forceinline__ int ld_volatile(const int32_t* p) { return *(volatile const int32_t*)p; }
 
 // Sum over the 32 lanes in a fixed butterfly order (deterministic).

@@ -10,6 +10,7 @@
 #include <cuda_fp16.h>
 
 #include "qsa_select.cuh"
+#include "qsa_checked.cuh"
 
 namespace qsa {
 

@@ -308,7 +308,7 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_
 #pragma unroll
             for (int h = 0; h < H; ++h)
               s += wr[u][h] * fmaxf(__uint_as_float(r[u][h]) + __uint_as_float(r[u][H + h]) * (1.0f / kLoScale), 0.0f);
-            if (QSA_GUARD(st, row < max_blocks)) scores[size_t(u) * score_stride + row] = s / sqrt_d;
+            scores[size_t(u) * score_stride + row] = s / sqrt_d;
           }
         }
       }
