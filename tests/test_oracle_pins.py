@@ -637,3 +637,24 @@ def test_lse_merge_over_any_cell_partition():
     assert np.all(np.isneginf(parts[3][1]))
     np.testing.assert_allclose(O.merge_partials(parts), O.sparse_attention(q, L.k, L.v, cells, shape),
                                rtol=0, atol=1e-12)
+
+
+def test_context_parallel_over_decode_steps_with_a_growing_tail():
+    """Tokens are appended to the last shard only; as its tail completes blocks they join the
+    shard's candidates, and every step still equals the single-device step."""
+    shape = O.QsaShape(d_idx=32, n_idx_heads=3, top_k_tokens=64, n_q_heads=4, n_kv_heads=2, head_dim=16)
+    L, q_idx, w, q = _cp_layer(5, 4 * 150 + 1, shape)
+    rng = np.random.default_rng(8)
+    starts = [0, 200, 400]
+    for step in range(9):
+        L.append_tokens(rng.standard_normal((1, shape.n_kv_heads, shape.head_dim)).astype(np.float16),
+                        rng.standard_normal((1, shape.n_kv_heads, shape.head_dim)).astype(np.float16),
+                        rng.standard_normal((1, shape.d_idx)).astype(np.float16))
+        L.update_pooled_cache()
+        q_idx = rng.standard_normal((shape.n_idx_heads, shape.d_idx)).astype(np.float16)
+        sel, out = _cp_step(L, starts, q_idx, w, q)
+        n = L.n
+        ref_sel = O.topk_blocks(O.block_scores(L.pooled.rows, q_idx, w, n, shape), shape.k_blocks)
+        np.testing.assert_array_equal(sel, ref_sel)
+        ref_out = O.sparse_attention(q, L.k, L.v, O.expand_cells(ref_sel, n), shape)
+        np.testing.assert_allclose(out, ref_out, rtol=0, atol=1e-12)
