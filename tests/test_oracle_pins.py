@@ -571,9 +571,9 @@ def test_step_inputs_range_equals_single_steps(first):
 
 # ---------------------------------------------------------------- context-parallel decomposition
 
-def _cp_layer(seed, n, shape):
+def _cp_layer(seed, n, shape, extra=4):
     rng = np.random.default_rng(seed)
-    L = O.OracleLayer(shape, max_ctx=n + 4)
+    L = O.OracleLayer(shape, max_ctx=n + extra)
     L.append_tokens(rng.standard_normal((n, shape.n_kv_heads, shape.head_dim)).astype(np.float16),
                     rng.standard_normal((n, shape.n_kv_heads, shape.head_dim)).astype(np.float16),
                     rng.standard_normal((n, shape.d_idx)).astype(np.float16))
@@ -643,7 +643,7 @@ def test_context_parallel_over_decode_steps_with_a_growing_tail():
     """Tokens are appended to the last shard only; as its tail completes blocks they join the
     shard's candidates, and every step still equals the single-device step."""
     shape = O.QsaShape(d_idx=32, n_idx_heads=3, top_k_tokens=64, n_q_heads=4, n_kv_heads=2, head_dim=16)
-    L, q_idx, w, q = _cp_layer(5, 4 * 150 + 1, shape)
+    L, q_idx, w, q = _cp_layer(5, 4 * 150 + 1, shape, extra=16)
     rng = np.random.default_rng(8)
     starts = [0, 200, 400]
     for step in range(9):
