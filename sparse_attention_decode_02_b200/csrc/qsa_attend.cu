@@ -806,16 +806,48 @@ constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
 void* g_noalloc_addr[kMaxDevices];  // device address of g_noalloc_scratch, per device
 int g_noalloc_sms[kMaxDevices];
+unsigned long long g_noalloc_ctx[kMaxDevices];  // id of the context the address belongs to
 
-// Once per device, with that device current: look up the array's device address (host
-// code cannot use the symbol itself, which is only a host-side stand-in).
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// Unique id of the calling thread's current context (0 if it cannot be read). A device
+// reset or a primary-context teardown gives the device a new context with a new id, and
+// the array a new address in it.
+unsigned long long current_ctx_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static bool looked_up = false;
+  if (!looked_up) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+    looked_up = true;
+  }
+  CUcontext c = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&c) != CUDA_SUCCESS || !c || get_id(c, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+// Once per device (and again if the device's context was replaced since), with that
+// device current: look up the array's device address (host code cannot use the symbol
+// itself, which is only a host-side stand-in).
 cudaError_t noalloc_setup(void** addr, int* n_sms) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  // 0 when no context is current on this thread yet (the lookup below makes it current)
+  const unsigned long long ctx_id = current_ctx_id();
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_addr[dev]) {
+  if (!g_noalloc_addr[dev] || ctx_id == 0 || g_noalloc_ctx[dev] != ctx_id) {
     int sms = 0;
     e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
@@ -824,6 +856,7 @@ cudaError_t noalloc_setup(void** addr, int* n_sms) {
     if (e != cudaSuccess) return e;
     g_noalloc_sms[dev] = sms;
     g_noalloc_addr[dev] = p;
+    g_noalloc_ctx[dev] = current_ctx_id();
   }
   *addr = g_noalloc_addr[dev];
   *n_sms = g_noalloc_sms[dev];

@@ -3,6 +3,9 @@ run the decode calls through the C ABI, and compare against the oracle with the
 tolerances the tests use."""
 from __future__ import annotations
 
+import json
+import os
+
 import numpy as np
 import torch
 
@@ -131,3 +134,15 @@ def assert_attention_close(gpu_out, ref_out):
         scale = max(np.abs(ref_out[i]).max(), 1e-6)
         err = np.abs(gpu_out[i] - ref_out[i]).max() / scale
         assert err <= ATTN_REL, f"head {i}: attention rel err {err:.3e}"
+
+
+def record_chain(case: str, step: int, flips: int, **extra):
+    """Appends one line (case, step, near-tie selection flips) to chain_flips.jsonl under
+    $QSA_ARTIFACT_DIR when that variable is set: the per-context flip counts of the
+    end-to-end chains, kept as a test artifact."""
+    d = os.environ.get("QSA_ARTIFACT_DIR")
+    if not d:
+        return
+    os.makedirs(d, exist_ok=True)
+    with open(os.path.join(d, "chain_flips.jsonl"), "a") as f:
+        f.write(json.dumps(dict(case=case, step=step, flips=flips, **extra)) + "\n")

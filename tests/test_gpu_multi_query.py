@@ -107,6 +107,12 @@ def test_multi_query_equals_single_token_steps_on_gpu():
         np.testing.assert_allclose(multi[u]["scores"][: n_u // 4], s1, rtol=0, atol=1e-6 * np.abs(s1).max())
         if H.selection_mismatch(multi[u]["sel"], s1, wl.k_blocks, H.TIE_GAP_REL) == 0:
             np.testing.assert_allclose(multi[u]["out"], single["out"], rtol=0, atol=1e-5)
+        # either way, each output matches the oracle attending over that query's own cells
+        k_all = np.concatenate([a.ref.k[:1018], x["k"]])
+        v_all = np.concatenate([a.ref.v[:1018], x["v"]])
+        for res in (multi[u], single):
+            H.assert_attention_close(res["out"], O.sparse_attention(x["q"][u], k_all, v_all,
+                                                                    O.expand_cells(res["sel"], n_u), a.ref.shape))
 
 
 def test_rollback_recomputes_dirty_blocks():
