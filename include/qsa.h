@@ -92,9 +92,17 @@ typedef struct {
    * nearest-even and saturated (an all-zero row: scale 1, zero codes); attention reads
    * code * scale. The indexer caches stay f16 either way. */
   int32_t kv_format;
+  /* How the indexer scan computes the dots q~_h . p_b (the scores are the same up to f32
+   * rounding; zero gives the default). QSA_SCAN_TENSOR (0): the 5th-generation tensor
+   * cores (tcgen05), the query split into f16 high and scaled low parts so it keeps ~22
+   * significant bits. QSA_SCAN_CUDA_CORES (1): the CUDA cores, an f32 query and packed
+   * f32 FMAs with warp-shuffle reductions; single-query scans only (the multi-query calls
+   * use the tensor cores), and a decode step with it takes four launches. */
+  int32_t scan_kind;
 } qsa_config;
 
 enum { QSA_KV_F16 = 0, QSA_KV_FP8 = 1 };
+enum { QSA_SCAN_TENSOR = 0, QSA_SCAN_CUDA_CORES = 1 };
 
 /* Caller-owned device buffers of one layer. Sizes come from qsa_buffer_bytes(). */
 typedef struct {
@@ -303,10 +311,21 @@ int32_t qsa_n_ctx(const qsa_ctx* ctx, int32_t layer);
  * reports a CUDA error. */
 qsa_status qsa_get_device_status(qsa_ctx* ctx, int32_t* status_out);
 
-/* One decode step of one layer, the whole hot path in four launches on `stream`:
- * qsa_decode_append(k, v, idx_key), the indexer scan of q_idx / w into the layer
- * workspace, the block top-k into sel_blocks / n_sel, and qsa_sparse_attend_selected(q)
- * into out. Arguments as in those calls; the same results as making them one by one. */
+/* One decode step of one layer, the whole hot path on `stream`: the append of the
+ * token (k, v, idx_key) with the incremental pooled update, the indexer scan of q_idx / w
+ * into the layer workspace, the block top-k into sel_blocks / n_sel, and the sparse
+ * attention of q over the selection into out. Arguments as in qsa_decode_append,
+ * qsa_index_topk and qsa_sparse_attend_selected; the results are bit-identical to making
+ * those three calls one by one.
+ * Launches: when the pooled cache is current up to the previous token (the library knows
+ * that from the calls made on the layer: after qsa_update_pooled_cache, qsa_decode_append,
+ * qsa_decode_step or qsa_rollback, not after qsa_append_token(s), qsa_restore_layer with
+ * blocks left to pool or qsa_invalidate_pooled_cache), three: the scan kernel itself
+ * appends the token and pools the block the token completes (Part 10, section
+ * "incremental pooled-key cache（COMMON-004）": only the new block is computed), then the
+ * selection, then the attention. Otherwise four: a separate append that pools every
+ * waiting block first. If the device state disagrees (the pooled cache is behind), the
+ * three-launch form appends nothing and reports QSA_ERR_STATE in the device status. */
 qsa_status qsa_decode_step(qsa_ctx* ctx, int32_t layer, const void* k, const void* v, const void* idx_key,
                            const void* q_idx, const float* w, const void* q, int32_t* sel_blocks,
                            int32_t* n_sel, float* out, qsa_stream_t stream);
@@ -326,7 +345,10 @@ qsa_status qsa_decode_step(qsa_ctx* ctx, int32_t layer, const void* k, const voi
  * The result is the same as qsa_sparse_attend's for the same inputs and shapes.
  * Scratch: one array of QSA_NOALLOC_SCRATCH_BYTES compiled into the library; every GPU
  * that loads the library holds it until the process exits. The first call on a device
- * looks up the array's device address (make that first call before any stream capture).
+ * looks up the array's device address (make that first call before any stream capture);
+ * later calls reuse it while the device keeps the same CUDA context, and look it up again
+ * after the context was replaced (a device reset or a primary-context teardown). With no
+ * valid cells the output rows are zero; a negative *n_cells counts as zero.
  * Every call shares the array and overwrites what the previous call left there, so
  * calls whose kernels overlap on the GPU (on different streams, or from several host
  * threads) race and must be serialised by the caller. Nothing here allocates: no

@@ -10,6 +10,10 @@ is newer than every source and header.
 -DQSA_CHECKED: bounds guards on the kernels' data-dependent writes record
 QSA_ERR_BAD_INDEX in the layer status and skip the access (a stand-in for a memory
 sanitizer). Point the binding at it with QSA_LIBRARY=<path to libqsa_checked.so>.
+
+--timeline builds libqsa_timeline.so (objects in _build_timeline/), compiled with
+-DQSA_TIMELINE: the decode-step kernels record %globaltimer marks for one chosen layer
+(csrc/qsa_timeline.cuh), read back through qsa_tl_arm_<kernel> / qsa_tl_read_<kernel>.
 """
 from __future__ import annotations
 
@@ -26,6 +30,7 @@ CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libqsa.so")
 LIB_CHECKED = os.path.join(PKG, "libqsa_checked.so")
+LIB_TIMELINE = os.path.join(PKG, "libqsa_timeline.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-O2",
@@ -53,15 +58,15 @@ def up_to_date(lib: str = LIB) -> bool:
     return all(os.path.getmtime(p) <= t for p in srcs + hdrs + [__file__])
 
 
-def build(force: bool = False, verbose: bool = False, checked: bool = False) -> str:
-    lib = LIB_CHECKED if checked else LIB
+def build(force: bool = False, verbose: bool = False, checked: bool = False, timeline: bool = False) -> str:
+    lib = LIB_CHECKED if checked else LIB_TIMELINE if timeline else LIB
     if not force and up_to_date(lib):
         return lib
     nvcc = _nvcc()
     srcs, _ = _inputs()
-    build_dir = BUILD + "_checked" if checked else BUILD
+    build_dir = BUILD + ("_checked" if checked else "_timeline" if timeline else "")
     os.makedirs(build_dir, exist_ok=True)
-    extra = ["-DQSA_CHECKED"] if checked else []
+    extra = (["-DQSA_CHECKED"] if checked else []) + (["-DQSA_TIMELINE"] if timeline else [])
 
     def compile_one(src):
         obj = os.path.join(build_dir, os.path.basename(src)[:-3] + ".o")
@@ -86,4 +91,5 @@ def build(force: bool = False, verbose: bool = False, checked: bool = False) -> 
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="--verbose" in sys.argv, checked="--checked" in sys.argv))
+    print(build(force="--force" in sys.argv, verbose="--verbose" in sys.argv, checked="--checked" in sys.argv,
+                timeline="--timeline" in sys.argv))

@@ -49,6 +49,8 @@ const char* config_problem(const qsa_config& c) {
   if (c.rope_pos_stride < 0 || c.rope_pos_stride > 16) return "rope_pos_stride must be 0..16";
   if (c.rope_pos_offset < 0 || c.rope_pos_offset > (1 << 20)) return "rope_pos_offset must be 0..1048576";
   if (c.kv_format != QSA_KV_F16 && c.kv_format != QSA_KV_FP8) return "kv_format must be QSA_KV_F16 or QSA_KV_FP8";
+  if (c.scan_kind != QSA_SCAN_TENSOR && c.scan_kind != QSA_SCAN_CUDA_CORES)
+    return "scan_kind must be QSA_SCAN_TENSOR or QSA_SCAN_CUDA_CORES";
   return nullptr;
 }
 
@@ -97,6 +99,7 @@ struct qsa_ctx {
     v.kv_scales = static_cast<float*>(l.buf.kv_scales);
     v.state = reinterpret_cast<DevState*>(wsp + ws.state);
     v.scores = reinterpret_cast<float*>(wsp + ws.scores);
+    v.hist = reinterpret_cast<uint32_t*>(wsp + ws.hist);
     v.part_o = reinterpret_cast<float*>(wsp + ws.part_o);
     v.part_ml = reinterpret_cast<float*>(wsp + ws.part_ml);
     v.split = split;
@@ -157,7 +160,8 @@ qsa_status qsa_create(const qsa_config* cfg, qsa_ctx** out) {
     delete ctx;
     return QSA_ERR_CUDA;
   }
-  if (init_kernel_attributes() != cudaSuccess || init_scan_attributes() != cudaSuccess) {
+  if (init_kernel_attributes() != cudaSuccess || init_scan_attributes() != cudaSuccess ||
+      init_scan_cc_attributes() != cudaSuccess) {
     delete ctx;
     return QSA_ERR_CUDA;
   }
@@ -200,7 +204,10 @@ qsa_status qsa_bind_layer(qsa_ctx* ctx, int32_t layer, const qsa_layer_buffers* 
   l.pooled_box_map = box_map;
   l.bound = true;
   l.pending_blocks = 0;
-  qsa_status st = ctx->cuda(launch_set_state(ctx->view(layer), 0, 0, kSetReset, (cudaStream_t)stream), "bind_layer");
+  const LayerView v = ctx->view(layer);
+  qsa_status st = ctx->cuda(cudaMemsetAsync(v.hist, 0, size_t(1 << kHistBits) * sizeof(uint32_t), (cudaStream_t)stream),
+                            "bind_layer: clear histogram");
+  if (st == QSA_OK) st = ctx->cuda(launch_set_state(v, 0, 0, kSetReset, (cudaStream_t)stream), "bind_layer");
   if (st != QSA_OK) l.bound = false;
   return st;
 }
@@ -264,7 +271,10 @@ qsa_status qsa_decode_append(qsa_ctx* ctx, int32_t layer, const void* k, const v
   QSA_CHECK_PTR(k, 16, "k");
   QSA_CHECK_PTR(v, 16, "v");
   QSA_CHECK_PTR(idx_key, 16, "idx_key");
-  return ctx->cuda(launch_decode_append(ctx->view(layer), k, v, idx_key, (cudaStream_t)stream), "decode_append");
+  qsa_status st = ctx->cuda(launch_decode_append(ctx->view(layer), k, v, idx_key, (cudaStream_t)stream),
+                            "decode_append");
+  if (st == QSA_OK) ctx->layers[layer].pending_blocks = 0;  // the call pools every completed block
+  return st;
 }
 
 qsa_status qsa_update_pooled_cache(qsa_ctx* ctx, int32_t layer, qsa_stream_t stream) {
@@ -300,8 +310,10 @@ qsa_status qsa_index_topk(qsa_ctx* ctx, int32_t layer, const void* q_idx, const 
   if (scores && !aligned(scores, 16)) return ctx->fail(QSA_ERR_INVALID_ARG, "scores must be 16-byte aligned");
   LayerView v = ctx->view(layer);
   float* s = scores ? scores : v.scores;
-  if (qsa_status st = ctx->cuda(launch_index_scan(v, q_idx, w, s, (cudaStream_t)stream), "index scan")) return st;
-  return ctx->cuda(launch_topk(v, s, sel_blocks, n_sel, (cudaStream_t)stream), "block top-k");
+  // the scan fills the score-key histogram the selection starts from (and clears)
+  if (qsa_status st = ctx->cuda(launch_index_scan(v, q_idx, w, s, (cudaStream_t)stream, 1, 0, v.hist), "index scan"))
+    return st;
+  return ctx->cuda(launch_topk(v, s, sel_blocks, n_sel, (cudaStream_t)stream, 1, 0, v.hist), "block top-k");
 }
 
 qsa_status qsa_index_scores(qsa_ctx* ctx, int32_t layer, const void* q_idx, const float* w, float* scores,
@@ -433,9 +445,24 @@ qsa_status qsa_decode_step(qsa_ctx* ctx, int32_t layer, const void* k, const voi
   QSA_CHECK_PTR(out, 16, "out");
   const LayerView lv = ctx->view(layer);
   const cudaStream_t s = (cudaStream_t)stream;
-  if (qsa_status st = ctx->cuda(launch_decode_append(lv, k, v, idx_key, s), "decode_step: append")) return st;
-  if (qsa_status st = ctx->cuda(launch_index_scan(lv, q_idx, w, lv.scores, s), "decode_step: index scan")) return st;
-  if (qsa_status st = ctx->cuda(launch_topk(lv, lv.scores, sel_blocks, n_sel, s), "decode_step: block top-k"))
+  Layer& l = ctx->layers[layer];
+  if (l.pending_blocks == 0 && ctx->cfg.scan_kind == QSA_SCAN_TENSOR) {
+    // the pooled cache is current up to the previous token: the scan kernel itself
+    // appends the token and pools the block it completes (three launches per step)
+    if (qsa_status st = ctx->cuda(launch_decode_scan(lv, k, v, idx_key, q_idx, w, lv.scores, lv.hist, s),
+                                  "decode_step: append + index scan"))
+      return st;
+  } else {
+    // blocks are waiting to be pooled (after a bulk append or an invalidation), or the
+    // layer scans on the CUDA cores: the separate append pools every waiting block first
+    if (qsa_status st = ctx->cuda(launch_decode_append(lv, k, v, idx_key, s), "decode_step: append")) return st;
+    l.pending_blocks = 0;
+    if (qsa_status st = ctx->cuda(launch_index_scan(lv, q_idx, w, lv.scores, s, 1, 0, lv.hist),
+                                  "decode_step: index scan"))
+      return st;
+  }
+  if (qsa_status st = ctx->cuda(launch_topk(lv, lv.scores, sel_blocks, n_sel, s, 1, 0, lv.hist),
+                                "decode_step: block top-k"))
     return st;
   return ctx->cuda(launch_attend_selected(lv, q, sel_blocks, n_sel, out, s), "decode_step: sparse attend");
 }
@@ -444,8 +471,9 @@ qsa_status qsa_rollback(qsa_ctx* ctx, int32_t layer, int32_t n_keep, qsa_stream_
   if (!ctx) return QSA_ERR_INVALID_ARG;
   if (qsa_status st = ctx->layer_ok(layer)) return st;
   if (n_keep < 0) return ctx->fail(QSA_ERR_INVALID_ARG, "n_keep must be >= 0");
-  Layer& l = ctx->layers[layer];
-  l.pending_blocks += 2;  // the invalidated tail blocks (sizes the next update's grid only)
+  // Dropping tokens never adds blocks to pool: the kept summaries [0, n_keep/4) stay valid
+  // and the pooled count is cut to them, so the count of blocks waiting to be pooled can
+  // only fall (pending_blocks stays an upper bound).
   return ctx->cuda(launch_set_state(ctx->view(layer), n_keep, 0, kSetRollback, (cudaStream_t)stream), "rollback");
 }
 

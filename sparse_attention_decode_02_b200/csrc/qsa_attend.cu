@@ -17,6 +17,7 @@
 #include <mutex>
 
 #include "qsa_device.cuh"
+#include "qsa_timeline.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -439,8 +440,10 @@ attn_cluster_kernel(DevState* st, const __half* __restrict__ q, const int32_t* _
   n_ids += u;
 
   pdl_launch_dependents();
+  if (tid == 0) QSA_TL(st, kTlAttn, kTlEntry);
   cluster_arrive_relaxed();  // paired with cluster_wait() before the partials are pushed
   pdl_wait();
+  if (tid == 0) QSA_TL(st, kTlAttn, kTlWait);
   const int n_full = ld_volatile(&st->n_ctx);
   const int c0 = rank * Lc;
   // this thread's id, loaded in the same round trip as the counts (clamped into the id
@@ -497,6 +500,7 @@ attn_cluster_kernel(DevState* st, const __half* __restrict__ q, const int32_t* _
     s_cell[i] = cell;
   }
   __syncthreads();
+  if (tid == 0) QSA_TL(st, kTlAttn2, 0);  // cells known
   // stage the selected K and V rows (rows of invalid or padding cells are zero-filled)
   if constexpr (!FP8) {
     for (int e = tid; e < LP * CH; e += kAcThreads) {
@@ -544,6 +548,7 @@ attn_cluster_kernel(DevState* st, const __half* __restrict__ q, const int32_t* _
   }
   cp_async_commit_wait_all();
   __syncthreads();
+  if (tid == 0) QSA_TL(st, kTlAttn, kTlA);  // rows staged
 
   // ---- logits = Q K^T: warp w takes 8-cell tiles w and w + 16 ----
   const float scale = 1.0f / sqrtf((float)D);
@@ -575,6 +580,7 @@ attn_cluster_kernel(DevState* st, const __half* __restrict__ q, const int32_t* _
   rmax = fmaxf(rmax, __shfl_xor_sync(0xffffffffu, rmax, 2));
   if (tq == 0) s_rmax[warp * 8 + gq] = rmax;
   __syncthreads();
+  if (tid == 0) QSA_TL(st, kTlAttn2, 1);  // logits done
   float m = -INFINITY;
 #pragma unroll
   for (int w = 0; w < 16; ++w) m = fmaxf(m, s_rmax[w * 8 + gq]);
@@ -627,7 +633,9 @@ attn_cluster_kernel(DevState* st, const __half* __restrict__ q, const int32_t* _
   constexpr int PER = (PAIRS + CS - 1) / CS;
   float2* s_in = reinterpret_cast<float2*>(smem + SM::in_off(Lc, CS));  // [CS][PER]
   __syncthreads();  // s_o, s_m and s_l are complete
+  if (tid == 0) QSA_TL(st, kTlAttn2, 2);  // P.V done
   cluster_wait();   // every CTA of the cluster has started: its shared memory may be written
+  if (tid == 0) QSA_TL(st, kTlAttn2, 3);
   for (int pidx = tid; pidx < PAIRS; pidx += kAcThreads) {
     const int h = pidx / (D / 2), d2 = pidx % (D / 2);
     const float2 v = *reinterpret_cast<const float2*>(s_o + h * D + 2 * d2);
@@ -639,7 +647,9 @@ attn_cluster_kernel(DevState* st, const __half* __restrict__ q, const int32_t* _
     dst[0] = s_m[h];
     dst[1] = s_l[h];
   }
+  if (tid == 0) QSA_TL(st, kTlAttn2, 4);  // pushed
   cluster.sync();  // release the pushes above, acquire every other CTA's
+  if (tid == 0) QSA_TL(st, kTlAttn, kTlB);
   for (int t = tid; t < PER; t += kAcThreads) {
     const int pidx = rank * PER + t;
     if (pidx >= PAIRS) break;
@@ -663,6 +673,7 @@ attn_cluster_kernel(DevState* st, const __half* __restrict__ q, const int32_t* _
     if (den > 0.0f) res = make_float2(a0 / den, a1 / den);
     *reinterpret_cast<float2*>(out + (size_t(g) * G + h) * D + 2 * d2) = res;
   }
+  if (tid == 0) QSA_TL(st, kTlAttn, kTlExit);
 }
 
 template <int D, int G, int CS, bool FB, bool FP8>

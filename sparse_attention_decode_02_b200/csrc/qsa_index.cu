@@ -11,6 +11,7 @@
 
 #include "qsa_select.cuh"
 #include "qsa_checked.cuh"
+#include "qsa_timeline.cuh"
 
 namespace qsa {
 
@@ -18,27 +19,35 @@ namespace qsa {
 // the selected blocks in ascending order. With gridDim.y = T > 1 (multi-query step),
 // cluster u selects for the query of token n_ctx - T + u from score row u into output
 // row u (rows of k_blocks ids, one count each).
+// With `hist` (single query), the selection starts from the scan's score-key histogram.
 template <int V>
 __global__ void __launch_bounds__(sel::kThreads, 1)
 block_topk_kernel(DevState* st, const float* __restrict__ scores, int32_t* __restrict__ sel_out,
-                  int32_t* __restrict__ n_sel, int k_blocks, int max_blocks, int score_stride) {
+                  int32_t* __restrict__ n_sel, int k_blocks, int max_blocks, int score_stride, uint32_t* hist) {
   const int rank = int(cooperative_groups::this_cluster().block_rank());
   const int u = blockIdx.y, n_back = gridDim.y - 1 - blockIdx.y;
   scores += size_t(u) * score_stride;
   sel_out += size_t(u) * k_blocks;
   n_sel += u;
   pdl_launch_dependents();
+  if (threadIdx.x == 0) QSA_TL(st, kTlTopk, kTlEntry);
   cluster_arrive_relaxed();  // paired inside cluster_select
   pdl_wait();
-  const sel::Result res = sel::cluster_select<V>(st, scores, k_blocks, max_blocks, n_back,
+  if (threadIdx.x == 0) QSA_TL(st, kTlTopk, kTlWait);
+  const sel::Result res = sel::cluster_select<V>(st, scores, gridDim.y == 1 ? hist : nullptr, k_blocks, max_blocks,
+                                                 n_back,
                                                  [&](uint32_t pos, int block) {
-                                                   if (QSA_GUARD(st, pos < uint32_t(k_blocks) && block < max_blocks))
+                                                   // bounds-checked in every build
+                                                   if (pos < uint32_t(k_blocks) && block < max_blocks)
                                                      sel_out[pos] = block;
+                                                   else
+                                                     record_status(st, QSA_ERR_BAD_INDEX);
                                                  });
   if (res.status == sel::kAll)
     for (int i = rank * sel::kThreads + threadIdx.x; i < res.n_blocks; i += sel::kCS * sel::kThreads) sel_out[i] = i;
   if (rank == 0 && threadIdx.x == 0)
     *n_sel = res.status == sel::kTopK ? k_blocks : res.status == sel::kAll ? res.n_blocks : 0;
+  if (threadIdx.x == 0) QSA_TL(st, kTlTopk, kTlExit);
 }
 
 namespace {
@@ -70,18 +79,19 @@ cudaError_t init_kernel_attributes() {
 }
 
 cudaError_t launch_topk(const LayerView& L, const float* scores, int32_t* sel_out, int32_t* n_sel, cudaStream_t s,
-                        int n_queries, int score_stride) {
+                        int n_queries, int score_stride, uint32_t* hist) {
+  if (n_queries != 1) hist = nullptr;
   const int max_blocks = L.cfg.max_ctx / kBlock;
   const int kb = L.cfg.top_k_tokens / kBlock;
   const dim3 grid(sel::kCS, n_queries), block(sel::kThreads);
   if (max_blocks <= sel::kCS * sel::kThreads * 8)
     return launch_pdl(block_topk_kernel<8>, grid, block, 0, s, sel::kCS, L.state, scores, sel_out, n_sel, kb,
-                      max_blocks, score_stride);
+                      max_blocks, score_stride, hist);
   if (max_blocks <= sel::kCS * sel::kThreads * 16)
     return launch_pdl(block_topk_kernel<16>, grid, block, 0, s, sel::kCS, L.state, scores, sel_out, n_sel, kb,
-                      max_blocks, score_stride);
+                      max_blocks, score_stride, hist);
   return launch_pdl(block_topk_kernel<32>, grid, block, 0, s, sel::kCS, L.state, scores, sel_out, n_sel, kb,
-                    max_blocks, score_stride);
+                    max_blocks, score_stride, hist);
 }
 
 }  // namespace qsa

@@ -19,6 +19,7 @@ constexpr int kTopkMaxK = kTopkThreads * 32 / kTopkCluster;  // largest top_k_to
 constexpr int kMaxQueries = 4;        // queries verified together by the multi-query calls
 constexpr int kAttnWarps = 8;         // warps per attention CTA
 constexpr int kAttnMaxCells = 64;     // cells per attention CTA (split size cap)
+constexpr int kHistBits = 11;         // score-key prefix bits the scan histograms for the selection
 
 // Device-resident sequence state of one layer; lives at the start of the workspace.
 struct DevState {
@@ -27,13 +28,16 @@ struct DevState {
   int32_t status;         // first device-side error (qsa_status), 0 if none
   uint32_t ticket_append; // last-CTA tickets of multi-CTA kernels (reset by the last CTA)
   uint32_t ticket_pool;
-  int32_t reserved[59];
+  // timeline build only (-DQSA_TIMELINE): [kernel][point][min, max] of the low 32 bits of
+  // %globaltimer (ns) that the CTAs of the step's kernels reached at each probe point
+  uint32_t timeline[5][5][2];  // scan, top-k, attention, top-k detail, attention detail
+  int32_t reserved[9];
 };
 static_assert(sizeof(DevState) == 256, "DevState must stay 256 bytes");
 
 // Byte offsets inside a layer's workspace (all 256-byte aligned).
 struct WorkspaceLayout {
-  size_t state, scores, part_o, part_ml, total;
+  size_t state, hist, scores, part_o, part_ml, total;
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -66,6 +70,8 @@ inline WorkspaceLayout workspace_layout(const qsa_config& c, int n_splits) {
   size_t off = 0;
   w.state = off;
   off += align256(sizeof(DevState));
+  w.hist = off;  // score-key prefix histogram of the last scan (zero between selections)
+  off += align256(size_t(1 << kHistBits) * sizeof(uint32_t));
   w.scores = off;  // kMaxQueries rows of score_stride_of(c) floats
   off += align256(size_t(kMaxQueries) * score_stride_of(c) * sizeof(float));
   w.part_o = off;
@@ -87,6 +93,7 @@ struct LayerView {
   float* kv_scales;       // [max_ctx][n_kv_heads][2] f32 with QSA_KV_FP8, else null
   DevState* state;
   float* scores;          // workspace scores
+  uint32_t* hist;         // workspace score-key prefix histogram
   float* part_o;
   float* part_ml;
   AttnSplit split;
@@ -109,10 +116,21 @@ cudaError_t launch_decode_append(const LayerView& L, const void* k, const void* 
 // The index/top-k/attention launchers take n_queries T >= 1: query t (t < T) belongs to
 // token n_ctx - T + t and sees only the first n_ctx - T + t + 1 tokens. Per-query inputs
 // and outputs are consecutive rows (scores: rows of score_stride floats).
+// With `hist` (single query only) the scan also fills the score-key prefix histogram and
+// the selection starts from it (and clears it for the next scan).
 cudaError_t launch_index_scan(const LayerView& L, const void* q_idx, const float* w,
-                              float* scores, cudaStream_t s, int n_queries = 1, int score_stride = 0);
+                              float* scores, cudaStream_t s, int n_queries = 1, int score_stride = 0,
+                              uint32_t* hist = nullptr);
 cudaError_t launch_topk(const LayerView& L, const float* scores, int32_t* sel, int32_t* n_sel,
-                        cudaStream_t s, int n_queries = 1, int score_stride = 0);
+                        cudaStream_t s, int n_queries = 1, int score_stride = 0, uint32_t* hist = nullptr);
+// The same scan on the CUDA cores (scan_kind = QSA_SCAN_CUDA_CORES; single query).
+cudaError_t init_scan_cc_attributes();
+cudaError_t launch_index_scan_cc(const LayerView& L, const void* q_idx, const float* w, float* scores,
+                                 uint32_t* hist, cudaStream_t s);
+// Decode step's first launch: append the token at n_ctx (pooling the block it completes)
+// and scan, filling `hist`. Needs the pooled cache current up to the token before.
+cudaError_t launch_decode_scan(const LayerView& L, const void* k, const void* v, const void* idx,
+                               const void* q_idx, const float* w, float* scores, uint32_t* hist, cudaStream_t s);
 cudaError_t launch_gather(const LayerView& L, const int32_t* sel, const int32_t* n_sel,
                           int32_t* cells, int32_t* n_cells, void* k_compact, void* v_compact,
                           cudaStream_t s);

@@ -19,11 +19,27 @@
 //    warps 0-3 read the accumulator back (one row per thread) and form the score.
 // No tile is re-read: every pooled byte crosses HBM once (plus at most 15 rows per CTA
 // of rounding to the 16-row box).
+//
+// Two options ride on the same kernel:
+//  - HIST: the epilogue also counts every score's 11-bit key prefix (the sign, exponent
+//    and two mantissa bits of the order-preserving key the selection ranks by) into a
+//    2048-bin histogram in the layer workspace, so the selection kernel starts from the
+//    bin that holds the K-th score instead of running its own first radix pass;
+//  - FUSED (the decode step): the kernel first appends the token (K/V row and indexer key
+//    at position n_ctx) and, when that token completes a block, pools the block (section
+//    "incremental pooled-key cache（COMMON-004）": only the new block is computed) before
+//    scoring it, so a decode step needs no separate append launch. A seventh warp of the
+//    CTA that owns the last rows does both; the new pooled row reaches the TMA loads
+//    through a proxy fence and an mbarrier. The CTAs publish the new length with a
+//    last-CTA ticket.
 #include <cuda.h>
 #include <cuda_fp16.h>
 
 #include "qsa_device.cuh"
+#include "qsa_pool.cuh"
+#include "qsa_select.cuh"
 #include "qsa_sm100.cuh"
+#include "qsa_timeline.cuh"
 
 namespace qsa {
 
@@ -33,8 +49,10 @@ using namespace sm100;
 
 constexpr int kAcc = 4;          // TMEM accumulators
 constexpr int kBoxRows = 16;     // TMA box height
-constexpr int kThreads = 192;    // warps 0-3 epilogue, warp 4 TMA, warp 5 MMA + TMEM owner
+// warps 0-3 epilogue, warp 4 TMA, warp 5 MMA + TMEM owner, warp 6 append + pool (FUSED)
+constexpr int kThreads = 224;
 constexpr float kLoScale = 4096.0f;
+constexpr int kHistBins = 1 << kHistBits;
 
 constexpr size_t kSmemMax = 227 * 1024;  // dynamic shared memory per CTA
 
@@ -53,8 +71,8 @@ struct ScanShape {
       ACC_COLS <= 32 ? 32 : ACC_COLS <= 64 ? 64 : ACC_COLS <= 128 ? 128 : ACC_COLS <= 256 ? 256 : 512;
   static constexpr uint32_t IDESC = idesc_f16_f32(128, N);
   // barriers and TMEM address (256 B), sin/cos (T*D floats), RoPE frequencies (D/2
-  // doubles), raw queries (T*H*D f16)
-  static constexpr int CTRL_BYTES = 256 + T * D * 4 + D / 2 * 8 + T * H * D * 2;
+  // doubles), raw queries (T*H*D f16), the score-prefix histogram, one pooled row (f32)
+  static constexpr int CTRL_BYTES = 256 + T * D * 4 + D / 2 * 8 + T * H * D * 2 + kHistBins * 4 + D * 4;
   static constexpr size_t FIXED = 1024 + size_t(B_BYTES) + CTRL_BYTES;
   // ring depth: 6 tiles where they fit (all single-query shapes), fewer for wide B operands
   static constexpr int STAGES = FIXED + 6 * size_t(TILE_BYTES) <= kSmemMax ? 6
@@ -76,12 +94,89 @@ __device__ __forceinline__ uint32_t sw128_offset(int n, int k, int half_bytes) {
 
 }  // namespace
 
-template <int D, int H, int T>
+// The fused decode step's token and caches (FUSED only).
+struct DecodeAppend {
+  const uint4* k;           // the token's K and V rows [Hkv][hd] f16 and indexer key [d] f16
+  const uint4* v;
+  const uint4* idx;
+  uint4* k_cache;           // caches (K/V in f16, or e4m3 codes with kv_scales)
+  uint4* v_cache;
+  uint4* idx_cache;
+  __half* pooled;           // the pooled cache the TMA maps describe
+  const float* gain;        // RMS-norm gain or null
+  float* kv_scales;
+  PoolRope rope;
+  float eps;
+  int kv_units, max_ctx, n_kv_heads, head_dim, fp8, gen;
+};
+
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Warp 6 of the CTA that owns the last rows, in a decode step: after the dependency wait,
+// appends the token at position n_old (K/V rows, FP8-quantised when the cache is, and the
+// raw indexer key) and, when the token completes block b = (n_old + 1)/4 - 1, pools that
+// block from its first three cached keys and the token's own key, writes the summary and
+// makes it visible to the TMA loads (proxy fence, then an arrival on pool_bar). The
+// summary is bit-identical to the one the pooling kernels compute.
+template <int D, bool GEN>
+__device__ __forceinline__ void decode_append_pool(const DecodeAppend& a, DevState* st, uint64_t* pool_bar,
+                                                   float* s_row, int lane) {
+  const PoolLane<D, GEN> c = pool_lane_consts<D, GEN>(lane, a.gain, a.rope.base, a.rope.dims, a.rope.interleaved);
+  pdl_wait();
+  const int n_old = ld_volatile(&st->n_ctx);
+  const int n_pooled = ld_volatile(&st->n_pooled);
+  if (n_old < 0 || n_old >= a.max_ctx || n_pooled != n_old / kBlock) return;  // the grid skips (reported there)
+  if (!a.fp8) {
+    for (int i = lane; i < a.kv_units; i += 32) {
+      a.k_cache[size_t(n_old) * a.kv_units + i] = a.k[i];
+      a.v_cache[size_t(n_old) * a.kv_units + i] = a.v[i];
+    }
+  } else {
+    const __half* kh = reinterpret_cast<const __half*>(a.k);
+    const __half* vh = reinterpret_cast<const __half*>(a.v);
+    for (int r = 0; r < 2 * a.n_kv_heads; ++r) {
+      const KvRow kr = kv_row(r, size_t(n_old), kh, vh, reinterpret_cast<unsigned char*>(a.k_cache),
+                              reinterpret_cast<unsigned char*>(a.v_cache), a.kv_scales, a.n_kv_heads, a.head_dim);
+      fp8_row_store(fp8_row_load(kr.src, a.head_dim, lane), kr.dst, kr.scale, a.head_dim, lane);
+    }
+  }
+  constexpr int IDX_UNITS = D * 2 / 16;
+  if (lane < IDX_UNITS) a.idx_cache[size_t(n_old) * IDX_UNITS + lane] = a.idx[lane];
+  const int n = n_old + 1;
+  if (n % kBlock) return;
+  const int b = n / kBlock - 1;
+  // raw keys of the block: three cached rows, then the token's own key (from the input)
+  PoolRaw<D> raw;
+  constexpr int P = D / 64, HALF = D / 2;
+  const __half* ic = reinterpret_cast<const __half*>(a.idx_cache);
+  const __half* key = reinterpret_cast<const __half*>(a.idx);
+#pragma unroll
+  for (int t = 0; t < kBlock; ++t) {
+    const __half* row = t < kBlock - 1 ? ic + (size_t(b) * kBlock + t) * D : key;
+    if constexpr (P == 2) {
+      raw.x1[t] = *reinterpret_cast<const __half2*>(row + lane * 2);
+      raw.x2[t] = *reinterpret_cast<const __half2*>(row + lane * 2 + HALF);
+    } else {
+      raw.x1[t] = __halves2half2(row[lane], __float2half_rn(0.0f));
+      raw.x2[t] = __halves2half2(row[lane + HALF], __float2half_rn(0.0f));
+    }
+  }
+  pool_finish<D, GEN>(b, lane, c, raw, a.pooled, a.eps, a.rope.pos, s_row);
+  fence_proxy_async_global();  // the summary, written through the generic proxy, is read by TMA
+  __syncwarp();
+  if (lane == 0) mbar_arrive(pool_bar);
+}
+
+template <int D, int H, int T, bool HIST, bool FUSED>
 __global__ void __launch_bounds__(kThreads, 1)
 index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_constant__ CUtensorMap map_box,
                      DevState* st, const __half* __restrict__ q_idx, const float* __restrict__ w,
-                     float* __restrict__ scores, float rope_base, int max_blocks, int rope_dims,
-                     int rope_interleaved, int rope_pos_stride, int score_stride) {
+                     float* __restrict__ scores, uint32_t* __restrict__ hist, float rope_base, int max_blocks,
+                     int rope_dims, int rope_interleaved, int rope_pos_stride, int score_stride, DecodeAppend app) {
+  static_assert(!(HIST || FUSED) || T == 1, "histogram and fused append serve the single-query step");
+  static_assert(!FUSED || HIST, "the decode step always fills the histogram");
   using S = ScanShape<D, H, T>;
   constexpr int kStages = S::STAGES;
   extern __shared__ unsigned char smem_raw[];
@@ -92,14 +187,18 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_
   uint64_t* empty = full + kStages;
   uint64_t* tfull = empty + kStages;
   uint64_t* tempty = tfull + kAcc;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tempty + kAcc);
-  float* s_cos = reinterpret_cast<float*>(tmem_holder + 4);
+  uint64_t* pool_bar = tempty + kAcc;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(pool_bar + 1);
+  float* s_cos = reinterpret_cast<float*>(smem + size_t(kStages) * S::TILE_BYTES + S::B_BYTES + 256);
   float* s_sin = s_cos + T * (D / 2);                                 // [T][D/2] each
   double* s_theta = reinterpret_cast<double*>(s_sin + T * (D / 2));   // D/2 doubles
   __half* s_q = reinterpret_cast<__half*>(s_theta + D / 2);           // raw queries, T x H x D
+  uint32_t* s_hist = reinterpret_cast<uint32_t*>(s_q + T * H * D);    // [kHistBins]
+  float* s_row = reinterpret_cast<float*>(s_hist + kHistBins);        // [D] (pooling, generic RoPE)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   pdl_launch_dependents();
+  if (threadIdx.x == 0) QSA_TL(st, kTlScan, kTlEntry);
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
@@ -109,6 +208,7 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_
       mbar_init(&tfull[a], 1);
       mbar_init(&tempty[a], 128);
     }
+    mbar_init(pool_bar, 1);
     fence_mbar_init();
   }
   if (warp == 5) {
@@ -122,7 +222,7 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_
     // the context length read here, before the dependency wait, may be one token stale,
     // which only shifts the prefetched range slightly. Prefetches change nothing that
     // later loads observe; the real loads below use the current length.
-    const int nb_hint = min(max(ld_volatile(&st->n_ctx), 0) / kBlock, max_blocks);
+    const int nb_hint = min(max(ld_volatile(&st->n_ctx) + (FUSED ? 1 : 0), 0) / kBlock, max_blocks);
     const int p0 = int((long long)blockIdx.x * nb_hint / gridDim.x);
     const int p1 = int((long long)(blockIdx.x + 1) * nb_hint / gridDim.x);
     for (int r = p0; r < p1; r += 128)
@@ -137,17 +237,35 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
 
-  pdl_wait();
-  const int n = ld_volatile(&st->n_ctx);
+  if (FUSED && warp == 6) {
+    // ---------------- warp 6: the decode step's append and new-block pooling ----------------
+    if (blockIdx.x == gridDim.x - 1) {
+      if (app.gen) decode_append_pool<D, true>(app, st, pool_bar, s_row, lane);
+      else decode_append_pool<D, false>(app, st, pool_bar, s_row, lane);
+    } else {
+      pdl_wait();
+    }
+  }
+  if (!(FUSED && warp == 6)) pdl_wait();
+  if (threadIdx.x == 0) QSA_TL(st, kTlScan, kTlWait);
+  const int n_old = ld_volatile(&st->n_ctx);
+  const int n_pooled = ld_volatile(&st->n_pooled);
+  // tokens the (last) query sees; the decode step's token is appended by this kernel
+  const int n = FUSED ? n_old + 1 : n_old;
+  bool state_ok = n_pooled == n_old / kBlock;
+  if (FUSED) state_ok = state_ok && n_old >= 0 && n_old < app.max_ctx;
+  if (!state_ok && blockIdx.x == 0 && threadIdx.x == 0)
+    record_status(st, FUSED && (n_old >= app.max_ctx) ? QSA_ERR_CAPACITY : QSA_ERR_STATE);
   const int n_blocks = n / kBlock;
-  const bool stale = ld_volatile(&st->n_pooled) != n_blocks;
-  if (stale && blockIdx.x == 0 && threadIdx.x == 0) record_status(st, QSA_ERR_STATE);
   const int r0 = int((long long)blockIdx.x * n_blocks / gridDim.x);
   const int r1 = int((long long)(blockIdx.x + 1) * n_blocks / gridDim.x);
-  const int n_rows = stale ? 0 : r1 - r0;
+  const int n_rows = state_ok ? r1 - r0 : 0;
   const int n_tiles = (n_rows + 127) / 128;
+  // the tile that holds the block this step completes (last CTA of a fused step), or -1
+  const int pool_tile = (FUSED && state_ok && n % kBlock == 0 && blockIdx.x == gridDim.x - 1)
+                            ? (n_blocks - 1 - r0) / 128 : -1;
 
-  if (n_tiles > 0) {
+  if (n_tiles > 0 && warp < 6) {
     if (warp == 4) {
       // ---------------- TMA producer ----------------
       if (lane == 0) {
@@ -156,6 +274,10 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_
         for (int t = 0; t < n_tiles && ok; ++t) {
           const int s = t % kStages;
           if (t >= kStages && !mbar_wait(&empty[s], ((t / kStages) - 1) & 1)) {
+            ok = false;
+            break;
+          }
+          if (FUSED && t == pool_tile && !mbar_wait(pool_bar, 0)) {  // the new summary is in memory
             ok = false;
             break;
           }
@@ -190,6 +312,7 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_
         for (int t = 0; t < n_tiles; ++t) {
           const int s = t % kStages, a = t % kAcc;
           if (!mbar_wait(&full[s], (t / kStages) & 1)) { ok = false; break; }
+          if (t == 0) QSA_TL(st, kTlScan, kTlA);  // first tile landed
           if (t >= kAcc && !mbar_wait(&tempty[a], ((t / kAcc) - 1) & 1)) { ok = false; break; }
           tc_fence_after();
           const uint32_t d_tmem = tmem_base + uint32_t(a * S::N);
@@ -220,6 +343,8 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_
 #pragma unroll
       for (int k = 0; k < (QV + 127) / 128; ++k)
         if (tid + k * 128 < QV) qraw[k] = reinterpret_cast<const uint4*>(q_idx)[tid + k * 128];
+      if constexpr (HIST)
+        for (int i = tid; i < kHistBins; i += 128) s_hist[i] = 0u;
       // query u belongs to token n - T + u: on the block-position scale it sits at
       // floor(stride * (n_u - 1) / 4), n_u = n - T + u + 1 (token n_u - 1 when stride = 4)
       const int half_r = rope_dims / 2;
@@ -308,11 +433,21 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_
 #pragma unroll
             for (int h = 0; h < H; ++h)
               s += wr[u][h] * fmaxf(__uint_as_float(r[u][h]) + __uint_as_float(r[u][H + h]) * (1.0f / kLoScale), 0.0f);
-            scores[size_t(u) * score_stride + row] = s / sqrt_d;
+            const float score = s / sqrt_d;
+            scores[size_t(u) * score_stride + row] = score;
+            if constexpr (HIST) atomicAdd(&s_hist[sel::score_key(score) >> (32 - kHistBits)], 1u);
           }
         }
       }
       if (!ok && tid == 0) record_status(st, QSA_ERR_TIMEOUT);
+      if (tid == 0) QSA_TL(st, kTlScan, kTlB);  // this thread's rows scored
+      if constexpr (HIST) {  // this CTA's counts into the layer's histogram
+        named_bar_sync(2, 128);
+        for (int i = tid; i < kHistBins; i += 128) {
+          const uint32_t c = s_hist[i];
+          if (c) atomicAdd(hist + i, c);
+        }
+      }
     }
   }
   tc_fence_before();
@@ -321,22 +456,38 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_
     tc_fence_after();
     tmem_dealloc(tmem_base, S::TMEM_COLS);
   }
+  if (threadIdx.x == 0) QSA_TL(st, kTlScan, kTlExit);
+  if (FUSED && state_ok && threadIdx.x == 0) {
+    // the last CTA to finish publishes the new length (every CTA has read the old one)
+    __threadfence();
+    const unsigned t = atomicAdd(&st->ticket_append, 1u);
+    if (t == gridDim.x - 1) {
+      st->n_ctx = n;
+      st->n_pooled = n / kBlock;
+      st->ticket_append = 0;
+      __threadfence();
+    }
+  }
 }
 
 // ---------------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------------
-template <int D, int H, int T>
+template <int D, int H, int T, bool HIST, bool FUSED>
 static cudaError_t set_scan_attr() {
-  return cudaFuncSetAttribute(index_scan_tc_kernel<D, H, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  return cudaFuncSetAttribute(index_scan_tc_kernel<D, H, T, HIST, FUSED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               (int)ScanShape<D, H, T>::SMEM);
 }
 
 template <int D, int H>
 static cudaError_t set_scan_attr_t() {
   cudaError_t e;
-  if ((e = set_scan_attr<D, H, 1>()) != cudaSuccess || (e = set_scan_attr<D, H, 2>()) != cudaSuccess ||
-      (e = set_scan_attr<D, H, 3>()) != cudaSuccess || (e = set_scan_attr<D, H, 4>()) != cudaSuccess)
+  if ((e = set_scan_attr<D, H, 1, false, false>()) != cudaSuccess ||
+      (e = set_scan_attr<D, H, 1, true, false>()) != cudaSuccess ||
+      (e = set_scan_attr<D, H, 1, true, true>()) != cudaSuccess ||
+      (e = set_scan_attr<D, H, 2, false, false>()) != cudaSuccess ||
+      (e = set_scan_attr<D, H, 3, false, false>()) != cudaSuccess ||
+      (e = set_scan_attr<D, H, 4, false, false>()) != cudaSuccess)
     return e;
   return cudaSuccess;
 }
@@ -381,44 +532,83 @@ cudaError_t encode_pooled_map(const qsa_config& c, void* pooled, int box_rows, C
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-template <int D, int H, int T>
+template <int D, int H, int T, bool HIST, bool FUSED>
 static cudaError_t launch_scan_tc(const LayerView& L, const void* q_idx, const float* w, float* scores,
-                                  cudaStream_t s, int score_stride) {
-  return launch_pdl(index_scan_tc_kernel<D, H, T>, dim3(L.n_sms), dim3(kThreads), ScanShape<D, H, T>::SMEM, s, 1,
-                    L.pooled_tile_map, L.pooled_box_map, L.state, (const __half*)q_idx, w, scores, L.cfg.rope_base,
-                    L.cfg.max_ctx / kBlock, L.cfg.rope_dims, L.cfg.rope_interleaved, L.cfg.rope_pos_stride,
-                    score_stride);
+                                  cudaStream_t s, int score_stride, uint32_t* hist, const DecodeAppend& app) {
+  return launch_pdl(index_scan_tc_kernel<D, H, T, HIST, FUSED>, dim3(L.n_sms), dim3(kThreads),
+                    ScanShape<D, H, T>::SMEM, s, 1, L.pooled_tile_map, L.pooled_box_map, L.state,
+                    (const __half*)q_idx, w, scores, hist, L.cfg.rope_base, L.cfg.max_ctx / kBlock, L.cfg.rope_dims,
+                    L.cfg.rope_interleaved, L.cfg.rope_pos_stride, score_stride, app);
 }
 
+// mode 0: plain scan of T queries; 1: single query with the histogram; 2: decode step
 template <int D, int H>
 static cudaError_t launch_scan_tc_t(const LayerView& L, const void* q_idx, const float* w, float* scores,
-                                    cudaStream_t s, int n_queries, int score_stride) {
+                                    cudaStream_t s, int n_queries, int score_stride, uint32_t* hist, int mode,
+                                    const DecodeAppend& app) {
+  if (mode == 2) return launch_scan_tc<D, H, 1, true, true>(L, q_idx, w, scores, s, score_stride, hist, app);
+  if (mode == 1) return launch_scan_tc<D, H, 1, true, false>(L, q_idx, w, scores, s, score_stride, hist, app);
   switch (n_queries) {
-    case 1: return launch_scan_tc<D, H, 1>(L, q_idx, w, scores, s, score_stride);
-    case 2: return launch_scan_tc<D, H, 2>(L, q_idx, w, scores, s, score_stride);
-    case 3: return launch_scan_tc<D, H, 3>(L, q_idx, w, scores, s, score_stride);
-    case 4: return launch_scan_tc<D, H, 4>(L, q_idx, w, scores, s, score_stride);
+    case 1: return launch_scan_tc<D, H, 1, false, false>(L, q_idx, w, scores, s, score_stride, hist, app);
+    case 2: return launch_scan_tc<D, H, 2, false, false>(L, q_idx, w, scores, s, score_stride, hist, app);
+    case 3: return launch_scan_tc<D, H, 3, false, false>(L, q_idx, w, scores, s, score_stride, hist, app);
+    case 4: return launch_scan_tc<D, H, 4, false, false>(L, q_idx, w, scores, s, score_stride, hist, app);
     default: return cudaErrorInvalidValue;
   }
 }
 
 template <int D>
 static cudaError_t launch_scan_tc_d(const LayerView& L, const void* q_idx, const float* w, float* scores,
-                                    cudaStream_t s, int n_queries, int score_stride) {
+                                    cudaStream_t s, int n_queries, int score_stride, uint32_t* hist, int mode,
+                                    const DecodeAppend& app) {
   switch (L.cfg.n_idx_heads) {
-    case 1: return launch_scan_tc_t<D, 1>(L, q_idx, w, scores, s, n_queries, score_stride);
-    case 2: return launch_scan_tc_t<D, 2>(L, q_idx, w, scores, s, n_queries, score_stride);
-    case 4: return launch_scan_tc_t<D, 4>(L, q_idx, w, scores, s, n_queries, score_stride);
-    case 8: return launch_scan_tc_t<D, 8>(L, q_idx, w, scores, s, n_queries, score_stride);
-    case 16: return launch_scan_tc_t<D, 16>(L, q_idx, w, scores, s, n_queries, score_stride);
+    case 1: return launch_scan_tc_t<D, 1>(L, q_idx, w, scores, s, n_queries, score_stride, hist, mode, app);
+    case 2: return launch_scan_tc_t<D, 2>(L, q_idx, w, scores, s, n_queries, score_stride, hist, mode, app);
+    case 4: return launch_scan_tc_t<D, 4>(L, q_idx, w, scores, s, n_queries, score_stride, hist, mode, app);
+    case 8: return launch_scan_tc_t<D, 8>(L, q_idx, w, scores, s, n_queries, score_stride, hist, mode, app);
+    case 16: return launch_scan_tc_t<D, 16>(L, q_idx, w, scores, s, n_queries, score_stride, hist, mode, app);
     default: return cudaErrorInvalidValue;
   }
 }
 
+static cudaError_t launch_scan_mode(const LayerView& L, const void* q_idx, const float* w, float* scores,
+                                    cudaStream_t s, int n_queries, int score_stride, uint32_t* hist, int mode,
+                                    const DecodeAppend& app) {
+  return L.cfg.d_idx == 128 ? launch_scan_tc_d<128>(L, q_idx, w, scores, s, n_queries, score_stride, hist, mode, app)
+                            : launch_scan_tc_d<64>(L, q_idx, w, scores, s, n_queries, score_stride, hist, mode, app);
+}
+
 cudaError_t launch_index_scan(const LayerView& L, const void* q_idx, const float* w, float* scores,
-                              cudaStream_t s, int n_queries, int score_stride) {
-  return L.cfg.d_idx == 128 ? launch_scan_tc_d<128>(L, q_idx, w, scores, s, n_queries, score_stride)
-                            : launch_scan_tc_d<64>(L, q_idx, w, scores, s, n_queries, score_stride);
+                              cudaStream_t s, int n_queries, int score_stride, uint32_t* hist) {
+  if (L.cfg.scan_kind == QSA_SCAN_CUDA_CORES && n_queries == 1)
+    return launch_index_scan_cc(L, q_idx, w, scores, hist, s);
+  const int mode = (hist && n_queries == 1) ? 1 : 0;
+  return launch_scan_mode(L, q_idx, w, scores, s, n_queries, score_stride, mode ? hist : nullptr, mode,
+                          DecodeAppend{});
+}
+
+cudaError_t launch_decode_scan(const LayerView& L, const void* k, const void* v, const void* idx, const void* q_idx,
+                               const float* w, float* scores, uint32_t* hist, cudaStream_t s) {
+  DecodeAppend app{};
+  app.k = static_cast<const uint4*>(k);
+  app.v = static_cast<const uint4*>(v);
+  app.idx = static_cast<const uint4*>(idx);
+  app.k_cache = static_cast<uint4*>(L.k_cache);
+  app.v_cache = static_cast<uint4*>(L.v_cache);
+  app.idx_cache = static_cast<uint4*>(L.idx_cache);
+  app.pooled = static_cast<__half*>(L.pooled_cache);
+  app.gain = L.rms_gain;
+  app.kv_scales = L.kv_scales;
+  app.rope = PoolRope{L.cfg.rope_base, L.cfg.rope_dims, L.cfg.rope_interleaved,
+                      RopePos{L.cfg.rope_pos_stride, L.cfg.rope_pos_offset}};
+  app.eps = L.cfg.rms_eps;
+  app.kv_units = L.cfg.n_kv_heads * L.cfg.head_dim * 2 / 16;
+  app.max_ctx = L.cfg.max_ctx;
+  app.n_kv_heads = L.cfg.n_kv_heads;
+  app.head_dim = L.cfg.head_dim;
+  app.fp8 = L.cfg.kv_format == QSA_KV_FP8;
+  app.gen = L.cfg.rope_dims != L.cfg.d_idx || L.cfg.rope_interleaved != 0;
+  return launch_scan_mode(L, q_idx, w, scores, s, 1, 0, hist, 2, app);
 }
 
 }  // namespace qsa

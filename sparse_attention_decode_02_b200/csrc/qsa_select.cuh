@@ -8,21 +8,23 @@
 // Rule of this library: the min(K, B) largest scores, ties to the lower block index,
 // output in ascending block order.
 //
-// An exact radix select on order-preserving 32-bit keys: 8-bit digits from the top,
-// stopping as soon as every key with the current prefix is needed. CTA r of the cluster
-// owns blocks [r*kTopkThreads*V, (r+1)*kTopkThreads*V), thread t the V consecutive blocks
-// starting at t*V, held in registers. Per pass, each CTA histograms its keys in shared
-// memory and pushes the histogram into every CTA's inbox with distributed-shared-memory
-// stores; after one cluster barrier each CTA adds the histograms from its own memory. The
-// output position of a selected block is the number of keys above the threshold before
-// it plus min(need, ties before it), so one packed prefix scan and one pushed exchange of
-// per-CTA totals give every position; ties are taken in block order. No CTA reads
-// another's shared memory.
+// An exact radix select on order-preserving 32-bit keys: 8-bit digits from the top (or
+// from the 11-bit bin the scan's histogram points at), stopping as soon as every key with
+// the current prefix is needed. CTA r of the cluster owns blocks
+// [r*kTopkThreads*V, (r+1)*kTopkThreads*V), thread t the V consecutive blocks starting at
+// t*V, held in registers. Per pass, each CTA histograms its keys in shared memory and
+// pushes the histogram into every CTA's inbox with distributed-shared-memory stores; after
+// one cluster barrier each CTA adds the histograms from its own memory. The output
+// position of a selected block is the number of keys above the threshold before it plus
+// min(need, ties before it); the per-CTA counts follow from the pushed histograms, so one
+// packed prefix scan inside the CTA gives every position; ties are taken in block order.
+// No CTA reads another's shared memory.
 #pragma once
 
 #include <cooperative_groups.h>
 
 #include "qsa_device.cuh"
+#include "qsa_timeline.cuh"
 
 namespace qsa {
 
@@ -87,21 +89,39 @@ struct Result {
 // emit(position, block) once per selected block (kTopK only) and returns the same result
 // in every thread of the cluster. Cluster-barrier pairing is complete on return on every
 // path.
+//
+// With `hist` (the 2048-bin histogram of the scores' 11-bit key prefixes that the scan
+// filled for exactly these blocks), the bin holding the K-th largest key comes from the
+// histogram and the radix passes only refine the keys inside that bin (bits 20..13,
+// 12..5, 4..0). Without it, or if its total does not match the block count (a scan whose
+// selection never ran), the passes start from the top byte. The histogram is cleared for
+// the next scan in either case.
+//
+// Output positions need, for every CTA, how many of its keys lie above the final
+// threshold and at it. Each CTA pushes its whole pass histogram (plus, in the first pass,
+// its count of keys above the starting bin) to every CTA, so each CTA derives every
+// other CTA's counts from its own inbox: no exchange of totals is needed.
 template <int V, class Emit>
-__device__ __forceinline__ Result cluster_select(DevState* st, const float* __restrict__ scores, int k_blocks,
-                                                 int max_blocks, int n_back, Emit&& emit) {
-  __shared__ uint32_t s_hist[256];          // this CTA's histogram of the pass
-  __shared__ uint32_t s_in[2][kCS][256];    // every CTA's histogram, double-buffered by pass
+__device__ __forceinline__ Result cluster_select(DevState* st, const float* __restrict__ scores, uint32_t* hist,
+                                                 int k_blocks, int max_blocks, int n_back, Emit&& emit) {
+  constexpr int kSlots = 257;                 // 256 digit bins + the first pass's count above
+  constexpr int kHB = 1 << kHistBits;         // 2048
+  static_assert(kThreads * 4 == kHB, "each thread reads 4 histogram bins");
+  static_assert(kThreads / 32 == kCS, "one warp per source CTA when reading the inbox");
+  __shared__ uint32_t s_hist[kSlots];          // this CTA's histogram of the pass
+  __shared__ uint32_t s_in[2][kCS][kSlots];    // every CTA's histogram, double-buffered by pass
   __shared__ uint32_t s_warp[32];
-  __shared__ uint32_t s_ctl[4];             // digit, count above the digit, count at the digit
-  __shared__ uint32_t s_all[2 * kCS];       // every CTA's (greater, equal) totals
+  __shared__ uint32_t s_ctl[4];                // digit, count above the digit, count at the digit
+  __shared__ uint32_t s_gt[kCS], s_eq[kCS];    // per CTA: keys above the threshold, keys at it
+  __shared__ uint32_t s_gt0;                   // this CTA's keys above the histogram's bin
 
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = int(cluster.block_rank());
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
   // this thread's V scores, read up to the buffer's capacity (max_ctx/4) in the same round
-  // trip as the state; blocks at or past n_ctx/4 are masked once the state is known
+  // trip as the state and the histogram; blocks at or past n_ctx/4 are masked once the
+  // state is known. Thread t reads bins [2044 - 4t, 2048 - 4t): thread 0 the top ones.
   const int base = rank * kThreads * V + tid * V;
   float f[V];
   if (base + V <= max_blocks) {
@@ -117,19 +137,34 @@ __device__ __forceinline__ Result cluster_select(DevState* st, const float* __re
 #pragma unroll
     for (int j = 0; j < V; ++j) f[j] = base + j < max_blocks ? scores[base + j] : 0.0f;
   }
+  uint4 h4 = make_uint4(0u, 0u, 0u, 0u);
+  if (hist) h4 = *reinterpret_cast<const uint4*>(hist + (kHB - 4 - 4 * tid));
   const int n_full = ld_volatile(&st->n_ctx);
   const int n_pooled = ld_volatile(&st->n_pooled);
 #pragma unroll
   for (int j = 0; j < V; ++j) asm volatile("" ::"f"(f[j]));  // keep the loads ahead of the branches
+  asm volatile("" ::"r"(h4.x), "r"(h4.y), "r"(h4.z), "r"(h4.w));
   const int n = n_full - n_back;
   const int n_blocks = n / kBlock;
+  // clears this CTA's slice of the histogram once every CTA of the cluster has read it
+  auto clear_hist = [&]() {
+    if (hist && tid < kHB / kCS) hist[rank * (kHB / kCS) + tid] = 0u;
+  };
   if (n_pooled != n_full / kBlock || n < 0) {  // uniform over the cluster
     if (rank == 0 && tid == 0) record_status(st, QSA_ERR_STATE);
     cluster_wait();
+    if (hist) {
+      cluster.sync();
+      clear_hist();
+    }
     return Result{kStale, n, 0};
   }
   if (n_blocks <= k_blocks) {  // uniform over the cluster
     cluster_wait();
+    if (hist) {
+      cluster.sync();
+      clear_hist();
+    }
     return Result{kAll, n, n_blocks};
   }
 
@@ -140,33 +175,78 @@ __device__ __forceinline__ Result cluster_select(DevState* st, const float* __re
     key[j] = score_key(f[j]);
     if (base + j < n_blocks) valid |= 1u << j;
   }
-  if (tid < 256) s_hist[tid] = 0;
-  cluster_wait();  // every CTA of the cluster has started: its shared memory may be written
+  if (tid < kSlots) s_hist[tid] = 0;
+  if (tid < kCS) s_gt[tid] = 0;
+  if (tid == 0) s_gt0 = 0;
 
+  // the starting prefix: the histogram's bin holding the K-th largest key, if the
+  // histogram counts exactly these blocks
   uint32_t prefix = 0, mask = 0, need = uint32_t(k_blocks);
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
-    __syncthreads();  // the local histogram is zeroed
+  int first_shift = 24;   // first refinement pass: bits [first_shift, first_shift + 8)
+  if (hist) {
+    const uint32_t c4 = h4.x + h4.y + h4.z + h4.w;
+    uint32_t total;
+    const uint32_t above = cta_exclusive_scan(c4, s_warp, &total);  // keys in higher bins
+    if (total == uint32_t(n_blocks)) {  // uniform: every thread sees the same total
+      // bins of this thread from the top: 2047-4t (h4.w), then h4.z, h4.y, h4.x
+      const uint32_t hb[4] = {h4.w, h4.z, h4.y, h4.x};
+      uint32_t acc = above;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if (acc < need && acc + hb[i] >= need) {
+          s_ctl[0] = uint32_t(kHB - 1 - 4 * tid - i);
+          s_ctl[1] = acc;
+        }
+        acc += hb[i];
+      }
+      __syncthreads();
+      const uint32_t b1 = s_ctl[0];
+      need -= s_ctl[1];
+      prefix = b1 << (32 - kHistBits);
+      mask = ~0u << (32 - kHistBits);
+      first_shift = 32 - kHistBits - 8;  // 13
+      uint32_t g0 = 0;
+#pragma unroll
+      for (int j = 0; j < V; ++j) g0 += ((valid >> j) & 1u) && (key[j] >> (32 - kHistBits)) > b1;
+      if (g0) atomicAdd(&s_gt0, g0);
+    }
+  }
+  if (tid == 0) QSA_TL(st, kTlTopk2, 0);  // loads and the histogram's bin done
+  cluster_wait();  // every CTA of the cluster has started: its shared memory may be written
+  if (tid == 0) QSA_TL(st, kTlTopk2, 1);
+
+  // radix passes over the keys that match the prefix, 8-bit digits (the last one narrower)
+  for (int pass = 0, shift = first_shift;; ++pass) {
+    const int bits = shift >= 0 ? 8 : 8 + shift;
+    shift = shift >= 0 ? shift : 0;
+    const uint32_t nb = 1u << bits;
+    __syncthreads();  // the local histogram is zeroed, s_gt0 complete
 #pragma unroll
     for (int j = 0; j < V; ++j)
-      if (((valid >> j) & 1u) && (key[j] & mask) == prefix) atomicAdd(&s_hist[(key[j] >> shift) & 255u], 1u);
+      if (((valid >> j) & 1u) && (key[j] & mask) == prefix) atomicAdd(&s_hist[(key[j] >> shift) & (nb - 1)], 1u);
+    if (pass == 0 && tid == 0) s_hist[256] = s_gt0;
     __syncthreads();
-    // push bin t into slot [rank][t] of every CTA's inbox for this pass, and clear it for
-    // the next pass. A CTA reuses an inbox buffer two passes later, after a barrier that
-    // every CTA passes only once all have finished reading it.
-    if (tid < 256) {
+    // push slot t into [rank][t] of every CTA's inbox for this pass, and clear it for the
+    // next pass. A CTA reuses an inbox buffer two passes later, after a barrier that every
+    // CTA passes only once all have finished reading it.
+    if (tid < kSlots) {
       const uint32_t mine = s_hist[tid];
       s_hist[tid] = 0;
 #pragma unroll
-      for (int r = 0; r < kCS; ++r) cluster.map_shared_rank(&s_in[pass & 1][0][0], r)[rank * 256 + tid] = mine;
+      for (int r = 0; r < kCS; ++r) cluster.map_shared_rank(&s_in[pass & 1][0][0], r)[rank * kSlots + tid] = mine;
     }
+    if (pass == 0 && tid == 0) QSA_TL(st, kTlTopk2, 2);  // pass 0 pushed
     cluster.sync();  // release the pushes, acquire every other CTA's
-    // thread t < 256 takes digit (255 - t): an inclusive prefix over t counts keys >= digit
+    if (pass == 0 && tid == 0) QSA_TL(st, kTlTopk, kTlA);
+    if (pass == 1 && tid == 0) QSA_TL(st, kTlTopk2, 3);
+    if (pass == 0) clear_hist();  // every CTA read the histogram before its first push
+    const uint32_t(*in)[kSlots] = s_in[pass & 1];
+    // thread t < nb takes digit (nb - 1 - t): an inclusive prefix over t counts keys >= digit
     uint32_t v = 0;
-    if (tid < 256) {
-      const int bin = 255 - tid;
+    if (tid < int(nb)) {
+      const int bin = int(nb) - 1 - tid;
 #pragma unroll
-      for (int r = 0; r < kCS; ++r) v += s_in[pass & 1][r][bin];
+      for (int r = 0; r < kCS; ++r) v += in[r][bin];
     }
     uint32_t x = v;
 #pragma unroll
@@ -176,22 +256,39 @@ __device__ __forceinline__ Result cluster_select(DevState* st, const float* __re
     }
     if (lane == 31 && warp < 8) s_warp[warp] = x;
     __syncthreads();
-    if (tid < 256) {
+    if (tid < int(nb)) {
       uint32_t excl = x - v;
 #pragma unroll
       for (int w = 0; w < 8; ++w) excl += w < warp ? s_warp[w] : 0u;
       if (excl < need && excl + v >= need) {
-        s_ctl[0] = uint32_t(255 - tid);
+        s_ctl[0] = uint32_t(int(nb) - 1 - tid);
         s_ctl[1] = excl;
         s_ctl[2] = v;
       }
     }
     __syncthreads();
+    const uint32_t d = s_ctl[0];
+    // per source CTA (warp r reads CTA r's row): its keys above the digit in this pass
+    // (plus its count above the histogram's bin), and at the digit
+    {
+      const int r = warp;
+      uint32_t a = 0;
+      for (int b = lane; b < int(nb); b += 32) a += b > int(d) ? in[r][b] : 0u;
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) a += __shfl_xor_sync(0xffffffffu, a, off);
+      if (lane == 0) {
+        s_gt[r] += a + (pass == 0 ? in[r][256] : 0u);
+        s_eq[r] = in[r][d];
+      }
+    }
     need -= s_ctl[1];
-    prefix |= s_ctl[0] << shift;
-    mask |= 255u << shift;
-    if (s_ctl[2] == need) break;  // every key with this prefix is selected (uniform)
+    prefix |= d << shift;
+    mask |= (nb - 1) << shift;
+    if (s_ctl[2] == need || shift == 0) break;  // uniform: the threshold is fixed
+    shift -= 8;
   }
+  __syncthreads();  // s_gt and s_eq complete
+  if (tid == 0) QSA_TL(st, kTlTopk, kTlB);
 
   // classify: above the threshold prefix, or equal to it (ties go by block order)
   uint32_t c_gt = 0, c_eq = 0;
@@ -204,17 +301,12 @@ __device__ __forceinline__ Result cluster_select(DevState* st, const float* __re
   }
   uint32_t tot;
   const uint32_t before = cta_exclusive_scan((c_gt << 16) | c_eq, s_warp, &tot);
-  if (tid < kCS) {  // push this CTA's totals to every CTA
-    uint32_t* dst = cluster.map_shared_rank(s_all, tid);
-    dst[2 * rank] = tot >> 16;
-    dst[2 * rank + 1] = tot & 0xffffu;
-  }
-  cluster.sync();
+  if (tid == 0) QSA_TL(st, kTlTopk2, 4);
   uint32_t gt_before = before >> 16, eq_before = before & 0xffffu;
 #pragma unroll
   for (int r = 0; r < kCS; ++r) {
-    gt_before += r < rank ? s_all[2 * r] : 0u;
-    eq_before += r < rank ? s_all[2 * r + 1] : 0u;
+    gt_before += r < rank ? s_gt[r] : 0u;
+    eq_before += r < rank ? s_eq[r] : 0u;
   }
 #pragma unroll
   for (int j = 0; j < V; ++j) {

@@ -1,0 +1,30 @@
+// Timeline probes of the timeline build (-DQSA_TIMELINE): each decode-step kernel records
+// in its layer's device state (DevState::timeline) the first and last value of
+// %globaltimer (low 32 bits, ns) that its CTAs reach at named points (entry, return from
+// the dependency wait, two phase ends, exit), with 32-bit atomic min/max. The host clears
+// the record (min slots to all ones, max slots to zero) and reads it back from the layer
+// workspace. The default build compiles every probe to nothing.
+#pragma once
+
+#include <stdint.h>
+
+#include "qsa_internal.h"
+
+namespace qsa {
+
+enum { kTlScan = 0, kTlTopk = 1, kTlAttn = 2, kTlTopk2 = 3, kTlAttn2 = 4 };
+enum { kTlEntry = 0, kTlWait = 1, kTlA = 2, kTlB = 3, kTlExit = 4 };
+
+#ifdef QSA_TIMELINE
+__device__ __forceinline__ void tl_mark(DevState* st, int kernel, int point) {
+  uint32_t t;
+  asm volatile("mov.u32 %0, %%globaltimer_lo;" : "=r"(t));
+  atomicMin(&st->timeline[kernel][point][0], t);
+  atomicMax(&st->timeline[kernel][point][1], t);
+}
+#define QSA_TL(st, kernel, point) ::qsa::tl_mark((st), (kernel), (point))
+#else
+#define QSA_TL(st, kernel, point) ((void)0)
+#endif
+
+}  // namespace qsa

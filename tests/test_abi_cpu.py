@@ -104,6 +104,13 @@ def test_fp8_buffer_sizes(lib):
     assert Q.buffer_bytes(bad, Q.QSA_BUF_KV) == 0
 
 
+def test_scan_kind_is_validated(lib):
+    cfg = Q.make_config(1, 4096, 128, 16, 2048, 32, 4, 128, scan_kind=Q.QSA_SCAN_CUDA_CORES)
+    assert Q.buffer_bytes(cfg, Q.QSA_BUF_KV) == 4096 * 4 * 128 * 2
+    cfg.scan_kind = 2
+    assert Q.buffer_bytes(cfg, Q.QSA_BUF_KV) == 0
+
+
 def test_null_arguments_are_rejected(lib):
     assert lib.qsa_create(None, None) == 1
     lib.qsa_destroy(None)  # no-op

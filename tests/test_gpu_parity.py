@@ -445,8 +445,9 @@ def test_decode_append_equals_append_then_update():
 
 @pytest.mark.slow
 def test_streaming_512_steps_12_layers():
-    """The streaming workload: from the 256k prefill, 512 fused decode steps on each of the 12
-    layers (128 block completions per layer). Every 128 steps the live pooled cache equals a
+    """The streaming workload: from the 256k prefill, 512 decode steps (qsa_decode_step, the
+    append and pooled update fused into the scan launch) on each of the 12 layers (128
+    block completions per layer). Every 128 steps the live pooled cache equals a
     full rebuild bit for bit; at steps 0, 127, 255, 383 and 511 the step's selection and
     attention match the oracle, whose pooled cache evolves incrementally every step."""
     wl = synth.workload("stream256k_12l")
@@ -463,9 +464,9 @@ def test_streaming_512_steps_12_layers():
         ref.update_pooled_cache()
         del pre
         for step, st in enumerate(synth.step_inputs_range(wl, layer, 0, wl.n_steps)):
-            qsa.decode_append(0, H.to_dev(st["k"]), H.to_dev(st["v"]), H.to_dev(st["idx"]))
-            g.index_topk(st["q_idx"], st["w"])
-            g.attend_selected(st["q"])
+            d = {k: H.to_dev(x) for k, x in st.items()}   # the bench's call: qsa_decode_step
+            qsa.decode_step(0, d["k"], d["v"], d["idx"], d["q_idx"], d["w"], d["q"], g.outs["sel"], g.outs["n_sel"],
+                            g.outs["out"])
             ref.append_tokens(st["k"][None], st["v"][None], st["idx"][None])
             ref.update_pooled_cache()
             n = ref.n
