@@ -6,8 +6,9 @@ the indexer-scan kernel itself appends the token and pools the block the token c
 computed), then the selection (starting from the scan's score-key histogram), then the
 attention. These tests hold it bit for bit to the separate calls (qsa_decode_append,
 qsa_index_topk, qsa_sparse_attend_selected) over several block completions, for the
-default layer, the RoPE switches and the FP8 K/V cache, check it against the oracle, and
-cover the four-launch form taken after a bulk append and the capacity limit.
+default layer, the RoPE switches and the FP8 K/V cache, check it against the oracle
+(adversarial tables for the histogram-started selection included), and cover the form
+taken after a bulk append and the capacity limit.
 """
 import numpy as np
 import pytest
@@ -146,3 +147,38 @@ def test_decode_step_reports_capacity_and_writes_nothing():
     assert (n, p) == (1024, 256) and status == 2  # QSA_ERR_CAPACITY
     for k, t in before.items():
         assert torch.equal(g.buf[k], t), k
+
+
+@pytest.mark.parametrize("table", ["repeats10", "allequal", "zeroquery", "random"])
+@pytest.mark.parametrize("wl_name,n0", [("tiny", 4 * 600 + 1), ("ctx256k_12l", 255181)])
+def test_decode_step_selection_on_adversarial_tables(wl_name, n0, table):
+    """The decode step's selection (started from the scan's score-key histogram) on pooled
+    tables that take every path of the radix passes: exact ties within and across CTAs
+    (rows repeating ten base rows, one row everywhere, a zero query so that every score is
+    0 and the whole key decides by block order) and plain N(0,1) rows. The selection must
+    be the oracle's on the same f16 table (ties to the lower block)."""
+    wl = synth.workload(wl_name)
+    qsa, g, pre = _layer(wl, n0, extra=8)
+    g.update()
+    B = n0 // 4
+    base = synth.random_pooled(wl, 0, 10, salt=3)
+    if table == "repeats10":
+        pooled = base[np.arange(B) % 10]
+    elif table == "allequal":
+        pooled = np.repeat(base[:1], B, axis=0)
+    else:
+        pooled = synth.random_pooled(wl, 0, B, salt=11)
+    g.buf["pooled_cache"][:B] = H.to_dev(pooled)
+    st = dict(synth.step_inputs(wl, 0, 0))   # n0 + 1 tokens: no block completes
+    if table == "zeroquery":
+        st["q_idx"] = np.zeros_like(st["q_idx"])
+    _decode_step(qsa, g, st)
+    torch.cuda.synchronize()
+    n = n0 + 1
+    assert n % 4 != 0 and g.state() == (n, B, 0)
+    got = g.outs["sel"][: int(g.outs["n_sel"][0])].cpu().numpy().astype(np.int64)
+    ref_scores = O.block_scores(pooled, st["q_idx"], st["w"], n, O.QsaShape.of(wl))
+    gap = 0.0 if table in ("repeats10", "allequal", "zeroquery") else H.TIE_GAP_REL
+    H.selection_mismatch(got, ref_scores, wl.k_blocks, gap)
+    if table in ("allequal", "zeroquery"):
+        assert got.tolist() == list(range(wl.k_blocks))
