@@ -680,6 +680,9 @@ template <int D, int G, int CS, bool FB, bool FP8>
 static cudaError_t set_ac_attr1(size_t smem) {
   cudaError_t e = cudaFuncSetAttribute(attn_cluster_kernel<D, G, CS, FB, FP8>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(attn_cluster_kernel<D, G, CS, FB, FP8>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             kCarveoutMaxShared);
   if (e == cudaSuccess && CS > 8)
     e = cudaFuncSetAttribute(attn_cluster_kernel<D, G, CS, FB, FP8>, cudaFuncAttributeNonPortableClusterSizeAllowed,
                              1);

@@ -104,6 +104,13 @@ __device__ __forceinline__ float sum_over_heads(float x) {
   return x;
 }
 
+// Preferred shared-memory carveout of every kernel of the decode step: the largest shared
+// memory configuration. The scan, selection and attention kernels overlap through
+// programmatic dependent launch, and CTAs of different kernels can share an SM only when
+// the SM's configuration holds both; the largest one lets a scan CTA start beside an
+// attention CTA (or a selection CTA beside a scan CTA) instead of waiting for it to exit.
+constexpr int kCarveoutMaxShared = 100;  // percent (cudaSharedmemCarveoutMaxShared)
+
 // Launch with programmatic stream serialization (PDL) and an optional cluster shape.
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,

@@ -53,7 +53,10 @@ block_topk_kernel(DevState* st, const float* __restrict__ scores, int32_t* __res
 namespace {
 template <int V>
 cudaError_t set_topk_attr() {
-  return cudaFuncSetAttribute(block_topk_kernel<V>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  cudaError_t e = cudaFuncSetAttribute(block_topk_kernel<V>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(block_topk_kernel<V>, cudaFuncAttributePreferredSharedMemoryCarveout, kCarveoutMaxShared);
+  return e;
 }
 }  // namespace
 

@@ -55,6 +55,10 @@ constexpr float kLoScale = 4096.0f;
 constexpr int kHistBins = 1 << kHistBits;
 
 constexpr size_t kSmemMax = 227 * 1024;  // dynamic shared memory per CTA
+#ifndef QSA_SCAN_STAGES
+#define QSA_SCAN_STAGES 3
+#endif
+constexpr int kScanStages = QSA_SCAN_STAGES;  // TMA ring depth (tiles of 128 rows)
 
 // Shapes of the scan for d = D, H indexer heads and T queries scored in one pass.
 template <int D, int H, int T>
@@ -74,8 +78,10 @@ struct ScanShape {
   // doubles), raw queries (T*H*D f16), the score-prefix histogram, one pooled row (f32)
   static constexpr int CTRL_BYTES = 256 + T * D * 4 + D / 2 * 8 + T * H * D * 2 + kHistBins * 4 + D * 4;
   static constexpr size_t FIXED = 1024 + size_t(B_BYTES) + CTRL_BYTES;
-  // ring depth: 6 tiles where they fit (all single-query shapes), fewer for wide B operands
-  static constexpr int STAGES = FIXED + 6 * size_t(TILE_BYTES) <= kSmemMax ? 6
+  // ring depth: kScanStages tiles where they fit, fewer for wide B operands. A short ring
+  // keeps the CTA small enough to be resident beside the attention and selection kernels'
+  // CTAs, so it can start (and prefetch) while they still run.
+  static constexpr int STAGES = FIXED + kScanStages * size_t(TILE_BYTES) <= kSmemMax ? kScanStages
                                 : FIXED + 5 * size_t(TILE_BYTES) <= kSmemMax ? 5 : 4;
   static constexpr size_t SMEM = FIXED + size_t(STAGES) * TILE_BYTES;
   static_assert(NQ <= 32, "the epilogue reads at most 32 accumulator columns per query");
@@ -458,14 +464,14 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_
   }
   if (threadIdx.x == 0) QSA_TL(st, kTlScan, kTlExit);
   if (FUSED && state_ok && threadIdx.x == 0) {
-    // the last CTA to finish publishes the new length (every CTA has read the old one)
-    __threadfence();
+    // the last CTA to finish publishes the new length: every CTA took its ticket after
+    // using the old one (no fence: the next kernel sees these writes once this grid
+    // completes)
     const unsigned t = atomicAdd(&st->ticket_append, 1u);
     if (t == gridDim.x - 1) {
       st->n_ctx = n;
       st->n_pooled = n / kBlock;
       st->ticket_append = 0;
-      __threadfence();
     }
   }
 }
@@ -475,8 +481,12 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_
 // ---------------------------------------------------------------------------------
 template <int D, int H, int T, bool HIST, bool FUSED>
 static cudaError_t set_scan_attr() {
-  return cudaFuncSetAttribute(index_scan_tc_kernel<D, H, T, HIST, FUSED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              (int)ScanShape<D, H, T>::SMEM);
+  cudaError_t e = cudaFuncSetAttribute(index_scan_tc_kernel<D, H, T, HIST, FUSED>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ScanShape<D, H, T>::SMEM);
+  if (e == cudaSuccess)  // the whole unified L1/shared array as shared memory (see qsa_device.cuh)
+    e = cudaFuncSetAttribute(index_scan_tc_kernel<D, H, T, HIST, FUSED>,
+                             cudaFuncAttributePreferredSharedMemoryCarveout, kCarveoutMaxShared);
+  return e;
 }
 
 template <int D, int H>
