@@ -330,6 +330,62 @@ qsa_status qsa_decode_step(qsa_ctx* ctx, int32_t layer, const void* k, const voi
                            const void* q_idx, const float* w, const void* q, int32_t* sel_blocks,
                            int32_t* n_sel, float* out, qsa_stream_t stream);
 
+/* ---- Context-parallel decode step (one layer sharded over devices) ----
+ * Part 10 (section "QSAとQSA indexerについて") handles long context by sparsity: the
+ * attended set stays at most 4K + 3 cells whatever the context length. For a context
+ * beyond one device, each device holds a contiguous, block-aligned shard of the layer as
+ * its own layer: global blocks [block_base, block_base + its n_ctx/4) and, on the last
+ * shard only, the open tail. Its config has rope_pos_offset = rope_pos_stride *
+ * block_base (plus the unsharded layer's own offset), so its blocks are pooled at their
+ * global positions; appends and pooled updates are the ordinary calls. One step:
+ *   1. every shard: qsa_cp_index_candidates (its local top-K as fixed-size slots);
+ *   2. the slots of all shards, shard by shard, gathered on every device (for instance an
+ *      all-gather of K floats and K ints per shard), then qsa_cp_select: the global
+ *      top-K, identical on every device;
+ *   3. every shard: qsa_cp_attend_partial over its part of the global selection;
+ *   4. the partials (out, lse) gathered, then qsa_cp_merge.
+ * The result equals the single-device step on the whole context: every block of the
+ * global top-K is in its own shard's local top-K, and candidates listed shard by shard in
+ * block order keep ties going to the lower block. The exchange itself is the caller's
+ * (NCCL or any collective); these calls only compute. */
+
+/* The shard's indexer scan with the query at global position n_global - 1 (rotated there,
+ * as the single-device scan rotates it at n_ctx - 1), then its local top-K:
+ *   cand_scores [top_k_tokens/4] f32, cand_blocks [top_k_tokens/4] i32: the selected
+ *   blocks' scores and GLOBAL ids (local id + block_base) in ascending block order; the
+ *   slots past the count hold -inf and -1; n_cand: a device i32, the count.
+ * Uses the layer workspace's score buffer. Requires the shard's pooled cache to be
+ * current (else QSA_ERR_STATE in the device status and n_cand = 0, all slots empty). */
+qsa_status qsa_cp_index_candidates(qsa_ctx* ctx, int32_t layer, const void* q_idx, const float* w, int32_t n_global,
+                                   int32_t block_base, float* cand_scores, int32_t* cand_blocks, int32_t* n_cand,
+                                   qsa_stream_t stream);
+
+/* The global top-K of every shard's slots: cand_scores [n_shards][k_blocks] f32 and
+ * cand_blocks [n_shards][k_blocks] i32 as qsa_cp_index_candidates writes them, shard by
+ * shard in block order. Rule of the single-device selection: the k_blocks largest scores,
+ * ties to the lower block, ascending; fewer candidates than k_blocks: all of them.
+ * Writes sel_blocks [k_blocks] (global ids) and n_sel (device i32). Needs no context:
+ * n_shards * k_blocks <= 8192 (QSA_ERR_UNSUPPORTED beyond), k_blocks <= 1024. */
+qsa_status qsa_cp_select(const float* cand_scores, const int32_t* cand_blocks, int32_t n_shards, int32_t k_blocks,
+                         int32_t* sel_blocks, int32_t* n_sel, qsa_stream_t stream);
+
+/* The shard's attention partial: over the blocks of the global selection (sel_blocks,
+ * n_sel from qsa_cp_select) that fall in [block_base, block_base + n_ctx/4), plus the
+ * shard's own open tail (the last shard's), like qsa_sparse_attend_selected:
+ *   out [n_q_heads][head_dim] f32: the normalised output over those cells;
+ *   lse [n_q_heads] f32: log sum_c exp(q_i . K[c] / sqrt(head_dim)); -inf and out = 0 when
+ *   the shard has no cell. Uses the layer workspace. */
+qsa_status qsa_cp_attend_partial(qsa_ctx* ctx, int32_t layer, const void* q, const int32_t* sel_blocks,
+                                 const int32_t* n_sel, int32_t block_base, float* out, float* lse,
+                                 qsa_stream_t stream);
+
+/* The exact merge of the shards' partials: o_parts [n_shards][n_q_heads][head_dim] f32,
+ * lse_parts [n_shards][n_q_heads] f32 -> out [n_q_heads][head_dim] f32,
+ * out = sum_r exp(lse_r - L) o_r / sum_r exp(lse_r - L), L = max_r lse_r (shards with lse
+ * -inf count 0; all of them: out = 0). Needs no context. */
+qsa_status qsa_cp_merge(const float* o_parts, const float* lse_parts, int32_t n_shards, int32_t n_q_heads,
+                        int32_t head_dim, float* out, qsa_stream_t stream);
+
 /* Size of the fixed scratch array behind qsa_sparse_attend_noalloc (1 MiB). */
 #define QSA_NOALLOC_SCRATCH_BYTES (1u << 20)
 

@@ -100,6 +100,8 @@ struct qsa_ctx {
     v.state = reinterpret_cast<DevState*>(wsp + ws.state);
     v.scores = reinterpret_cast<float*>(wsp + ws.scores);
     v.hist = reinterpret_cast<uint32_t*>(wsp + ws.hist);
+    v.cp_count = reinterpret_cast<int32_t*>(wsp + ws.cp);
+    v.cp_sel = v.cp_count + 16;
     v.part_o = reinterpret_cast<float*>(wsp + ws.part_o);
     v.part_ml = reinterpret_cast<float*>(wsp + ws.part_ml);
     v.split = split;
@@ -475,6 +477,69 @@ qsa_status qsa_rollback(qsa_ctx* ctx, int32_t layer, int32_t n_keep, qsa_stream_
   // and the pooled count is cut to them, so the count of blocks waiting to be pooled can
   // only fall (pending_blocks stays an upper bound).
   return ctx->cuda(launch_set_state(ctx->view(layer), n_keep, 0, kSetRollback, (cudaStream_t)stream), "rollback");
+}
+
+qsa_status qsa_cp_index_candidates(qsa_ctx* ctx, int32_t layer, const void* q_idx, const float* w, int32_t n_global,
+                                   int32_t block_base, float* cand_scores, int32_t* cand_blocks, int32_t* n_cand,
+                                   qsa_stream_t stream) {
+  if (!ctx) return QSA_ERR_INVALID_ARG;
+  if (qsa_status st = ctx->layer_ok(layer)) return st;
+  QSA_CHECK_PTR(q_idx, 16, "q_idx");
+  QSA_CHECK_PTR(w, 4, "w");
+  QSA_CHECK_PTR(cand_scores, 16, "cand_scores");
+  QSA_CHECK_PTR(cand_blocks, 16, "cand_blocks");
+  QSA_CHECK_PTR(n_cand, 4, "n_cand");
+  if (n_global < 1) return ctx->fail(QSA_ERR_INVALID_ARG, "n_global must be >= 1");
+  if (block_base < 0) return ctx->fail(QSA_ERR_INVALID_ARG, "block_base must be >= 0");
+  const LayerView v = ctx->view(layer);
+  const cudaStream_t s = (cudaStream_t)stream;
+  if (qsa_status st = ctx->cuda(launch_index_scan(v, q_idx, w, v.scores, s, 1, 0, v.hist, n_global),
+                                "cp_index_candidates: index scan"))
+    return st;
+  return ctx->cuda(launch_topk(v, v.scores, cand_blocks, n_cand, s, 1, 0, v.hist, cand_scores, block_base),
+                   "cp_index_candidates: local top-k");
+}
+
+qsa_status qsa_cp_attend_partial(qsa_ctx* ctx, int32_t layer, const void* q, const int32_t* sel_blocks,
+                                 const int32_t* n_sel, int32_t block_base, float* out, float* lse,
+                                 qsa_stream_t stream) {
+  if (!ctx) return QSA_ERR_INVALID_ARG;
+  if (qsa_status st = ctx->layer_ok(layer)) return st;
+  QSA_CHECK_PTR(q, 16, "q");
+  QSA_CHECK_PTR(sel_blocks, 4, "sel_blocks");
+  QSA_CHECK_PTR(n_sel, 4, "n_sel");
+  QSA_CHECK_PTR(out, 16, "out");
+  QSA_CHECK_PTR(lse, 4, "lse");
+  if (block_base < 0) return ctx->fail(QSA_ERR_INVALID_ARG, "block_base must be >= 0");
+  const LayerView v = ctx->view(layer);
+  const cudaStream_t s = (cudaStream_t)stream;
+  if (qsa_status st = ctx->cuda(launch_cp_filter(v, sel_blocks, n_sel, block_base, v.cp_sel, v.cp_count, s),
+                                "cp_attend_partial: this shard's blocks"))
+    return st;
+  return ctx->cuda(launch_attend_selected(v, q, v.cp_sel, v.cp_count, out, s, 1, lse), "cp_attend_partial: attend");
+}
+
+qsa_status qsa_cp_select(const float* cand_scores, const int32_t* cand_blocks, int32_t n_shards, int32_t k_blocks,
+                         int32_t* sel_blocks, int32_t* n_sel, qsa_stream_t stream) {
+  if (!cand_scores || !cand_blocks || !sel_blocks || !n_sel || !aligned(cand_scores, 4) || !aligned(cand_blocks, 4) ||
+      !aligned(sel_blocks, 4) || !aligned(n_sel, 4))
+    return QSA_ERR_INVALID_ARG;
+  if (n_shards < 1 || k_blocks < 1 || k_blocks > kTopkMaxK) return QSA_ERR_INVALID_ARG;
+  if (n_shards * k_blocks > 8192) return QSA_ERR_UNSUPPORTED;
+  return launch_cp_select(cand_scores, cand_blocks, n_shards, k_blocks, sel_blocks, n_sel, (cudaStream_t)stream) ==
+                 cudaSuccess
+             ? QSA_OK
+             : QSA_ERR_CUDA;
+}
+
+qsa_status qsa_cp_merge(const float* o_parts, const float* lse_parts, int32_t n_shards, int32_t n_q_heads,
+                        int32_t head_dim, float* out, qsa_stream_t stream) {
+  if (!o_parts || !lse_parts || !out || !aligned(o_parts, 4) || !aligned(lse_parts, 4) || !aligned(out, 4))
+    return QSA_ERR_INVALID_ARG;
+  if (n_shards < 1 || n_q_heads < 1 || head_dim < 1) return QSA_ERR_INVALID_ARG;
+  return launch_cp_merge(o_parts, lse_parts, n_shards, n_q_heads, head_dim, out, (cudaStream_t)stream) == cudaSuccess
+             ? QSA_OK
+             : QSA_ERR_CUDA;
 }
 
 qsa_status qsa_sparse_attend_selected(qsa_ctx* ctx, int32_t layer, const void* q, const int32_t* sel_blocks,

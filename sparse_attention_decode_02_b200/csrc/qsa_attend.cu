@@ -406,7 +406,7 @@ __global__ void __launch_bounds__(kAcThreads, 1)
 attn_cluster_kernel(DevState* st, const __half* __restrict__ q, const int32_t* __restrict__ ids,
                     const int32_t* __restrict__ n_ids, const void* __restrict__ kc_raw,
                     const void* __restrict__ vc_raw, float* __restrict__ out, int n_kv_heads, int cells_per_cta,
-                    int max_cells, int k_blocks, const float* __restrict__ kv_scales) {
+                    int max_cells, int k_blocks, const float* __restrict__ kv_scales, float* __restrict__ lse_out) {
   const __half* __restrict__ kc = static_cast<const __half*>(kc_raw);
   const __half* __restrict__ vc = static_cast<const __half*>(vc_raw);
   using SM = AcSmem<D, G>;
@@ -436,6 +436,7 @@ attn_cluster_kernel(DevState* st, const __half* __restrict__ q, const int32_t* _
   const int u = blockIdx.y, n_back = gridDim.y - 1 - blockIdx.y;
   q += size_t(u) * n_kv_heads * G * D;
   out += size_t(u) * n_kv_heads * G * D;
+  if (lse_out) lse_out += size_t(u) * n_kv_heads * G;
   ids += size_t(u) * (FROM_BLOCKS ? k_blocks : max_cells);
   n_ids += u;
 
@@ -672,6 +673,9 @@ attn_cluster_kernel(DevState* st, const __half* __restrict__ q, const int32_t* _
     float2 res = make_float2(0.0f, 0.0f);
     if (den > 0.0f) res = make_float2(a0 / den, a1 / den);
     *reinterpret_cast<float2*>(out + (size_t(g) * G + h) * D + 2 * d2) = res;
+    // log-sum-exp of the head's scaled logits over all its cells (a context-parallel
+    // shard's partial): max + log(sum of exp(logit - max)); -inf with no cells
+    if (lse_out && d2 == 0) lse_out[size_t(g) * G + h] = den > 0.0f ? M + logf(den) : -INFINITY;
   }
   if (tid == 0) QSA_TL(st, kTlAttn, kTlExit);
 }
@@ -697,7 +701,7 @@ static cudaError_t set_ac_attr(size_t smem) {
 
 template <int D, int G, int CS>
 static cudaError_t launch_ac(const LayerView& L, bool from_blocks, const void* q, const int32_t* ids,
-                             const int32_t* n_ids, float* out, cudaStream_t s, int n_queries) {
+                             const int32_t* n_ids, float* out, cudaStream_t s, int n_queries, float* lse) {
   const int lc = L.attn_cells_per_cta;
   const size_t smem = AcSmem<D, G>::bytes(lc, CS);
   const dim3 grid(L.cfg.n_kv_heads * CS, n_queries), block(kAcThreads);
@@ -706,7 +710,7 @@ static cudaError_t launch_ac(const LayerView& L, bool from_blocks, const void* q
   const float* scl = L.kv_scales;
 #define QSA_AC_LAUNCH(FB, F8)                                                                                    \
   launch_pdl(attn_cluster_kernel<D, G, CS, FB, F8>, grid, block, smem, s, CS, L.state, (const __half*)q, ids, n_ids, \
-             (const void*)L.k_cache, (const void*)L.v_cache, out, L.cfg.n_kv_heads, lc, mc, kb, scl)
+             (const void*)L.k_cache, (const void*)L.v_cache, out, L.cfg.n_kv_heads, lc, mc, kb, scl, lse)
   if (from_blocks) return fp8 ? QSA_AC_LAUNCH(true, true) : QSA_AC_LAUNCH(true, false);
   return fp8 ? QSA_AC_LAUNCH(false, true) : QSA_AC_LAUNCH(false, false);
 #undef QSA_AC_LAUNCH
@@ -714,33 +718,33 @@ static cudaError_t launch_ac(const LayerView& L, bool from_blocks, const void* q
 
 template <int D, int G>
 static cudaError_t launch_ac_g(const LayerView& L, bool fb, const void* q, const int32_t* ids, const int32_t* n_ids,
-                               float* out, cudaStream_t s, int nq) {
-  return L.attn_cluster == 16 ? launch_ac<D, G, 16>(L, fb, q, ids, n_ids, out, s, nq)
-                              : launch_ac<D, G, 8>(L, fb, q, ids, n_ids, out, s, nq);
+                               float* out, cudaStream_t s, int nq, float* lse) {
+  return L.attn_cluster == 16 ? launch_ac<D, G, 16>(L, fb, q, ids, n_ids, out, s, nq, lse)
+                              : launch_ac<D, G, 8>(L, fb, q, ids, n_ids, out, s, nq, lse);
 }
 
 template <int D>
 static cudaError_t launch_ac_d(const LayerView& L, bool fb, const void* q, const int32_t* ids, const int32_t* n_ids,
-                               float* out, cudaStream_t s, int nq) {
+                               float* out, cudaStream_t s, int nq, float* lse) {
   switch (L.cfg.n_q_heads / L.cfg.n_kv_heads) {
-    case 1: return launch_ac_g<D, 1>(L, fb, q, ids, n_ids, out, s, nq);
-    case 2: return launch_ac_g<D, 2>(L, fb, q, ids, n_ids, out, s, nq);
-    case 4: return launch_ac_g<D, 4>(L, fb, q, ids, n_ids, out, s, nq);
-    case 8: return launch_ac_g<D, 8>(L, fb, q, ids, n_ids, out, s, nq);
+    case 1: return launch_ac_g<D, 1>(L, fb, q, ids, n_ids, out, s, nq, lse);
+    case 2: return launch_ac_g<D, 2>(L, fb, q, ids, n_ids, out, s, nq, lse);
+    case 4: return launch_ac_g<D, 4>(L, fb, q, ids, n_ids, out, s, nq, lse);
+    case 8: return launch_ac_g<D, 8>(L, fb, q, ids, n_ids, out, s, nq, lse);
     default: return cudaErrorInvalidValue;
   }
 }
 
 cudaError_t launch_attend(const LayerView& L, const void* q, const int32_t* cells, const int32_t* n_cells, float* out,
                           cudaStream_t s) {
-  return L.cfg.head_dim == 128 ? launch_ac_d<128>(L, false, q, cells, n_cells, out, s, 1)
-                               : launch_ac_d<64>(L, false, q, cells, n_cells, out, s, 1);
+  return L.cfg.head_dim == 128 ? launch_ac_d<128>(L, false, q, cells, n_cells, out, s, 1, nullptr)
+                               : launch_ac_d<64>(L, false, q, cells, n_cells, out, s, 1, nullptr);
 }
 
 cudaError_t launch_attend_selected(const LayerView& L, const void* q, const int32_t* sel, const int32_t* n_sel,
-                                   float* out, cudaStream_t s, int n_queries) {
-  return L.cfg.head_dim == 128 ? launch_ac_d<128>(L, true, q, sel, n_sel, out, s, n_queries)
-                               : launch_ac_d<64>(L, true, q, sel, n_sel, out, s, n_queries);
+                                   float* out, cudaStream_t s, int n_queries, float* lse) {
+  return L.cfg.head_dim == 128 ? launch_ac_d<128>(L, true, q, sel, n_sel, out, s, n_queries, lse)
+                               : launch_ac_d<64>(L, true, q, sel, n_sel, out, s, n_queries, lse);
 }
 
 // Cluster size and cells per CTA for a configuration, plus the kernel attributes they

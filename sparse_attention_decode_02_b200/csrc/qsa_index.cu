@@ -20,10 +20,12 @@ namespace qsa {
 // cluster u selects for the query of token n_ctx - T + u from score row u into output
 // row u (rows of k_blocks ids, one count each).
 // With `hist` (single query), the selection starts from the scan's score-key histogram.
+// With sel_scores (single query): a context-parallel shard's candidate slots, below.
 template <int V>
 __global__ void __launch_bounds__(sel::kThreads, 1)
 block_topk_kernel(DevState* st, const float* __restrict__ scores, int32_t* __restrict__ sel_out,
-                  int32_t* __restrict__ n_sel, int k_blocks, int max_blocks, int score_stride, uint32_t* hist) {
+                  int32_t* __restrict__ n_sel, int k_blocks, int max_blocks, int score_stride, uint32_t* hist,
+                  float* __restrict__ sel_scores, int block_base) {
   const int rank = int(cooperative_groups::this_cluster().block_rank());
   const int u = blockIdx.y, n_back = gridDim.y - 1 - blockIdx.y;
   scores += size_t(u) * score_stride;
@@ -38,15 +40,27 @@ block_topk_kernel(DevState* st, const float* __restrict__ scores, int32_t* __res
                                                  n_back,
                                                  [&](uint32_t pos, int block) {
                                                    // bounds-checked in every build
-                                                   if (pos < uint32_t(k_blocks) && block < max_blocks)
-                                                     sel_out[pos] = block;
-                                                   else
+                                                   if (pos < uint32_t(k_blocks) && block < max_blocks) {
+                                                     sel_out[pos] = block + block_base;
+                                                     if (sel_scores) sel_scores[pos] = scores[block];
+                                                   } else {
                                                      record_status(st, QSA_ERR_BAD_INDEX);
+                                                   }
                                                  });
   if (res.status == sel::kAll)
-    for (int i = rank * sel::kThreads + threadIdx.x; i < res.n_blocks; i += sel::kCS * sel::kThreads) sel_out[i] = i;
-  if (rank == 0 && threadIdx.x == 0)
-    *n_sel = res.status == sel::kTopK ? k_blocks : res.status == sel::kAll ? res.n_blocks : 0;
+    for (int i = rank * sel::kThreads + threadIdx.x; i < res.n_blocks; i += sel::kCS * sel::kThreads) {
+      sel_out[i] = i + block_base;
+      if (sel_scores) sel_scores[i] = scores[i];
+    }
+  const int count = res.status == sel::kTopK ? k_blocks : res.status == sel::kAll ? res.n_blocks : 0;
+  if (rank == 0 && threadIdx.x == 0) *n_sel = count;
+  // candidate slots: the positions past the count hold score -inf and block -1
+  if (sel_scores)
+    for (int i = rank * sel::kThreads + threadIdx.x; i < k_blocks; i += sel::kCS * sel::kThreads)
+      if (i >= count) {
+        sel_scores[i] = -INFINITY;
+        sel_out[i] = -1;
+      }
   if (threadIdx.x == 0) QSA_TL(st, kTlTopk, kTlExit);
 }
 
@@ -82,19 +96,19 @@ cudaError_t init_kernel_attributes() {
 }
 
 cudaError_t launch_topk(const LayerView& L, const float* scores, int32_t* sel_out, int32_t* n_sel, cudaStream_t s,
-                        int n_queries, int score_stride, uint32_t* hist) {
-  if (n_queries != 1) hist = nullptr;
+                        int n_queries, int score_stride, uint32_t* hist, float* sel_scores, int block_base) {
+  if (n_queries != 1) hist = nullptr, sel_scores = nullptr, block_base = 0;
   const int max_blocks = L.cfg.max_ctx / kBlock;
   const int kb = L.cfg.top_k_tokens / kBlock;
   const dim3 grid(sel::kCS, n_queries), block(sel::kThreads);
   if (max_blocks <= sel::kCS * sel::kThreads * 8)
     return launch_pdl(block_topk_kernel<8>, grid, block, 0, s, sel::kCS, L.state, scores, sel_out, n_sel, kb,
-                      max_blocks, score_stride, hist);
+                      max_blocks, score_stride, hist, sel_scores, block_base);
   if (max_blocks <= sel::kCS * sel::kThreads * 16)
     return launch_pdl(block_topk_kernel<16>, grid, block, 0, s, sel::kCS, L.state, scores, sel_out, n_sel, kb,
-                      max_blocks, score_stride, hist);
+                      max_blocks, score_stride, hist, sel_scores, block_base);
   return launch_pdl(block_topk_kernel<32>, grid, block, 0, s, sel::kCS, L.state, scores, sel_out, n_sel, kb,
-                    max_blocks, score_stride, hist);
+                    max_blocks, score_stride, hist, sel_scores, block_base);
 }
 
 }  // namespace qsa

@@ -37,7 +37,7 @@ static_assert(sizeof(DevState) == 256, "DevState must stay 256 bytes");
 
 // Byte offsets inside a layer's workspace (all 256-byte aligned).
 struct WorkspaceLayout {
-  size_t state, hist, scores, part_o, part_ml, total;
+  size_t state, hist, cp, scores, part_o, part_ml, total;
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -72,6 +72,8 @@ inline WorkspaceLayout workspace_layout(const qsa_config& c, int n_splits) {
   off += align256(sizeof(DevState));
   w.hist = off;  // score-key prefix histogram of the last scan (zero between selections)
   off += align256(size_t(1 << kHistBits) * sizeof(uint32_t));
+  w.cp = off;    // a context-parallel shard's part of the global selection: count, then ids
+  off += align256(size_t(16 + kTopkMaxK) * sizeof(int32_t));
   w.scores = off;  // kMaxQueries rows of score_stride_of(c) floats
   off += align256(size_t(kMaxQueries) * score_stride_of(c) * sizeof(float));
   w.part_o = off;
@@ -94,6 +96,8 @@ struct LayerView {
   DevState* state;
   float* scores;          // workspace scores
   uint32_t* hist;         // workspace score-key prefix histogram
+  int32_t* cp_count;      // workspace: a context-parallel shard's selected-block count
+  int32_t* cp_sel;        //            and its local block ids
   float* part_o;
   float* part_ml;
   AttnSplit split;
@@ -118,15 +122,21 @@ cudaError_t launch_decode_append(const LayerView& L, const void* k, const void* 
 // and outputs are consecutive rows (scores: rows of score_stride floats).
 // With `hist` (single query only) the scan also fills the score-key prefix histogram and
 // the selection starts from it (and clears it for the next scan).
+// q_n > 0 (single query): the query belongs to token q_n - 1 of a longer sequence (a
+// context-parallel shard's scan), else to token n_ctx - 1.
 cudaError_t launch_index_scan(const LayerView& L, const void* q_idx, const float* w,
                               float* scores, cudaStream_t s, int n_queries = 1, int score_stride = 0,
-                              uint32_t* hist = nullptr);
+                              uint32_t* hist = nullptr, int q_n = 0);
+// With sel_scores (single query), the selection also writes each selected block's score,
+// adds block_base to the written ids and pads positions past n_sel with -inf / -1 (the
+// fixed-size candidate slots of a context-parallel shard).
 cudaError_t launch_topk(const LayerView& L, const float* scores, int32_t* sel, int32_t* n_sel,
-                        cudaStream_t s, int n_queries = 1, int score_stride = 0, uint32_t* hist = nullptr);
+                        cudaStream_t s, int n_queries = 1, int score_stride = 0, uint32_t* hist = nullptr,
+                        float* sel_scores = nullptr, int block_base = 0);
 // The same scan on the CUDA cores (scan_kind = QSA_SCAN_CUDA_CORES; single query).
 cudaError_t init_scan_cc_attributes();
 cudaError_t launch_index_scan_cc(const LayerView& L, const void* q_idx, const float* w, float* scores,
-                                 uint32_t* hist, cudaStream_t s);
+                                 uint32_t* hist, cudaStream_t s, int q_n = 0);
 // Decode step's first launch: append the token at n_ctx (pooling the block it completes)
 // and scan, filling `hist`. Needs the pooled cache current up to the token before.
 cudaError_t launch_decode_scan(const LayerView& L, const void* k, const void* v, const void* idx,
@@ -136,8 +146,17 @@ cudaError_t launch_gather(const LayerView& L, const int32_t* sel, const int32_t*
                           cudaStream_t s);
 cudaError_t launch_attend(const LayerView& L, const void* q, const int32_t* cells,
                           const int32_t* n_cells, float* out, cudaStream_t s);
+// With lse (single query): also the log-sum-exp of each head's scaled logits over its cells.
 cudaError_t launch_attend_selected(const LayerView& L, const void* q, const int32_t* sel,
-                                   const int32_t* n_sel, float* out, cudaStream_t s, int n_queries = 1);
+                                   const int32_t* n_sel, float* out, cudaStream_t s, int n_queries = 1,
+                                   float* lse = nullptr);
+// context-parallel step (qsa_cp.cu)
+cudaError_t launch_cp_select(const float* cand_scores, const int32_t* cand_blocks, int n_shards, int k_blocks,
+                             int32_t* sel, int32_t* n_sel, cudaStream_t s);
+cudaError_t launch_cp_filter(const LayerView& L, const int32_t* sel_global, const int32_t* n_sel_global,
+                             int block_base, int32_t* sel_local, int32_t* n_local, cudaStream_t s);
+cudaError_t launch_cp_merge(const float* o_parts, const float* lse_parts, int n_shards, int n_q_heads, int head_dim,
+                            float* out, cudaStream_t s);
 cudaError_t launch_attend_split(const LayerView& L, const void* q, const int32_t* cells,
                                 const int32_t* n_cells, float* out, cudaStream_t s);
 cudaError_t plan_attention(const qsa_config& c, int* cluster, int* cells_per_cta);

@@ -86,7 +86,8 @@ template <int D, int H, bool HIST>
 __global__ void __launch_bounds__(kCcThreads, 1)
 index_scan_cc_kernel(DevState* st, const __half* __restrict__ pooled, const __half* __restrict__ q_idx,
                      const float* __restrict__ w, float* __restrict__ scores, uint32_t* __restrict__ hist,
-                     float rope_base, int max_blocks, int rope_dims, int rope_interleaved, int rope_pos_stride) {
+                     float rope_base, int max_blocks, int rope_dims, int rope_interleaved, int rope_pos_stride,
+                     int q_n) {
   constexpr int LPR = D / 8;            // lanes per row (16 bytes each)
   constexpr int RPW = 32 / LPR;         // rows per warp per pass
   constexpr int NV = H < LPR ? 1 : H / LPR;  // reduced values per lane
@@ -140,7 +141,8 @@ index_scan_cc_kernel(DevState* st, const __half* __restrict__ pooled, const __ha
 
   // the rotated query (position of token n-1 on the block-position scale), f32
   const int half_r = rope_dims / 2;
-  const double qpos = n > 0 ? (double)(((long long)rope_pos_stride * (n - 1)) / kBlock) : 0.0;
+  const int nq = q_n > 0 ? q_n : n;  // the query's token count (a shard's query sits in a longer sequence)
+  const double qpos = nq > 0 ? (double)(((long long)rope_pos_stride * (nq - 1)) / kBlock) : 0.0;
   for (int f = tid; f < half_r; f += kCcThreads) {
     double sd, cd;
     sincos(qpos * s_theta[f], &sd, &cd);
@@ -243,24 +245,24 @@ cudaError_t set_cc_attr() {
 
 template <int D, int H>
 cudaError_t launch_cc(const LayerView& L, const void* q_idx, const float* w, float* scores, uint32_t* hist,
-                      cudaStream_t s) {
+                      cudaStream_t s, int q_n) {
   const auto args = [&](auto kernel) {
     return launch_pdl(kernel, dim3(L.n_sms), dim3(kCcThreads), cc_smem<D, H>(), s, 1, L.state,
                       (const __half*)L.pooled_cache, (const __half*)q_idx, w, scores, hist, L.cfg.rope_base,
-                      L.cfg.max_ctx / kBlock, L.cfg.rope_dims, L.cfg.rope_interleaved, L.cfg.rope_pos_stride);
+                      L.cfg.max_ctx / kBlock, L.cfg.rope_dims, L.cfg.rope_interleaved, L.cfg.rope_pos_stride, q_n);
   };
   return hist ? args(index_scan_cc_kernel<D, H, true>) : args(index_scan_cc_kernel<D, H, false>);
 }
 
 template <int D>
 cudaError_t launch_cc_d(const LayerView& L, const void* q_idx, const float* w, float* scores, uint32_t* hist,
-                        cudaStream_t s) {
+                        cudaStream_t s, int q_n) {
   switch (L.cfg.n_idx_heads) {
-    case 1: return launch_cc<D, 1>(L, q_idx, w, scores, hist, s);
-    case 2: return launch_cc<D, 2>(L, q_idx, w, scores, hist, s);
-    case 4: return launch_cc<D, 4>(L, q_idx, w, scores, hist, s);
-    case 8: return launch_cc<D, 8>(L, q_idx, w, scores, hist, s);
-    case 16: return launch_cc<D, 16>(L, q_idx, w, scores, hist, s);
+    case 1: return launch_cc<D, 1>(L, q_idx, w, scores, hist, s, q_n);
+    case 2: return launch_cc<D, 2>(L, q_idx, w, scores, hist, s, q_n);
+    case 4: return launch_cc<D, 4>(L, q_idx, w, scores, hist, s, q_n);
+    case 8: return launch_cc<D, 8>(L, q_idx, w, scores, hist, s, q_n);
+    case 16: return launch_cc<D, 16>(L, q_idx, w, scores, hist, s, q_n);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -278,9 +280,9 @@ cudaError_t init_scan_cc_attributes() {
 }
 
 cudaError_t launch_index_scan_cc(const LayerView& L, const void* q_idx, const float* w, float* scores,
-                                 uint32_t* hist, cudaStream_t s) {
-  return L.cfg.d_idx == 128 ? launch_cc_d<128>(L, q_idx, w, scores, hist, s)
-                            : launch_cc_d<64>(L, q_idx, w, scores, hist, s);
+                                 uint32_t* hist, cudaStream_t s, int q_n) {
+  return L.cfg.d_idx == 128 ? launch_cc_d<128>(L, q_idx, w, scores, hist, s, q_n)
+                            : launch_cc_d<64>(L, q_idx, w, scores, hist, s, q_n);
 }
 
 }  // namespace qsa

@@ -180,7 +180,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_constant__ CUtensorMap map_box,
                      DevState* st, const __half* __restrict__ q_idx, const float* __restrict__ w,
                      float* __restrict__ scores, uint32_t* __restrict__ hist, float rope_base, int max_blocks,
-                     int rope_dims, int rope_interleaved, int rope_pos_stride, int score_stride, DecodeAppend app) {
+                     int rope_dims, int rope_interleaved, int rope_pos_stride, int score_stride, DecodeAppend app,
+                     int q_n) {
   static_assert(!(HIST || FUSED) || T == 1, "histogram and fused append serve the single-query step");
   static_assert(!FUSED || HIST, "the decode step always fills the histogram");
   using S = ScanShape<D, H, T>;
@@ -356,7 +357,9 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_
       const int half_r = rope_dims / 2;
       for (int i = tid; i < T * half_r; i += 128) {
         const int u = i / half_r, f = i % half_r;
-        const int n_u = n - (T - 1 - u);
+        // q_n > 0: the query belongs to token q_n - 1 of a longer sequence whose blocks this
+        // layer holds a contiguous part of (a context-parallel shard)
+        const int n_u = (q_n > 0 ? q_n : n) - (T - 1 - u);
         const double qpos = n_u > 0 ? (double)(((long long)rope_pos_stride * (n_u - 1)) / kBlock) : 0.0;
         double sd, cd;
         sincos(qpos * s_theta[f], &sd, &cd);
@@ -544,22 +547,23 @@ cudaError_t encode_pooled_map(const qsa_config& c, void* pooled, int box_rows, C
 
 template <int D, int H, int T, bool HIST, bool FUSED>
 static cudaError_t launch_scan_tc(const LayerView& L, const void* q_idx, const float* w, float* scores,
-                                  cudaStream_t s, int score_stride, uint32_t* hist, const DecodeAppend& app) {
+                                  cudaStream_t s, int score_stride, uint32_t* hist, const DecodeAppend& app,
+                                  int q_n = 0) {
   return launch_pdl(index_scan_tc_kernel<D, H, T, HIST, FUSED>, dim3(L.n_sms), dim3(kThreads),
                     ScanShape<D, H, T>::SMEM, s, 1, L.pooled_tile_map, L.pooled_box_map, L.state,
                     (const __half*)q_idx, w, scores, hist, L.cfg.rope_base, L.cfg.max_ctx / kBlock, L.cfg.rope_dims,
-                    L.cfg.rope_interleaved, L.cfg.rope_pos_stride, score_stride, app);
+                    L.cfg.rope_interleaved, L.cfg.rope_pos_stride, score_stride, app, q_n);
 }
 
 // mode 0: plain scan of T queries; 1: single query with the histogram; 2: decode step
 template <int D, int H>
 static cudaError_t launch_scan_tc_t(const LayerView& L, const void* q_idx, const float* w, float* scores,
                                     cudaStream_t s, int n_queries, int score_stride, uint32_t* hist, int mode,
-                                    const DecodeAppend& app) {
+                                    const DecodeAppend& app, int q_n) {
   if (mode == 2) return launch_scan_tc<D, H, 1, true, true>(L, q_idx, w, scores, s, score_stride, hist, app);
-  if (mode == 1) return launch_scan_tc<D, H, 1, true, false>(L, q_idx, w, scores, s, score_stride, hist, app);
+  if (mode == 1) return launch_scan_tc<D, H, 1, true, false>(L, q_idx, w, scores, s, score_stride, hist, app, q_n);
   switch (n_queries) {
-    case 1: return launch_scan_tc<D, H, 1, false, false>(L, q_idx, w, scores, s, score_stride, hist, app);
+    case 1: return launch_scan_tc<D, H, 1, false, false>(L, q_idx, w, scores, s, score_stride, hist, app, q_n);
     case 2: return launch_scan_tc<D, H, 2, false, false>(L, q_idx, w, scores, s, score_stride, hist, app);
     case 3: return launch_scan_tc<D, H, 3, false, false>(L, q_idx, w, scores, s, score_stride, hist, app);
     case 4: return launch_scan_tc<D, H, 4, false, false>(L, q_idx, w, scores, s, score_stride, hist, app);
@@ -570,31 +574,32 @@ static cudaError_t launch_scan_tc_t(const LayerView& L, const void* q_idx, const
 template <int D>
 static cudaError_t launch_scan_tc_d(const LayerView& L, const void* q_idx, const float* w, float* scores,
                                     cudaStream_t s, int n_queries, int score_stride, uint32_t* hist, int mode,
-                                    const DecodeAppend& app) {
+                                    const DecodeAppend& app, int q_n) {
   switch (L.cfg.n_idx_heads) {
-    case 1: return launch_scan_tc_t<D, 1>(L, q_idx, w, scores, s, n_queries, score_stride, hist, mode, app);
-    case 2: return launch_scan_tc_t<D, 2>(L, q_idx, w, scores, s, n_queries, score_stride, hist, mode, app);
-    case 4: return launch_scan_tc_t<D, 4>(L, q_idx, w, scores, s, n_queries, score_stride, hist, mode, app);
-    case 8: return launch_scan_tc_t<D, 8>(L, q_idx, w, scores, s, n_queries, score_stride, hist, mode, app);
-    case 16: return launch_scan_tc_t<D, 16>(L, q_idx, w, scores, s, n_queries, score_stride, hist, mode, app);
+    case 1: return launch_scan_tc_t<D, 1>(L, q_idx, w, scores, s, n_queries, score_stride, hist, mode, app, q_n);
+    case 2: return launch_scan_tc_t<D, 2>(L, q_idx, w, scores, s, n_queries, score_stride, hist, mode, app, q_n);
+    case 4: return launch_scan_tc_t<D, 4>(L, q_idx, w, scores, s, n_queries, score_stride, hist, mode, app, q_n);
+    case 8: return launch_scan_tc_t<D, 8>(L, q_idx, w, scores, s, n_queries, score_stride, hist, mode, app, q_n);
+    case 16: return launch_scan_tc_t<D, 16>(L, q_idx, w, scores, s, n_queries, score_stride, hist, mode, app, q_n);
     default: return cudaErrorInvalidValue;
   }
 }
 
 static cudaError_t launch_scan_mode(const LayerView& L, const void* q_idx, const float* w, float* scores,
                                     cudaStream_t s, int n_queries, int score_stride, uint32_t* hist, int mode,
-                                    const DecodeAppend& app) {
-  return L.cfg.d_idx == 128 ? launch_scan_tc_d<128>(L, q_idx, w, scores, s, n_queries, score_stride, hist, mode, app)
-                            : launch_scan_tc_d<64>(L, q_idx, w, scores, s, n_queries, score_stride, hist, mode, app);
+                                    const DecodeAppend& app, int q_n = 0) {
+  return L.cfg.d_idx == 128
+             ? launch_scan_tc_d<128>(L, q_idx, w, scores, s, n_queries, score_stride, hist, mode, app, q_n)
+             : launch_scan_tc_d<64>(L, q_idx, w, scores, s, n_queries, score_stride, hist, mode, app, q_n);
 }
 
 cudaError_t launch_index_scan(const LayerView& L, const void* q_idx, const float* w, float* scores,
-                              cudaStream_t s, int n_queries, int score_stride, uint32_t* hist) {
+                              cudaStream_t s, int n_queries, int score_stride, uint32_t* hist, int q_n) {
   if (L.cfg.scan_kind == QSA_SCAN_CUDA_CORES && n_queries == 1)
-    return launch_index_scan_cc(L, q_idx, w, scores, hist, s);
+    return launch_index_scan_cc(L, q_idx, w, scores, hist, s, q_n);
   const int mode = (hist && n_queries == 1) ? 1 : 0;
   return launch_scan_mode(L, q_idx, w, scores, s, n_queries, score_stride, mode ? hist : nullptr, mode,
-                          DecodeAppend{});
+                          DecodeAppend{}, n_queries == 1 ? q_n : 0);
 }
 
 cudaError_t launch_decode_scan(const LayerView& L, const void* k, const void* v, const void* idx, const void* q_idx,

@@ -76,6 +76,10 @@ SIGNATURES = {
     "qsa_n_ctx": (_I, [_P, _I]),
     "qsa_get_device_status": (_I, [_P, ctypes.POINTER(_I)]),
     "qsa_decode_step": (_I, [_P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "qsa_cp_index_candidates": (_I, [_P, _I, _P, _P, _I, _I, _P, _P, _P, _P]),
+    "qsa_cp_select": (_I, [_P, _P, _I, _I, _P, _P, _P]),
+    "qsa_cp_attend_partial": (_I, [_P, _I, _P, _P, _P, _I, _P, _P, _P]),
+    "qsa_cp_merge": (_I, [_P, _P, _I, _I, _I, _P, _P]),
 }
 
 _lib = None
@@ -237,6 +241,20 @@ class Qsa:
                                              _ptr(w), _ptr(q), _ptr(sel_blocks), _ptr(n_sel), _ptr(out),
                                              _stream(stream)))
 
+    def cp_index_candidates(self, layer, q_idx, w, n_global, block_base, cand_scores, cand_blocks, n_cand,
+                            stream=None):
+        """A context-parallel shard's scan (query at global position n_global - 1) and its
+        local top-K as fixed-size slots of scores and global block ids."""
+        self._check(self.lib.qsa_cp_index_candidates(self.handle, layer, _ptr(q_idx), _ptr(w), int(n_global),
+                                                     int(block_base), _ptr(cand_scores), _ptr(cand_blocks),
+                                                     _ptr(n_cand), _stream(stream)))
+
+    def cp_attend_partial(self, layer, q, sel_blocks, n_sel, block_base, out, lse, stream=None):
+        """A context-parallel shard's attention over its part of the global selection:
+        normalised output and per-head log-sum-exp."""
+        self._check(self.lib.qsa_cp_attend_partial(self.handle, layer, _ptr(q), _ptr(sel_blocks), _ptr(n_sel),
+                                                   int(block_base), _ptr(out), _ptr(lse), _stream(stream)))
+
     def n_ctx(self, layer) -> int:
         """Tokens in the layer's caches (synchronises the device)."""
         n = self.lib.qsa_n_ctx(self.handle, layer)
@@ -249,6 +267,22 @@ class Qsa:
         st = c_int32()
         self._check(self.lib.qsa_get_device_status(self.handle, ctypes.byref(st)))
         return st.value
+
+
+def cp_select(cand_scores, cand_blocks, n_shards, k_blocks, sel_blocks, n_sel, stream=None):
+    """qsa_cp_select: the global top-K of every shard's candidate slots."""
+    st = load_library().qsa_cp_select(_ptr(cand_scores), _ptr(cand_blocks), int(n_shards), int(k_blocks),
+                                      _ptr(sel_blocks), _ptr(n_sel), _stream(stream))
+    if st != QSA_OK:
+        raise QsaError(st, "qsa_cp_select failed")
+
+
+def cp_merge(o_parts, lse_parts, n_shards, n_q_heads, head_dim, out, stream=None):
+    """qsa_cp_merge: the exact merge of the shards' attention partials."""
+    st = load_library().qsa_cp_merge(_ptr(o_parts), _ptr(lse_parts), int(n_shards), int(n_q_heads), int(head_dim),
+                                     _ptr(out), _stream(stream))
+    if st != QSA_OK:
+        raise QsaError(st, "qsa_cp_merge failed")
 
 
 def sparse_attend_noalloc(q, k_cache, v_cache, n_ctx, cells, n_cells, out, n_q_heads, n_kv_heads, head_dim,

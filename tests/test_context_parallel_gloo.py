@@ -7,7 +7,9 @@ over its selected cells. The candidates travel as fixed-size slots (K scores pad
 -inf, K block ids padded with -1) through all_gather; every rank merges them with the
 selection rule; the partials travel through all_gather and merge exactly. Rank 0 checks
 the result against the single-device definition. This pins the protocol the sharded
-kernels will follow; the kernels themselves are not built.
+kernels follow (qsa_cp_index_candidates, qsa_cp_select, qsa_cp_attend_partial,
+qsa_cp_merge; their GPU parity, with the shards emulated on one GPU, is in
+test_gpu_context_parallel.py).
 """
 import json
 import os
