@@ -56,6 +56,8 @@ Readings taken where the pages are silent (each one is listed in the design note
      §COMMON-004: speculative writes must not corrupt the cached range).
   R12 FP8 K/V cache (optional): per (token, KV head) row, scale = amax/448 and e4m3 codes
      of x * 448/amax (nearest-even, saturating); attention reads code * scale.
+  R13 8-bit pooled keys (optional): each f16 summary p_b (R5) is stored as e4m3 codes with
+     one f32 scale, by the R12 rule applied to the row; the indexer scores code * scale.
 
 Also stated here: the sharded (context-parallel) form of one step, whose local top-K
 candidates, merged selection and (o, lse) partials reproduce the single-device step.
@@ -404,6 +406,12 @@ def quantize_kv_rows(rows):
 _E4M3_TABLE = np.array([e4m3_value(c) for c in range(256)])
 
 
+def pooled_fp8_rows(pooled_f16):
+    """8-bit pooled keys (R13): the f16 summaries [B, d] as e4m3 codes [B, d] and one f32
+    scale per row [B], by the R12 rule."""
+    return quantize_kv_rows(np.asarray(pooled_f16, np.float16))
+
+
 def dequantize_kv_rows(codes, scales) -> np.ndarray:
     """code * scale in float64."""
     return _E4M3_TABLE[np.asarray(codes)] * np.asarray(scales, dtype=np.float64)[..., None]
@@ -416,11 +424,12 @@ def dequantize_kv_rows(codes, scales) -> np.ndarray:
 class OracleLayer:
     """One QSA layer's caches and the decode-step calls, in plain numpy."""
 
-    def __init__(self, shape: QsaShape, max_ctx: int, gain=None, kv_fp8: bool = False):
+    def __init__(self, shape: QsaShape, max_ctx: int, gain=None, kv_fp8: bool = False, pooled_fp8: bool = False):
         self.shape = shape
         self.max_ctx = max_ctx
         self.gain = gain
         self.kv_fp8 = kv_fp8
+        self.pooled_fp8 = pooled_fp8
         kv_shape = (max_ctx, shape.n_kv_heads, shape.head_dim)
         # attention reads self.k / self.v: the f16 rows, or code * scale (reading R12)
         self.k = np.zeros(kv_shape, dtype=np.float64 if kv_fp8 else np.float16)
@@ -454,10 +463,19 @@ class OracleLayer:
     def update_pooled_cache(self) -> int:
         return self.pooled.update(self.idx, self.n, self.shape, self.gain)
 
+    @property
+    def scored_rows(self) -> np.ndarray:
+        """What the indexer scores: the f16 summaries, or with 8-bit pooled keys their
+        e4m3 codes * scale (R13)."""
+        if not self.pooled_fp8:
+            return self.pooled.rows
+        codes, scales = pooled_fp8_rows(self.pooled.rows)
+        return dequantize_kv_rows(codes, scales)
+
     def scores(self, q_idx, w) -> np.ndarray:
         if self.pooled.n_pooled != self.n // BLOCK:
             raise ValueError("pooled cache is stale")
-        return block_scores(self.pooled.rows, q_idx, w, self.n, self.shape)
+        return block_scores(self.scored_rows, q_idx, w, self.n, self.shape)
 
     def index_topk(self, q_idx, w):
         s = self.scores(q_idx, w)
@@ -487,7 +505,7 @@ class OracleLayer:
         outs = []
         for t in range(T):
             n_t = self.n - T + t + 1
-            s = block_scores(self.pooled.rows, q_idx[t], w[t], n_t, self.shape)
+            s = block_scores(self.scored_rows, q_idx[t], w[t], n_t, self.shape)
             sel = topk_blocks(s, self.shape.k_blocks)
             cells = expand_cells(sel, n_t)
             outs.append({"sel": sel, "scores": s, "cells": cells, "out": self.attend(q[t], cells)})

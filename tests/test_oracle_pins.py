@@ -555,6 +555,58 @@ def test_fp8_layer_is_exact_on_e4m3_grid_rows():
     np.testing.assert_array_equal(a.attend(q, cells), b.attend(q, cells))
 
 
+def _pooled_layers(rows, n, pooled_fp8):
+    """An oracle layer whose pooled cache holds `rows` (f16) for a context of n tokens."""
+    L = O.OracleLayer(SMALL, 4 * len(rows) + 8, pooled_fp8=pooled_fp8)
+    L.n = n
+    L.pooled.rows[: len(rows)] = rows
+    L.pooled.n_pooled = n // 4
+    return L
+
+
+def test_pooled_fp8_is_exact_on_e4m3_grid_rows():
+    """Summaries on the e4m3 grid whose largest magnitude is 448 quantise with scale 1 and
+    no rounding: the 8-bit pooled keys then score exactly like the f16 ones (reading R13)."""
+    rng = np.random.default_rng(51)
+    grid = np.array([O.e4m3_value(c) for c in range(256) if not np.isnan(O.e4m3_value(c))])
+    grid = grid[np.abs(grid) <= 8]
+    rows = rng.choice(grid, (20, SMALL.d_idx)).astype(np.float16)
+    rows[:, 2] = 448.0
+    codes, scales = O.pooled_fp8_rows(rows)
+    assert np.all(scales == 1.0)
+    np.testing.assert_array_equal(O.dequantize_kv_rows(codes, scales), rows.astype(np.float64))
+    q_idx = rng.standard_normal((SMALL.n_idx_heads, SMALL.d_idx)).astype(np.float16)
+    w = rng.random(SMALL.n_idx_heads).astype(np.float32)
+    a, b = _pooled_layers(rows, 81, False), _pooled_layers(rows, 81, True)
+    np.testing.assert_array_equal(a.scores(q_idx, w), b.scores(q_idx, w))
+
+
+def test_pooled_fp8_scores_within_the_quantisation_bound():
+    """Every element moves by at most 2^-4 of itself (or half a subnormal quantum), so a
+    score moves by at most sum_h w_h * sum_e |q~_he| * bound_e / sqrt(d); and the scores
+    use code * scale, not the f16 rows (a plain reading of R13 against R12's rule)."""
+    rng = np.random.default_rng(52)
+    rows = rng.standard_normal((40, SMALL.d_idx)).astype(np.float16)
+    q_idx = rng.standard_normal((SMALL.n_idx_heads, SMALL.d_idx)).astype(np.float16)
+    w = rng.random(SMALL.n_idx_heads).astype(np.float32)
+    n = 4 * 40 + 1
+    f16, f8 = _pooled_layers(rows, n, False), _pooled_layers(rows, n, True)
+    s16, s8 = f16.scores(q_idx, w), f8.scores(q_idx, w)
+    codes, scales = O.pooled_fp8_rows(rows)
+    x = rows.astype(np.float64)
+    bound = np.maximum(np.abs(x) * 2.0 ** -4, 2.0 ** -10 * scales[:, None].astype(np.float64))
+    q = np.abs(O.indexer_query(q_idx, n, SMALL))                        # [H, d]
+    limit = (bound @ q.T) @ w.astype(np.float64) / np.sqrt(SMALL.d_idx)  # [B]
+    assert np.all(np.abs(s8 - s16) <= limit * (1 + 1e-9) + 1e-12)
+    assert np.abs(s8 - s16).max() > 0   # the rows are not on the grid: the 8-bit scores differ
+    # a needle row aligned with every head's query still wins under the 8-bit keys
+    needle = O.indexer_query(q_idx, n, SMALL).sum(axis=0)
+    rows2 = rows.copy()
+    rows2[17] = (needle / np.abs(needle).max() * 4).astype(np.float16)
+    f8b = _pooled_layers(rows2, n, True)
+    assert 17 in O.topk_blocks(f8b.scores(q_idx, w), 1)
+
+
 # ---------------------------------------------------------------- seeded inputs
 
 @pytest.mark.parametrize("first", [250, 258048 - 255181 - 5])   # the second range crosses a chunk boundary
