@@ -181,7 +181,7 @@ def max_over_ranks(x, world):
 class Workbench:
     """L bound layers prefilled with the workload's context and graph-captured steps."""
 
-    def __init__(self, wl, n_layers, n_graph_steps, extra_steps, rank, kv_format=0):
+    def __init__(self, wl, n_layers, n_graph_steps, extra_steps, rank, kv_format=0, pooled_format=0):
         import torch
 
         import synth
@@ -189,7 +189,8 @@ class Workbench:
         self.torch, self.Q, self.wl, self.L = torch, Q, wl, n_layers
         max_ctx = int(math.ceil((wl.n_prefill + n_graph_steps + extra_steps + 8) / 4) * 4)
         self.cfg = Q.make_config(n_layers, max_ctx, wl.d_idx, wl.n_idx_heads, wl.top_k_tokens, wl.n_q_heads,
-                                 wl.n_kv_heads, wl.head_dim, wl.rope_base, wl.rms_eps, kv_format=kv_format)
+                                 wl.n_kv_heads, wl.head_dim, wl.rope_base, wl.rms_eps, kv_format=kv_format,
+                                 pooled_format=pooled_format)
         self.qsa = Q.Qsa(self.cfg)
         self.bufs, self.outs = [], []
         for layer in range(n_layers):
@@ -355,10 +356,12 @@ def run_multi_query(wb, wl, n_layers, T=4, steps_per_graph=8, replays=4):
 
 
 def run_ours(wl, n_layers, K, W, rank, world, e2e_steps, sample_clocks, local, multi_query=False, kv_format=0,
+             pooled_format=0,
              spread_reps=0):
     import torch
     G = max(d for d in range(1, 33) if K % d == 0)       # steps per timed graph
-    wb = Workbench(wl, n_layers, W + K, extra_steps=e2e_steps + 128, rank=rank, kv_format=kv_format)
+    wb = Workbench(wl, n_layers, W + K, extra_steps=e2e_steps + 128, rank=rank, kv_format=kv_format,
+                   pooled_format=pooled_format)
     warm = [wb.capture([s]) for s in range(W)]
     timed = [wb.capture(list(range(W + j * G, W + (j + 1) * G))) for j in range(K // G)]
     torch.cuda.synchronize()
@@ -599,14 +602,16 @@ def ncu_traffic(stage):
         return None
 
 
-def stage_bytes(wl, n_ctx, kv_fp8=False):
+def stage_bytes(wl, n_ctx, kv_fp8=False, pooled_fp8=False):
     """Algorithmic HBM bytes per launch of each stage at context n_ctx (per layer). With an
-    FP8 K/V cache a row is head_dim code bytes plus its 4-byte scale."""
+    FP8 K/V cache a row is head_dim code bytes plus its 4-byte scale; with 8-bit pooled keys
+    a pooled row is d_idx code bytes plus its 4-byte scale."""
     B = n_ctx // 4
+    pooled_row = wl.d_idx + 4 if pooled_fp8 else wl.d_idx * 2
     kv_row = wl.n_kv_heads * (wl.head_dim + 4 if kv_fp8 else wl.head_dim * 2)
     n_cells = 4 * min(wl.k_blocks, B) + n_ctx % 4
     return {
-        "index_scan": B * wl.d_idx * 2 + B * 4 + wl.n_idx_heads * (wl.d_idx * 2 + 4),
+        "index_scan": B * pooled_row + B * 4 + wl.n_idx_heads * (wl.d_idx * 2 + 4),
         "block_topk": B * 4 + wl.k_blocks * 4,
         "sparse_attend": wl.k_blocks * 4 + n_cells * 2 * (kv_row // wl.n_kv_heads) * wl.n_kv_heads
                          + wl.n_q_heads * wl.head_dim * (2 + 4),
@@ -724,6 +729,24 @@ def main_ours(args):
         del r8
         torch.cuda.empty_cache()
 
+    # the same step with 8-bit pooled keys (e4m3 codes + per-row scale): the scan reads half
+    pooled_fp8 = None
+    if not args.profile_case and not args.no_fp8 and wl.d_idx == 128:
+        torch.cuda.empty_cache()
+        k8 = max(500, min(K // 5, 1000))
+        k8 -= k8 % 25
+        r8 = run_ours(wl, wl.n_layers, k8, 5, rank, world, 0, sample_clocks=False, local=local, pooled_format=1)
+        b8 = stage_bytes(wl, r8["n_ctx_instr"], pooled_fp8=True)
+        s8 = r8["iso_us"]["index_scan"]
+        pooled_fp8 = {"value": round(world * wl.n_layers * k8 / (r8["ms"] / 1e3), 1), "unit": UNIT, "steps": k8,
+                      "ms_per_step": round(r8["ms"] / k8, 5), "scan_us": round(s8, 3),
+                      "scan_bytes": int(b8["index_scan"]),
+                      "scan_gbs": round(b8["index_scan"] / (s8 * 1e-6) / 1e9, 1),
+                      "scan_us_f16": round(per["index_scan"], 3),
+                      "stages_us": {k: round(v, 3) for k, v in r8["per_launch_us"].items()}}
+        del r8
+        torch.cuda.empty_cache()
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(wl)
@@ -751,6 +774,7 @@ def main_ours(args):
             "multi_query": main["multi_query"],
             "scan_ab": main["scan_ab"],
             "kv_fp8": kv_fp8,
+            "pooled_fp8": pooled_fp8,
             "hbm_gbs_step": round(world * wl.n_layers * K * sum(sb.values()) / (main["ms"] / 1e3) / 1e9, 1),
         }
         print(json.dumps(line))

@@ -99,10 +99,18 @@ typedef struct {
    * f32 FMAs with warp-shuffle reductions; single-query scans only (the multi-query calls
    * use the tensor cores), and a decode step with it takes four launches. */
   int32_t scan_kind;
+  /* Storage of the pooled-key cache (the other half of the 8-bit option the tuning post's
+   * section "KV cacheをQ8_0にしてみる" tried). QSA_POOLED_F16 (0): f16 summaries.
+   * QSA_POOLED_FP8 (1): each f16 summary stored as d_idx e4m3 codes and one f32 scale per
+   * row (pooled_scales), by the QSA_KV_FP8 rule; the indexer scores code * scale, on the
+   * tensor cores with 8-bit operands (d_idx 128, QSA_SCAN_TENSOR and single-query scans
+   * only: otherwise QSA_ERR_UNSUPPORTED). The scan then reads half the bytes. */
+  int32_t pooled_format;
 } qsa_config;
 
 enum { QSA_KV_F16 = 0, QSA_KV_FP8 = 1 };
 enum { QSA_SCAN_TENSOR = 0, QSA_SCAN_CUDA_CORES = 1 };
+enum { QSA_POOLED_F16 = 0, QSA_POOLED_FP8 = 1 };
 
 /* Caller-owned device buffers of one layer. Sizes come from qsa_buffer_bytes(). */
 typedef struct {
@@ -110,11 +118,14 @@ typedef struct {
                              QSA_KV_FP8), token-major                                   */
   void* v_cache;          /* same layout as k_cache                                     */
   void* idx_cache;        /* [max_ctx][d_idx] f16: raw per-token indexer keys           */
-  void* pooled_cache;     /* [max_ctx/4][d_idx] f16: pooled summaries p_b               */
+  void* pooled_cache;     /* [max_ctx/4][d_idx] f16: pooled summaries p_b (e4m3 bytes
+                             with QSA_POOLED_FP8)                                        */
   const float* rms_gain;  /* [d_idx] f32 RMS-norm gain, or NULL for unit gain           */
   void* workspace;        /* device state + scratch; QSA_BUF_WORKSPACE bytes            */
   void* kv_scales;        /* QSA_KV_FP8 only: [max_ctx][n_kv_heads][2] f32, the K and V
                              scales of each row; NULL with QSA_KV_F16                   */
+  void* pooled_scales;    /* QSA_POOLED_FP8 only: [max_ctx/4] f32, the scale of each
+                             pooled row (pooled_cache then holds e4m3 codes); NULL otherwise */
 } qsa_layer_buffers;
 
 enum {
@@ -125,7 +136,8 @@ enum {
   QSA_BUF_MAX_CELLS = 4,  /* not bytes: max cells per step = 4*(top_k_tokens/4) + 3 */
   QSA_BUF_SCORE_STRIDE = 5, /* not bytes: floats per row of a multi-query score table
                                (max_ctx/4 rounded up to a multiple of 64) */
-  QSA_BUF_KV_SCALES = 6   /* bytes of kv_scales (0 with QSA_KV_F16)      */
+  QSA_BUF_KV_SCALES = 6,  /* bytes of kv_scales (0 with QSA_KV_F16)      */
+  QSA_BUF_POOLED_SCALES = 7 /* bytes of pooled_scales (0 with QSA_POOLED_F16) */
 };
 
 typedef struct qsa_ctx qsa_ctx;

@@ -51,6 +51,10 @@ const char* config_problem(const qsa_config& c) {
   if (c.kv_format != QSA_KV_F16 && c.kv_format != QSA_KV_FP8) return "kv_format must be QSA_KV_F16 or QSA_KV_FP8";
   if (c.scan_kind != QSA_SCAN_TENSOR && c.scan_kind != QSA_SCAN_CUDA_CORES)
     return "scan_kind must be QSA_SCAN_TENSOR or QSA_SCAN_CUDA_CORES";
+  if (c.pooled_format != QSA_POOLED_F16 && c.pooled_format != QSA_POOLED_FP8)
+    return "pooled_format must be QSA_POOLED_F16 or QSA_POOLED_FP8";
+  if (c.pooled_format == QSA_POOLED_FP8 && (c.d_idx != 128 || c.scan_kind != QSA_SCAN_TENSOR))
+    return "QSA_POOLED_FP8 needs d_idx 128 and the tensor-core scan";
   return nullptr;
 }
 
@@ -97,6 +101,7 @@ struct qsa_ctx {
     v.pooled_cache = l.buf.pooled_cache;
     v.rms_gain = l.buf.rms_gain;
     v.kv_scales = static_cast<float*>(l.buf.kv_scales);
+    v.pooled_scales = static_cast<float*>(l.buf.pooled_scales);
     v.state = reinterpret_cast<DevState*>(wsp + ws.state);
     v.scores = reinterpret_cast<float*>(wsp + ws.scores);
     v.hist = reinterpret_cast<uint32_t*>(wsp + ws.hist);
@@ -130,7 +135,8 @@ size_t qsa_buffer_bytes(const qsa_config* cfg, int32_t which) {
     case QSA_BUF_KV: return size_t(c.max_ctx) * c.n_kv_heads * c.head_dim * (c.kv_format == QSA_KV_FP8 ? 1 : 2);
     case QSA_BUF_KV_SCALES: return c.kv_format == QSA_KV_FP8 ? size_t(c.max_ctx) * c.n_kv_heads * 2 * 4 : 0;
     case QSA_BUF_IDX: return size_t(c.max_ctx) * c.d_idx * 2;
-    case QSA_BUF_POOLED: return size_t(c.max_ctx / kBlock) * c.d_idx * 2;
+    case QSA_BUF_POOLED: return size_t(c.max_ctx / kBlock) * c.d_idx * (c.pooled_format == QSA_POOLED_FP8 ? 1 : 2);
+    case QSA_BUF_POOLED_SCALES: return c.pooled_format == QSA_POOLED_FP8 ? size_t(c.max_ctx / kBlock) * 4 : 0;
     case QSA_BUF_WORKSPACE: {
       int dev = 0, sms = 0;
       if (cudaGetDevice(&dev) != cudaSuccess ||
@@ -195,6 +201,7 @@ qsa_status qsa_bind_layer(qsa_ctx* ctx, int32_t layer, const qsa_layer_buffers* 
   if (buf->rms_gain && !aligned(buf->rms_gain, 16))
     return ctx->fail(QSA_ERR_INVALID_ARG, "rms_gain must be 16-byte aligned");
   if (ctx->cfg.kv_format == QSA_KV_FP8) QSA_CHECK_PTR(buf->kv_scales, 16, "kv_scales");
+  if (ctx->cfg.pooled_format == QSA_POOLED_FP8) QSA_CHECK_PTR(buf->pooled_scales, 16, "pooled_scales");
   Layer& l = ctx->layers[layer];
   CUtensorMap tile_map, box_map;
   if (qsa_status st = ctx->cuda(encode_pooled_map(ctx->cfg, buf->pooled_cache, 128, &tile_map), "bind_layer: pooled TMA map"))
@@ -372,6 +379,8 @@ qsa_status qsa_index_topk_multi(qsa_ctx* ctx, int32_t layer, int32_t n_queries, 
   if (qsa_status st = ctx->layer_ok(layer)) return st;
   if (n_queries < 1 || n_queries > kMaxQueries)
     return ctx->fail(QSA_ERR_INVALID_ARG, "n_queries %d outside [1, %d]", n_queries, kMaxQueries);
+  if (n_queries > 1 && ctx->cfg.pooled_format == QSA_POOLED_FP8)
+    return ctx->fail(QSA_ERR_UNSUPPORTED, "8-bit pooled keys are scanned one query at a time");
   QSA_CHECK_PTR(q_idx, 16, "q_idx");
   QSA_CHECK_PTR(w, 4, "w");
   QSA_CHECK_PTR(sel_blocks, 16, "sel_blocks");

@@ -121,7 +121,7 @@ constexpr int kPoolThreads = 256;
 // Pools blocks [n_pooled, n_ctx/4), one warp per block, grid-stride.
 template <int D, bool GEN>
 __global__ void __launch_bounds__(kPoolThreads) pool_update_kernel(DevState* st, const __half* __restrict__ ic,
-                                                                   __half* __restrict__ pc,
+                                                                   PooledOut pc,
                                                                    const float* __restrict__ gain, float eps,
                                                                    PoolRope rope, int max_blocks) {
   __shared__ float s_rows[GEN ? kPoolThreads / 32 : 1][GEN ? D : 1];
@@ -169,7 +169,7 @@ template <int D, bool GEN, bool FP8>
 __global__ void __launch_bounds__(kPoolThreads) decode_append_kernel(DevState* st, uint4* kc, uint4* vc, uint4* ic,
                                                                      const uint4* k, const uint4* v,
                                                                      const uint4* idx, int kv_units, int max_ctx,
-                                                                     __half* __restrict__ pc,
+                                                                     PooledOut pc,
                                                                      const float* __restrict__ gain, float eps,
                                                                      PoolRope rope, float* kv_scales, int n_kv_heads,
                                                                      int hd) {
@@ -251,7 +251,7 @@ static cudaError_t launch_decode_append_d(const LayerView& L, const void* k, con
 #define QSA_DA_LAUNCH(F8)                                                                                         \
   launch_pdl(decode_append_kernel<D, GEN, F8>, dim3(1), dim3(kPoolThreads), 0, s, 1, L.state, (uint4*)L.k_cache,     \
              (uint4*)L.v_cache, (uint4*)L.idx_cache, (const uint4*)k, (const uint4*)v, (const uint4*)idx, kv_units, \
-             L.cfg.max_ctx, (__half*)L.pooled_cache, L.rms_gain, L.cfg.rms_eps, pool_rope(L.cfg), L.kv_scales,    \
+             L.cfg.max_ctx, pooled_out(L), L.rms_gain, L.cfg.rms_eps, pool_rope(L.cfg), L.kv_scales,    \
              L.cfg.n_kv_heads, L.cfg.head_dim)
   return L.cfg.kv_format == QSA_KV_FP8 ? QSA_DA_LAUNCH(true) : QSA_DA_LAUNCH(false);
 #undef QSA_DA_LAUNCH
@@ -267,7 +267,7 @@ cudaError_t launch_decode_append(const LayerView& L, const void* k, const void* 
 template <int D, bool GEN>
 static cudaError_t launch_pool_update_d(const LayerView& L, int grid, cudaStream_t s) {
   return launch_pdl(pool_update_kernel<D, GEN>, dim3(grid), dim3(kPoolThreads), 0, s, 1, L.state,
-                    (const __half*)L.idx_cache, (__half*)L.pooled_cache, L.rms_gain, L.cfg.rms_eps, pool_rope(L.cfg),
+                    (const __half*)L.idx_cache, pooled_out(L), L.rms_gain, L.cfg.rms_eps, pool_rope(L.cfg),
                     L.cfg.max_ctx / kBlock);
 }
 

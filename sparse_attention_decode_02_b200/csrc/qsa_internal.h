@@ -93,6 +93,7 @@ struct LayerView {
   void* pooled_cache;
   const float* rms_gain;
   float* kv_scales;       // [max_ctx][n_kv_heads][2] f32 with QSA_KV_FP8, else null
+  float* pooled_scales;   // [max_ctx/4] f32 with QSA_POOLED_FP8, else null
   DevState* state;
   float* scores;          // workspace scores
   uint32_t* hist;         // workspace score-key prefix histogram

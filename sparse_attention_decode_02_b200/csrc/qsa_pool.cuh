@@ -168,12 +168,28 @@ __device__ __forceinline__ void pool_load(int b, int lane, const __half* ic, Poo
   }
 }
 
+// Where a summary goes: the f16 pooled cache, or with 8-bit pooled keys (scale != null)
+// its e4m3 codes and the row's scale.
+struct PooledOut {
+  __half* f16;
+  unsigned char* fp8;
+  float* scale;
+};
+
+// The layer's pooled cache in the form its pooled_format stores.
+inline PooledOut pooled_out(const LayerView& L) {
+  const bool fp8 = L.cfg.pooled_format == QSA_POOLED_FP8;
+  return PooledOut{fp8 ? nullptr : static_cast<__half*>(L.pooled_cache),
+                   fp8 ? static_cast<unsigned char*>(L.pooled_cache) : nullptr, fp8 ? L.pooled_scales : nullptr};
+}
+
 // Summary of block b from its raw keys: mean (summed in token order), RMSNorm, RoPE at
-// the block position, f16 store. GEN kernels pass s_row, D floats of shared memory owned
-// by the warp.
+// the block position, f16 store (or the f16 row quantised to e4m3 codes and one scale by
+// the FP8 K/V rule, for 8-bit pooled keys). GEN kernels pass s_row, D floats of shared
+// memory owned by the warp.
 template <int D, bool GEN>
 __device__ __forceinline__ void pool_finish(int b, int lane, const PoolLane<D, GEN>& c, const PoolRaw<D>& raw,
-                                            __half* __restrict__ pc, float eps, RopePos rp, float* s_row) {
+                                            const PooledOut& out, float eps, RopePos rp, float* s_row) {
   constexpr int P = D / 64;
   constexpr int HALF = D / 2;
   float m1[P], m2[P];
@@ -238,20 +254,36 @@ __device__ __forceinline__ void pool_finish(int b, int lane, const PoolLane<D, G
     }
   }
   if constexpr (P == 2) {
-    *reinterpret_cast<__half2*>(pc + size_t(b) * D + lane * 2) = __halves2half2(o1[0], o1[1]);
-    *reinterpret_cast<__half2*>(pc + size_t(b) * D + lane * 2 + HALF) = __halves2half2(o2[0], o2[1]);
+    if (out.scale) {  // 8-bit pooled keys (d_idx 128): scale = amax/448, codes of x * 448/amax
+      const float x0 = __half2float(o1[0]), x1 = __half2float(o1[1]);
+      const float x2 = __half2float(o2[0]), x3 = __half2float(o2[1]);
+      const float m = warp_max(fmaxf(fmaxf(fabsf(x0), fabsf(x1)), fmaxf(fabsf(x2), fabsf(x3))));
+      const float scale = m > 0.0f ? m / 448.0f : 1.0f;
+      const float mult = m > 0.0f ? 448.0f / m : 0.0f;
+      const uint32_t p0 = __nv_cvt_float2_to_fp8x2(make_float2(__fmul_rn(x0, mult), __fmul_rn(x1, mult)),
+                                                   __NV_SATFINITE, __NV_E4M3);
+      const uint32_t p1 = __nv_cvt_float2_to_fp8x2(make_float2(__fmul_rn(x2, mult), __fmul_rn(x3, mult)),
+                                                   __NV_SATFINITE, __NV_E4M3);
+      unsigned char* row = out.fp8 + size_t(b) * D;
+      *reinterpret_cast<uint16_t*>(row + lane * 2) = uint16_t(p0);
+      *reinterpret_cast<uint16_t*>(row + lane * 2 + HALF) = uint16_t(p1);
+      if (lane == 0) out.scale[b] = scale;
+      return;
+    }
+    *reinterpret_cast<__half2*>(out.f16 + size_t(b) * D + lane * 2) = __halves2half2(o1[0], o1[1]);
+    *reinterpret_cast<__half2*>(out.f16 + size_t(b) * D + lane * 2 + HALF) = __halves2half2(o2[0], o2[1]);
   } else {
-    pc[size_t(b) * D + lane] = o1[0];
-    pc[size_t(b) * D + lane + HALF] = o2[0];
+    out.f16[size_t(b) * D + lane] = o1[0];
+    out.f16[size_t(b) * D + lane + HALF] = o2[0];
   }
 }
 
 template <int D, bool GEN>
 __device__ __forceinline__ void pool_one_block(int b, int lane, const PoolLane<D, GEN>& c, const __half* ic,
-                                               __half* __restrict__ pc, float eps, RopePos rp, float* s_row) {
+                                               const PooledOut& out, float eps, RopePos rp, float* s_row) {
   PoolRaw<D> raw;
   pool_load<D>(b, lane, ic, raw);
-  pool_finish<D, GEN>(b, lane, c, raw, pc, eps, rp, s_row);
+  pool_finish<D, GEN>(b, lane, c, raw, out, eps, rp, s_row);
 }
 
 // RoPE settings of a layer as the pooling kernels take them.

@@ -47,8 +47,8 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kAcc = 4;          // TMEM accumulators
 constexpr int kBoxRows = 16;     // TMA box height
+constexpr int kF8Terms = 5;      // e4m3 terms of the query with 8-bit pooled keys (4 bits each)
 // warps 0-3 epilogue, warp 4 TMA, warp 5 MMA + TMEM owner, warp 6 append + pool (FUSED)
 constexpr int kThreads = 224;
 constexpr float kLoScale = 4096.0f;
@@ -60,23 +60,30 @@ constexpr size_t kSmemMax = 227 * 1024;  // dynamic shared memory per CTA
 #endif
 constexpr int kScanStages = QSA_SCAN_STAGES;  // TMA ring depth (tiles of 128 rows)
 
-// Shapes of the scan for d = D, H indexer heads and T queries scored in one pass.
-template <int D, int H, int T>
+// Shapes of the scan for d = D, H indexer heads and T queries scored in one pass; F8:
+// 8-bit pooled keys (e4m3 rows, the query as kF8Terms e4m3 terms).
+template <int D, int H, int T, bool F8 = false>
 struct ScanShape {
-  static constexpr int HALVES = D / 64;                  // one 128-byte swizzle span = 64 f16
-  static constexpr int NQ = 2 * H < 16 ? 16 : 2 * H;     // B rows per query: hi rows, lo rows, zero pad
-  static constexpr int N = T * NQ;                       // MMA N
-  static constexpr int TILE_BYTES = 128 * D * 2;         // A tile: 128 rows
-  static constexpr int HALF_BYTES = 128 * 128;           // 128 rows x 128 bytes
+  static constexpr int ESIZE = F8 ? 1 : 2;                // bytes per pooled element
+  static constexpr int HALVES = D * ESIZE / 128;          // 128-byte swizzle spans per row
+  static constexpr int TERMS = F8 ? kF8Terms : 2;        // query terms: hi and lo, or e4m3 terms
+  static constexpr int NQ = (TERMS * H + 15) / 16 * 16;  // B rows per query (term-major), zero pad
+  static constexpr int N = T * NQ;                        // MMA N
+  static constexpr int K_STEPS = D * ESIZE / 32;          // MMAs per tile: 32 bytes of K each
+  static constexpr int ACC = F8 ? 2 : 4;                  // TMEM accumulators
+  static constexpr int TILE_BYTES = 128 * D * ESIZE;      // A tile: 128 rows
+  static constexpr int HALF_BYTES = 128 * 128;            // 128 rows x 128 bytes
   static constexpr int B_HALF_BYTES = N * 128;
-  static constexpr int B_BYTES = N * D * 2;
-  static constexpr int ACC_COLS = kAcc * N;
+  static constexpr int B_BYTES = N * D * ESIZE;
+  static constexpr int ACC_COLS = ACC * N;
   static constexpr int TMEM_COLS =
       ACC_COLS <= 32 ? 32 : ACC_COLS <= 64 ? 64 : ACC_COLS <= 128 ? 128 : ACC_COLS <= 256 ? 256 : 512;
   static constexpr uint32_t IDESC = idesc_f16_f32(128, N);
   // barriers and TMEM address (256 B), sin/cos (T*D floats), RoPE frequencies (D/2
-  // doubles), raw queries (T*H*D f16), the score-prefix histogram, one pooled row (f32)
-  static constexpr int CTRL_BYTES = 256 + T * D * 4 + D / 2 * 8 + T * H * D * 2 + kHistBins * 4 + D * 4;
+  // doubles), raw queries (T*H*D f16), the score-prefix histogram, one pooled row (f32),
+  // the rotated query in f32 (8-bit keys: T*H*D floats)
+  static constexpr int CTRL_BYTES =
+      256 + T * D * 4 + D / 2 * 8 + T * H * D * 2 + kHistBins * 4 + D * 4 + (F8 ? T * H * D * 4 : 0);
   static constexpr size_t FIXED = 1024 + size_t(B_BYTES) + CTRL_BYTES;
   // ring depth: kScanStages tiles where they fit, fewer for wide B operands. A short ring
   // keeps the CTA small enough to be resident beside the attention and selection kernels'
@@ -84,7 +91,8 @@ struct ScanShape {
   static constexpr int STAGES = FIXED + kScanStages * size_t(TILE_BYTES) <= kSmemMax ? kScanStages
                                 : FIXED + 5 * size_t(TILE_BYTES) <= kSmemMax ? 5 : 4;
   static constexpr size_t SMEM = FIXED + size_t(STAGES) * TILE_BYTES;
-  static_assert(NQ <= 32, "the epilogue reads at most 32 accumulator columns per query");
+  static_assert(NQ <= 80 && NQ % 16 == 0, "the epilogue reads the query's columns 16 at a time");
+  static_assert(!F8 || (T == 1 && D == 128), "8-bit pooled keys: one query, d_idx 128");
   static_assert(N <= 256 && ACC_COLS <= 512, "MMA N and TMEM columns");
   static_assert(SMEM <= kSmemMax, "shared memory");
   static_assert(TILE_BYTES % 1024 == 0 && B_HALF_BYTES % 1024 == 0, "1024-byte swizzle atoms");
@@ -98,6 +106,22 @@ __device__ __forceinline__ uint32_t sw128_offset(int n, int k, int half_bytes) {
   return uint32_t(j * half_bytes + (n >> 3) * 1024 + (n & 7) * 128 + (((c >> 3) ^ (n & 7)) << 4) + ((c & 7) << 1));
 }
 
+// The same for a one-byte element at column k < 128 (one 128-byte span).
+__device__ __forceinline__ uint32_t sw128_offset_b(int n, int k) {
+  return uint32_t((n >> 3) * 1024 + (n & 7) * 128 + (((k >> 4) ^ (n & 7)) << 4) + (k & 15));
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T with e4m3 operands (kind::f8f6f4), issued by one thread.
+__device__ __forceinline__ void mma_f8_ss(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}"
+      ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 }  // namespace
 
 // The fused decode step's token and caches (FUSED only).
@@ -108,7 +132,7 @@ struct DecodeAppend {
   uint4* k_cache;           // caches (K/V in f16, or e4m3 codes with kv_scales)
   uint4* v_cache;
   uint4* idx_cache;
-  __half* pooled;           // the pooled cache the TMA maps describe
+  PooledOut pooled;         // the pooled cache the TMA maps describe (f16, or e4m3 + scales)
   const float* gain;        // RMS-norm gain or null
   float* kv_scales;
   PoolRope rope;
@@ -175,16 +199,17 @@ __device__ __forceinline__ void decode_append_pool(const DecodeAppend& a, DevSta
   if (lane == 0) mbar_arrive(pool_bar);
 }
 
-template <int D, int H, int T, bool HIST, bool FUSED>
+template <int D, int H, int T, bool HIST, bool FUSED, bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
 index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_constant__ CUtensorMap map_box,
                      DevState* st, const __half* __restrict__ q_idx, const float* __restrict__ w,
                      float* __restrict__ scores, uint32_t* __restrict__ hist, float rope_base, int max_blocks,
                      int rope_dims, int rope_interleaved, int rope_pos_stride, int score_stride, DecodeAppend app,
-                     int q_n) {
+                     int q_n, const float* pooled_scales) {
   static_assert(!(HIST || FUSED) || T == 1, "histogram and fused append serve the single-query step");
   static_assert(!FUSED || HIST, "the decode step always fills the histogram");
-  using S = ScanShape<D, H, T>;
+  using S = ScanShape<D, H, T, F8>;
+  constexpr int kAcc = S::ACC;
   constexpr int kStages = S::STAGES;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -196,6 +221,8 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_
   uint64_t* tempty = tfull + kAcc;
   uint64_t* pool_bar = tempty + kAcc;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(pool_bar + 1);
+  float* s_qmax = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(full) + 192);  // [4] (8-bit keys)
+  static_assert((2 * kStages + 2 * kAcc + 1) * 8 + 4 <= 192, "barriers below the query-max slots");
   float* s_cos = reinterpret_cast<float*>(smem + size_t(kStages) * S::TILE_BYTES + S::B_BYTES + 256);
   float* s_sin = s_cos + T * (D / 2);                                 // [T][D/2] each
   double* s_theta = reinterpret_cast<double*>(s_sin + T * (D / 2));   // D/2 doubles
@@ -234,7 +261,7 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_
     const int p1 = int((long long)(blockIdx.x + 1) * nb_hint / gridDim.x);
     for (int r = p0; r < p1; r += 128)
 #pragma unroll
-      for (int j = 0; j < S::HALVES; ++j) tma_prefetch_l2_2d(&map_tile, j * 64, r);
+      for (int j = 0; j < S::HALVES; ++j) tma_prefetch_l2_2d(&map_tile, j * (128 / S::ESIZE), r);
   }
   // RoPE frequencies do not depend on the previous kernel: compute them before waiting on it
   for (int i = threadIdx.x; i < rope_dims / 2; i += blockDim.x)
@@ -294,14 +321,14 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_
             mbar_arrive_expect_tx(&full[s], uint32_t(S::TILE_BYTES));
 #pragma unroll
             for (int j = 0; j < S::HALVES; ++j)
-              tma_load_2d(dst + j * S::HALF_BYTES, &map_tile, j * 64, r0 + t * 128, &full[s]);
+              tma_load_2d(dst + j * S::HALF_BYTES, &map_tile, j * (128 / S::ESIZE), r0 + t * 128, &full[s]);
           } else {            // ragged tail: 16-row boxes, at most 15 rows past the range
             const int boxes = (rows + kBoxRows - 1) / kBoxRows;
             mbar_arrive_expect_tx(&full[s], uint32_t(boxes * kBoxRows * 128 * S::HALVES));
 #pragma unroll
             for (int j = 0; j < S::HALVES; ++j)
               for (int b = 0; b < boxes; ++b)
-                tma_load_2d(dst + j * S::HALF_BYTES + b * kBoxRows * 128, &map_box, j * 64,
+                tma_load_2d(dst + j * S::HALF_BYTES + b * kBoxRows * 128, &map_box, j * (128 / S::ESIZE),
                             r0 + t * 128 + b * kBoxRows, &full[s]);
           }
           ++issued;
@@ -326,11 +353,12 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_
           const uint32_t a0 = smem_u32(sA + size_t(s) * S::TILE_BYTES);
           const uint32_t b0 = smem_u32(sB);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const int j = kk >> 2, kin = kk & 3;  // 64-column half, 16-column step inside it
+          for (int kk = 0; kk < S::K_STEPS; ++kk) {
+            const int j = kk >> 2, kin = kk & 3;  // 128-byte span, 32-byte K step inside it
             const uint64_t adesc = smem_desc_sw128(a0 + j * S::HALF_BYTES + kin * 32);
             const uint64_t bdesc = smem_desc_sw128(b0 + j * S::B_HALF_BYTES + kin * 32);
-            mma_f16_ss(d_tmem, adesc, bdesc, S::IDESC, kk > 0 ? 1u : 0u);
+            if constexpr (F8) mma_f8_ss(d_tmem, adesc, bdesc, S::IDESC, kk > 0 ? 1u : 0u);
+            else mma_f16_ss(d_tmem, adesc, bdesc, S::IDESC, kk > 0 ? 1u : 0u);
           }
           tc_commit(&empty[s]);
           tc_commit(&tfull[a]);
@@ -352,6 +380,21 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_
         if (tid + k * 128 < QV) qraw[k] = reinterpret_cast<const uint4*>(q_idx)[tid + k * 128];
       if constexpr (HIST)
         for (int i = tid; i < kHistBins; i += 128) s_hist[i] = 0u;
+      if constexpr (F8) {  // largest |raw query element|: sets the power-of-2 prescale below
+        float m = 0.0f;
+#pragma unroll
+        for (int k = 0; k < (QV + 127) / 128; ++k)
+          if (tid + k * 128 < QV) {
+            const __half2* hv = reinterpret_cast<const __half2*>(&qraw[k]);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float2 f = __half22float2(hv[i]);
+              m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+            }
+          }
+        m = warp_max(m);
+        if (lane == 0) s_qmax[warp] = m;
+      }
       // query u belongs to token n - T + u: on the block-position scale it sits at
       // floor(stride * (n_u - 1) / 4), n_u = n - T + u + 1 (token n_u - 1 when stride = 4)
       const int half_r = rope_dims / 2;
@@ -370,13 +413,36 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_
       for (int k = 0; k < (QV + 127) / 128; ++k)
         if (tid + k * 128 < QV) reinterpret_cast<uint4*>(s_q)[tid + k * 128] = qraw[k];
       named_bar_sync(2, 128);
-      // rotated element e of head h of query u -> high f16 part in B row u*NQ + h, scaled
-      // residual in row u*NQ + H + h
+      // 8-bit keys: the rotated query times pre = 2^k, k set so that the largest raw element
+      // lands in [64, 128); a rotated element is at most sqrt(2) times that, inside e4m3's
+      // range (448). Each element becomes kF8Terms e4m3 terms, x_0 = pre * q~,
+      // v_t = e4m3(x_t), x_{t+1} = (x_t - v_t) * 16 (both steps exact in f32), so that
+      // pre * q~ = sum_t v_t 16^-t up to the last term's rounding (~2^-20 relative); term t
+      // of head h is B row t*H + h and its dots are weighted by 16^-t in the epilogue.
+      float pre = 1.0f;
+      if constexpr (F8) {
+        const float m = fmaxf(fmaxf(s_qmax[0], s_qmax[1]), fmaxf(s_qmax[2], s_qmax[3]));
+        int ex = 0;
+        (void)frexpf(m, &ex);
+        if (m > 0.0f) pre = ldexpf(1.0f, 7 - ex);
+      }
+      // rotated element e of head h of query u -> f16: high part in B row u*NQ + h, scaled
+      // residual in row u*NQ + H + h; e4m3: terms in rows t*H + h
       auto put = [&](int u, int h, int e, float r) {
-        const __half hi = __float2half_rn(r);
-        const __half lo = __float2half_rn((r - __half2float(hi)) * kLoScale);
-        *reinterpret_cast<__half*>(sB + sw128_offset(u * S::NQ + h, e, S::B_HALF_BYTES)) = hi;
-        *reinterpret_cast<__half*>(sB + sw128_offset(u * S::NQ + H + h, e, S::B_HALF_BYTES)) = lo;
+        if constexpr (F8) {
+          float x = r * pre;
+#pragma unroll
+          for (int t = 0; t < kF8Terms; ++t) {
+            const __nv_fp8_storage_t v = __nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E4M3);
+            sB[sw128_offset_b(t * H + h, e)] = v;
+            x = (x - __half2float(__half(__nv_cvt_fp8_to_halfraw(v, __NV_E4M3)))) * 16.0f;
+          }
+        } else {
+          const __half hi = __float2half_rn(r);
+          const __half lo = __float2half_rn((r - __half2float(hi)) * kLoScale);
+          *reinterpret_cast<__half*>(sB + sw128_offset(u * S::NQ + h, e, S::B_HALF_BYTES)) = hi;
+          *reinterpret_cast<__half*>(sB + sw128_offset(u * S::NQ + H + h, e, S::B_HALF_BYTES)) = lo;
+        }
       };
       if (rope_dims == D && !rope_interleaved) {  // NeoX pairs (i, i + D/2) over all dims
         for (int e = tid; e < T * H * (D / 2); e += 128) {
@@ -402,12 +468,15 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_
           put(u, h, k, r);
         }
       }
-      constexpr int PAD = S::NQ - 2 * H;  // zero rows after each query's hi and lo rows
+      constexpr int USED = S::TERMS * H;
+      constexpr int PAD = S::NQ - USED;  // zero rows after each query's term rows
       if constexpr (PAD > 0) {
         for (int e = tid; e < T * PAD * D; e += 128) {
           const int u = e / (PAD * D), rem = e % (PAD * D);
-          *reinterpret_cast<__half*>(sB + sw128_offset(u * S::NQ + 2 * H + rem / D, rem % D, S::B_HALF_BYTES)) =
-              __float2half_rn(0.0f);
+          if constexpr (F8) sB[sw128_offset_b(USED + rem / D, rem % D)] = 0;
+          else
+            *reinterpret_cast<__half*>(sB + sw128_offset(u * S::NQ + USED + rem / D, rem % D, S::B_HALF_BYTES)) =
+                __float2half_rn(0.0f);
         }
       }
       fence_proxy_async_smem();
@@ -419,30 +488,52 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_
 #pragma unroll
         for (int h = 0; h < H; ++h) wr[u][h] = w[u * H + h];
       const float sqrt_d = sqrtf((float)D);
+      const float unscale = 1.0f / pre;  // a power of 2: exact
       bool ok = true;
       for (int t = 0; t < n_tiles; ++t) {
         const int a = t % kAcc;
+        const int row = r0 + t * 128 + tid;
+        // 8-bit keys: the row's scale (the block this step pools: once warp 6 has written it)
+        float row_scale = 1.0f;
+        if constexpr (F8)
+          if (row < r1 && t != pool_tile) row_scale = pooled_scales[row];
         if (!mbar_wait(&tfull[a], (t / kAcc) & 1)) { ok = false; break; }
+        if constexpr (F8)
+          if (row < r1 && t == pool_tile && mbar_wait(pool_bar, 0)) row_scale = pooled_scales[row];
         tc_fence_after();
         const uint32_t taddr = tmem_base + (uint32_t(32 * warp) << 16) + uint32_t(a * S::N);
         uint32_t r[T][S::NQ];  // query u's columns [u*NQ, (u+1)*NQ) of this row
 #pragma unroll
         for (int u = 0; u < T; ++u) {
-          if constexpr (S::NQ == 32) tmem_ld_32x32b_x32(taddr + uint32_t(u * S::NQ), r[u]);
-          else tmem_ld_32x32b_x16(taddr + uint32_t(u * S::NQ), r[u]);
+#pragma unroll
+          for (int c = 0; c < S::NQ / 32; ++c)
+            tmem_ld_32x32b_x32(taddr + uint32_t(u * S::NQ + 32 * c), reinterpret_cast<uint32_t(&)[32]>(r[u][32 * c]));
+          if constexpr (S::NQ % 32 != 0)
+            tmem_ld_32x32b_x16(taddr + uint32_t(u * S::NQ + S::NQ / 32 * 32),
+                               reinterpret_cast<uint32_t(&)[16]>(r[u][S::NQ / 32 * 32]));
         }
         tmem_ld_wait();
         tc_fence_before();
         mbar_arrive(&tempty[a]);
-        const int row = r0 + t * 128 + tid;
         if (row < r1) {
 #pragma unroll
           for (int u = 0; u < T; ++u) {
             float s = 0.0f;
 #pragma unroll
-            for (int h = 0; h < H; ++h)
-              s += wr[u][h] * fmaxf(__uint_as_float(r[u][h]) + __uint_as_float(r[u][H + h]) * (1.0f / kLoScale), 0.0f);
-            const float score = s / sqrt_d;
+            for (int h = 0; h < H; ++h) {
+              float dot;
+              if constexpr (F8) {  // sum_t acc_t 16^-t, smallest term first
+                dot = __uint_as_float(r[u][(kF8Terms - 1) * H + h]);
+#pragma unroll
+                for (int tt = kF8Terms - 2; tt >= 0; --tt) dot = fmaf(dot, 1.0f / 16.0f, __uint_as_float(r[u][tt * H + h]));
+              } else {
+                dot = __uint_as_float(r[u][h]) + __uint_as_float(r[u][H + h]) * (1.0f / kLoScale);
+              }
+              s += wr[u][h] * fmaxf(dot, 0.0f);
+            }
+            // 8-bit keys: the dots were of pre * q~ with the codes; scale and prescale are
+            // positive, so they come out of the max(0, .) unchanged
+            const float score = F8 ? s * (row_scale * unscale) / sqrt_d : s / sqrt_d;
             scores[size_t(u) * score_stride + row] = score;
             if constexpr (HIST) atomicAdd(&s_hist[sel::score_key(score) >> (32 - kHistBits)], 1u);
           }
@@ -482,12 +573,13 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_
 // ---------------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------------
-template <int D, int H, int T, bool HIST, bool FUSED>
+template <int D, int H, int T, bool HIST, bool FUSED, bool F8 = false>
 static cudaError_t set_scan_attr() {
-  cudaError_t e = cudaFuncSetAttribute(index_scan_tc_kernel<D, H, T, HIST, FUSED>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ScanShape<D, H, T>::SMEM);
+  cudaError_t e = cudaFuncSetAttribute(index_scan_tc_kernel<D, H, T, HIST, FUSED, F8>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)ScanShape<D, H, T, F8>::SMEM);
   if (e == cudaSuccess)  // the whole unified L1/shared array as shared memory (see qsa_device.cuh)
-    e = cudaFuncSetAttribute(index_scan_tc_kernel<D, H, T, HIST, FUSED>,
+    e = cudaFuncSetAttribute(index_scan_tc_kernel<D, H, T, HIST, FUSED, F8>,
                              cudaFuncAttributePreferredSharedMemoryCarveout, kCarveoutMaxShared);
   return e;
 }
@@ -502,6 +594,12 @@ static cudaError_t set_scan_attr_t() {
       (e = set_scan_attr<D, H, 3, false, false>()) != cudaSuccess ||
       (e = set_scan_attr<D, H, 4, false, false>()) != cudaSuccess)
     return e;
+  if constexpr (D == 128) {  // 8-bit pooled keys: single query
+    if ((e = set_scan_attr<D, H, 1, false, false, true>()) != cudaSuccess ||
+        (e = set_scan_attr<D, H, 1, true, false, true>()) != cudaSuccess ||
+        (e = set_scan_attr<D, H, 1, true, true, true>()) != cudaSuccess)
+      return e;
+  }
   return cudaSuccess;
 }
 
@@ -523,8 +621,8 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-// TMA descriptor of a layer's pooled cache: rows = max_ctx/4 blocks of d_idx f16,
-// box_rows x 64-column boxes written with the 128-byte swizzle.
+// TMA descriptor of a layer's pooled cache: rows = max_ctx/4 blocks of d_idx f16 (or e4m3
+// codes with QSA_POOLED_FP8), box_rows x 128-byte boxes written with the 128-byte swizzle.
 cudaError_t encode_pooled_map(const qsa_config& c, void* pooled, int box_rows, CUtensorMap* out) {
   static EncodeTiledFn fn = nullptr;
   if (!fn) {
@@ -536,23 +634,26 @@ cudaError_t encode_pooled_map(const qsa_config& c, void* pooled, int box_rows, C
     fn = reinterpret_cast<EncodeTiledFn>(p);
   }
   const cuuint64_t dims[2] = {cuuint64_t(c.d_idx), cuuint64_t(c.max_ctx / kBlock)};
-  const cuuint64_t strides[1] = {cuuint64_t(c.d_idx) * 2};
-  const cuuint32_t box[2] = {64, cuuint32_t(box_rows)};
+  const bool fp8 = c.pooled_format == QSA_POOLED_FP8;
+  const cuuint64_t strides[1] = {cuuint64_t(c.d_idx) * (fp8 ? 1 : 2)};
+  const cuuint32_t box[2] = {fp8 ? 128u : 64u, cuuint32_t(box_rows)};
   const cuuint32_t estr[2] = {1, 1};
-  const CUresult r = fn(out, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, pooled, dims, strides, box, estr,
+  const CUresult r = fn(out, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, pooled, dims,
+                        strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-template <int D, int H, int T, bool HIST, bool FUSED>
+template <int D, int H, int T, bool HIST, bool FUSED, bool F8 = false>
 static cudaError_t launch_scan_tc(const LayerView& L, const void* q_idx, const float* w, float* scores,
                                   cudaStream_t s, int score_stride, uint32_t* hist, const DecodeAppend& app,
                                   int q_n = 0) {
-  return launch_pdl(index_scan_tc_kernel<D, H, T, HIST, FUSED>, dim3(L.n_sms), dim3(kThreads),
-                    ScanShape<D, H, T>::SMEM, s, 1, L.pooled_tile_map, L.pooled_box_map, L.state,
+  return launch_pdl(index_scan_tc_kernel<D, H, T, HIST, FUSED, F8>, dim3(L.n_sms), dim3(kThreads),
+                    ScanShape<D, H, T, F8>::SMEM, s, 1, L.pooled_tile_map, L.pooled_box_map, L.state,
                     (const __half*)q_idx, w, scores, hist, L.cfg.rope_base, L.cfg.max_ctx / kBlock, L.cfg.rope_dims,
-                    L.cfg.rope_interleaved, L.cfg.rope_pos_stride, score_stride, app, q_n);
+                    L.cfg.rope_interleaved, L.cfg.rope_pos_stride, score_stride, app, q_n,
+                    (const float*)L.pooled_scales);
 }
 
 // mode 0: plain scan of T queries; 1: single query with the histogram; 2: decode step
@@ -560,6 +661,16 @@ template <int D, int H>
 static cudaError_t launch_scan_tc_t(const LayerView& L, const void* q_idx, const float* w, float* scores,
                                     cudaStream_t s, int n_queries, int score_stride, uint32_t* hist, int mode,
                                     const DecodeAppend& app, int q_n) {
+  if (L.cfg.pooled_format == QSA_POOLED_FP8) {  // single query (checked by the callers)
+    if constexpr (D == 128) {
+      if (n_queries != 1) return cudaErrorInvalidValue;
+      if (mode == 2) return launch_scan_tc<D, H, 1, true, true, true>(L, q_idx, w, scores, s, score_stride, hist, app);
+      if (mode == 1)
+        return launch_scan_tc<D, H, 1, true, false, true>(L, q_idx, w, scores, s, score_stride, hist, app, q_n);
+      return launch_scan_tc<D, H, 1, false, false, true>(L, q_idx, w, scores, s, score_stride, hist, app, q_n);
+    }
+    return cudaErrorInvalidValue;
+  }
   if (mode == 2) return launch_scan_tc<D, H, 1, true, true>(L, q_idx, w, scores, s, score_stride, hist, app);
   if (mode == 1) return launch_scan_tc<D, H, 1, true, false>(L, q_idx, w, scores, s, score_stride, hist, app, q_n);
   switch (n_queries) {
@@ -611,7 +722,7 @@ cudaError_t launch_decode_scan(const LayerView& L, const void* k, const void* v,
   app.k_cache = static_cast<uint4*>(L.k_cache);
   app.v_cache = static_cast<uint4*>(L.v_cache);
   app.idx_cache = static_cast<uint4*>(L.idx_cache);
-  app.pooled = static_cast<__half*>(L.pooled_cache);
+  app.pooled = pooled_out(L);
   app.gain = L.rms_gain;
   app.kv_scales = L.kv_scales;
   app.rope = PoolRope{L.cfg.rope_base, L.cfg.rope_dims, L.cfg.rope_interleaved,

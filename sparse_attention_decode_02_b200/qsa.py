@@ -19,9 +19,10 @@ STATUS_NAMES = {0: "QSA_OK", 1: "QSA_ERR_INVALID_ARG", 2: "QSA_ERR_CAPACITY", 3:
                 4: "QSA_ERR_CUDA", 5: "QSA_ERR_UNSUPPORTED", 6: "QSA_ERR_BAD_INDEX",
                 7: "QSA_ERR_TIMEOUT"}
 (QSA_BUF_KV, QSA_BUF_IDX, QSA_BUF_POOLED, QSA_BUF_WORKSPACE, QSA_BUF_MAX_CELLS, QSA_BUF_SCORE_STRIDE,
- QSA_BUF_KV_SCALES) = range(7)
+ QSA_BUF_KV_SCALES, QSA_BUF_POOLED_SCALES) = range(8)
 QSA_KV_F16, QSA_KV_FP8 = 0, 1
 QSA_SCAN_TENSOR, QSA_SCAN_CUDA_CORES = 0, 1
+QSA_POOLED_F16, QSA_POOLED_FP8 = 0, 1
 QSA_MAX_QUERIES = 4
 
 
@@ -37,13 +38,13 @@ class QsaConfig(ctypes.Structure):
                 ("n_kv_heads", c_int32), ("head_dim", c_int32), ("rope_base", c_float),
                 ("rms_eps", c_float), ("rope_dims", c_int32), ("rope_interleaved", c_int32),
                 ("rope_pos_stride", c_int32), ("rope_pos_offset", c_int32), ("kv_format", c_int32),
-                ("scan_kind", c_int32)]
+                ("scan_kind", c_int32), ("pooled_format", c_int32)]
 
 
 class QsaLayerBuffers(ctypes.Structure):
     _fields_ = [("k_cache", c_void_p), ("v_cache", c_void_p), ("idx_cache", c_void_p),
                 ("pooled_cache", c_void_p), ("rms_gain", c_void_p), ("workspace", c_void_p),
-                ("kv_scales", c_void_p)]
+                ("kv_scales", c_void_p), ("pooled_scales", c_void_p)]
 
 
 _P = c_void_p
@@ -124,10 +125,11 @@ def _stream(stream):
 
 def make_config(n_layers, max_ctx, d_idx, n_idx_heads, top_k_tokens, n_q_heads, n_kv_heads, head_dim,
                 rope_base=10000.0, rms_eps=1e-6, rope_dims=0, rope_interleaved=False, rope_pos_stride=4,
-                rope_pos_offset=0, kv_format=QSA_KV_F16, scan_kind=QSA_SCAN_TENSOR) -> QsaConfig:
+                rope_pos_offset=0, kv_format=QSA_KV_F16, scan_kind=QSA_SCAN_TENSOR,
+                pooled_format=QSA_POOLED_F16) -> QsaConfig:
     return QsaConfig(n_layers, max_ctx, d_idx, n_idx_heads, top_k_tokens, n_q_heads, n_kv_heads, head_dim,
                      rope_base, rms_eps, rope_dims, int(bool(rope_interleaved)), rope_pos_stride, rope_pos_offset,
-                     kv_format, scan_kind)
+                     kv_format, scan_kind, pooled_format)
 
 
 def buffer_bytes(cfg: QsaConfig, which: int) -> int:
@@ -166,9 +168,9 @@ class Qsa:
         return buffer_bytes(self.cfg, which)
 
     def bind_layer(self, layer, k_cache, v_cache, idx_cache, pooled_cache, workspace, rms_gain=None,
-                   kv_scales=None, stream=None):
+                   kv_scales=None, pooled_scales=None, stream=None):
         b = QsaLayerBuffers(_ptr(k_cache), _ptr(v_cache), _ptr(idx_cache), _ptr(pooled_cache),
-                            _ptr(rms_gain), _ptr(workspace), _ptr(kv_scales))
+                            _ptr(rms_gain), _ptr(workspace), _ptr(kv_scales), _ptr(pooled_scales))
         self._check(self.lib.qsa_bind_layer(self.handle, layer, ctypes.byref(b), _stream(stream)))
 
     def restore_layer(self, layer, n_ctx, n_pooled, stream=None):
@@ -307,12 +309,16 @@ def alloc_layer(cfg: QsaConfig, device="cuda"):
         "k_cache": torch.zeros(shape, dtype=kv_dtype, device=device),
         "v_cache": torch.zeros(shape, dtype=kv_dtype, device=device),
         "idx_cache": torch.zeros(cfg.max_ctx, cfg.d_idx, dtype=torch.float16, device=device),
-        "pooled_cache": torch.zeros(cfg.max_ctx // 4, cfg.d_idx, dtype=torch.float16, device=device),
+        "pooled_cache": torch.zeros(cfg.max_ctx // 4, cfg.d_idx, device=device,
+                                    dtype=torch.uint8 if cfg.pooled_format == QSA_POOLED_FP8 else torch.float16),
         "workspace": torch.zeros(buffer_bytes(cfg, QSA_BUF_WORKSPACE), dtype=torch.uint8, device=device),
     }
     assert bufs["k_cache"].numel() * bufs["k_cache"].element_size() == buffer_bytes(cfg, QSA_BUF_KV)
     if fp8:
         bufs["kv_scales"] = torch.zeros(cfg.max_ctx, cfg.n_kv_heads, 2, dtype=torch.float32, device=device)
+    if cfg.pooled_format == QSA_POOLED_FP8:
+        bufs["pooled_scales"] = torch.zeros(cfg.max_ctx // 4, dtype=torch.float32, device=device)
+    assert bufs["pooled_cache"].numel() * bufs["pooled_cache"].element_size() == buffer_bytes(cfg, QSA_BUF_POOLED)
     return bufs
 
 

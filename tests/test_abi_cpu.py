@@ -125,7 +125,7 @@ def test_null_arguments_are_rejected(lib):
 
 def test_layer_bytes_is_buffer_bytes(lib):
     cfg = Q.make_config(12, 255184 + 512, 128, 16, 2048, 32, 4, 128)
-    for which in range(7):
+    for which in range(8):
         assert lib.qsa_layer_bytes(ctypes.byref(cfg), which) == Q.buffer_bytes(cfg, which)
 
 
