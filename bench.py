@@ -190,7 +190,7 @@ class Workbench:
         max_ctx = int(math.ceil((wl.n_prefill + n_graph_steps + extra_steps + 8) / 4) * 4)
         self.cfg = Q.make_config(n_layers, max_ctx, wl.d_idx, wl.n_idx_heads, wl.top_k_tokens, wl.n_q_heads,
                                  wl.n_kv_heads, wl.head_dim, wl.rope_base, wl.rms_eps, kv_format=kv_format,
-                                 pooled_format=pooled_format)
+                                 pooled_format=pooled_format, early_inputs=Q.QSA_INPUTS_EARLY)
         self.qsa = Q.Qsa(self.cfg)
         self.bufs, self.outs = [], []
         for layer in range(n_layers):
@@ -762,6 +762,7 @@ def main_ours(args):
                        "batch": 1, "parallelism": f"replicas x{world}",
                        "l2": "inputs larger than L2 (each step reads ~20.6 MB per layer x 12 layers)",
                        "graph_steps_per_replay": main["graph_steps"],
+                       "early_inputs": "step inputs are staged (device copies) before the graph that reads them",
                        "timed_graphs": "each replayed once untimed and rolled back before the timed region"},
             "roofline": roofline,
             "cpu_baseline": cpu,

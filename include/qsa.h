@@ -106,11 +106,20 @@ typedef struct {
    * tensor cores with 8-bit operands (d_idx 128, QSA_SCAN_TENSOR and single-query scans
    * only: otherwise QSA_ERR_UNSUPPORTED). The scan then reads half the bytes. */
   int32_t pooled_format;
+  /* When a call may read its inputs (token rows, queries, head weights).
+   * QSA_INPUTS_ORDERED (0): only after the previous work on the stream has completed.
+   * QSA_INPUTS_EARLY (1): the caller guarantees that every input of a call is complete in
+   * device memory before the call's first kernel can start: written by copies or by
+   * kernels that finish first, never by a kernel on the same stream that lets its
+   * dependents start early (programmatic dependent launch). The indexer scan then loads
+   * and splits the query while the previous kernel still runs. Results are identical. */
+  int32_t early_inputs;
 } qsa_config;
 
 enum { QSA_KV_F16 = 0, QSA_KV_FP8 = 1 };
 enum { QSA_SCAN_TENSOR = 0, QSA_SCAN_CUDA_CORES = 1 };
 enum { QSA_POOLED_F16 = 0, QSA_POOLED_FP8 = 1 };
+enum { QSA_INPUTS_ORDERED = 0, QSA_INPUTS_EARLY = 1 };
 
 /* Caller-owned device buffers of one layer. Sizes come from qsa_buffer_bytes(). */
 typedef struct {

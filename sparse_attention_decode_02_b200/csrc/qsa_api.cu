@@ -55,6 +55,8 @@ const char* config_problem(const qsa_config& c) {
     return "pooled_format must be QSA_POOLED_F16 or QSA_POOLED_FP8";
   if (c.pooled_format == QSA_POOLED_FP8 && (c.d_idx != 128 || c.scan_kind != QSA_SCAN_TENSOR))
     return "QSA_POOLED_FP8 needs d_idx 128 and the tensor-core scan";
+  if (c.early_inputs != QSA_INPUTS_ORDERED && c.early_inputs != QSA_INPUTS_EARLY)
+    return "early_inputs must be QSA_INPUTS_ORDERED or QSA_INPUTS_EARLY";
   return nullptr;
 }
 

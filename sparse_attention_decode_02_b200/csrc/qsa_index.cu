@@ -31,13 +31,18 @@ block_topk_kernel(DevState* st, const float* __restrict__ scores, int32_t* __res
   scores += size_t(u) * score_stride;
   sel_out += size_t(u) * k_blocks;
   n_sel += u;
+  __shared__ uint64_t s_gather_bar;  // CTA 0: every CTA's candidates have landed (histogram path)
+  if (threadIdx.x == 0) {
+    sm100::mbar_init(&s_gather_bar, sel::kCS);
+    sm100::fence_mbar_init();
+  }
   pdl_launch_dependents();
   if (threadIdx.x == 0) QSA_TL(st, kTlTopk, kTlEntry);
   cluster_arrive_relaxed();  // paired inside cluster_select
   pdl_wait();
   if (threadIdx.x == 0) QSA_TL(st, kTlTopk, kTlWait);
   const sel::Result res = sel::cluster_select<V>(st, scores, gridDim.y == 1 ? hist : nullptr, k_blocks, max_blocks,
-                                                 n_back,
+                                                 n_back, &s_gather_bar,
                                                  [&](uint32_t pos, int block) {
                                                    // bounds-checked in every build
                                                    if (pos < uint32_t(k_blocks) && block < max_blocks) {

@@ -28,12 +28,18 @@ struct DevState {
   int32_t status;         // first device-side error (qsa_status), 0 if none
   uint32_t ticket_append; // last-CTA tickets of multi-CTA kernels (reset by the last CTA)
   uint32_t ticket_pool;
-  // timeline build only (-DQSA_TIMELINE): [kernel][point][min, max] of the low 32 bits of
-  // %globaltimer (ns) that the CTAs of the step's kernels reached at each probe point
-  uint32_t timeline[5][5][2];  // scan, top-k, attention, top-k detail, attention detail
-  int32_t reserved[9];
+  int32_t reserved[59];
 };
 static_assert(sizeof(DevState) == 256, "DevState must stay 256 bytes");
+
+// Timeline build only (-DQSA_TIMELINE): right after a layer's DevState in its workspace,
+// [kernel][point][min, max] of the low 32 bits of %globaltimer (ns) that the CTAs of the
+// step's kernels reached at each probe point (kernels: scan, top-k, attention, and detail
+// rows of each).
+constexpr int kTimelineKernels = 8, kTimelinePoints = 5;
+constexpr size_t kTimelineOffset = sizeof(DevState);
+constexpr size_t kTimelineBytes = 512;
+static_assert(kTimelineKernels * kTimelinePoints * 2 * 4 <= kTimelineBytes, "timeline region");
 
 // Byte offsets inside a layer's workspace (all 256-byte aligned).
 struct WorkspaceLayout {
@@ -70,6 +76,7 @@ inline WorkspaceLayout workspace_layout(const qsa_config& c, int n_splits) {
   size_t off = 0;
   w.state = off;
   off += align256(sizeof(DevState));
+  off += kTimelineBytes;  // the timeline build's probe record (kTimelineOffset)
   w.hist = off;  // score-key prefix histogram of the last scan (zero between selections)
   off += align256(size_t(1 << kHistBits) * sizeof(uint32_t));
   w.cp = off;    // a context-parallel shard's part of the global selection: count, then ids

@@ -205,7 +205,7 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_
                      DevState* st, const __half* __restrict__ q_idx, const float* __restrict__ w,
                      float* __restrict__ scores, uint32_t* __restrict__ hist, float rope_base, int max_blocks,
                      int rope_dims, int rope_interleaved, int rope_pos_stride, int score_stride, DecodeAppend app,
-                     int q_n, const float* pooled_scales) {
+                     int q_n, const float* pooled_scales, int early) {
   static_assert(!(HIST || FUSED) || T == 1, "histogram and fused append serve the single-query step");
   static_assert(!FUSED || HIST, "the decode step always fills the histogram");
   using S = ScanShape<D, H, T, F8>;
@@ -222,6 +222,7 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_
   uint64_t* pool_bar = tempty + kAcc;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(pool_bar + 1);
   float* s_qmax = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(full) + 192);  // [4] (8-bit keys)
+  int* s_nspec = reinterpret_cast<int*>(reinterpret_cast<unsigned char*>(full) + 208);     // early B operand
   static_assert((2 * kStages + 2 * kAcc + 1) * 8 + 4 <= 192, "barriers below the query-max slots");
   float* s_cos = reinterpret_cast<float*>(smem + size_t(kStages) * S::TILE_BYTES + S::B_BYTES + 256);
   float* s_sin = s_cos + T * (D / 2);                                 // [T][D/2] each
@@ -270,6 +271,140 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+
+  // ---- warps 0-3: the B operand, the query rotated at the position of token n_pos - 1
+  // (its last query) and split (f16 high and low parts, or e4m3 terms) ----
+  const int tid = threadIdx.x;  // 0..127 in warps 0-3
+  float pre = 1.0f;             // 8-bit keys: the query's power-of-2 prescale
+  auto build_b = [&](int n_pos) {
+    // raw queries: T*H*D f16 = T*H*D/8 16-byte vectors, all loads in flight at once
+    constexpr int QV = T * H * D / 8;
+    uint4 qraw[(QV + 127) / 128];
+#pragma unroll
+    for (int k = 0; k < (QV + 127) / 128; ++k)
+      if (tid + k * 128 < QV) qraw[k] = reinterpret_cast<const uint4*>(q_idx)[tid + k * 128];
+    if constexpr (F8) {  // largest |raw query element|: sets the power-of-2 prescale below
+      float m = 0.0f;
+#pragma unroll
+      for (int k = 0; k < (QV + 127) / 128; ++k)
+        if (tid + k * 128 < QV) {
+          const __half2* hv = reinterpret_cast<const __half2*>(&qraw[k]);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 f = __half22float2(hv[i]);
+            m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+          }
+        }
+      m = warp_max(m);
+      if (lane == 0) s_qmax[warp] = m;
+    }
+    // query u belongs to token n_pos - T + u: on the block-position scale it sits at
+    // floor(stride * (n_u - 1) / 4), n_u = n_pos - T + u + 1 (token n_u - 1 when stride = 4)
+    const int half_r = rope_dims / 2;
+    for (int i = tid; i < T * half_r; i += 128) {
+      const int u = i / half_r, f = i % half_r;
+      const int n_u = n_pos - (T - 1 - u);
+      const double qpos = n_u > 0 ? (double)(((long long)rope_pos_stride * (n_u - 1)) / kBlock) : 0.0;
+      double sd, cd;
+      sincos(qpos * s_theta[f], &sd, &cd);
+      s_cos[u * (D / 2) + f] = (float)cd;
+      s_sin[u * (D / 2) + f] = (float)sd;
+    }
+    if (tid == 0) QSA_TL(st, kTlScan2, 1);  // this thread's sin/cos done
+#pragma unroll
+    for (int k = 0; k < (QV + 127) / 128; ++k)
+      if (tid + k * 128 < QV) reinterpret_cast<uint4*>(s_q)[tid + k * 128] = qraw[k];
+    if (tid == 0) QSA_TL(st, kTlScan2, 0);  // this thread's query loads landed
+    named_bar_sync(2, 128);
+    // 8-bit keys: the rotated query times pre = 2^k, k set so that the largest raw element
+    // lands in [64, 128); a rotated element is at most sqrt(2) times that, inside e4m3's
+    // range (448). Each element becomes kF8Terms e4m3 terms, x_0 = pre * q~,
+    // v_t = e4m3(x_t), x_{t+1} = (x_t - v_t) * 16 (both steps exact in f32), so that
+    // pre * q~ = sum_t v_t 16^-t up to the last term's rounding (~2^-20 relative); term t
+    // of head h is B row t*H + h and its dots are weighted by 16^-t in the epilogue.
+    pre = 1.0f;
+    if constexpr (F8) {
+      const float m = fmaxf(fmaxf(s_qmax[0], s_qmax[1]), fmaxf(s_qmax[2], s_qmax[3]));
+      int ex = 0;
+      (void)frexpf(m, &ex);
+      if (m > 0.0f) pre = ldexpf(1.0f, 7 - ex);
+    }
+    // rotated element e of head h of query u -> f16: high part in B row u*NQ + h, scaled
+    // residual in row u*NQ + H + h; e4m3: terms in rows t*H + h
+    auto put = [&](int u, int h, int e, float r) {
+      if constexpr (F8) {
+        float x = r * pre;
+#pragma unroll
+        for (int t = 0; t < kF8Terms; ++t) {
+          const __nv_fp8_storage_t v = __nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E4M3);
+          sB[sw128_offset_b(t * H + h, e)] = v;
+          x = (x - __half2float(__half(__nv_cvt_fp8_to_halfraw(v, __NV_E4M3)))) * 16.0f;
+        }
+      } else {
+        const __half hi = __float2half_rn(r);
+        const __half lo = __float2half_rn((r - __half2float(hi)) * kLoScale);
+        *reinterpret_cast<__half*>(sB + sw128_offset(u * S::NQ + h, e, S::B_HALF_BYTES)) = hi;
+        *reinterpret_cast<__half*>(sB + sw128_offset(u * S::NQ + H + h, e, S::B_HALF_BYTES)) = lo;
+      }
+    };
+    if (rope_dims == D && !rope_interleaved) {  // NeoX pairs (i, i + D/2) over all dims
+      for (int e = tid; e < T * H * (D / 2); e += 128) {
+        const int uh = e / (D / 2), i = e % (D / 2);
+        const int u = uh / H, h = uh % H;
+        const __half* x = s_q + uh * D;
+        const float c = s_cos[u * (D / 2) + i], sn = s_sin[u * (D / 2) + i];
+        const float x1 = __half2float(x[i]);
+        const float x2 = __half2float(x[i + D / 2]);
+        put(u, h, i, x1 * c - x2 * sn);
+        put(u, h, i + D / 2, x1 * sn + x2 * c);
+      }
+    } else {  // partial rotary or interleaved pairs: one element at a time
+      for (int e = tid; e < T * H * D; e += 128) {
+        const int uh = e / D, k = e % D;
+        const int u = uh / H, h = uh % H;
+        const __half* x = s_q + uh * D;
+        const RopeSlot sl = rope_slot(k, rope_dims, rope_interleaved != 0);
+        const float xk = __half2float(x[k]);
+        float r = xk;
+        if (sl.freq >= 0)
+          r = xk * s_cos[u * (D / 2) + sl.freq] + sl.sign * __half2float(x[sl.partner]) * s_sin[u * (D / 2) + sl.freq];
+        put(u, h, k, r);
+      }
+    }
+    constexpr int USED = S::TERMS * H;
+    constexpr int PAD = S::NQ - USED;  // zero rows after each query's term rows
+    if constexpr (PAD > 0) {
+      for (int e = tid; e < T * PAD * D; e += 128) {
+        const int u = e / (PAD * D), rem = e % (PAD * D);
+        if constexpr (F8) sB[sw128_offset_b(USED + rem / D, rem % D)] = 0;
+        else
+          *reinterpret_cast<__half*>(sB + sw128_offset(u * S::NQ + USED + rem / D, rem % D, S::B_HALF_BYTES)) =
+              __float2half_rn(0.0f);
+      }
+    }
+  };
+  float wr[T][H];  // indexer head weights
+  auto load_w = [&]() {
+#pragma unroll
+    for (int u = 0; u < T; ++u)
+#pragma unroll
+      for (int h = 0; h < H; ++h) wr[u][h] = w[u * H + h];
+  };
+  // Inputs complete at launch (early): build the B operand and load the weights before the
+  // dependency wait, at the position the state holds now (the previous kernel on the stream
+  // does not change it, except in a sequence like append-then-scan of the same layer, where
+  // the position is checked after the wait and the operand rebuilt).
+  int pos_built = -1;
+  if (early && warp < 4) {
+    if (tid == 0) *s_nspec = ld_volatile(&st->n_ctx) + (FUSED ? 1 : 0);
+    named_bar_sync(2, 128);
+    pos_built = q_n > 0 ? q_n : *s_nspec;
+    build_b(pos_built);
+    load_w();
+  }
+  if (warp < 4 && HIST)
+    for (int i = tid; i < kHistBins; i += 128) s_hist[i] = 0u;
+
 
   if (FUSED && warp == 6) {
     // ---------------- warp 6: the decode step's append and new-block pooling ----------------
@@ -331,6 +466,7 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_
                 tma_load_2d(dst + j * S::HALF_BYTES + b * kBoxRows * 128, &map_box, j * (128 / S::ESIZE),
                             r0 + t * 128 + b * kBoxRows, &full[s]);
           }
+          if (t == 0) QSA_TL(st, kTlScan2, 3);  // first tile's loads issued
           ++issued;
         }
         if (!ok) record_status(st, QSA_ERR_TIMEOUT);
@@ -364,6 +500,7 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_
           tc_commit(&tfull[a]);
           last = t;
         }
+        if (last >= 0) QSA_TL(st, kTlScan2, 4);  // last tile's MMAs issued
         if (!ok) record_status(st, QSA_ERR_TIMEOUT);
         // the tensor core must be done with TMEM before it is freed
         if (last >= 0) mbar_wait(&tfull[last % kAcc], (last / kAcc) & 1);
@@ -371,122 +508,18 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_
       __syncwarp();
     } else {
       // ---------------- warps 0-3: rotated, split query -> B operand; then epilogue ----------------
-      const int tid = threadIdx.x;  // 0..127
-      // raw queries: T*H*D f16 = T*H*D/8 16-byte vectors, all loads in flight at once
-      constexpr int QV = T * H * D / 8;
-      uint4 qraw[(QV + 127) / 128];
-#pragma unroll
-      for (int k = 0; k < (QV + 127) / 128; ++k)
-        if (tid + k * 128 < QV) qraw[k] = reinterpret_cast<const uint4*>(q_idx)[tid + k * 128];
-      if constexpr (HIST)
-        for (int i = tid; i < kHistBins; i += 128) s_hist[i] = 0u;
-      if constexpr (F8) {  // largest |raw query element|: sets the power-of-2 prescale below
-        float m = 0.0f;
-#pragma unroll
-        for (int k = 0; k < (QV + 127) / 128; ++k)
-          if (tid + k * 128 < QV) {
-            const __half2* hv = reinterpret_cast<const __half2*>(&qraw[k]);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const float2 f = __half22float2(hv[i]);
-              m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
-            }
-          }
-        m = warp_max(m);
-        if (lane == 0) s_qmax[warp] = m;
-      }
-      // query u belongs to token n - T + u: on the block-position scale it sits at
-      // floor(stride * (n_u - 1) / 4), n_u = n - T + u + 1 (token n_u - 1 when stride = 4)
-      const int half_r = rope_dims / 2;
-      for (int i = tid; i < T * half_r; i += 128) {
-        const int u = i / half_r, f = i % half_r;
-        // q_n > 0: the query belongs to token q_n - 1 of a longer sequence whose blocks this
-        // layer holds a contiguous part of (a context-parallel shard)
-        const int n_u = (q_n > 0 ? q_n : n) - (T - 1 - u);
-        const double qpos = n_u > 0 ? (double)(((long long)rope_pos_stride * (n_u - 1)) / kBlock) : 0.0;
-        double sd, cd;
-        sincos(qpos * s_theta[f], &sd, &cd);
-        s_cos[u * (D / 2) + f] = (float)cd;
-        s_sin[u * (D / 2) + f] = (float)sd;
-      }
-#pragma unroll
-      for (int k = 0; k < (QV + 127) / 128; ++k)
-        if (tid + k * 128 < QV) reinterpret_cast<uint4*>(s_q)[tid + k * 128] = qraw[k];
-      named_bar_sync(2, 128);
-      // 8-bit keys: the rotated query times pre = 2^k, k set so that the largest raw element
-      // lands in [64, 128); a rotated element is at most sqrt(2) times that, inside e4m3's
-      // range (448). Each element becomes kF8Terms e4m3 terms, x_0 = pre * q~,
-      // v_t = e4m3(x_t), x_{t+1} = (x_t - v_t) * 16 (both steps exact in f32), so that
-      // pre * q~ = sum_t v_t 16^-t up to the last term's rounding (~2^-20 relative); term t
-      // of head h is B row t*H + h and its dots are weighted by 16^-t in the epilogue.
-      float pre = 1.0f;
-      if constexpr (F8) {
-        const float m = fmaxf(fmaxf(s_qmax[0], s_qmax[1]), fmaxf(s_qmax[2], s_qmax[3]));
-        int ex = 0;
-        (void)frexpf(m, &ex);
-        if (m > 0.0f) pre = ldexpf(1.0f, 7 - ex);
-      }
-      // rotated element e of head h of query u -> f16: high part in B row u*NQ + h, scaled
-      // residual in row u*NQ + H + h; e4m3: terms in rows t*H + h
-      auto put = [&](int u, int h, int e, float r) {
-        if constexpr (F8) {
-          float x = r * pre;
-#pragma unroll
-          for (int t = 0; t < kF8Terms; ++t) {
-            const __nv_fp8_storage_t v = __nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E4M3);
-            sB[sw128_offset_b(t * H + h, e)] = v;
-            x = (x - __half2float(__half(__nv_cvt_fp8_to_halfraw(v, __NV_E4M3)))) * 16.0f;
-          }
-        } else {
-          const __half hi = __float2half_rn(r);
-          const __half lo = __float2half_rn((r - __half2float(hi)) * kLoScale);
-          *reinterpret_cast<__half*>(sB + sw128_offset(u * S::NQ + h, e, S::B_HALF_BYTES)) = hi;
-          *reinterpret_cast<__half*>(sB + sw128_offset(u * S::NQ + H + h, e, S::B_HALF_BYTES)) = lo;
-        }
-      };
-      if (rope_dims == D && !rope_interleaved) {  // NeoX pairs (i, i + D/2) over all dims
-        for (int e = tid; e < T * H * (D / 2); e += 128) {
-          const int uh = e / (D / 2), i = e % (D / 2);
-          const int u = uh / H, h = uh % H;
-          const __half* x = s_q + uh * D;
-          const float c = s_cos[u * (D / 2) + i], sn = s_sin[u * (D / 2) + i];
-          const float x1 = __half2float(x[i]);
-          const float x2 = __half2float(x[i + D / 2]);
-          put(u, h, i, x1 * c - x2 * sn);
-          put(u, h, i + D / 2, x1 * sn + x2 * c);
-        }
-      } else {  // partial rotary or interleaved pairs: one element at a time
-        for (int e = tid; e < T * H * D; e += 128) {
-          const int uh = e / D, k = e % D;
-          const int u = uh / H, h = uh % H;
-          const __half* x = s_q + uh * D;
-          const RopeSlot sl = rope_slot(k, rope_dims, rope_interleaved != 0);
-          const float xk = __half2float(x[k]);
-          float r = xk;
-          if (sl.freq >= 0)
-            r = xk * s_cos[u * (D / 2) + sl.freq] + sl.sign * __half2float(x[sl.partner]) * s_sin[u * (D / 2) + sl.freq];
-          put(u, h, k, r);
-        }
-      }
-      constexpr int USED = S::TERMS * H;
-      constexpr int PAD = S::NQ - USED;  // zero rows after each query's term rows
-      if constexpr (PAD > 0) {
-        for (int e = tid; e < T * PAD * D; e += 128) {
-          const int u = e / (PAD * D), rem = e % (PAD * D);
-          if constexpr (F8) sB[sw128_offset_b(USED + rem / D, rem % D)] = 0;
-          else
-            *reinterpret_cast<__half*>(sB + sw128_offset(u * S::NQ + USED + rem / D, rem % D, S::B_HALF_BYTES)) =
-                __float2half_rn(0.0f);
-        }
+      // the query's position: q_n > 0 when it belongs to token q_n - 1 of a longer sequence
+      // whose blocks this layer holds a contiguous part of (a context-parallel shard)
+      const int pos = q_n > 0 ? q_n : n;  // uniform
+      if (pos != pos_built) {
+        if (pos_built >= 0) named_bar_sync(2, 128);  // every thread is done with the first build
+        build_b(pos);
+        load_w();
       }
       fence_proxy_async_smem();
       named_bar_sync(1, 160);
+      if (tid == 0) QSA_TL(st, kTlScan2, 2);  // B operand built
 
-      float wr[T][H];
-#pragma unroll
-      for (int u = 0; u < T; ++u)
-#pragma unroll
-        for (int h = 0; h < H; ++h) wr[u][h] = w[u * H + h];
       const float sqrt_d = sqrtf((float)D);
       const float unscale = 1.0f / pre;  // a power of 2: exact
       bool ok = true;
@@ -653,7 +686,7 @@ static cudaError_t launch_scan_tc(const LayerView& L, const void* q_idx, const f
                     ScanShape<D, H, T, F8>::SMEM, s, 1, L.pooled_tile_map, L.pooled_box_map, L.state,
                     (const __half*)q_idx, w, scores, hist, L.cfg.rope_base, L.cfg.max_ctx / kBlock, L.cfg.rope_dims,
                     L.cfg.rope_interleaved, L.cfg.rope_pos_stride, score_stride, app, q_n,
-                    (const float*)L.pooled_scales);
+                    (const float*)L.pooled_scales, L.cfg.early_inputs);
 }
 
 // mode 0: plain scan of T queries; 1: single query with the histogram; 2: decode step

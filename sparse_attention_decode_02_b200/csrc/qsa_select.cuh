@@ -8,9 +8,11 @@
 // Rule of this library: the min(K, B) largest scores, ties to the lower block index,
 // output in ascending block order.
 //
-// An exact radix select on order-preserving 32-bit keys: 8-bit digits from the top (or
-// from the 11-bit bin the scan's histogram points at), stopping as soon as every key with
-// the current prefix is needed. CTA r of the cluster owns blocks
+// An exact radix select on order-preserving 32-bit keys: 8-bit digits from the top,
+// stopping as soon as every key with the current prefix is needed. When the scan's 11-bit
+// histogram gives the bin of the K-th key, the CTAs send the keys at or above that bin to
+// CTA 0, which refines inside the bin on its own (gather_finish); otherwise every CTA takes
+// part in every pass as follows. CTA r of the cluster owns blocks
 // [r*kTopkThreads*V, (r+1)*kTopkThreads*V), thread t the V consecutive blocks starting at
 // t*V, held in registers. Per pass, each CTA histograms its keys in shared memory and
 // pushes the histogram into every CTA's inbox with distributed-shared-memory stores; after
@@ -24,6 +26,7 @@
 #include <cooperative_groups.h>
 
 #include "qsa_device.cuh"
+#include "qsa_sm100.cuh"
 #include "qsa_timeline.cuh"
 
 namespace qsa {
@@ -73,6 +76,46 @@ __device__ __forceinline__ uint32_t cta_exclusive_scan(uint32_t v, uint32_t* s_w
   return s_warp[warp] + x - v;
 }
 
+// ---- distributed shared memory: stores into CTA 0 that count on its mbarrier ----
+// shared::cluster address of `p` (a variable of this CTA's shared memory) in CTA `r`
+__device__ __forceinline__ uint32_t cluster_addr(const void* p, uint32_t r) {
+  uint32_t a;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(sm100::smem_u32(p)), "r"(r));
+  return a;
+}
+// 8 (4) bytes into another CTA's shared memory; completion is counted in bytes on `bar`,
+// an mbarrier in that CTA
+__device__ __forceinline__ void st_async_v2(uint32_t addr, uint32_t a, uint32_t b, uint32_t bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.u32 [%0], {%1, %2}, [%3];"
+               ::"r"(addr), "r"(a), "r"(b), "r"(bar) : "memory");
+}
+__device__ __forceinline__ void st_async_u32(uint32_t addr, uint32_t a, uint32_t bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.u32 [%0], %1, [%2];"
+               ::"r"(addr), "r"(a), "r"(bar) : "memory");
+}
+// one arrival on another CTA's mbarrier, announcing `bytes` of st_async data
+__device__ __forceinline__ void mbar_arrive_expect_tx_remote(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+// wait (bounded, like sm100::mbar_wait) for a phase of this CTA's mbarrier that other
+// CTAs of the cluster complete; their data is visible on return
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity) {
+  const unsigned long long t0 = sm100::globaltimer();
+  for (uint32_t i = 0;; ++i) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(sm100::smem_u32(bar)), "r"(parity)
+        : "memory");
+    if (ok) return true;
+    if ((i & 255u) == 255u && sm100::globaltimer() - t0 > sm100::kWaitLimitNs) return false;
+  }
+}
+
 enum { kStale = 0, kAll = 1, kTopK = 2 };
 
 struct Result {
@@ -83,6 +126,191 @@ struct Result {
   int n_blocks;
 };
 
+// The selection's finish once the histogram has given the bin b1 holding the K-th largest
+// key (prefix = b1's key bits, mask = its 11 bits, need = K minus the keys above b1):
+// every CTA sends its keys at or above b1 with their blocks (in block order) and its count
+// into CTA 0's shared memory with asynchronous remote stores that count on an mbarrier
+// there; CTA 0 waits on that mbarrier alone (no cluster-wide barrier on the way), refines
+// the threshold inside b1 with radix passes on the remaining 21 bits over the gathered
+// keys, and emits the selection: keys above the threshold, then ties by lower block, at
+// positions from one prefix scan in block order. A CTA with more candidates than its
+// region holds (a table of near-ties) sends an overflow mark instead, and CTA 0 then runs
+// the same passes over every block's score read from memory, kThreads * 8 at a time.
+// Every CTA arrives on a final cluster barrier once its data is in place (CTA 0: once it
+// has everything) and waits on it before leaving, so no CTA exits while stores into its
+// shared memory may still arrive.
+template <int V, class ClearHist, class Emit>
+__device__ __forceinline__ Result gather_finish(DevState* st, const float* __restrict__ scores, const uint32_t (&key)[V],
+                                             uint32_t valid, int base, int n, int n_blocks, uint32_t prefix,
+                                             uint32_t mask, uint32_t need, uint64_t* gather_bar, void* region,
+                                             uint32_t* s_hist, uint32_t* s_warp, uint32_t* s_ctl, ClearHist&& clear_hist,
+                                             Emit&& emit) {
+  constexpr uint32_t kCap = 256;               // candidates per source CTA in CTA 0's region
+  constexpr uint32_t kOverflow = 0xffffffffu;
+  constexpr int kP = 8;                        // items per thread held at once
+  constexpr uint32_t kChunk = uint32_t(kThreads) * kP;
+  static_assert(kCS * kCap <= kChunk, "the gathered candidates fit one chunk");
+  __shared__ uint32_t s_cnt[kCS];
+  uint2* s_cand = static_cast<uint2*>(region);  // [kCS][kCap]
+  const int rank = int(cg::this_cluster().block_rank());
+  const int tid = threadIdx.x;
+
+  // this CTA's candidates: keys at or above b1, in block order
+  uint32_t c = 0;
+#pragma unroll
+  for (int j = 0; j < V; ++j) c += ((valid >> j) & 1u) && key[j] >= prefix;
+  uint32_t tot;
+  uint32_t off = cta_exclusive_scan(c, s_warp, &tot);
+  cluster_wait();  // every CTA of the cluster has started: CTA 0's mbarrier is initialised
+  const uint32_t bar0 = cluster_addr(gather_bar, 0);
+  const bool fits = tot <= kCap;  // uniform in the CTA
+  if (fits && c) {
+    const uint32_t dst = cluster_addr(s_cand + size_t(rank) * kCap, 0);
+#pragma unroll
+    for (int j = 0; j < V; ++j)
+      if (((valid >> j) & 1u) && key[j] >= prefix) st_async_v2(dst + 8u * off++, key[j], uint32_t(base + j), bar0);
+  }
+  if (tid == 0) {
+    st_async_u32(cluster_addr(&s_cnt[rank], 0), fits ? tot : kOverflow, bar0);
+    mbar_arrive_expect_tx_remote(bar0, 4u + (fits ? 8u * tot : 0u));
+  }
+  if (rank != 0) {
+    cluster_arrive_release();
+    cluster_wait();
+    clear_hist();
+    return Result{kTopK, n, n_blocks};  // CTA 0 writes the selection
+  }
+
+  // ---------------- CTA 0 ----------------
+  if (!mbar_wait_cluster(gather_bar, 0)) {
+    if (tid == 0) record_status(st, QSA_ERR_TIMEOUT);
+    (void)mbar_wait_cluster(gather_bar, 0);  // stores still in flight land before this CTA leaves
+    cluster_arrive_release();
+    cluster_wait();
+    clear_hist();
+    return Result{kStale, n, 0};
+  }
+  cluster_arrive_release();  // every source's data is here: the sources may leave
+  if (tid == 0) QSA_TL(st, kTlTopk, kTlA);
+  bool over = false;
+  uint32_t n_items = 0;
+#pragma unroll
+  for (int r = 0; r < kCS; ++r) {
+    const uint32_t x = s_cnt[r];
+    over |= x == kOverflow;
+    n_items += x;
+  }
+  int n_chunks = 1;
+  uint32_t per = (n_items + kThreads - 1) / kThreads;
+  if (over) {  // every block from memory
+    n_items = uint32_t(n_blocks);
+    n_chunks = int((n_items + kChunk - 1) / kChunk);
+    per = kP;
+  }
+  uint32_t ik[kP], ib[kP], iv = 0;
+  // items [ch * kChunk + tid * per, + per) into registers: thread order is block order
+  auto load = [&](int ch) {
+    const uint32_t i0 = uint32_t(ch) * kChunk + uint32_t(tid) * per;
+    iv = 0;
+    if (!over) {
+      int r = 0;
+      uint32_t pre = 0;  // items in the regions before r
+#pragma unroll
+      for (int j = 0; j < kP; ++j) {
+        const uint32_t i = i0 + uint32_t(j);
+        ik[j] = 0u;
+        ib[j] = 0u;
+        if (uint32_t(j) < per && i < n_items) {
+          while (pre + s_cnt[r] <= i) pre += s_cnt[r++];
+          const uint2 e = s_cand[size_t(r) * kCap + (i - pre)];
+          ik[j] = e.x;
+          ib[j] = e.y;
+          iv |= 1u << j;
+        }
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < kP; ++j) {
+        const uint32_t i = i0 + uint32_t(j);
+        ik[j] = i < n_items ? score_key(__ldcg(scores + i)) : 0u;
+        ib[j] = i;
+        if (i < n_items) iv |= 1u << j;
+      }
+    }
+  };
+  if (n_chunks == 1) load(0);
+  if (tid == 0) QSA_TL(st, kTlTopk2, 1);  // candidates in registers
+
+  // radix passes inside b1: bits 20..13, 12..5, 4..0
+  for (int shift = 32 - kHistBits - 8;; shift -= 8) {
+    const int bits = shift >= 0 ? 8 : 8 + shift;
+    shift = shift >= 0 ? shift : 0;
+    const uint32_t nb = 1u << bits;
+    if (tid < 256) s_hist[tid] = 0u;
+    __syncthreads();
+    for (int ch = 0; ch < n_chunks; ++ch) {
+      if (n_chunks > 1) load(ch);
+#pragma unroll
+      for (int j = 0; j < kP; ++j)
+        if (((iv >> j) & 1u) && (ik[j] & mask) == prefix) atomicAdd(&s_hist[(ik[j] >> shift) & (nb - 1)], 1u);
+    }
+    __syncthreads();
+    // thread t < nb takes digit nb - 1 - t: an inclusive prefix over t counts keys >= digit
+    const uint32_t v = tid < int(nb) ? s_hist[nb - 1 - tid] : 0u;
+    uint32_t tt;
+    const uint32_t excl = cta_exclusive_scan(v, s_warp, &tt);
+    if (tid < int(nb) && excl < need && excl + v >= need) {
+      s_ctl[0] = nb - 1 - uint32_t(tid);
+      s_ctl[1] = excl;
+      s_ctl[2] = v;
+    }
+    __syncthreads();
+    need -= s_ctl[1];
+    prefix |= s_ctl[0] << shift;
+    mask |= (nb - 1) << shift;
+    const bool done = s_ctl[2] == need || shift == 0;
+    __syncthreads();  // s_ctl and s_hist are rewritten by the next pass
+    if (tid == 0) QSA_TL(st, kTlTopk2, 2);  // a pass done
+    if (done) break;
+  }
+  if (tid == 0) QSA_TL(st, kTlTopk, kTlB);
+
+  // output: keys above the threshold, and the first `need` keys at it in block order
+  uint32_t gt_base = 0, eq_base = 0;
+  for (int ch = 0; ch < n_chunks; ++ch) {
+    if (n_chunks > 1) load(ch);
+    uint32_t c_gt = 0, c_eq = 0;
+#pragma unroll
+    for (int j = 0; j < kP; ++j) {
+      if (!((iv >> j) & 1u)) continue;
+      const uint32_t km = ik[j] & mask;
+      c_gt += km > prefix;
+      c_eq += km == prefix;
+    }
+    uint32_t t2;
+    const uint32_t before = cta_exclusive_scan((c_gt << 16) | c_eq, s_warp, &t2);
+    uint32_t gt_b = gt_base + (before >> 16), eq_b = eq_base + (before & 0xffffu);
+#pragma unroll
+    for (int j = 0; j < kP; ++j) {
+      if (!((iv >> j) & 1u)) continue;
+      const uint32_t km = ik[j] & mask;
+      if (km > prefix) {
+        emit(gt_b + min(need, eq_b), int(ib[j]));
+        ++gt_b;
+      } else if (km == prefix) {
+        if (eq_b < need) emit(gt_b + eq_b, int(ib[j]));
+        ++eq_b;
+      }
+    }
+    gt_base += t2 >> 16;
+    eq_base += t2 & 0xffffu;
+  }
+  if (tid == 0) QSA_TL(st, kTlTopk2, 4);
+  cluster_wait();
+  clear_hist();
+  return Result{kTopK, n, n_blocks};
+}
+
 // Preconditions: every thread of the cluster executed cluster_arrive_relaxed() and then
 // pdl_wait(). Selects among the blocks completed within the first n_ctx - n_back tokens
 // (n_back > 0: a query of an earlier token of a multi-query step). Calls
@@ -92,10 +320,11 @@ struct Result {
 //
 // With `hist` (the 2048-bin histogram of the scores' 11-bit key prefixes that the scan
 // filled for exactly these blocks), the bin holding the K-th largest key comes from the
-// histogram and the radix passes only refine the keys inside that bin (bits 20..13,
-// 12..5, 4..0). Without it, or if its total does not match the block count (a scan whose
-// selection never ran), the passes start from the top byte. The histogram is cleared for
-// the next scan in either case.
+// histogram and gather_finish completes the selection in CTA 0 (gather_bar: its mbarrier,
+// initialised for kCS arrivals before the cluster's first arrive). Without it, or if its
+// total does not match the block count (a scan whose selection never ran), the radix
+// passes below run on every CTA from the top byte. The histogram is cleared for the next
+// scan in either case.
 //
 // Output positions need, for every CTA, how many of its keys lie above the final
 // threshold and at it. Each CTA pushes its whole pass histogram (plus, in the first pass,
@@ -103,13 +332,16 @@ struct Result {
 // other CTA's counts from its own inbox: no exchange of totals is needed.
 template <int V, class Emit>
 __device__ __forceinline__ Result cluster_select(DevState* st, const float* __restrict__ scores, uint32_t* hist,
-                                                 int k_blocks, int max_blocks, int n_back, Emit&& emit) {
+                                                 int k_blocks, int max_blocks, int n_back, uint64_t* gather_bar,
+                                                 Emit&& emit) {
   constexpr int kSlots = 257;                 // 256 digit bins + the first pass's count above
   constexpr int kHB = 1 << kHistBits;         // 2048
   static_assert(kThreads * 4 == kHB, "each thread reads 4 histogram bins");
   static_assert(kThreads / 32 == kCS, "one warp per source CTA when reading the inbox");
   __shared__ uint32_t s_hist[kSlots];          // this CTA's histogram of the pass
-  __shared__ uint32_t s_in[2][kCS][kSlots];    // every CTA's histogram, double-buffered by pass
+  // every CTA's histogram, double-buffered by pass; on the histogram path, CTA 0's
+  // region for every CTA's candidates instead
+  __shared__ __align__(16) uint32_t s_in[2][kCS][kSlots];
   __shared__ uint32_t s_warp[32];
   __shared__ uint32_t s_ctl[4];                // digit, count above the digit, count at the digit
   __shared__ uint32_t s_gt[kCS], s_eq[kCS];    // per CTA: keys above the threshold, keys at it
@@ -210,6 +442,11 @@ __device__ __forceinline__ Result cluster_select(DevState* st, const float* __re
       for (int j = 0; j < V; ++j) g0 += ((valid >> j) & 1u) && (key[j] >> (32 - kHistBits)) > b1;
       if (g0) atomicAdd(&s_gt0, g0);
     }
+  }
+  if (first_shift != 24) {  // uniform: the histogram gave the bin; finish in CTA 0
+    if (tid == 0) QSA_TL(st, kTlTopk2, 0);  // loads and the histogram's bin done
+    return gather_finish<V>(st, scores, key, valid, base, n, n_blocks, prefix, mask, need, gather_bar,
+                            static_cast<void*>(&s_in[0][0][0]), s_hist, s_warp, s_ctl, clear_hist, emit);
   }
   if (tid == 0) QSA_TL(st, kTlTopk2, 0);  // loads and the histogram's bin done
   cluster_wait();  // every CTA of the cluster has started: its shared memory may be written

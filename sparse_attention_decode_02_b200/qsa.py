@@ -23,6 +23,7 @@ STATUS_NAMES = {0: "QSA_OK", 1: "QSA_ERR_INVALID_ARG", 2: "QSA_ERR_CAPACITY", 3:
 QSA_KV_F16, QSA_KV_FP8 = 0, 1
 QSA_SCAN_TENSOR, QSA_SCAN_CUDA_CORES = 0, 1
 QSA_POOLED_F16, QSA_POOLED_FP8 = 0, 1
+QSA_INPUTS_ORDERED, QSA_INPUTS_EARLY = 0, 1
 QSA_MAX_QUERIES = 4
 
 
@@ -38,7 +39,7 @@ class QsaConfig(ctypes.Structure):
                 ("n_kv_heads", c_int32), ("head_dim", c_int32), ("rope_base", c_float),
                 ("rms_eps", c_float), ("rope_dims", c_int32), ("rope_interleaved", c_int32),
                 ("rope_pos_stride", c_int32), ("rope_pos_offset", c_int32), ("kv_format", c_int32),
-                ("scan_kind", c_int32), ("pooled_format", c_int32)]
+                ("scan_kind", c_int32), ("pooled_format", c_int32), ("early_inputs", c_int32)]
 
 
 class QsaLayerBuffers(ctypes.Structure):
@@ -126,10 +127,10 @@ def _stream(stream):
 def make_config(n_layers, max_ctx, d_idx, n_idx_heads, top_k_tokens, n_q_heads, n_kv_heads, head_dim,
                 rope_base=10000.0, rms_eps=1e-6, rope_dims=0, rope_interleaved=False, rope_pos_stride=4,
                 rope_pos_offset=0, kv_format=QSA_KV_F16, scan_kind=QSA_SCAN_TENSOR,
-                pooled_format=QSA_POOLED_F16) -> QsaConfig:
+                pooled_format=QSA_POOLED_F16, early_inputs=QSA_INPUTS_ORDERED) -> QsaConfig:
     return QsaConfig(n_layers, max_ctx, d_idx, n_idx_heads, top_k_tokens, n_q_heads, n_kv_heads, head_dim,
                      rope_base, rms_eps, rope_dims, int(bool(rope_interleaved)), rope_pos_stride, rope_pos_offset,
-                     kv_format, scan_kind, pooled_format)
+                     kv_format, scan_kind, pooled_format, early_inputs)
 
 
 def buffer_bytes(cfg: QsaConfig, which: int) -> int:

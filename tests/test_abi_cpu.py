@@ -111,6 +111,17 @@ def test_scan_kind_is_validated(lib):
     assert Q.buffer_bytes(cfg, Q.QSA_BUF_KV) == 0
 
 
+def test_pooled_format_and_early_inputs_are_validated(lib):
+    cfg = Q.make_config(1, 4096, 128, 16, 2048, 32, 4, 128, pooled_format=Q.QSA_POOLED_FP8,
+                        early_inputs=Q.QSA_INPUTS_EARLY)
+    assert Q.buffer_bytes(cfg, Q.QSA_BUF_POOLED) == 1024 * 128
+    assert Q.buffer_bytes(cfg, Q.QSA_BUF_POOLED_SCALES) == 1024 * 4
+    cfg.early_inputs = 2
+    assert Q.buffer_bytes(cfg, Q.QSA_BUF_POOLED) == 0
+    d64 = Q.make_config(1, 4096, 64, 16, 2048, 32, 4, 128, pooled_format=Q.QSA_POOLED_FP8)
+    assert Q.buffer_bytes(d64, Q.QSA_BUF_POOLED) == 0  # 8-bit pooled keys need d_idx 128
+
+
 def test_null_arguments_are_rejected(lib):
     assert lib.qsa_create(None, None) == 1
     lib.qsa_destroy(None)  # no-op

@@ -182,3 +182,35 @@ def test_decode_step_selection_on_adversarial_tables(wl_name, n0, table):
     H.selection_mismatch(got, ref_scores, wl.k_blocks, gap)
     if table in ("allequal", "zeroquery"):
         assert got.tolist() == list(range(wl.k_blocks))
+
+
+@pytest.mark.parametrize("wl_name,kw", [("tiny", {}), ("tiny", dict(rope_dims=32, rope_pos_stride=1)),
+                                        ("ctx64k", {}), ("ctx64k", dict(pooled_format=1))],
+                         ids=["tiny", "tiny-partial-rope", "ctx64k", "ctx64k-fp8-pooled"])
+def test_early_inputs_give_identical_results(wl_name, kw):
+    """early_inputs = QSA_INPUTS_EARLY (the scan prepares the query before waiting for the
+    previous kernel) against the default, bit for bit: the decode step over block
+    completions, and the separate calls, where the append that precedes the scan changes
+    the length after the scan read it early (the scan then rebuilds the query operand)."""
+    wl = synth.workload(wl_name)
+    n0 = 1017 if wl_name == "tiny" else 8193
+    qa, ga, _ = _layer(wl, n0, extra=24, early_inputs=1, **kw)
+    qb, gb, _ = _layer(wl, n0, extra=24, **kw)
+    ga.update()
+    gb.update()
+    for step in range(12):
+        st = synth.step_inputs(wl, 0, step)
+        if step % 2 == 0:
+            _decode_step(qa, ga, st)
+            _decode_step(qb, gb, st)
+        else:
+            _separate(qa, ga, st)
+            _separate(qb, gb, st)
+        torch.cuda.synchronize()
+        na, nb = int(ga.outs["n_sel"][0]), int(gb.outs["n_sel"][0])
+        assert na == nb
+        assert torch.equal(ga.outs["sel"][:na], gb.outs["sel"][:nb]), f"step {step}: selection"
+        assert torch.equal(ga.outs["out"], gb.outs["out"]), f"step {step}: attention output"
+        if step % 2:
+            assert torch.equal(ga.scores, gb.scores), f"step {step}: scores"
+        assert ga.state() == gb.state() == (n0 + step + 1, (n0 + step + 1) // 4, 0)
