@@ -30,11 +30,6 @@ __device__ __forceinline__ void cluster_arrive_relaxed() {
   asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 }
 __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
-// Arrive with release semantics: this thread's earlier writes are visible to every thread
-// of the cluster that returns from the matching wait.
-__device__ __forceinline__ void cluster_arrive_release() {
-  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-}
 
 // Rotation pair of element e of an indexer key or query whose first R dims are rotary
 // (Part 10, section "QSA indexer": RoPE at the block position). NeoX style pairs

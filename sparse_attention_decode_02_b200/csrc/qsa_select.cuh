@@ -93,9 +93,10 @@ __device__ __forceinline__ void st_async_u32(uint32_t addr, uint32_t a, uint32_t
   asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.u32 [%0], %1, [%2];"
                ::"r"(addr), "r"(a), "r"(bar) : "memory");
 }
-// one arrival on another CTA's mbarrier, announcing `bytes` of st_async data
+// one arrival on another CTA's mbarrier, announcing `bytes` of st_async data (no ordering
+// of its own: the data's arrival is what the bytes count)
 __device__ __forceinline__ void mbar_arrive_expect_tx_remote(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+  asm volatile("mbarrier.arrive.expect_tx.relaxed.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
                : "memory");
 }
 // wait (bounded, like sm100::mbar_wait) for a phase of this CTA's mbarrier that other
@@ -116,6 +117,12 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
   }
 }
 
+__device__ __forceinline__ uint32_t lanemask_lt() {
+  uint32_t m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
 enum { kStale = 0, kAll = 1, kTopK = 2 };
 
 struct Result {
@@ -132,8 +139,10 @@ struct Result {
 // into CTA 0's shared memory with asynchronous remote stores that count on an mbarrier
 // there; CTA 0 waits on that mbarrier alone (no cluster-wide barrier on the way), refines
 // the threshold inside b1 with radix passes on the remaining 21 bits over the gathered
-// keys, and emits the selection: keys above the threshold, then ties by lower block, at
-// positions from one prefix scan in block order. A CTA with more candidates than its
+// keys, and emits the selection: keys above the threshold, then ties by lower block. In
+// CTA 0, warp r holds CTA r's keys (lane l the items l + 32k), so the positions in block
+// order come from warp ballots plus one exchange of per-warp counts; one warp scans each
+// pass's digit counts. A CTA with more candidates than its
 // region holds (a table of near-ties) sends an overflow mark instead, and CTA 0 then runs
 // the same passes over every block's score read from memory, kThreads * 8 at a time.
 // Every CTA arrives on a final cluster barrier once its data is in place (CTA 0: once it
@@ -149,7 +158,7 @@ __device__ __forceinline__ Result gather_finish(DevState* st, const float* __res
   constexpr uint32_t kOverflow = 0xffffffffu;
   constexpr int kP = 8;                        // items per thread held at once
   constexpr uint32_t kChunk = uint32_t(kThreads) * kP;
-  static_assert(kCS * kCap <= kChunk, "the gathered candidates fit one chunk");
+  static_assert(kCap == 32 * kP && kThreads / 32 == kCS, "warp r holds CTA r's region, 8 items per lane");
   __shared__ uint32_t s_cnt[kCS];
   uint2* s_cand = static_cast<uint2*>(region);  // [kCS][kCap]
   const int rank = int(cg::this_cluster().block_rank());
@@ -174,8 +183,10 @@ __device__ __forceinline__ Result gather_finish(DevState* st, const float* __res
     st_async_u32(cluster_addr(&s_cnt[rank], 0), fits ? tot : kOverflow, bar0);
     mbar_arrive_expect_tx_remote(bar0, 4u + (fits ? 8u * tot : 0u));
   }
+  // the final cluster barrier only keeps every CTA alive until CTA 0 holds all the data:
+  // it orders nothing, so its arrive is relaxed
   if (rank != 0) {
-    cluster_arrive_release();
+    cluster_arrive_relaxed();
     cluster_wait();
     clear_hist();
     return Result{kTopK, n, n_blocks};  // CTA 0 writes the selection
@@ -185,127 +196,205 @@ __device__ __forceinline__ Result gather_finish(DevState* st, const float* __res
   if (!mbar_wait_cluster(gather_bar, 0)) {
     if (tid == 0) record_status(st, QSA_ERR_TIMEOUT);
     (void)mbar_wait_cluster(gather_bar, 0);  // stores still in flight land before this CTA leaves
-    cluster_arrive_release();
+    cluster_arrive_relaxed();
     cluster_wait();
     clear_hist();
     return Result{kStale, n, 0};
   }
-  cluster_arrive_release();  // every source's data is here: the sources may leave
+  cluster_arrive_relaxed();  // every source's data is here: the sources may leave
   if (tid == 0) QSA_TL(st, kTlTopk, kTlA);
+#ifdef QSA_TIMELINE
+  const long long cyc0 = clock64();
+#define QSA_CYC(pt) if (tid == 0) QSA_TL_VALUE(st, kTlCycles, pt, uint32_t(clock64() - cyc0))
+#else
+#define QSA_CYC(pt) ((void)0)
+#endif
   bool over = false;
-  uint32_t n_items = 0;
 #pragma unroll
-  for (int r = 0; r < kCS; ++r) {
-    const uint32_t x = s_cnt[r];
-    over |= x == kOverflow;
-    n_items += x;
-  }
-  int n_chunks = 1;
-  uint32_t per = (n_items + kThreads - 1) / kThreads;
-  if (over) {  // every block from memory
-    n_items = uint32_t(n_blocks);
-    n_chunks = int((n_items + kChunk - 1) / kChunk);
-    per = kP;
-  }
-  uint32_t ik[kP], ib[kP], iv = 0;
-  // items [ch * kChunk + tid * per, + per) into registers: thread order is block order
-  auto load = [&](int ch) {
-    const uint32_t i0 = uint32_t(ch) * kChunk + uint32_t(tid) * per;
-    iv = 0;
-    if (!over) {
-      int r = 0;
-      uint32_t pre = 0;  // items in the regions before r
+  for (int r = 0; r < kCS; ++r) over |= s_cnt[r] == kOverflow;
+  if (!over) {
+    // ---- warp r takes CTA r's candidates, lane l its items l + 32k (k < 8), in shared
+    // memory where they landed; the candidates' order (block order) is region, then item:
+    // k, then lane. The passes hold the keys in registers; the output loop stays rolled
+    // and reads shared memory: it runs once per launch, so its instruction fetch costs
+    // more than those loads. ----
+    const int warp = tid >> 5, lane = tid & 31;
+    const uint32_t lt = lanemask_lt();
+    const uint32_t cnt = s_cnt[warp];
+    const uint2* mine = s_cand + size_t(warp) * kCap;
+    uint32_t ik[kP], iv = 0;  // the keys, in registers for the passes
 #pragma unroll
-      for (int j = 0; j < kP; ++j) {
-        const uint32_t i = i0 + uint32_t(j);
-        ik[j] = 0u;
-        ib[j] = 0u;
-        if (uint32_t(j) < per && i < n_items) {
-          while (pre + s_cnt[r] <= i) pre += s_cnt[r++];
-          const uint2 e = s_cand[size_t(r) * kCap + (i - pre)];
-          ik[j] = e.x;
-          ib[j] = e.y;
-          iv |= 1u << j;
+    for (int k = 0; k < kP; ++k) {
+      const uint32_t i = uint32_t(lane + 32 * k);
+      ik[k] = i < cnt ? mine[i].x : 0u;
+      iv |= (i < cnt ? 1u : 0u) << k;
+    }
+    if (tid == 0) QSA_TL(st, kTlTopk2, 1);
+    QSA_CYC(0);
+    // radix passes inside b1 (bits 20..13, 12..5, 4..0); warp 0 scans the digit counts
+    for (int shift = 32 - kHistBits - 8;; shift -= 8) {
+      const int bits = shift >= 0 ? 8 : 8 + shift;
+      shift = shift >= 0 ? shift : 0;
+      const uint32_t nb = 1u << bits;
+      if (tid < 256) s_hist[tid] = 0u;
+      __syncthreads();
+#pragma unroll
+      for (int k = 0; k < kP; ++k)
+        if (((iv >> k) & 1u) && (ik[k] & mask) == prefix) atomicAdd(&s_hist[(ik[k] >> shift) & (nb - 1)], 1u);
+      __syncthreads();
+      if (warp == 0) {  // lane l: digits nb-1-8l .. nb-8-8l (from the top), 8 per lane
+        uint32_t cq[8], sum = 0;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const int d = int(nb) - 1 - (8 * lane + q);
+          cq[q] = d >= 0 ? s_hist[d] : 0u;
+          sum += cq[q];
+        }
+        uint32_t x = sum;  // inclusive scan of the lane sums
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const uint32_t y = __shfl_up_sync(0xffffffffu, x, off);
+          if (lane >= off) x += y;
+        }
+        uint32_t acc = x - sum;  // keys in higher digits than this lane's first
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          if (acc < need && acc + cq[q] >= need) {
+            s_ctl[0] = nb - 1 - uint32_t(8 * lane + q);
+            s_ctl[1] = acc;
+            s_ctl[2] = cq[q];
+          }
+          acc += cq[q];
         }
       }
-    } else {
+      __syncthreads();
+      need -= s_ctl[1];
+      prefix |= s_ctl[0] << shift;
+      mask |= (nb - 1) << shift;
+      // s_ctl is rewritten only after the next pass's two barriers, which every thread
+      // reaches after reading it here
+      if (tid == 0) QSA_TL(st, kTlTopk2, 2);  // a pass done
+      if (shift == 32 - kHistBits - 8) QSA_CYC(1);
+      if (s_ctl[2] == need || shift == 0) break;
+    }
+    if (tid == 0) QSA_TL(st, kTlTopk, kTlB);
+    QSA_CYC(2);
+    // output: keys above the threshold, then the first `need` keys at it in block order
+    uint32_t g_w = 0, e_w = 0;  // this lane's counts, then the warp's (region's)
 #pragma unroll
+    for (int k = 0; k < kP; ++k) {
+      const uint32_t km = ik[k] & mask;
+      g_w += ((iv >> k) & 1u) && km > prefix;
+      e_w += ((iv >> k) & 1u) && km == prefix;
+    }
+    uint32_t ge = (g_w << 16) | e_w;
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) ge += __shfl_xor_sync(0xffffffffu, ge, off);
+    __syncthreads();  // s_warp's previous readers are done
+    if (lane == 0) s_warp[warp] = ge;
+    __syncthreads();
+    uint32_t before = lane < warp ? s_warp[lane] : 0u;  // regions before this one
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) before += __shfl_xor_sync(0xffffffffu, before, off);
+    uint32_t gt_b = before >> 16, eq_b = before & 0xffffu;
+#pragma unroll 1
+    for (uint32_t i0 = 0; i0 < cnt; i0 += 32) {
+      const uint32_t i = i0 + uint32_t(lane);
+      const uint2 e = i < cnt ? mine[i] : make_uint2(0u, 0u);
+      const uint32_t km = e.x & mask;
+      const bool gt = i < cnt && km > prefix, eq = i < cnt && km == prefix;
+      const uint32_t bg = __ballot_sync(0xffffffffu, gt), be = __ballot_sync(0xffffffffu, eq);
+      const uint32_t g = gt_b + __popc(bg & lt), q = eq_b + __popc(be & lt);
+      if (gt) emit(g + min(need, q), int(e.y));
+      else if (eq && q < need) emit(g + q, int(e.y));
+      gt_b += __popc(bg);
+      eq_b += __popc(be);
+    }
+  } else {
+    // ---- a CTA overflowed its region: every block's score from memory, kChunk at a time ----
+    const uint32_t n_items = uint32_t(n_blocks);
+    const int n_chunks = int((n_items + kChunk - 1) / kChunk);
+    uint32_t ik[kP], ib[kP], iv = 0;
+    // blocks [ch * kChunk + tid * kP, + kP) into registers: thread order is block order
+    auto load = [&](int ch) {
+      const uint32_t i0 = uint32_t(ch) * kChunk + uint32_t(tid) * kP;
+      iv = 0;
+  #pragma unroll
       for (int j = 0; j < kP; ++j) {
         const uint32_t i = i0 + uint32_t(j);
         ik[j] = i < n_items ? score_key(__ldcg(scores + i)) : 0u;
         ib[j] = i;
         if (i < n_items) iv |= 1u << j;
       }
-    }
-  };
-  if (n_chunks == 1) load(0);
-  if (tid == 0) QSA_TL(st, kTlTopk2, 1);  // candidates in registers
+    };
+    if (n_chunks == 1) load(0);
 
-  // radix passes inside b1: bits 20..13, 12..5, 4..0
-  for (int shift = 32 - kHistBits - 8;; shift -= 8) {
-    const int bits = shift >= 0 ? 8 : 8 + shift;
-    shift = shift >= 0 ? shift : 0;
-    const uint32_t nb = 1u << bits;
-    if (tid < 256) s_hist[tid] = 0u;
-    __syncthreads();
+    // radix passes inside b1: bits 20..13, 12..5, 4..0
+    for (int shift = 32 - kHistBits - 8;; shift -= 8) {
+      const int bits = shift >= 0 ? 8 : 8 + shift;
+      shift = shift >= 0 ? shift : 0;
+      const uint32_t nb = 1u << bits;
+      if (tid < 256) s_hist[tid] = 0u;
+      __syncthreads();
+      for (int ch = 0; ch < n_chunks; ++ch) {
+        if (n_chunks > 1) load(ch);
+  #pragma unroll
+        for (int j = 0; j < kP; ++j)
+          if (((iv >> j) & 1u) && (ik[j] & mask) == prefix) atomicAdd(&s_hist[(ik[j] >> shift) & (nb - 1)], 1u);
+      }
+      __syncthreads();
+      // thread t < nb takes digit nb - 1 - t: an inclusive prefix over t counts keys >= digit
+      const uint32_t v = tid < int(nb) ? s_hist[nb - 1 - tid] : 0u;
+      uint32_t tt;
+      const uint32_t excl = cta_exclusive_scan(v, s_warp, &tt);
+      if (tid < int(nb) && excl < need && excl + v >= need) {
+        s_ctl[0] = nb - 1 - uint32_t(tid);
+        s_ctl[1] = excl;
+        s_ctl[2] = v;
+      }
+      __syncthreads();
+      need -= s_ctl[1];
+      prefix |= s_ctl[0] << shift;
+      mask |= (nb - 1) << shift;
+      const bool done = s_ctl[2] == need || shift == 0;
+      __syncthreads();  // s_ctl and s_hist are rewritten by the next pass
+      if (done) break;
+    }
+
+    // output: keys above the threshold, and the first `need` keys at it in block order
+    uint32_t gt_base = 0, eq_base = 0;
     for (int ch = 0; ch < n_chunks; ++ch) {
       if (n_chunks > 1) load(ch);
-#pragma unroll
-      for (int j = 0; j < kP; ++j)
-        if (((iv >> j) & 1u) && (ik[j] & mask) == prefix) atomicAdd(&s_hist[(ik[j] >> shift) & (nb - 1)], 1u);
-    }
-    __syncthreads();
-    // thread t < nb takes digit nb - 1 - t: an inclusive prefix over t counts keys >= digit
-    const uint32_t v = tid < int(nb) ? s_hist[nb - 1 - tid] : 0u;
-    uint32_t tt;
-    const uint32_t excl = cta_exclusive_scan(v, s_warp, &tt);
-    if (tid < int(nb) && excl < need && excl + v >= need) {
-      s_ctl[0] = nb - 1 - uint32_t(tid);
-      s_ctl[1] = excl;
-      s_ctl[2] = v;
-    }
-    __syncthreads();
-    need -= s_ctl[1];
-    prefix |= s_ctl[0] << shift;
-    mask |= (nb - 1) << shift;
-    const bool done = s_ctl[2] == need || shift == 0;
-    __syncthreads();  // s_ctl and s_hist are rewritten by the next pass
-    if (tid == 0) QSA_TL(st, kTlTopk2, 2);  // a pass done
-    if (done) break;
-  }
-  if (tid == 0) QSA_TL(st, kTlTopk, kTlB);
-
-  // output: keys above the threshold, and the first `need` keys at it in block order
-  uint32_t gt_base = 0, eq_base = 0;
-  for (int ch = 0; ch < n_chunks; ++ch) {
-    if (n_chunks > 1) load(ch);
-    uint32_t c_gt = 0, c_eq = 0;
-#pragma unroll
-    for (int j = 0; j < kP; ++j) {
-      if (!((iv >> j) & 1u)) continue;
-      const uint32_t km = ik[j] & mask;
-      c_gt += km > prefix;
-      c_eq += km == prefix;
-    }
-    uint32_t t2;
-    const uint32_t before = cta_exclusive_scan((c_gt << 16) | c_eq, s_warp, &t2);
-    uint32_t gt_b = gt_base + (before >> 16), eq_b = eq_base + (before & 0xffffu);
-#pragma unroll
-    for (int j = 0; j < kP; ++j) {
-      if (!((iv >> j) & 1u)) continue;
-      const uint32_t km = ik[j] & mask;
-      if (km > prefix) {
-        emit(gt_b + min(need, eq_b), int(ib[j]));
-        ++gt_b;
-      } else if (km == prefix) {
-        if (eq_b < need) emit(gt_b + eq_b, int(ib[j]));
-        ++eq_b;
+      uint32_t c_gt = 0, c_eq = 0;
+  #pragma unroll
+      for (int j = 0; j < kP; ++j) {
+        if (!((iv >> j) & 1u)) continue;
+        const uint32_t km = ik[j] & mask;
+        c_gt += km > prefix;
+        c_eq += km == prefix;
       }
+      uint32_t t2;
+      const uint32_t before = cta_exclusive_scan((c_gt << 16) | c_eq, s_warp, &t2);
+      uint32_t gt_b = gt_base + (before >> 16), eq_b = eq_base + (before & 0xffffu);
+  #pragma unroll
+      for (int j = 0; j < kP; ++j) {
+        if (!((iv >> j) & 1u)) continue;
+        const uint32_t km = ik[j] & mask;
+        if (km > prefix) {
+          emit(gt_b + min(need, eq_b), int(ib[j]));
+          ++gt_b;
+        } else if (km == prefix) {
+          if (eq_b < need) emit(gt_b + eq_b, int(ib[j]));
+          ++eq_b;
+        }
+      }
+      gt_base += t2 >> 16;
+      eq_base += t2 & 0xffffu;
     }
-    gt_base += t2 >> 16;
-    eq_base += t2 & 0xffffu;
   }
+  QSA_CYC(3);
   if (tid == 0) QSA_TL(st, kTlTopk2, 4);
+#undef QSA_CYC
   cluster_wait();
   clear_hist();
   return Result{kTopK, n, n_blocks};
