@@ -123,6 +123,32 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
   return m;
 }
 
+// The same prefix sum with one barrier: warp scans, warp totals through s_warp, and each
+// warp adds the totals of the warps before it with shuffles. The caller keeps s_warp
+// unwritten until every thread has returned (a barrier lies between two calls).
+__device__ __forceinline__ uint32_t cta_exclusive_scan_1(uint32_t v, uint32_t* s_warp, uint32_t* total) {
+  constexpr int W = kThreads / 32;
+  static_assert(W <= 32, "one warp total per lane");
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t x = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, x, off);
+    if (lane >= off) x += y;
+  }
+  if (lane == 31) s_warp[warp] = x;
+  __syncthreads();
+  const uint32_t w = lane < W ? s_warp[lane] : 0u;
+  uint32_t before = lane < warp ? w : 0u, all = w;
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) {
+    before += __shfl_xor_sync(0xffffffffu, before, off);
+    all += __shfl_xor_sync(0xffffffffu, all, off);
+  }
+  *total = all;
+  return before + x - v;
+}
+
 enum { kStale = 0, kAll = 1, kTopK = 2 };
 
 struct Result {
@@ -169,7 +195,7 @@ __device__ __forceinline__ Result gather_finish(DevState* st, const float* __res
 #pragma unroll
   for (int j = 0; j < V; ++j) c += ((valid >> j) & 1u) && key[j] >= prefix;
   uint32_t tot;
-  uint32_t off = cta_exclusive_scan(c, s_warp, &tot);
+  uint32_t off = cta_exclusive_scan_1(c, s_warp, &tot);  // a barrier since the last s_warp use
   cluster_wait();  // every CTA of the cluster has started: CTA 0's mbarrier is initialised
   const uint32_t bar0 = cluster_addr(gather_bar, 0);
   const bool fits = tot <= kCap;  // uniform in the CTA
@@ -416,17 +442,17 @@ __device__ __forceinline__ Result gather_finish(DevState* st, const float* __res
 // scan in either case.
 //
 // Output positions need, for every CTA, how many of its keys lie above the final
-// threshold and at it. Each CTA pushes its whole pass histogram (plus, in the first pass,
-// its count of keys above the starting bin) to every CTA, so each CTA derives every
-// other CTA's counts from its own inbox: no exchange of totals is needed.
+// threshold and at it. Each CTA pushes its whole pass histogram to every CTA, so each CTA
+// derives every other CTA's counts from its own inbox: no exchange of totals is needed.
 template <int V, class Emit>
 __device__ __forceinline__ Result cluster_select(DevState* st, const float* __restrict__ scores, uint32_t* hist,
                                                  int k_blocks, int max_blocks, int n_back, uint64_t* gather_bar,
                                                  Emit&& emit) {
-  constexpr int kSlots = 257;                 // 256 digit bins + the first pass's count above
+  constexpr int kSlots = 256;                 // digit bins of a pass
   constexpr int kHB = 1 << kHistBits;         // 2048
   static_assert(kThreads * 4 == kHB, "each thread reads 4 histogram bins");
   static_assert(kThreads / 32 == kCS, "one warp per source CTA when reading the inbox");
+  static_assert(2 * kCS * kSlots * 4 >= kCS * 256 * 8, "the inbox holds CTA 0's candidate regions");
   __shared__ uint32_t s_hist[kSlots];          // this CTA's histogram of the pass
   // every CTA's histogram, double-buffered by pass; on the histogram path, CTA 0's
   // region for every CTA's candidates instead
@@ -434,7 +460,6 @@ __device__ __forceinline__ Result cluster_select(DevState* st, const float* __re
   __shared__ uint32_t s_warp[32];
   __shared__ uint32_t s_ctl[4];                // digit, count above the digit, count at the digit
   __shared__ uint32_t s_gt[kCS], s_eq[kCS];    // per CTA: keys above the threshold, keys at it
-  __shared__ uint32_t s_gt0;                   // this CTA's keys above the histogram's bin
 
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = int(cluster.block_rank());
@@ -498,7 +523,6 @@ __device__ __forceinline__ Result cluster_select(DevState* st, const float* __re
   }
   if (tid < kSlots) s_hist[tid] = 0;
   if (tid < kCS) s_gt[tid] = 0;
-  if (tid == 0) s_gt0 = 0;
 
   // the starting prefix: the histogram's bin holding the K-th largest key, if the
   // histogram counts exactly these blocks
@@ -507,7 +531,8 @@ __device__ __forceinline__ Result cluster_select(DevState* st, const float* __re
   if (hist) {
     const uint32_t c4 = h4.x + h4.y + h4.z + h4.w;
     uint32_t total;
-    const uint32_t above = cta_exclusive_scan(c4, s_warp, &total);  // keys in higher bins
+    __syncthreads();  // s_warp's previous readers are done
+    const uint32_t above = cta_exclusive_scan_1(c4, s_warp, &total);  // keys in higher bins
     if (total == uint32_t(n_blocks)) {  // uniform: every thread sees the same total
       // bins of this thread from the top: 2047-4t (h4.w), then h4.z, h4.y, h4.x
       const uint32_t hb[4] = {h4.w, h4.z, h4.y, h4.x};
@@ -526,10 +551,6 @@ __device__ __forceinline__ Result cluster_select(DevState* st, const float* __re
       prefix = b1 << (32 - kHistBits);
       mask = ~0u << (32 - kHistBits);
       first_shift = 32 - kHistBits - 8;  // 13
-      uint32_t g0 = 0;
-#pragma unroll
-      for (int j = 0; j < V; ++j) g0 += ((valid >> j) & 1u) && (key[j] >> (32 - kHistBits)) > b1;
-      if (g0) atomicAdd(&s_gt0, g0);
     }
   }
   if (first_shift != 24) {  // uniform: the histogram gave the bin; finish in CTA 0
@@ -546,11 +567,10 @@ __device__ __forceinline__ Result cluster_select(DevState* st, const float* __re
     const int bits = shift >= 0 ? 8 : 8 + shift;
     shift = shift >= 0 ? shift : 0;
     const uint32_t nb = 1u << bits;
-    __syncthreads();  // the local histogram is zeroed, s_gt0 complete
+    __syncthreads();  // the local histogram is zeroed
 #pragma unroll
     for (int j = 0; j < V; ++j)
       if (((valid >> j) & 1u) && (key[j] & mask) == prefix) atomicAdd(&s_hist[(key[j] >> shift) & (nb - 1)], 1u);
-    if (pass == 0 && tid == 0) s_hist[256] = s_gt0;
     __syncthreads();
     // push slot t into [rank][t] of every CTA's inbox for this pass, and clear it for the
     // next pass. A CTA reuses an inbox buffer two passes later, after a barrier that every
@@ -594,8 +614,8 @@ __device__ __forceinline__ Result cluster_select(DevState* st, const float* __re
     }
     __syncthreads();
     const uint32_t d = s_ctl[0];
-    // per source CTA (warp r reads CTA r's row): its keys above the digit in this pass
-    // (plus its count above the histogram's bin), and at the digit
+    // per source CTA (warp r reads CTA r's row): its keys above the digit in this pass,
+    // and at the digit
     {
       const int r = warp;
       uint32_t a = 0;
@@ -603,7 +623,7 @@ __device__ __forceinline__ Result cluster_select(DevState* st, const float* __re
 #pragma unroll
       for (int off = 16; off >= 1; off >>= 1) a += __shfl_xor_sync(0xffffffffu, a, off);
       if (lane == 0) {
-        s_gt[r] += a + (pass == 0 ? in[r][256] : 0u);
+        s_gt[r] += a;
         s_eq[r] = in[r][d];
       }
     }
