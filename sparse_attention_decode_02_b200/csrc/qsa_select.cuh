@@ -13,8 +13,9 @@
 // histogram gives the bin of the K-th key, the CTAs send the keys at or above that bin to
 // CTA 0, which refines inside the bin on its own (gather_finish); otherwise every CTA takes
 // part in every pass as follows. CTA r of the cluster owns blocks
-// [r*kTopkThreads*V, (r+1)*kTopkThreads*V), thread t the V consecutive blocks starting at
-// t*V, held in registers. Per pass, each CTA histograms its keys in shared memory and
+// [r*kTopkThreads*P, (r+1)*kTopkThreads*P), thread t the P consecutive blocks starting at
+// t*P, held in registers (P <= V: the smallest power of two that spreads the layer's
+// capacity over the whole cluster). Per pass, each CTA histograms its keys in shared memory and
 // pushes the histogram into every CTA's inbox with distributed-shared-memory stores; after
 // one cluster barrier each CTA adds the histograms from its own memory. The output
 // position of a selected block is the number of keys above the threshold before it plus
@@ -465,15 +466,20 @@ __device__ __forceinline__ Result cluster_select(DevState* st, const float* __re
   const int rank = int(cluster.block_rank());
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
-  // this thread's V scores, read up to the buffer's capacity (max_ctx/4) in the same round
-  // trip as the state and the histogram; blocks at or past n_ctx/4 are masked once the
-  // state is known. Thread t reads bins [2044 - 4t, 2048 - 4t): thread 0 the top ones.
-  const int base = rank * kThreads * V + tid * V;
+  // this thread's P <= V scores (P: the smallest power of two that covers the buffer's
+  // capacity max_ctx/4 with every CTA of the cluster, so a shorter context still spreads
+  // over all of them), read in the same round trip as the state and the histogram; blocks
+  // at or past n_ctx/4 are masked once the state is known. Thread t reads histogram bins
+  // [2044 - 4t, 2048 - 4t): thread 0 the top ones.
+  int P = 1;
+  while (P < V && kCS * kThreads * P < max_blocks) P <<= 1;
+  const int base = (rank * kThreads + tid) * P;
   float f[V];
-  if (base + V <= max_blocks) {
+  if (P >= 4 && base + P <= max_blocks) {  // whole 16-byte vectors (base is a multiple of 4)
 #pragma unroll
     for (int j = 0; j < V; j += 4) {
-      const float4 x = *reinterpret_cast<const float4*>(scores + base + j);
+      float4 x = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      if (j < P) x = *reinterpret_cast<const float4*>(scores + base + j);
       f[j] = x.x;
       f[j + 1] = x.y;
       f[j + 2] = x.z;
@@ -481,7 +487,7 @@ __device__ __forceinline__ Result cluster_select(DevState* st, const float* __re
     }
   } else {
 #pragma unroll
-    for (int j = 0; j < V; ++j) f[j] = base + j < max_blocks ? scores[base + j] : 0.0f;
+    for (int j = 0; j < V; ++j) f[j] = j < P && base + j < max_blocks ? scores[base + j] : 0.0f;
   }
   uint4 h4 = make_uint4(0u, 0u, 0u, 0u);
   if (hist) h4 = *reinterpret_cast<const uint4*>(hist + (kHB - 4 - 4 * tid));
@@ -519,7 +525,7 @@ __device__ __forceinline__ Result cluster_select(DevState* st, const float* __re
 #pragma unroll
   for (int j = 0; j < V; ++j) {
     key[j] = score_key(f[j]);
-    if (base + j < n_blocks) valid |= 1u << j;
+    if (j < P && base + j < n_blocks) valid |= 1u << j;
   }
   if (tid < kSlots) s_hist[tid] = 0;
   if (tid < kCS) s_gt[tid] = 0;
