@@ -651,31 +651,34 @@ attn_cluster_kernel(DevState* st, const __half* __restrict__ q, const int32_t* _
   if (tid == 0) QSA_TL(st, kTlAttn2, 4);  // pushed
   cluster.sync();  // release the pushes above, acquire every other CTA's
   if (tid == 0) QSA_TL(st, kTlAttn, kTlB);
-  for (int t = tid; t < PER; t += kAcThreads) {
+  // CS lanes per output pair, lane r merging source CTA r's partial; shuffles within the
+  // aligned CS-lane group combine them (max, then the weighted sums)
+  static_assert(PAIRS % CS == 0 && (PER * CS) % 32 == 0 && 32 % CS == 0, "whole warps, aligned lane groups");
+  for (int i = tid; i < PER * CS; i += kAcThreads) {
+    const int t = i / CS, r = i % CS;
     const int pidx = rank * PER + t;
-    if (pidx >= PAIRS) break;
     const int h = pidx / (D / 2), d2 = pidx % (D / 2);
-    float M = -INFINITY;
+    const float mr = s_stage[(r * G + h) * 2];
+    float M = mr;
 #pragma unroll
-    for (int r = 0; r < CS; ++r) M = fmaxf(M, s_stage[(r * G + h) * 2]);
-    float a0 = 0.0f, a1 = 0.0f, den = 0.0f;
-    if (M != -INFINITY) {
+    for (int off = CS / 2; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    const float e = (M == -INFINITY || mr == -INFINITY) ? 0.0f : expf(mr - M);
+    const float2 o = s_in[r * PER + t];
+    float a0 = e * o.x, a1 = e * o.y, den = e * s_stage[(r * G + h) * 2 + 1];
 #pragma unroll
-      for (int r = 0; r < CS; ++r) {
-        const float mr = s_stage[(r * G + h) * 2];
-        const float e = mr == -INFINITY ? 0.0f : expf(mr - M);
-        const float2 o = s_in[r * PER + t];
-        a0 = fmaf(e, o.x, a0);
-        a1 = fmaf(e, o.y, a1);
-        den = fmaf(e, s_stage[(r * G + h) * 2 + 1], den);
-      }
+    for (int off = CS / 2; off >= 1; off >>= 1) {
+      a0 += __shfl_xor_sync(0xffffffffu, a0, off);
+      a1 += __shfl_xor_sync(0xffffffffu, a1, off);
+      den += __shfl_xor_sync(0xffffffffu, den, off);
     }
-    float2 res = make_float2(0.0f, 0.0f);
-    if (den > 0.0f) res = make_float2(a0 / den, a1 / den);
-    *reinterpret_cast<float2*>(out + (size_t(g) * G + h) * D + 2 * d2) = res;
-    // log-sum-exp of the head's scaled logits over all its cells (a context-parallel
-    // shard's partial): max + log(sum of exp(logit - max)); -inf with no cells
-    if (lse_out && d2 == 0) lse_out[size_t(g) * G + h] = den > 0.0f ? M + logf(den) : -INFINITY;
+    if (r == 0) {
+      float2 res = make_float2(0.0f, 0.0f);
+      if (den > 0.0f) res = make_float2(a0 / den, a1 / den);
+      *reinterpret_cast<float2*>(out + (size_t(g) * G + h) * D + 2 * d2) = res;
+      // log-sum-exp of the head's scaled logits over all its cells (a context-parallel
+      // shard's partial): max + log(sum of exp(logit - max)); -inf with no cells
+      if (lse_out && d2 == 0) lse_out[size_t(g) * G + h] = den > 0.0f ? M + logf(den) : -INFINITY;
+    }
   }
   if (tid == 0) QSA_TL(st, kTlAttn, kTlExit);
 }
