@@ -459,9 +459,11 @@ qsa_status qsa_decode_step(qsa_ctx* ctx, int32_t layer, const void* k, const voi
   const LayerView lv = ctx->view(layer);
   const cudaStream_t s = (cudaStream_t)stream;
   Layer& l = ctx->layers[layer];
-  if (l.pending_blocks == 0 && ctx->cfg.scan_kind == QSA_SCAN_TENSOR) {
+  const bool fused = l.pending_blocks == 0 && ctx->cfg.scan_kind == QSA_SCAN_TENSOR;
+  if (fused) {
     // the pooled cache is current up to the previous token: the scan kernel itself
-    // appends the token and pools the block it completes (three launches per step)
+    // appends the token and pools the block it completes (three launches per step); the
+    // selection then advances the state past the token
     if (qsa_status st = ctx->cuda(launch_decode_scan(lv, k, v, idx_key, q_idx, w, lv.scores, lv.hist, s),
                                   "decode_step: append + index scan"))
       return st;
@@ -474,7 +476,7 @@ qsa_status qsa_decode_step(qsa_ctx* ctx, int32_t layer, const void* k, const voi
                                   "decode_step: index scan"))
       return st;
   }
-  if (qsa_status st = ctx->cuda(launch_topk(lv, lv.scores, sel_blocks, n_sel, s, 1, 0, lv.hist),
+  if (qsa_status st = ctx->cuda(launch_topk(lv, lv.scores, sel_blocks, n_sel, s, 1, 0, lv.hist, nullptr, 0, fused),
                                 "decode_step: block top-k"))
     return st;
   return ctx->cuda(launch_attend_selected(lv, q, sel_blocks, n_sel, out, s), "decode_step: sparse attend");

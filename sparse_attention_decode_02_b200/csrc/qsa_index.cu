@@ -25,7 +25,7 @@ template <int V>
 __global__ void __launch_bounds__(sel::kThreads, 1)
 block_topk_kernel(DevState* st, const float* __restrict__ scores, int32_t* __restrict__ sel_out,
                   int32_t* __restrict__ n_sel, int k_blocks, int max_blocks, int score_stride, uint32_t* hist,
-                  float* __restrict__ sel_scores, int block_base) {
+                  float* __restrict__ sel_scores, int block_base, int fused_max_ctx) {
   const int rank = int(cooperative_groups::this_cluster().block_rank());
   const int u = blockIdx.y, n_back = gridDim.y - 1 - blockIdx.y;
   scores += size_t(u) * score_stride;
@@ -42,7 +42,7 @@ block_topk_kernel(DevState* st, const float* __restrict__ scores, int32_t* __res
   pdl_wait();
   if (threadIdx.x == 0) QSA_TL(st, kTlTopk, kTlWait);
   const sel::Result res = sel::cluster_select<V>(st, scores, gridDim.y == 1 ? hist : nullptr, k_blocks, max_blocks,
-                                                 n_back, &s_gather_bar,
+                                                 n_back, &s_gather_bar, gridDim.y == 1 ? fused_max_ctx : 0,
                                                  [&](uint32_t pos, int block) {
                                                    // bounds-checked in every build
                                                    if (pos < uint32_t(k_blocks) && block < max_blocks) {
@@ -101,19 +101,21 @@ cudaError_t init_kernel_attributes() {
 }
 
 cudaError_t launch_topk(const LayerView& L, const float* scores, int32_t* sel_out, int32_t* n_sel, cudaStream_t s,
-                        int n_queries, int score_stride, uint32_t* hist, float* sel_scores, int block_base) {
-  if (n_queries != 1) hist = nullptr, sel_scores = nullptr, block_base = 0;
+                        int n_queries, int score_stride, uint32_t* hist, float* sel_scores, int block_base,
+                        bool after_fused_scan) {
+  if (n_queries != 1) hist = nullptr, sel_scores = nullptr, block_base = 0, after_fused_scan = false;
   const int max_blocks = L.cfg.max_ctx / kBlock;
   const int kb = L.cfg.top_k_tokens / kBlock;
+  const int fused_max_ctx = after_fused_scan ? L.cfg.max_ctx : 0;
   const dim3 grid(sel::kCS, n_queries), block(sel::kThreads);
   if (max_blocks <= sel::kCS * sel::kThreads * 8)
     return launch_pdl(block_topk_kernel<8>, grid, block, 0, s, sel::kCS, L.state, scores, sel_out, n_sel, kb,
-                      max_blocks, score_stride, hist, sel_scores, block_base);
+                      max_blocks, score_stride, hist, sel_scores, block_base, fused_max_ctx);
   if (max_blocks <= sel::kCS * sel::kThreads * 16)
     return launch_pdl(block_topk_kernel<16>, grid, block, 0, s, sel::kCS, L.state, scores, sel_out, n_sel, kb,
-                      max_blocks, score_stride, hist, sel_scores, block_base);
+                      max_blocks, score_stride, hist, sel_scores, block_base, fused_max_ctx);
   return launch_pdl(block_topk_kernel<32>, grid, block, 0, s, sel::kCS, L.state, scores, sel_out, n_sel, kb,
-                    max_blocks, score_stride, hist, sel_scores, block_base);
+                    max_blocks, score_stride, hist, sel_scores, block_base, fused_max_ctx);
 }
 
 }  // namespace qsa

@@ -137,10 +137,12 @@ cudaError_t launch_index_scan(const LayerView& L, const void* q_idx, const float
                               uint32_t* hist = nullptr, int q_n = 0);
 // With sel_scores (single query), the selection also writes each selected block's score,
 // adds block_base to the written ids and pads positions past n_sel with -inf / -1 (the
-// fixed-size candidate slots of a context-parallel shard).
+// fixed-size candidate slots of a context-parallel shard). after_fused_scan: the scan
+// before it was the decode step's (launch_decode_scan), which appended the token without
+// advancing the state; the selection counts that token and advances the state.
 cudaError_t launch_topk(const LayerView& L, const float* scores, int32_t* sel, int32_t* n_sel,
                         cudaStream_t s, int n_queries = 1, int score_stride = 0, uint32_t* hist = nullptr,
-                        float* sel_scores = nullptr, int block_base = 0);
+                        float* sel_scores = nullptr, int block_base = 0, bool after_fused_scan = false);
 // The same scan on the CUDA cores (scan_kind = QSA_SCAN_CUDA_CORES; single query).
 cudaError_t init_scan_cc_attributes();
 cudaError_t launch_index_scan_cc(const LayerView& L, const void* q_idx, const float* w, float* scores,

@@ -30,8 +30,9 @@
 //    "incremental pooled-key cache（COMMON-004）": only the new block is computed) before
 //    scoring it, so a decode step needs no separate append launch. A seventh warp of the
 //    CTA that owns the last rows does both; the new pooled row reaches the TMA loads
-//    through a proxy fence and an mbarrier. The CTAs publish the new length with a
-//    last-CTA ticket.
+//    through a proxy fence and an mbarrier. The state is left for the selection kernel
+//    that follows to advance (it counts the appended token), so the CTAs leave without a
+//    ticket round trip.
 #include <cuda.h>
 #include <cuda_fp16.h>
 
@@ -590,17 +591,6 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_
     tmem_dealloc(tmem_base, S::TMEM_COLS);
   }
   if (threadIdx.x == 0) QSA_TL(st, kTlScan, kTlExit);
-  if (FUSED && state_ok && threadIdx.x == 0) {
-    // the last CTA to finish publishes the new length: every CTA took its ticket after
-    // using the old one (no fence: the next kernel sees these writes once this grid
-    // completes)
-    const unsigned t = atomicAdd(&st->ticket_append, 1u);
-    if (t == gridDim.x - 1) {
-      st->n_ctx = n;
-      st->n_pooled = n / kBlock;
-      st->ticket_append = 0;
-    }
-  }
 }
 
 // ---------------------------------------------------------------------------------

@@ -448,7 +448,7 @@ __device__ __forceinline__ Result gather_finish(DevState* st, const float* __res
 template <int V, class Emit>
 __device__ __forceinline__ Result cluster_select(DevState* st, const float* __restrict__ scores, uint32_t* hist,
                                                  int k_blocks, int max_blocks, int n_back, uint64_t* gather_bar,
-                                                 Emit&& emit) {
+                                                 int fused_max_ctx, Emit&& emit) {
   constexpr int kSlots = 256;                 // digit bins of a pass
   constexpr int kHB = 1 << kHistBits;         // 2048
   static_assert(kThreads * 4 == kHB, "each thread reads 4 histogram bins");
@@ -491,18 +491,31 @@ __device__ __forceinline__ Result cluster_select(DevState* st, const float* __re
   }
   uint4 h4 = make_uint4(0u, 0u, 0u, 0u);
   if (hist) h4 = *reinterpret_cast<const uint4*>(hist + (kHB - 4 - 4 * tid));
-  const int n_full = ld_volatile(&st->n_ctx);
+  const int n_state = ld_volatile(&st->n_ctx);
   const int n_pooled = ld_volatile(&st->n_pooled);
 #pragma unroll
   for (int j = 0; j < V; ++j) asm volatile("" ::"f"(f[j]));  // keep the loads ahead of the branches
   asm volatile("" ::"r"(h4.x), "r"(h4.y), "r"(h4.z), "r"(h4.w));
+  // fused_max_ctx > 0: the decode step's scan appended token n_state (under the same
+  // conditions as here) and scored with it, leaving the state for this kernel to advance
+  const bool appended = fused_max_ctx > 0 && n_state >= 0 && n_state < fused_max_ctx &&
+                        n_pooled == n_state / kBlock;
+  const int n_full = appended ? n_state + 1 : n_state;
   const int n = n_full - n_back;
   const int n_blocks = n / kBlock;
   // clears this CTA's slice of the histogram once every CTA of the cluster has read it
   auto clear_hist = [&]() {
     if (hist && tid < kHB / kCS) hist[rank * (kHB / kCS) + tid] = 0u;
   };
-  if (n_pooled != n_full / kBlock || n < 0) {  // uniform over the cluster
+  // advances the state past the appended token, once every CTA has read it (each caller
+  // is past a point that every CTA of the cluster reaches only after its state read)
+  auto publish = [&]() {
+    if (appended && rank == 0 && tid == 0) {
+      st->n_ctx = n_full;
+      st->n_pooled = n_full / kBlock;
+    }
+  };
+  if (n_pooled != n_state / kBlock || n < 0 || (fused_max_ctx > 0 && !appended)) {  // uniform over the cluster
     if (rank == 0 && tid == 0) record_status(st, QSA_ERR_STATE);
     cluster_wait();
     if (hist) {
@@ -513,9 +526,10 @@ __device__ __forceinline__ Result cluster_select(DevState* st, const float* __re
   }
   if (n_blocks <= k_blocks) {  // uniform over the cluster
     cluster_wait();
-    if (hist) {
+    if (hist || appended) {
       cluster.sync();
       clear_hist();
+      publish();
     }
     return Result{kAll, n, n_blocks};
   }
@@ -561,8 +575,10 @@ __device__ __forceinline__ Result cluster_select(DevState* st, const float* __re
   }
   if (first_shift != 24) {  // uniform: the histogram gave the bin; finish in CTA 0
     if (tid == 0) QSA_TL(st, kTlTopk2, 0);  // loads and the histogram's bin done
-    return gather_finish<V>(st, scores, key, valid, base, n, n_blocks, prefix, mask, need, gather_bar,
-                            static_cast<void*>(&s_in[0][0][0]), s_hist, s_warp, s_ctl, clear_hist, emit);
+    const Result r = gather_finish<V>(st, scores, key, valid, base, n, n_blocks, prefix, mask, need, gather_bar,
+                                      static_cast<void*>(&s_in[0][0][0]), s_hist, s_warp, s_ctl, clear_hist, emit);
+    publish();  // CTA 0 returns after the final cluster barrier
+    return r;
   }
   if (tid == 0) QSA_TL(st, kTlTopk2, 0);  // loads and the histogram's bin done
   cluster_wait();  // every CTA of the cluster has started: its shared memory may be written
@@ -672,6 +688,7 @@ __device__ __forceinline__ Result cluster_select(DevState* st, const float* __re
       ++eq_before;
     }
   }
+  publish();  // every CTA passed a cluster barrier after its state read
   return Result{kTopK, n, n_blocks};
 }
 
