@@ -17,6 +17,7 @@
 #include <mutex>
 
 #include "qsa_device.cuh"
+#include "qsa_sm100.cuh"
 #include "qsa_timeline.cuh"
 
 namespace cg = cooperative_groups;
@@ -428,6 +429,7 @@ attn_cluster_kernel(DevState* st, const __half* __restrict__ q, const int32_t* _
   int* s_cell = reinterpret_cast<int*>(smem + SM::cell_off(Lc));
   float* s_stage = reinterpret_cast<float*>(smem + SM::stage_off(Lc));  // [CS][G][2] merged (m, l)
 
+  __shared__ uint64_t s_merge_bar;  // this CTA's slice: every CTA's partial has landed
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = int(cluster.block_rank());
   const int g = blockIdx.x / CS;
@@ -440,6 +442,10 @@ attn_cluster_kernel(DevState* st, const __half* __restrict__ q, const int32_t* _
   ids += size_t(u) * (FROM_BLOCKS ? k_blocks : max_cells);
   n_ids += u;
 
+  if (tid == 0) {  // one arrival per source CTA, plus the bytes each announces
+    sm100::mbar_init(&s_merge_bar, CS);
+    sm100::fence_mbar_init();
+  }
   pdl_launch_dependents();
   if (tid == 0) QSA_TL(st, kTlAttn, kTlEntry);
   cluster_arrive_relaxed();  // paired with cluster_wait() before the partials are pushed
@@ -626,10 +632,12 @@ attn_cluster_kernel(DevState* st, const __half* __restrict__ q, const int32_t* _
     if (gq < G) *reinterpret_cast<float2*>(s_o + gq * D + warp * 8 + 2 * tq) = make_float2(acc[0], acc[1]);
   }
   // ---- merge: CTA r owns output pairs [r*PER, (r+1)*PER) (2 dims of one head each).
-  //      Every CTA pushes its (max, sum) per head and its partial of each slice into the
-  //      owner's shared memory with DSMEM stores; after one cluster barrier each owner
-  //      merges its slice from local memory. Nothing reads another CTA's shared memory
-  //      after the barrier, so no second barrier is needed before exiting. ----
+  //      Every CTA sends its (max, sum) per head and its partial of each slice into the
+  //      owner's shared memory with st.async, whose bytes count on the owner's mbarrier,
+  //      and announces them with one arrival there; each owner waits on its own mbarrier
+  //      (no cluster-wide barrier on the way) and merges its slice from local memory. A
+  //      relaxed cluster barrier, arrived once a CTA holds all its data, keeps every CTA
+  //      alive until then. ----
   constexpr int PAIRS = G * (D / 2);
   constexpr int PER = (PAIRS + CS - 1) / CS;
   float2* s_in = reinterpret_cast<float2*>(smem + SM::in_off(Lc, CS));  // [CS][PER]
@@ -638,18 +646,24 @@ attn_cluster_kernel(DevState* st, const __half* __restrict__ q, const int32_t* _
   cluster_wait();   // every CTA of the cluster has started: its shared memory may be written
   if (tid == 0) QSA_TL(st, kTlAttn2, 3);
   for (int pidx = tid; pidx < PAIRS; pidx += kAcThreads) {
-    const int h = pidx / (D / 2), d2 = pidx % (D / 2);
+    const int h = pidx / (D / 2), d2 = pidx % (D / 2), owner = pidx / PER;
     const float2 v = *reinterpret_cast<const float2*>(s_o + h * D + 2 * d2);
-    *(cluster.map_shared_rank(s_in, pidx / PER) + rank * PER + pidx % PER) = v;
+    sm100::st_async_v2(sm100::cluster_addr(s_in + rank * PER + pidx % PER, owner), __float_as_uint(v.x),
+                       __float_as_uint(v.y), sm100::cluster_addr(&s_merge_bar, owner));
   }
   for (int t = tid; t < CS * G; t += kAcThreads) {
     const int owner = t / G, h = t % G;
-    float* dst = cluster.map_shared_rank(s_stage, owner) + (rank * G + h) * 2;
-    dst[0] = s_m[h];
-    dst[1] = s_l[h];
+    sm100::st_async_v2(sm100::cluster_addr(s_stage + (rank * G + h) * 2, owner), __float_as_uint(s_m[h]),
+                       __float_as_uint(s_l[h]), sm100::cluster_addr(&s_merge_bar, owner));
   }
+  // every source sends each owner PER output pairs and G (max, sum) pairs
+  if (tid < CS) sm100::mbar_arrive_expect_tx_remote(sm100::cluster_addr(&s_merge_bar, tid), uint32_t(PER + G) * 8u);
   if (tid == 0) QSA_TL(st, kTlAttn2, 4);  // pushed
-  cluster.sync();  // release the pushes above, acquire every other CTA's
+  if (!sm100::mbar_wait_cluster(&s_merge_bar, 0)) {
+    if (tid == 0) record_status(st, QSA_ERR_TIMEOUT);
+    (void)sm100::mbar_wait_cluster(&s_merge_bar, 0);  // stores still in flight land before this CTA leaves
+  }
+  cluster_arrive_relaxed();  // this CTA's data is all here; paired with the wait before exit
   if (tid == 0) QSA_TL(st, kTlAttn, kTlB);
   // CS lanes per output pair, lane r merging source CTA r's partial; shuffles within the
   // aligned CS-lane group combine them (max, then the weighted sums)
@@ -680,6 +694,7 @@ attn_cluster_kernel(DevState* st, const __half* __restrict__ q, const int32_t* _
       if (lse_out && d2 == 0) lse_out[size_t(g) * G + h] = den > 0.0f ? M + logf(den) : -INFINITY;
     }
   }
+  cluster_wait();  // every CTA holds its data: nothing is still arriving anywhere
   if (tid == 0) QSA_TL(st, kTlAttn, kTlExit);
 }
 

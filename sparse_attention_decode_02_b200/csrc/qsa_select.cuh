@@ -77,47 +77,6 @@ __device__ __forceinline__ uint32_t cta_exclusive_scan(uint32_t v, uint32_t* s_w
   return s_warp[warp] + x - v;
 }
 
-// ---- distributed shared memory: stores into CTA 0 that count on its mbarrier ----
-// shared::cluster address of `p` (a variable of this CTA's shared memory) in CTA `r`
-__device__ __forceinline__ uint32_t cluster_addr(const void* p, uint32_t r) {
-  uint32_t a;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(sm100::smem_u32(p)), "r"(r));
-  return a;
-}
-// 8 (4) bytes into another CTA's shared memory; completion is counted in bytes on `bar`,
-// an mbarrier in that CTA
-__device__ __forceinline__ void st_async_v2(uint32_t addr, uint32_t a, uint32_t b, uint32_t bar) {
-  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.u32 [%0], {%1, %2}, [%3];"
-               ::"r"(addr), "r"(a), "r"(b), "r"(bar) : "memory");
-}
-__device__ __forceinline__ void st_async_u32(uint32_t addr, uint32_t a, uint32_t bar) {
-  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.u32 [%0], %1, [%2];"
-               ::"r"(addr), "r"(a), "r"(bar) : "memory");
-}
-// one arrival on another CTA's mbarrier, announcing `bytes` of st_async data (no ordering
-// of its own: the data's arrival is what the bytes count)
-__device__ __forceinline__ void mbar_arrive_expect_tx_remote(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.relaxed.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-               : "memory");
-}
-// wait (bounded, like sm100::mbar_wait) for a phase of this CTA's mbarrier that other
-// CTAs of the cluster complete; their data is visible on return
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity) {
-  const unsigned long long t0 = sm100::globaltimer();
-  for (uint32_t i = 0;; ++i) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(sm100::smem_u32(bar)), "r"(parity)
-        : "memory");
-    if (ok) return true;
-    if ((i & 255u) == 255u && sm100::globaltimer() - t0 > sm100::kWaitLimitNs) return false;
-  }
-}
-
 __device__ __forceinline__ uint32_t lanemask_lt() {
   uint32_t m;
   asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
@@ -198,17 +157,17 @@ __device__ __forceinline__ Result gather_finish(DevState* st, const float* __res
   uint32_t tot;
   uint32_t off = cta_exclusive_scan_1(c, s_warp, &tot);  // a barrier since the last s_warp use
   cluster_wait();  // every CTA of the cluster has started: CTA 0's mbarrier is initialised
-  const uint32_t bar0 = cluster_addr(gather_bar, 0);
+  const uint32_t bar0 = sm100::cluster_addr(gather_bar, 0);
   const bool fits = tot <= kCap;  // uniform in the CTA
   if (fits && c) {
-    const uint32_t dst = cluster_addr(s_cand + size_t(rank) * kCap, 0);
+    const uint32_t dst = sm100::cluster_addr(s_cand + size_t(rank) * kCap, 0);
 #pragma unroll
     for (int j = 0; j < V; ++j)
-      if (((valid >> j) & 1u) && key[j] >= prefix) st_async_v2(dst + 8u * off++, key[j], uint32_t(base + j), bar0);
+      if (((valid >> j) & 1u) && key[j] >= prefix) sm100::st_async_v2(dst + 8u * off++, key[j], uint32_t(base + j), bar0);
   }
   if (tid == 0) {
-    st_async_u32(cluster_addr(&s_cnt[rank], 0), fits ? tot : kOverflow, bar0);
-    mbar_arrive_expect_tx_remote(bar0, 4u + (fits ? 8u * tot : 0u));
+    sm100::st_async_u32(sm100::cluster_addr(&s_cnt[rank], 0), fits ? tot : kOverflow, bar0);
+    sm100::mbar_arrive_expect_tx_remote(bar0, 4u + (fits ? 8u * tot : 0u));
   }
   // the final cluster barrier only keeps every CTA alive until CTA 0 holds all the data:
   // it orders nothing, so its arrive is relaxed
@@ -220,9 +179,9 @@ __device__ __forceinline__ Result gather_finish(DevState* st, const float* __res
   }
 
   // ---------------- CTA 0 ----------------
-  if (!mbar_wait_cluster(gather_bar, 0)) {
+  if (!sm100::mbar_wait_cluster(gather_bar, 0)) {
     if (tid == 0) record_status(st, QSA_ERR_TIMEOUT);
-    (void)mbar_wait_cluster(gather_bar, 0);  // stores still in flight land before this CTA leaves
+    (void)sm100::mbar_wait_cluster(gather_bar, 0);  // stores still in flight land before this CTA leaves
     cluster_arrive_relaxed();
     cluster_wait();
     clear_hist();

@@ -63,6 +63,47 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
+// ---- distributed shared memory: stores into another CTA that count on its mbarrier ----
+// shared::cluster address of `p` (a variable of this CTA's shared memory) in CTA `r`
+__device__ __forceinline__ uint32_t cluster_addr(const void* p, uint32_t r) {
+  uint32_t a;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(smem_u32(p)), "r"(r));
+  return a;
+}
+// 8 (4) bytes into another CTA's shared memory; completion is counted in bytes on `bar`,
+// an mbarrier in that CTA
+__device__ __forceinline__ void st_async_v2(uint32_t addr, uint32_t a, uint32_t b, uint32_t bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.u32 [%0], {%1, %2}, [%3];"
+               ::"r"(addr), "r"(a), "r"(b), "r"(bar) : "memory");
+}
+__device__ __forceinline__ void st_async_u32(uint32_t addr, uint32_t a, uint32_t bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.u32 [%0], %1, [%2];"
+               ::"r"(addr), "r"(a), "r"(bar) : "memory");
+}
+// one arrival on another CTA's mbarrier, announcing `bytes` of st_async data (no ordering
+// of its own: the data's arrival is what the bytes count)
+__device__ __forceinline__ void mbar_arrive_expect_tx_remote(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.relaxed.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+// wait (bounded, like sm100::mbar_wait) for a phase of this CTA's mbarrier that other
+// CTAs of the cluster complete; their data is visible on return
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity) {
+  const unsigned long long t0 = globaltimer();
+  for (uint32_t i = 0;; ++i) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    if (ok) return true;
+    if ((i & 255u) == 255u && globaltimer() - t0 > kWaitLimitNs) return false;
+  }
+}
+
 // ---- TMA ----------------------------------------------------------------------------
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
