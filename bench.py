@@ -58,6 +58,7 @@ def parse_args():
     ap.add_argument("--no-by-ctx", action="store_true", help="skip the 64k/128k lines")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-fp8", action="store_true", help="skip the FP8 K/V cache line")
+    ap.add_argument("--no-cp", action="store_true", help="skip the context-parallel line")
     ap.add_argument("--e2e-steps", type=int, default=300)
     ap.add_argument("--spread-replays", type=int, default=200,
                     help="replays of one step timed alone for the median / p10 / p90")
@@ -534,6 +535,107 @@ def run_ours(wl, n_layers, K, W, rank, world, e2e_steps, sample_clocks, local, m
             "graph_steps": G}
 
 
+def run_context_parallel(wl, shard_counts=(2, 4), reps=20):
+    """Row f3: one layer of the workload split into S contiguous block-aligned shards, each
+    its own library context on this GPU (the shards run one after another; the all-gathers
+    between devices are replaced by one stacked buffer). Times the sharded step, each of
+    its calls alone, and the same layer's single-device step, and checks that the sharded
+    selection equals the single-device one and the merged output matches it."""
+    import torch
+
+    import synth
+    import sparse_attention_decode_02_b200 as Q
+    n = wl.n_prefill
+    K = wl.k_blocks
+    pre = synth.device_prefill(wl, 0)
+    packed, views = synth.device_steps(wl, 1, 1)
+    q_idx, w, q = views["q_idx"][0, 0], views["w"][0, 0], views["q"][0, 0]
+    stream = torch.cuda.current_stream()
+
+    def timed(calls, r=reps):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(r):
+                calls()
+        g.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        g.replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return 1e3 * a.elapsed_time(b) / r
+
+    def layer(t0, t1, offset):
+        cfg = Q.make_config(1, (t1 - t0 + 7) // 4 * 4, wl.d_idx, wl.n_idx_heads, wl.top_k_tokens, wl.n_q_heads,
+                            wl.n_kv_heads, wl.head_dim, wl.rope_base, wl.rms_eps, rope_pos_offset=offset,
+                            early_inputs=Q.QSA_INPUTS_EARLY)
+        qsa = Q.Qsa(cfg)
+        bufs = Q.alloc_layer(cfg)
+        qsa.bind_layer(0, **bufs)
+        qsa.append_tokens(0, pre["k"][t0:t1], pre["v"][t0:t1], pre["idx"][t0:t1])
+        qsa.update_pooled_cache(0)
+        return qsa, bufs
+
+    one, one_bufs = layer(0, n, 0)
+    outs = Q.alloc_step_outputs(one.cfg)
+    scores = torch.zeros(one.cfg.max_ctx // 4, dtype=torch.float32, device="cuda")
+
+    def single():
+        one.index_topk(0, q_idx, w, outs["sel"], outs["n_sel"], scores)
+        one.sparse_attend_selected(0, q, outs["sel"], outs["n_sel"], outs["out"])
+
+    single_us = timed(single)
+    ref_sel = outs["sel"][: int(outs["n_sel"][0])].clone()
+    ref_out = outs["out"].clone()
+    lines = {}
+    for S in shard_counts:
+        bounds = [4 * ((r * (n // 4)) // S) for r in range(S)] + [n]
+        shards = [layer(bounds[r], bounds[r + 1], bounds[r]) for r in range(S)]
+        cand_s = torch.empty(S, K, dtype=torch.float32, device="cuda")
+        cand_b = torch.empty(S, K, dtype=torch.int32, device="cuda")
+        n_cand = torch.empty(S, dtype=torch.int32, device="cuda")
+        sel = torch.empty(K, dtype=torch.int32, device="cuda")
+        n_sel = torch.empty(1, dtype=torch.int32, device="cuda")
+        o_parts = torch.empty(S, wl.n_q_heads, wl.head_dim, dtype=torch.float32, device="cuda")
+        lse_parts = torch.empty(S, wl.n_q_heads, dtype=torch.float32, device="cuda")
+        out = torch.empty(wl.n_q_heads, wl.head_dim, dtype=torch.float32, device="cuda")
+        cand = [lambda r=r: shards[r][0].cp_index_candidates(0, q_idx, w, n, bounds[r] // 4, cand_s[r], cand_b[r],
+                                                              n_cand[r:r + 1]) for r in range(S)]
+        select = lambda: Q.cp_select(cand_s, cand_b, S, K, sel, n_sel)
+        attend = [lambda r=r: shards[r][0].cp_attend_partial(0, q, sel, n_sel, bounds[r] // 4, o_parts[r],
+                                                             lse_parts[r]) for r in range(S)]
+        merge = lambda: Q.cp_merge(o_parts, lse_parts, S, wl.n_q_heads, wl.head_dim, out)
+
+        def step():
+            for c in cand:
+                c()
+            select()
+            for a in attend:
+                a()
+            merge()
+
+        step_us = timed(step)
+        assert torch.equal(sel[: int(n_sel[0])], ref_sel), "sharded selection differs from the single device's"
+        err = ((out - ref_out).abs().amax(dim=1) / ref_out.abs().amax(dim=1).clamp_min(1e-6)).max().item()
+        assert err < 2e-3, err
+        cand_us = [timed(c) for c in cand]
+        att_us = [timed(a) for a in attend]
+        sel_us, merge_us = timed(select), timed(merge)
+        lines[f"x{S}"] = {
+            "shards": S, "sharded_step_us_one_gpu": round(step_us, 3),
+            "candidates_us": [round(x, 3) for x in cand_us], "select_us": round(sel_us, 3),
+            "attend_partial_us": [round(x, 3) for x in att_us], "merge_us": round(merge_us, 3),
+            "per_device_us": round(max(cand_us) + sel_us + max(att_us) + merge_us, 3),
+            "merged_out_rel_err": float(f"{err:.2e}")}
+        del shards
+        torch.cuda.empty_cache()
+    return {"layer_ctx": n, "single_device_us": round(single_us, 3), "reps": reps,
+            "per_device_us": "slowest shard's candidates + select + slowest shard's attention + merge, "
+                             "each timed alone; the two all-gathers between devices are not included",
+            **lines}
+
+
 def scan_ab(wb, n_layers, peak, reps=5):
     """The indexer scan both ways on the same pooled caches, isolated back to back over the
     layers: the tensor-core scan (the default) and the CUDA-core scan (f32 query, packed
@@ -747,6 +849,13 @@ def main_ours(args):
         del r8
         torch.cuda.empty_cache()
 
+    # row f3: the context-parallel step, shards emulated as contexts on this GPU
+    context_parallel = None
+    if not args.profile_case and not args.no_cp and world == 1:
+        torch.cuda.empty_cache()
+        context_parallel = run_context_parallel(synth.workload(wl.name, n_layers=1))
+        torch.cuda.empty_cache()
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(wl)
@@ -774,6 +883,7 @@ def main_ours(args):
             "bulk_pool": dict(main["bulk_pool"], frac=round(main["bulk_pool"]["gbs"] / peak, 4)) if main["bulk_pool"] else None,
             "multi_query": main["multi_query"],
             "scan_ab": main["scan_ab"],
+            "context_parallel": context_parallel,
             "kv_fp8": kv_fp8,
             "pooled_fp8": pooled_fp8,
             "hbm_gbs_step": round(world * wl.n_layers * K * sum(sb.values()) / (main["ms"] / 1e3) / 1e9, 1),
