@@ -216,7 +216,8 @@ qsa_status qsa_bind_layer(qsa_ctx* ctx, int32_t layer, const qsa_layer_buffers* 
   l.bound = true;
   l.pending_blocks = 0;
   const LayerView v = ctx->view(layer);
-  qsa_status st = ctx->cuda(cudaMemsetAsync(v.hist, 0, size_t(1 << kHistBits) * sizeof(uint32_t), (cudaStream_t)stream),
+  qsa_status st = ctx->cuda(cudaMemsetAsync(v.hist, 0, size_t(kMaxQueries) * (1 << kHistBits) * sizeof(uint32_t),
+                                            (cudaStream_t)stream),
                             "bind_layer: clear histogram");
   if (st == QSA_OK) st = ctx->cuda(launch_set_state(v, 0, 0, kSetReset, (cudaStream_t)stream), "bind_layer");
   if (st != QSA_OK) l.bound = false;
@@ -391,10 +392,10 @@ qsa_status qsa_index_topk_multi(qsa_ctx* ctx, int32_t layer, int32_t n_queries, 
   LayerView v = ctx->view(layer);
   const int stride = score_stride_of(ctx->cfg);
   float* s = scores ? scores : v.scores;
-  if (qsa_status st = ctx->cuda(launch_index_scan(v, q_idx, w, s, (cudaStream_t)stream, n_queries, stride),
+  if (qsa_status st = ctx->cuda(launch_index_scan(v, q_idx, w, s, (cudaStream_t)stream, n_queries, stride, v.hist),
                                 "index scan (multi-query)"))
     return st;
-  return ctx->cuda(launch_topk(v, s, sel_blocks, n_sel, (cudaStream_t)stream, n_queries, stride),
+  return ctx->cuda(launch_topk(v, s, sel_blocks, n_sel, (cudaStream_t)stream, n_queries, stride, v.hist),
                    "block top-k (multi-query)");
 }
 

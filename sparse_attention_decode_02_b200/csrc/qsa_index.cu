@@ -19,7 +19,7 @@ namespace qsa {
 // the selected blocks in ascending order. With gridDim.y = T > 1 (multi-query step),
 // cluster u selects for the query of token n_ctx - T + u from score row u into output
 // row u (rows of k_blocks ids, one count each).
-// With `hist` (single query), the selection starts from the scan's score-key histogram.
+// With `hist`, cluster u starts from query u's score-key histogram (hist + u * 2048).
 // With sel_scores (single query): a context-parallel shard's candidate slots, below.
 template <int V>
 __global__ void __launch_bounds__(sel::kThreads, 1)
@@ -41,7 +41,9 @@ block_topk_kernel(DevState* st, const float* __restrict__ scores, int32_t* __res
   cluster_arrive_relaxed();  // paired inside cluster_select
   pdl_wait();
   if (threadIdx.x == 0) QSA_TL(st, kTlTopk, kTlWait);
-  const sel::Result res = sel::cluster_select<V>(st, scores, gridDim.y == 1 ? hist : nullptr, k_blocks, max_blocks,
+  // query u's histogram (the multi-query scan fills one per query)
+  const sel::Result res = sel::cluster_select<V>(st, scores, hist ? hist + size_t(u) * (1u << kHistBits) : nullptr,
+                                                 k_blocks, max_blocks,
                                                  n_back, &s_gather_bar, gridDim.y == 1 ? fused_max_ctx : 0,
                                                  [&](uint32_t pos, int block) {
                                                    // bounds-checked in every build
@@ -103,7 +105,7 @@ cudaError_t init_kernel_attributes() {
 cudaError_t launch_topk(const LayerView& L, const float* scores, int32_t* sel_out, int32_t* n_sel, cudaStream_t s,
                         int n_queries, int score_stride, uint32_t* hist, float* sel_scores, int block_base,
                         bool after_fused_scan) {
-  if (n_queries != 1) hist = nullptr, sel_scores = nullptr, block_base = 0, after_fused_scan = false;
+  if (n_queries != 1) sel_scores = nullptr, block_base = 0, after_fused_scan = false;
   const int max_blocks = L.cfg.max_ctx / kBlock;
   const int kb = L.cfg.top_k_tokens / kBlock;
   const int fused_max_ctx = after_fused_scan ? L.cfg.max_ctx : 0;

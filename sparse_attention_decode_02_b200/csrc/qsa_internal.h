@@ -77,8 +77,8 @@ inline WorkspaceLayout workspace_layout(const qsa_config& c, int n_splits) {
   w.state = off;
   off += align256(sizeof(DevState));
   off += kTimelineBytes;  // the timeline build's probe record (kTimelineOffset)
-  w.hist = off;  // score-key prefix histogram of the last scan (zero between selections)
-  off += align256(size_t(1 << kHistBits) * sizeof(uint32_t));
+  w.hist = off;  // score-key prefix histograms of the last scan, one per query (zero between selections)
+  off += align256(size_t(kMaxQueries) * (1 << kHistBits) * sizeof(uint32_t));
   w.cp = off;    // a context-parallel shard's part of the global selection: count, then ids
   off += align256(size_t(16 + kTopkMaxK) * sizeof(int32_t));
   w.scores = off;  // kMaxQueries rows of score_stride_of(c) floats

@@ -84,7 +84,7 @@ struct ScanShape {
   // doubles), raw queries (T*H*D f16), the score-prefix histogram, one pooled row (f32),
   // the rotated query in f32 (8-bit keys: T*H*D floats)
   static constexpr int CTRL_BYTES =
-      256 + T * D * 4 + D / 2 * 8 + T * H * D * 2 + kHistBins * 4 + D * 4 + (F8 ? T * H * D * 4 : 0);
+      256 + T * D * 4 + D / 2 * 8 + T * H * D * 2 + T * kHistBins * 4 + D * 4 + (F8 ? T * H * D * 4 : 0);
   static constexpr size_t FIXED = 1024 + size_t(B_BYTES) + CTRL_BYTES;
   // ring depth: kScanStages tiles where they fit, fewer for wide B operands. A short ring
   // keeps the CTA small enough to be resident beside the attention and selection kernels'
@@ -207,7 +207,7 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_
                      float* __restrict__ scores, uint32_t* __restrict__ hist, float rope_base, int max_blocks,
                      int rope_dims, int rope_interleaved, int rope_pos_stride, int score_stride, DecodeAppend app,
                      int q_n, const float* pooled_scales, int early) {
-  static_assert(!(HIST || FUSED) || T == 1, "histogram and fused append serve the single-query step");
+  static_assert(!FUSED || T == 1, "the fused append serves the single-query step");
   static_assert(!FUSED || HIST, "the decode step always fills the histogram");
   using S = ScanShape<D, H, T, F8>;
   constexpr int kAcc = S::ACC;
@@ -229,8 +229,8 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_
   float* s_sin = s_cos + T * (D / 2);                                 // [T][D/2] each
   double* s_theta = reinterpret_cast<double*>(s_sin + T * (D / 2));   // D/2 doubles
   __half* s_q = reinterpret_cast<__half*>(s_theta + D / 2);           // raw queries, T x H x D
-  uint32_t* s_hist = reinterpret_cast<uint32_t*>(s_q + T * H * D);    // [kHistBins]
-  float* s_row = reinterpret_cast<float*>(s_hist + kHistBins);        // [D] (pooling, generic RoPE)
+  uint32_t* s_hist = reinterpret_cast<uint32_t*>(s_q + T * H * D);    // [T][kHistBins]
+  float* s_row = reinterpret_cast<float*>(s_hist + T * kHistBins);    // [D] (pooling, generic RoPE)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   pdl_launch_dependents();
@@ -404,7 +404,7 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_
     load_w();
   }
   if (warp < 4 && HIST)
-    for (int i = tid; i < kHistBins; i += 128) s_hist[i] = 0u;
+    for (int i = tid; i < T * kHistBins; i += 128) s_hist[i] = 0u;
 
 
   if (FUSED && warp == 6) {
@@ -569,7 +569,10 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_
             // positive, so they come out of the max(0, .) unchanged
             const float score = F8 ? s * (row_scale * unscale) / sqrt_d : s / sqrt_d;
             scores[size_t(u) * score_stride + row] = score;
-            if constexpr (HIST) atomicAdd(&s_hist[sel::score_key(score) >> (32 - kHistBits)], 1u);
+            // query u counts only the blocks its own n_u = n - (T-1-u) tokens complete
+            if constexpr (HIST)
+              if (row < (n - (T - 1 - u)) / kBlock)
+                atomicAdd(&s_hist[u * kHistBins + (sel::score_key(score) >> (32 - kHistBits))], 1u);
           }
         }
       }
@@ -577,9 +580,9 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_
       if (tid == 0) QSA_TL(st, kTlScan, kTlB);  // this thread's rows scored
       if constexpr (HIST) {  // this CTA's counts into the layer's histogram
         named_bar_sync(2, 128);
-        for (int i = tid; i < kHistBins; i += 128) {
+        for (int i = tid; i < T * kHistBins; i += 128) {
           const uint32_t c = s_hist[i];
-          if (c) atomicAdd(hist + i, c);
+          if (c) atomicAdd(hist + i, c);  // query u's bins at hist + u * kHistBins
         }
       }
     }
@@ -615,7 +618,10 @@ static cudaError_t set_scan_attr_t() {
       (e = set_scan_attr<D, H, 1, true, true>()) != cudaSuccess ||
       (e = set_scan_attr<D, H, 2, false, false>()) != cudaSuccess ||
       (e = set_scan_attr<D, H, 3, false, false>()) != cudaSuccess ||
-      (e = set_scan_attr<D, H, 4, false, false>()) != cudaSuccess)
+      (e = set_scan_attr<D, H, 4, false, false>()) != cudaSuccess ||
+      (e = set_scan_attr<D, H, 2, true, false>()) != cudaSuccess ||
+      (e = set_scan_attr<D, H, 3, true, false>()) != cudaSuccess ||
+      (e = set_scan_attr<D, H, 4, true, false>()) != cudaSuccess)
     return e;
   if constexpr (D == 128) {  // 8-bit pooled keys: single query
     if ((e = set_scan_attr<D, H, 1, false, false, true>()) != cudaSuccess ||
@@ -695,7 +701,15 @@ static cudaError_t launch_scan_tc_t(const LayerView& L, const void* q_idx, const
     return cudaErrorInvalidValue;
   }
   if (mode == 2) return launch_scan_tc<D, H, 1, true, true>(L, q_idx, w, scores, s, score_stride, hist, app);
-  if (mode == 1) return launch_scan_tc<D, H, 1, true, false>(L, q_idx, w, scores, s, score_stride, hist, app, q_n);
+  if (mode == 1) {  // with the score-key histograms (one per query)
+    switch (n_queries) {
+      case 1: return launch_scan_tc<D, H, 1, true, false>(L, q_idx, w, scores, s, score_stride, hist, app, q_n);
+      case 2: return launch_scan_tc<D, H, 2, true, false>(L, q_idx, w, scores, s, score_stride, hist, app);
+      case 3: return launch_scan_tc<D, H, 3, true, false>(L, q_idx, w, scores, s, score_stride, hist, app);
+      case 4: return launch_scan_tc<D, H, 4, true, false>(L, q_idx, w, scores, s, score_stride, hist, app);
+      default: return cudaErrorInvalidValue;
+    }
+  }
   switch (n_queries) {
     case 1: return launch_scan_tc<D, H, 1, false, false>(L, q_idx, w, scores, s, score_stride, hist, app, q_n);
     case 2: return launch_scan_tc<D, H, 2, false, false>(L, q_idx, w, scores, s, score_stride, hist, app);
@@ -731,9 +745,9 @@ cudaError_t launch_index_scan(const LayerView& L, const void* q_idx, const float
                               cudaStream_t s, int n_queries, int score_stride, uint32_t* hist, int q_n) {
   if (L.cfg.scan_kind == QSA_SCAN_CUDA_CORES && n_queries == 1)
     return launch_index_scan_cc(L, q_idx, w, scores, hist, s, q_n);
-  const int mode = (hist && n_queries == 1) ? 1 : 0;
-  return launch_scan_mode(L, q_idx, w, scores, s, n_queries, score_stride, mode ? hist : nullptr, mode,
-                          DecodeAppend{}, n_queries == 1 ? q_n : 0);
+  const int mode = hist ? 1 : 0;
+  return launch_scan_mode(L, q_idx, w, scores, s, n_queries, score_stride, hist, mode, DecodeAppend{},
+                          n_queries == 1 ? q_n : 0);
 }
 
 cudaError_t launch_decode_scan(const LayerView& L, const void* k, const void* v, const void* idx, const void* q_idx,
