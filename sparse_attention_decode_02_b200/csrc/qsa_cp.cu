@@ -61,14 +61,18 @@ __device__ __forceinline__ uint32_t cp_exclusive_scan(uint32_t v, uint32_t* s_wa
 // with block id -1 is empty), listed shard by shard, each shard's in ascending block order.
 // Rule: the K largest scores, ties to the lower block, output ascending; fewer than K
 // candidates: all of them. Thread t holds slots [8t, 8t + 8), so slot order is thread order.
+// A 2048-bin histogram of the keys' top 11 bits gives the bin of the K-th key; radix passes
+// over the remaining 21 bits (8, 8, 5) refine inside it, warp 0 scanning each pass's
+// digit counts; one packed prefix scan places every selected slot.
 __global__ void __launch_bounds__(kCpThreads) cp_select_kernel(const float* __restrict__ cand_scores,
                                                                const int32_t* __restrict__ cand_blocks,
                                                                int n_slots, int k_blocks, int32_t* __restrict__ sel,
                                                                int32_t* __restrict__ n_sel) {
-  __shared__ uint32_t s_hist[256];
+  constexpr int kHB = 2048;
+  __shared__ uint32_t s_h[kHB];
   __shared__ uint32_t s_warp[33];
   __shared__ uint32_t s_ctl[4];
-  const int tid = threadIdx.x, base = tid * kCpPer;
+  const int tid = threadIdx.x, base = tid * kCpPer, lane = tid & 31, warp = tid >> 5;
   pdl_launch_dependents();
   pdl_wait();
   uint32_t key[kCpPer];
@@ -81,36 +85,74 @@ __global__ void __launch_bounds__(kCpThreads) cp_select_kernel(const float* __re
     key[j] = i < n_slots ? sel::score_key(cand_scores[i]) : 0u;
     if (blk[j] >= 0) valid |= 1u << j;
   }
+  for (int i = tid; i < kHB; i += kCpThreads) s_h[i] = 0u;
+  __syncthreads();
+#pragma unroll
+  for (int j = 0; j < kCpPer; ++j)
+    if ((valid >> j) & 1u) atomicAdd(&s_h[key[j] >> 21], 1u);
+  __syncthreads();
+  // thread t holds bins 2047 - 2t and 2046 - 2t (from the top); keys above them come first
+  const uint32_t h0 = s_h[kHB - 1 - 2 * tid], h1 = s_h[kHB - 2 - 2 * tid];
   uint32_t total;
-  (void)cp_exclusive_scan(__popc(valid), s_warp, &total);
+  const uint32_t above = cp_exclusive_scan(h0 + h1, s_warp, &total);
   uint32_t prefix = 0, mask = 0, need = uint32_t(k_blocks);
   const bool all = total <= uint32_t(k_blocks);  // uniform
   if (all) {
-    mask = 0;  // every valid slot is "at the threshold" and taken
-    need = total;
+    need = total;  // mask 0: every valid slot is "at the threshold" and taken
   } else {
-    for (int shift = 24;; shift -= 8) {
-      if (tid < 256) s_hist[tid] = 0;
+    if (above < need && above + h0 >= need) {
+      s_ctl[0] = uint32_t(kHB - 1 - 2 * tid);
+      s_ctl[1] = above;
+    } else if (above + h0 < need && above + h0 + h1 >= need) {
+      s_ctl[0] = uint32_t(kHB - 2 - 2 * tid);
+      s_ctl[1] = above + h0;
+    }
+    __syncthreads();
+    prefix = s_ctl[0] << 21;
+    mask = ~0u << 21;
+    need -= s_ctl[1];
+    __syncthreads();  // s_ctl is rewritten below
+    for (int shift = 13;; shift -= 8) {  // bits 20..13, 12..5, 4..0
+      const int bits = shift >= 0 ? 8 : 8 + shift;
+      shift = shift >= 0 ? shift : 0;
+      const uint32_t nb = 1u << bits;
+      if (tid < 256) s_h[tid] = 0u;
       __syncthreads();
 #pragma unroll
       for (int j = 0; j < kCpPer; ++j)
-        if (((valid >> j) & 1u) && (key[j] & mask) == prefix) atomicAdd(&s_hist[(key[j] >> shift) & 255u], 1u);
+        if (((valid >> j) & 1u) && (key[j] & mask) == prefix) atomicAdd(&s_h[(key[j] >> shift) & (nb - 1)], 1u);
       __syncthreads();
-      // thread t < 256 takes digit 255 - t: an inclusive prefix over t counts keys >= digit
-      const uint32_t v = tid < 256 ? s_hist[255 - tid] : 0u;
-      uint32_t tt;
-      const uint32_t excl = cp_exclusive_scan(v, s_warp, &tt);
-      if (tid < 256 && excl < need && excl + v >= need) {
-        s_ctl[0] = uint32_t(255 - tid);
-        s_ctl[1] = excl;
-        s_ctl[2] = v;
+      if (warp == 0) {  // lane l: digits nb-1-8l .. nb-8-8l (from the top)
+        uint32_t cq[8], sum = 0;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const int d = int(nb) - 1 - (8 * lane + q);
+          cq[q] = d >= 0 ? s_h[d] : 0u;
+          sum += cq[q];
+        }
+        uint32_t x = sum;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const uint32_t y = __shfl_up_sync(0xffffffffu, x, off);
+          if (lane >= off) x += y;
+        }
+        uint32_t acc = x - sum;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          if (acc < need && acc + cq[q] >= need) {
+            s_ctl[0] = nb - 1 - uint32_t(8 * lane + q);
+            s_ctl[1] = acc;
+            s_ctl[2] = cq[q];
+          }
+          acc += cq[q];
+        }
       }
       __syncthreads();
       need -= s_ctl[1];
       prefix |= s_ctl[0] << shift;
-      mask |= 255u << shift;
+      mask |= (nb - 1) << shift;
       const bool done = s_ctl[2] == need || shift == 0;
-      __syncthreads();
+      __syncthreads();  // s_ctl and s_h are rewritten by the next pass
       if (done) break;
     }
   }
