@@ -156,6 +156,7 @@ __device__ __forceinline__ Result gather_finish(DevState* st, const float* __res
   for (int j = 0; j < V; ++j) c += ((valid >> j) & 1u) && key[j] >= prefix;
   uint32_t tot;
   uint32_t off = cta_exclusive_scan_1(c, s_warp, &tot);  // a barrier since the last s_warp use
+  if (rank == 1 && tid == 0) QSA_TL(st, kTlTopk3, 2);  // candidate offsets known
   cluster_wait();  // every CTA of the cluster has started: CTA 0's mbarrier is initialised
   const uint32_t bar0 = sm100::cluster_addr(gather_bar, 0);
   const bool fits = tot <= kCap;  // uniform in the CTA
@@ -168,6 +169,7 @@ __device__ __forceinline__ Result gather_finish(DevState* st, const float* __res
   if (tid == 0) {
     sm100::st_async_u32(sm100::cluster_addr(&s_cnt[rank], 0), fits ? tot : kOverflow, bar0);
     sm100::mbar_arrive_expect_tx_remote(bar0, 4u + (fits ? 8u * tot : 0u));
+    if (rank == 1) QSA_TL(st, kTlTopk3, 3);  // sent
   }
   // the final cluster barrier only keeps every CTA alive until CTA 0 holds all the data:
   // it orders nothing, so its arrive is relaxed
@@ -455,6 +457,7 @@ __device__ __forceinline__ Result cluster_select(DevState* st, const float* __re
 #pragma unroll
   for (int j = 0; j < V; ++j) asm volatile("" ::"f"(f[j]));  // keep the loads ahead of the branches
   asm volatile("" ::"r"(h4.x), "r"(h4.y), "r"(h4.z), "r"(h4.w));
+  if (rank == 1 && tid == 0) QSA_TL(st, kTlTopk3, 0);  // a source CTA's loads issued
   // fused_max_ctx > 0: the decode step's scan appended token n_state (under the same
   // conditions as here) and scored with it, leaving the state for this kernel to advance
   const bool appended = fused_max_ctx > 0 && n_state >= 0 && n_state < fused_max_ctx &&
@@ -511,6 +514,7 @@ __device__ __forceinline__ Result cluster_select(DevState* st, const float* __re
     const uint32_t c4 = h4.x + h4.y + h4.z + h4.w;
     uint32_t total;
     __syncthreads();  // s_warp's previous readers are done
+    if (rank == 1 && tid == 0) QSA_TL(st, kTlTopk3, 4);  // every warp's loads landed
     const uint32_t above = cta_exclusive_scan_1(c4, s_warp, &total);  // keys in higher bins
     if (total == uint32_t(n_blocks)) {  // uniform: every thread sees the same total
       // bins of this thread from the top: 2047-4t (h4.w), then h4.z, h4.y, h4.x
@@ -530,6 +534,7 @@ __device__ __forceinline__ Result cluster_select(DevState* st, const float* __re
       prefix = b1 << (32 - kHistBits);
       mask = ~0u << (32 - kHistBits);
       first_shift = 32 - kHistBits - 8;  // 13
+      if (rank == 1 && tid == 0) QSA_TL(st, kTlTopk3, 1);  // the bin found
     }
   }
   if (first_shift != 24) {  // uniform: the histogram gave the bin; finish in CTA 0
