@@ -204,8 +204,8 @@ __device__ __forceinline__ Result gather_finish(DevState* st, const float* __res
     // ---- warp r takes CTA r's candidates, lane l its items l + 32k (k < 8), in shared
     // memory where they landed; the candidates' order (block order) is region, then item:
     // k, then lane. The passes hold the keys in registers; the output loop stays rolled
-    // and reads shared memory: it runs once per launch, so its instruction fetch costs
-    // more than those loads. ----
+    // and reads them from shared memory again (measured faster than the unrolled loop
+    // over the registers). ----
     const int warp = tid >> 5, lane = tid & 31;
     const uint32_t lt = lanemask_lt();
     const uint32_t cnt = s_cnt[warp];
