@@ -36,7 +36,7 @@ static_assert(sizeof(DevState) == 256, "DevState must stay 256 bytes");
 // [kernel][point][min, max] of the low 32 bits of %globaltimer (ns) that the CTAs of the
 // step's kernels reached at each probe point (kernels: scan, top-k, attention, and detail
 // rows of each).
-constexpr int kTimelineKernels = 8, kTimelinePoints = 5;
+constexpr int kTimelineKernels = 10, kTimelinePoints = 5;
 constexpr size_t kTimelineOffset = sizeof(DevState);
 constexpr size_t kTimelineBytes = 512;
 static_assert(kTimelineKernels * kTimelinePoints * 2 * 4 <= kTimelineBytes, "timeline region");

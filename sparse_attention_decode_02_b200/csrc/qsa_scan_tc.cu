@@ -580,15 +580,26 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_
       if (tid == 0) QSA_TL(st, kTlScan, kTlB);  // this thread's rows scored
       if constexpr (HIST) {  // this CTA's counts into the layer's histogram
         named_bar_sync(2, 128);
-        for (int i = tid; i < T * kHistBins; i += 128) {
-          const uint32_t c = s_hist[i];
-          if (c) atomicAdd(hist + i, c);  // query u's bins at hist + u * kHistBins
+        // thread t: kPer consecutive bins, read 4 at a time, one reduction per non-zero
+        // bin; query u's bins sit at hist + u * kHistBins
+        constexpr int kPer = T * kHistBins / 128;
+        static_assert(kPer % 4 == 0, "whole 16-byte vectors");
+#pragma unroll 1
+        for (int v = 0; v < kPer / 4; ++v) {
+          const uint4 c4 = reinterpret_cast<const uint4*>(s_hist + tid * kPer)[v];
+          uint32_t* dst = hist + tid * kPer + 4 * v;
+          if (c4.x) atomicAdd(dst, c4.x);
+          if (c4.y) atomicAdd(dst + 1, c4.y);
+          if (c4.z) atomicAdd(dst + 2, c4.z);
+          if (c4.w) atomicAdd(dst + 3, c4.w);
         }
+        if (tid == 0) QSA_TL(st, kTlScan3, 0);  // histogram flushed (this thread's part)
       }
     }
   }
   tc_fence_before();
   __syncthreads();
+  if (threadIdx.x == 0) QSA_TL(st, kTlScan3, 1);  // every warp done
   if (warp == 5) {
     tc_fence_after();
     tmem_dealloc(tmem_base, S::TMEM_COLS);

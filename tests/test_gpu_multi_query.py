@@ -165,3 +165,19 @@ def test_multi_query_limits_and_short_context():
         p.qsa.rollback(0, -1)
     p.qsa.rollback(0, 100)
     assert p.g.state()[:2] == (2, 0)
+
+
+@pytest.mark.parametrize("T", [2, 4])
+def test_multi_query_early_inputs_identical(T):
+    """early_inputs (the scan builds the T-query operand before its dependency wait; here
+    the append and pooled update right before it move the length, so the operand is
+    rebuilt after the wait) against the default, bit for bit, over several draft rounds."""
+    a = Pair("tiny", 4 * 250 + 1, max_extra=32, early_inputs=1)
+    b = Pair("tiny", 4 * 250 + 1, max_extra=32)
+    for r in range(4):
+        x = _drafts(a.wl, T, step0=T * r)
+        ga, gb = a.gpu_multi(x), b.gpu_multi(x)
+        for u in range(T):
+            np.testing.assert_array_equal(ga[u]["sel"], gb[u]["sel"])
+            np.testing.assert_array_equal(ga[u]["scores"], gb[u]["scores"])
+            np.testing.assert_array_equal(ga[u]["out"], gb[u]["out"])
