@@ -221,10 +221,11 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_
   uint64_t* tfull = empty + kStages;
   uint64_t* tempty = tfull + kAcc;
   uint64_t* pool_bar = tempty + kAcc;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(pool_bar + 1);
+  uint64_t* spec_bar = pool_bar + 1;  // the first tile loaded at the hinted range
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(spec_bar + 1);
   float* s_qmax = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(full) + 192);  // [4] (8-bit keys)
   int* s_nspec = reinterpret_cast<int*>(reinterpret_cast<unsigned char*>(full) + 208);     // early B operand
-  static_assert((2 * kStages + 2 * kAcc + 1) * 8 + 4 <= 192, "barriers below the query-max slots");
+  static_assert((2 * kStages + 2 * kAcc + 2) * 8 + 4 <= 192, "barriers below the query-max slots");
   float* s_cos = reinterpret_cast<float*>(smem + size_t(kStages) * S::TILE_BYTES + S::B_BYTES + 256);
   float* s_sin = s_cos + T * (D / 2);                                 // [T][D/2] each
   double* s_theta = reinterpret_cast<double*>(s_sin + T * (D / 2));   // D/2 doubles
@@ -245,12 +246,14 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_
       mbar_init(&tempty[a], 128);
     }
     mbar_init(pool_bar, 1);
+    mbar_init(spec_bar, 1);
     fence_mbar_init();
   }
   if (warp == 5) {
     tmem_alloc(tmem_holder, S::TMEM_COLS);
     tmem_relinquish();
   }
+  int spec_r0 = 0, spec_r1 = 0;  // warp 4 lane 0: this CTA's range at the hinted length
   if (warp == 4 && lane == 0) {
     tma_prefetch_desc(&map_tile);
     tma_prefetch_desc(&map_box);
@@ -261,10 +264,30 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_
     const int nb_hint = min(max(ld_volatile(&st->n_ctx) + (FUSED ? 1 : 0), 0) / kBlock, max_blocks);
     const int p0 = int((long long)blockIdx.x * nb_hint / gridDim.x);
     const int p1 = int((long long)(blockIdx.x + 1) * nb_hint / gridDim.x);
+    spec_r0 = p0;
+    spec_r1 = p1;
     for (int r = p0; r < p1; r += 128)
 #pragma unroll
       for (int j = 0; j < S::HALVES; ++j) tma_prefetch_l2_2d(&map_tile, j * (128 / S::ESIZE), r);
   }
+  // TMA loads of `rows` pooled rows from row0 into ring stage s, completing on bar
+  auto issue_tile = [&](int s, int row0, int rows, uint64_t* bar) {
+    unsigned char* dst = sA + size_t(s) * S::TILE_BYTES;
+    if (rows == 128) {  // whole tile: one 128-row box per 128-byte span
+      mbar_arrive_expect_tx(bar, uint32_t(S::TILE_BYTES));
+#pragma unroll
+      for (int j = 0; j < S::HALVES; ++j)
+        tma_load_2d(dst + j * S::HALF_BYTES, &map_tile, j * (128 / S::ESIZE), row0, bar);
+    } else {            // ragged tail: 16-row boxes, at most 15 rows past the range
+      const int boxes = (rows + kBoxRows - 1) / kBoxRows;
+      mbar_arrive_expect_tx(bar, uint32_t(boxes * kBoxRows * 128 * S::HALVES));
+#pragma unroll
+      for (int j = 0; j < S::HALVES; ++j)
+        for (int b = 0; b < boxes; ++b)
+          tma_load_2d(dst + j * S::HALF_BYTES + b * kBoxRows * 128, &map_box, j * (128 / S::ESIZE),
+                      row0 + b * kBoxRows, bar);
+    }
+  };
   // RoPE frequencies do not depend on the previous kernel: compute them before waiting on it
   for (int i = threadIdx.x; i < rope_dims / 2; i += blockDim.x)
     s_theta[i] = pow((double)rope_base, -2.0 * (double)i / (double)rope_dims);
@@ -418,6 +441,14 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_
   }
   if (!(FUSED && warp == 6)) pdl_wait();
   if (threadIdx.x == 0) QSA_TL(st, kTlScan, kTlWait);
+  // The first tile at the hinted range, issued now (the data is safe to read: the wait is
+  // behind us) instead of after the state read; it is used only if the state confirms the
+  // range. Not in the CTA whose rows a decode step's new block may join.
+  bool spec_issued = false, spec_done = false;
+  if (warp == 4 && lane == 0 && spec_r1 > spec_r0 && !(FUSED && blockIdx.x == gridDim.x - 1)) {
+    issue_tile(0, spec_r0, min(128, spec_r1 - spec_r0), spec_bar);
+    spec_issued = true;
+  }
   const int n_old = ld_volatile(&st->n_ctx);
   const int n_pooled = ld_volatile(&st->n_pooled);
   // tokens the (last) query sees; the decode step's token is appended by this kernel
@@ -451,28 +482,28 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_
             ok = false;
             break;
           }
-          const int rows = min(128, n_rows - t * 128);
-          unsigned char* dst = sA + size_t(s) * S::TILE_BYTES;
-          if (rows == 128) {  // whole tile: one 128-row box per 64-column half
-            mbar_arrive_expect_tx(&full[s], uint32_t(S::TILE_BYTES));
-#pragma unroll
-            for (int j = 0; j < S::HALVES; ++j)
-              tma_load_2d(dst + j * S::HALF_BYTES, &map_tile, j * (128 / S::ESIZE), r0 + t * 128, &full[s]);
-          } else {            // ragged tail: 16-row boxes, at most 15 rows past the range
-            const int boxes = (rows + kBoxRows - 1) / kBoxRows;
-            mbar_arrive_expect_tx(&full[s], uint32_t(boxes * kBoxRows * 128 * S::HALVES));
-#pragma unroll
-            for (int j = 0; j < S::HALVES; ++j)
-              for (int b = 0; b < boxes; ++b)
-                tma_load_2d(dst + j * S::HALF_BYTES + b * kBoxRows * 128, &map_box, j * (128 / S::ESIZE),
-                            r0 + t * 128 + b * kBoxRows, &full[s]);
+          if (t == 0 && spec_issued) {
+            spec_done = true;
+            if (!mbar_wait(spec_bar, 0)) {  // the early tile has landed, whatever its rows
+              ok = false;
+              break;
+            }
+            if (spec_r0 == r0 && spec_r1 == r0 + n_rows) {  // the hinted range was right
+              mbar_arrive(&full[0]);
+              QSA_TL(st, kTlScan2, 3);
+              ++issued;
+              continue;
+            }
           }
+          issue_tile(s, r0 + t * 128, min(128, n_rows - t * 128), &full[s]);
           if (t == 0) QSA_TL(st, kTlScan2, 3);  // first tile's loads issued
           ++issued;
         }
         if (!ok) record_status(st, QSA_ERR_TIMEOUT);
         // every fill this thread started must land before the CTA's shared memory is released
         for (int t = max(0, issued - kStages); t < issued; ++t) mbar_wait(&full[t % kStages], (t / kStages) & 1);
+        if (spec_issued && !spec_done) mbar_wait(spec_bar, 0);
+        spec_done = true;
       }
     } else if (warp == 5) {
       // ---------------- MMA issuer ----------------
@@ -597,6 +628,7 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap map_tile, const __grid_
       }
     }
   }
+  if (spec_issued && !spec_done) mbar_wait(spec_bar, 0);  // no tiles here: the early tile lands first
   tc_fence_before();
   __syncthreads();
   if (threadIdx.x == 0) QSA_TL(st, kTlScan3, 1);  // every warp done
