@@ -33,3 +33,31 @@ def test_stage_bytes_fp8_rows_carry_their_scale():
 def test_measured_peaks_have_a_source():
     peak, src = bench.measured_peaks()
     assert peak > 1000 and isinstance(src, str) and src
+
+
+def test_stage_bytes_8bit_pooled_keys_carry_their_scale():
+    wl = synth.workload("ctx256k_12l")
+    n = 255_182
+    B = n // 4
+    b8 = bench.stage_bytes(wl, n, pooled_fp8=True)
+    # every pooled row once as d code bytes plus its f32 scale, the scores out, the query in
+    assert b8["index_scan"] == B * (128 + 4) + B * 4 + 16 * (128 * 2 + 4)
+    assert b8["sparse_attend"] == bench.stage_bytes(wl, n)["sparse_attend"]   # attention unchanged
+
+
+def test_ncu_traffic_is_tied_to_the_sources(tmp_path, monkeypatch):
+    """The counters file's traffic is reported only while the hash of the kernel's sources
+    matches; an edited source makes it null."""
+    import json
+    src = tmp_path / "k.cu"
+    src.write_text("kernel v1")
+    import hashlib
+    h = hashlib.sha256(b"kernel v1").hexdigest()
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "profiles" / "ncu_counters.json").write_text(json.dumps(
+        {"kernels": {"index_scan": {"sources": ["k.cu"], "dram_bytes": 123, "sources_sha256": h}}}))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.ncu_traffic("index_scan") == 123
+    src.write_text("kernel v2")
+    assert bench.ncu_traffic("index_scan") is None
+    assert bench.ncu_traffic("block_topk") is None
