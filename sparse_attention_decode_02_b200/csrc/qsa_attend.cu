@@ -337,7 +337,9 @@ __device__ __forceinline__ void cp_async_commit_wait_all() {
 // Warp-level tensor-core helpers (f16 inputs, f32 accumulation). The contractions here
 // are tiny (8 query heads x ~129 cells per CTA), below the 64/128-row tiles of tcgen05,
 // so the warp-synchronous m16n8k16 form is used; it keeps the logits and P.V off the
-// CUDA cores, whose issue rate bounded this kernel.
+// CUDA cores, whose issue rate bounded this kernel. Both products are taken transposed
+// (cells, resp. output dims, as the 16 MMA rows and the query heads as the 8 columns),
+// so that no MMA row is padding.
 __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                           uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -355,9 +357,9 @@ __device__ __forceinline__ void ldsm_x2(uint32_t (&r)[2], const void* p) {
                : "=r"(r[0]), "=r"(r[1])
                : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(p))));
 }
-__device__ __forceinline__ void ldsm_x2_trans(uint32_t (&r)[2], const void* p) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];"
-               : "=r"(r[0]), "=r"(r[1])
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
                : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(p))));
 }
 
@@ -381,7 +383,9 @@ struct AcSmem {
   __host__ __device__ static int per(int cs) { return (G * (D / 2) + cs - 1) / cs; }
   // inbox of this CTA's output slice: [cs source CTAs][per] float2
   __host__ __device__ static size_t in_off(int lc, int cs) { return (stage_off(lc) + size_t(cs) * G * 2 * 4 + 15) / 16 * 16; }
-  __host__ __device__ static size_t bytes(int lc, int cs) { return in_off(lc, cs) + size_t(cs) * per(cs) * 8; }
+  // the query rows of this KV head (8 rows, heads >= G zero), staged with the K/V rows
+  __host__ __device__ static size_t q_off(int lc, int cs) { return in_off(lc, cs) + size_t(cs) * per(cs) * 8; }
+  __host__ __device__ static size_t bytes(int lc, int cs) { return q_off(lc, cs) + size_t(8) * RS * 2; }
 };
 
 // FP8 (K/V cache in e4m3 with a per-row scale): each staged row is converted to f16 as
@@ -402,8 +406,10 @@ __device__ __forceinline__ uint4 fp8x16_to_half(uint4 codes, float scale, int ha
   return make_uint4(r[0], r[1], r[2], r[3]);
 }
 
+// The register cap keeps a CTA (512 threads) small enough to share an SM with a CTA of
+// the next layer's scan, which launches while this kernel runs.
 template <int D, int G, int CS, bool FROM_BLOCKS, bool FP8>
-__global__ void __launch_bounds__(kAcThreads, 1)
+__global__ void __maxnreg__(80)
 attn_cluster_kernel(DevState* st, const __half* __restrict__ q, const int32_t* __restrict__ ids,
                     const int32_t* __restrict__ n_ids, const void* __restrict__ kc_raw,
                     const void* __restrict__ vc_raw, float* __restrict__ out, int n_kv_heads, int cells_per_cta,
@@ -427,6 +433,7 @@ attn_cluster_kernel(DevState* st, const __half* __restrict__ q, const int32_t* _
   float* s_m = reinterpret_cast<float*>(smem + SM::ml_off(Lc));       // [G], then s_l [G]
   float* s_l = s_m + G;
   int* s_cell = reinterpret_cast<int*>(smem + SM::cell_off(Lc));
+  __half* sQ = reinterpret_cast<__half*>(smem + SM::q_off(Lc, CS));
   float* s_stage = reinterpret_cast<float*>(smem + SM::stage_off(Lc));  // [CS][G][2] merged (m, l)
 
   __shared__ uint64_t s_merge_bar;  // this CTA's slice: every CTA's partial has landed
@@ -449,187 +456,259 @@ attn_cluster_kernel(DevState* st, const __half* __restrict__ q, const int32_t* _
   pdl_launch_dependents();
   if (tid == 0) QSA_TL(st, kTlAttn, kTlEntry);
   cluster_arrive_relaxed();  // paired with cluster_wait() before the partials are pushed
-  pdl_wait();
-  if (tid == 0) QSA_TL(st, kTlAttn, kTlWait);
-  const int n_full = ld_volatile(&st->n_ctx);
-  const int c0 = rank * Lc;
-  // this thread's id, loaded in the same round trip as the counts (clamped into the id
-  // buffer, checked against the counts below)
-  int id_spec = 0;
-  if (tid < Lc) {
-    const int ci = c0 + tid;
-    id_spec = FROM_BLOCKS ? ids[min(ci / kBlock, k_blocks - 1)] : ids[min(ci, max_cells - 1)];
-  }
-  const int n_ids_v = *n_ids;
-  asm volatile("" ::"r"(id_spec), "r"(n_ids_v), "r"(n_full));  // keep the loads ahead of the branches
-  int n = n_full - n_back;  // tokens this query sees
-  if (n < 0) {
-    if (rank == 0 && tid == 0) record_status(st, QSA_ERR_STATE);
-    n = 0;
-  }
-  const int n_blocks = n / kBlock;
-  int total, ns = 0;
-  if constexpr (FROM_BLOCKS) {
-    ns = n_ids_v;
-    if (ns < 0 || ns > k_blocks) {
-      if (blockIdx.x == 0 && tid == 0) record_status(st, QSA_ERR_BAD_INDEX);
-      ns = ns < 0 ? 0 : k_blocks;
-    }
-    total = kBlock * ns + (n - kBlock * n_blocks);
-  } else {
-    total = n_ids_v;
-    if (total < 0 || total > max_cells) {
-      if (blockIdx.x == 0 && tid == 0) record_status(st, QSA_ERR_BAD_INDEX);
-      total = total < 0 ? 0 : max_cells;
-    }
-  }
-  const int cnt = max(0, min(Lc, total - c0));
-
-  for (int i = tid; i < LP; i += kAcThreads) {
-    int cell = -1;
-    if (i < cnt) {
-      const int ci = c0 + i;
+  // Two passes over the same code: pass 0 runs before the dependency wait with no cells
+  // (zero rows, nothing read from global memory, only this CTA's shared memory written),
+  // so that the instructions of the staging, logits and P.V phases are in the SM's
+  // instruction cache when pass 1 runs them on the selected cells. The pass number goes
+  // through a register move the compiler cannot see into, so that it keeps one copy of
+  // the loop body instead of peeling the first pass.
+#ifdef QSA_TIMELINE
+  long long cyc0 = 0;  // clock64 deltas from the cells known, min..max over the CTAs
+#define QSA_ACYC(pt) if (tid == 0) QSA_TL_VALUE(st, kTlAttnCyc, pt, uint32_t(clock64() - cyc0))
+#else
+#define QSA_ACYC(pt) ((void)0)
+#endif
+#pragma unroll 1
+  for (int pass_i = 0; pass_i < 2; ++pass_i) {
+    int pass;
+    asm volatile("mov.b32 %0, %1;" : "=r"(pass) : "r"(pass_i));
+    const int c0 = rank * Lc;
+    int n = 0, n_blocks = 0, ns = 0, id_spec = 0, cnt = 0;
+    if (pass) {
+      pdl_wait();
+      if (tid == 0) QSA_TL(st, kTlAttn, kTlWait);
+      const int n_full = ld_volatile(&st->n_ctx);
+      // this thread's id, loaded in the same round trip as the counts (clamped into the
+      // id buffer, checked against the counts below)
+      if (tid < Lc) {
+        const int ci = c0 + tid;
+        id_spec = FROM_BLOCKS ? ids[min(ci / kBlock, k_blocks - 1)] : ids[min(ci, max_cells - 1)];
+      }
+      const int n_ids_v = *n_ids;
+      asm volatile("" ::"r"(id_spec), "r"(n_ids_v), "r"(n_full));  // keep the loads ahead of the branches
+      n = n_full - n_back;  // tokens this query sees
+      if (n < 0) {
+        if (rank == 0 && tid == 0) record_status(st, QSA_ERR_STATE);
+        n = 0;
+      }
+      n_blocks = n / kBlock;
+      int total;
       if constexpr (FROM_BLOCKS) {
-        if (ci < kBlock * ns) {
-          const int b = i == tid ? id_spec : ids[ci / kBlock];
-          cell = (b >= 0 && b < n_blocks) ? kBlock * b + ci % kBlock : -1;
-        } else {
-          cell = kBlock * n_blocks + (ci - kBlock * ns);
+        ns = n_ids_v;
+        if (ns < 0 || ns > k_blocks) {
+          if (blockIdx.x == 0 && tid == 0) record_status(st, QSA_ERR_BAD_INDEX);
+          ns = ns < 0 ? 0 : k_blocks;
         }
+        total = kBlock * ns + (n - kBlock * n_blocks);
       } else {
-        cell = i == tid ? id_spec : ids[ci];
+        total = n_ids_v;
+        if (total < 0 || total > max_cells) {
+          if (blockIdx.x == 0 && tid == 0) record_status(st, QSA_ERR_BAD_INDEX);
+          total = total < 0 ? 0 : max_cells;
+        }
       }
-      if (cell < 0 || cell >= n) {
-        record_status(st, QSA_ERR_BAD_INDEX);
-        cell = -1;
-      }
+      cnt = max(0, min(Lc, total - c0));
     }
-    s_cell[i] = cell;
-  }
-  __syncthreads();
-  if (tid == 0) QSA_TL(st, kTlAttn2, 0);  // cells known
-  // stage the selected K and V rows (rows of invalid or padding cells are zero-filled)
-  if constexpr (!FP8) {
-    for (int e = tid; e < LP * CH; e += kAcThreads) {
-      const int i = e / CH, ch = e % CH;
-      const int cell = s_cell[i];
-      const size_t off = cell >= 0 ? ((size_t(cell) * n_kv_heads + g) * D + ch * 8) : 0;
-      cp_async_16(sK + size_t(i) * RS + ch * 8, kc + off, cell >= 0 ? 16 : 0);
-      cp_async_16(sV + size_t(i) * RS + ch * 8, vc + off, cell >= 0 ? 16 : 0);
-    }
-  } else {
-    // 16 e4m3 codes per 16-byte load; a row is D/16 of them
-    constexpr int CH8 = D / 16;
-    const unsigned char* kc8 = static_cast<const unsigned char*>(kc_raw);
-    const unsigned char* vc8 = static_cast<const unsigned char*>(vc_raw);
-#pragma unroll 2
-    for (int e = tid; e < LP * CH8; e += kAcThreads) {
-      const int i = e / CH8, ch = e % CH8;
-      const int cell = s_cell[i];
-      uint4 kq = make_uint4(0u, 0u, 0u, 0u), vq = kq;
-      float2 sc = make_float2(0.0f, 0.0f);
-      if (cell >= 0) {
-        const size_t row = size_t(cell) * n_kv_heads + g;
-        kq = *reinterpret_cast<const uint4*>(kc8 + row * D + ch * 16);
-        vq = *reinterpret_cast<const uint4*>(vc8 + row * D + ch * 16);
-        sc = *reinterpret_cast<const float2*>(kv_scales + row * 2);
-      }
-      __half* kd = sK + size_t(i) * RS + ch * 16;
-      __half* vd = sV + size_t(i) * RS + ch * 16;
-      *reinterpret_cast<uint4*>(kd) = fp8x16_to_half(kq, sc.x, 0);
-      *reinterpret_cast<uint4*>(kd + 8) = fp8x16_to_half(kq, sc.x, 1);
-      *reinterpret_cast<uint4*>(vd) = fp8x16_to_half(vq, sc.y, 0);
-      *reinterpret_cast<uint4*>(vd + 8) = fp8x16_to_half(vq, sc.y, 1);
-    }
-  }
-  // query fragments (A operand, rows = the G heads of KV head g, rows >= G zero)
-  uint32_t qa[KSTEPS][2];
-#pragma unroll
-  for (int ks = 0; ks < KSTEPS; ++ks) {
-    qa[ks][0] = qa[ks][1] = 0u;
-    if (gq < G) {
-      const __half* qr = q + (size_t(g) * G + gq) * D + ks * 16 + 2 * tq;
-      qa[ks][0] = *reinterpret_cast<const uint32_t*>(qr);
-      qa[ks][1] = *reinterpret_cast<const uint32_t*>(qr + 8);
-    }
-  }
-  cp_async_commit_wait_all();
-  __syncthreads();
-  if (tid == 0) QSA_TL(st, kTlAttn, kTlA);  // rows staged
 
-  // ---- logits = Q K^T: warp w takes 8-cell tiles w and w + 16 ----
-  const float scale = 1.0f / sqrtf((float)D);
-  const int NT = LP / 8;  // <= 32
-  float lg[2][2];
-  float rmax = -INFINITY;
+    for (int i = tid; i < LP; i += kAcThreads) {
+      int cell = -1;
+      if (i < cnt) {
+        const int ci = c0 + i;
+        if constexpr (FROM_BLOCKS) {
+          if (ci < kBlock * ns) {
+            const int b = i == tid ? id_spec : ids[ci / kBlock];
+            cell = (b >= 0 && b < n_blocks) ? kBlock * b + ci % kBlock : -1;
+          } else {
+            cell = kBlock * n_blocks + (ci - kBlock * ns);
+          }
+        } else {
+          cell = i == tid ? id_spec : ids[ci];
+        }
+        if (cell < 0 || cell >= n) {
+          record_status(st, QSA_ERR_BAD_INDEX);
+          cell = -1;
+        }
+      }
+      s_cell[i] = cell;
+    }
+    __syncthreads();
+    if (pass && tid == 0) QSA_TL(st, kTlAttn2, 0);  // cells known
+#ifdef QSA_TIMELINE
+    cyc0 = clock64();
+#endif
+    // stage the selected K and V rows (rows of invalid or padding cells are zero-filled)
+    if constexpr (!FP8) {
+      for (int e = tid; e < LP * CH; e += kAcThreads) {
+        const int i = e / CH, ch = e % CH;
+        const int cell = s_cell[i];
+        const size_t off = cell >= 0 ? ((size_t(cell) * n_kv_heads + g) * D + ch * 8) : 0;
+        cp_async_16(sK + size_t(i) * RS + ch * 8, kc + off, cell >= 0 ? 16 : 0);
+        cp_async_16(sV + size_t(i) * RS + ch * 8, vc + off, cell >= 0 ? 16 : 0);
+      }
+    } else {
+      // 16 e4m3 codes per 16-byte load; a row is D/16 of them
+      constexpr int CH8 = D / 16;
+      const unsigned char* kc8 = static_cast<const unsigned char*>(kc_raw);
+      const unsigned char* vc8 = static_cast<const unsigned char*>(vc_raw);
+#pragma unroll 2
+      for (int e = tid; e < LP * CH8; e += kAcThreads) {
+        const int i = e / CH8, ch = e % CH8;
+        const int cell = s_cell[i];
+        uint4 kq = make_uint4(0u, 0u, 0u, 0u), vq = kq;
+        float2 sc = make_float2(0.0f, 0.0f);
+        if (cell >= 0) {
+          const size_t row = size_t(cell) * n_kv_heads + g;
+          kq = *reinterpret_cast<const uint4*>(kc8 + row * D + ch * 16);
+          vq = *reinterpret_cast<const uint4*>(vc8 + row * D + ch * 16);
+          sc = *reinterpret_cast<const float2*>(kv_scales + row * 2);
+        }
+        __half* kd = sK + size_t(i) * RS + ch * 16;
+        __half* vd = sV + size_t(i) * RS + ch * 16;
+        *reinterpret_cast<uint4*>(kd) = fp8x16_to_half(kq, sc.x, 0);
+        *reinterpret_cast<uint4*>(kd + 8) = fp8x16_to_half(kq, sc.x, 1);
+        *reinterpret_cast<uint4*>(vd) = fp8x16_to_half(vq, sc.y, 0);
+        *reinterpret_cast<uint4*>(vd + 8) = fp8x16_to_half(vq, sc.y, 1);
+      }
+    }
+    // the query rows of KV head g in the same copy group (rows >= G zero-filled), so that
+    // they arrive with the K/V rows instead of after them
+    for (int e = tid; e < 8 * CH; e += kAcThreads) {
+      const int h = e / CH, ch = e % CH;
+      const bool ok = pass && h < G;
+      cp_async_16(sQ + h * RS + ch * 8, q + (ok ? (size_t(g) * G + h) * D + ch * 8 : 0), ok ? 16 : 0);
+    }
+    cp_async_commit_wait_all();
+    __syncthreads();
+    if (pass && tid == 0) QSA_TL(st, kTlAttn, kTlA);  // rows staged
+    if (pass) QSA_ACYC(0);
+
+    // ---- logits^T = K q^T: warp w takes cells [16w, 16w+16) as the 16 MMA rows, the
+    //      query heads are the 8 columns, so no MMA row is padding. Lane (gq, tq) holds
+    //      cells 16w+gq and 16w+gq+8 for heads 2tq and 2tq+1. ----
+    const float scale = 1.0f / sqrtf((float)D);
+    const int MT = LP / 16;  // <= 16 cell tiles
+    float lg[2][2];          // [cell gq, gq + 8][head 2tq, 2tq + 1]
+    float rmax[2] = {-INFINITY, -INFINITY};
 #pragma unroll
-  for (int tt = 0; tt < 2; ++tt) {
-    lg[tt][0] = lg[tt][1] = -INFINITY;
-    const int nt = warp + 16 * tt;
-    if (nt >= NT) continue;  // warp-uniform
-    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    const __half* kb = sK + size_t(nt * 8 + (lane & 7)) * RS + (lane >> 3) * 8;
+    for (int r = 0; r < 2; ++r) lg[r][0] = lg[r][1] = -INFINITY;
+    if (warp < MT) {  // warp-uniform
+      // B fragments (column n = query head n): two k-steps per ldmatrix.x4 of the query rows
+      uint32_t qb[KSTEPS][2];
+      const __half* qrow = sQ + size_t(lane & 7) * RS + (lane >> 3) * 8;
 #pragma unroll
-    for (int ks = 0; ks < KSTEPS; ks += 2) {
-      uint32_t b[4];
-      ldsm_x4(b, kb + ks * 16);  // cells nt*8.., dims ks*16 + {0,8,16,24}..
-      mma_16816(acc, qa[ks][0], 0u, qa[ks][1], 0u, b[0], b[1]);
-      mma_16816(acc, qa[ks + 1][0], 0u, qa[ks + 1][1], 0u, b[2], b[3]);
+      for (int ks = 0; ks < KSTEPS; ks += 2) {
+        uint32_t t[4];
+        ldsm_x4(t, qrow + ks * 16);  // heads 0..7, dims ks*16 + {0..7, 8..15, 16..23, 24..31}
+        qb[ks][0] = t[0];
+        qb[ks][1] = t[1];
+        qb[ks + 1][0] = t[2];
+        qb[ks + 1][1] = t[3];
+      }
+      // two accumulators (even and odd k-steps) halve the dependent MMA chain
+      float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f}, acc1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      const __half* ka = sK + size_t(warp * 16 + (lane & 15)) * RS + (lane >> 4) * 8;
+#pragma unroll
+      for (int ks = 0; ks < KSTEPS; ks += 2) {
+        uint32_t a[4], a1[4];
+        ldsm_x4(a, ka + ks * 16);  // cells 16w + {0..7, 8..15}, dims ks*16 + {0..7, 8..15}
+        ldsm_x4(a1, ka + ks * 16 + 16);
+        mma_16816(acc, a[0], a[1], a[2], a[3], qb[ks][0], qb[ks][1]);
+        mma_16816(acc1, a1[0], a1[1], a1[2], a1[3], qb[ks + 1][0], qb[ks + 1][1]);
+      }
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[c] += acc1[c];
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int i = warp * 16 + gq + 8 * r;
+        const bool valid = i < cnt && s_cell[i] >= 0;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          lg[r][c] = (valid && 2 * tq + c < G) ? acc[2 * r + c] * scale : -INFINITY;
+          rmax[c] = fmaxf(rmax[c], lg[r][c]);
+        }
+      }
     }
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
-      const int i = nt * 8 + 2 * tq + c;
-      lg[tt][c] = (i < cnt && s_cell[i] >= 0) ? acc[c] * scale : -INFINITY;
-      rmax = fmaxf(rmax, lg[tt][c]);
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) rmax[c] = fmaxf(rmax[c], __shfl_xor_sync(0xffffffffu, rmax[c], off));
     }
-  }
-  rmax = fmaxf(rmax, __shfl_xor_sync(0xffffffffu, rmax, 1));
-  rmax = fmaxf(rmax, __shfl_xor_sync(0xffffffffu, rmax, 2));
-  if (tq == 0) s_rmax[warp * 8 + gq] = rmax;
-  __syncthreads();
-  if (tid == 0) QSA_TL(st, kTlAttn2, 1);  // logits done
-  float m = -INFINITY;
-#pragma unroll
-  for (int w = 0; w < 16; ++w) m = fmaxf(m, s_rmax[w * 8 + gq]);
-  // probabilities, rounded to f16 for the P.V product; the row sums use the rounded values
-  float psum = 0.0f;
-#pragma unroll
-  for (int tt = 0; tt < 2; ++tt) {
-    const int nt = warp + 16 * tt;
-    if (nt >= NT) continue;
-    const float p0 = m == -INFINITY ? 0.0f : expf(lg[tt][0] - m);
-    const float p1 = m == -INFINITY ? 0.0f : expf(lg[tt][1] - m);
-    const __half2 h = __floats2half2_rn(p0, p1);
-    *reinterpret_cast<__half2*>(sP + size_t(gq) * PS + nt * 8 + 2 * tq) = h;
-    const float2 r = __half22float2(h);
-    psum += r.x + r.y;
-  }
-  psum += __shfl_xor_sync(0xffffffffu, psum, 1);
-  psum += __shfl_xor_sync(0xffffffffu, psum, 2);
-  if (tq == 0) s_rsum[warp * 8 + gq] = psum;
-  __syncthreads();
-  if (tid < G) {
-    float mm = -INFINITY, ll = 0.0f;
+    if (gq == 0) *reinterpret_cast<float2*>(s_rmax + warp * 8 + 2 * tq) = make_float2(rmax[0], rmax[1]);
+    __syncthreads();
+    if (pass && tid == 0) QSA_TL(st, kTlAttn2, 1);  // logits done
+    if (pass) QSA_ACYC(1);
+    float m[2] = {-INFINITY, -INFINITY};
 #pragma unroll
     for (int w = 0; w < 16; ++w) {
-      mm = fmaxf(mm, s_rmax[w * 8 + tid]);
-      ll += s_rsum[w * 8 + tid];
+      const float2 mw = *reinterpret_cast<const float2*>(s_rmax + w * 8 + 2 * tq);
+      m[0] = fmaxf(m[0], mw.x);
+      m[1] = fmaxf(m[1], mw.y);
     }
-    s_m[tid] = mm;
-    s_l[tid] = ll;
-  }
-  // ---- unnormalised P.V: warp w takes output dims [8w, 8w+8), all cells ----
-  if (warp < D / 8) {
-    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    const __half* pb = sP + size_t(lane & 7) * PS + ((lane >> 3) & 1) * 8;
-    const __half* vb = sV + size_t((lane & 7) + ((lane >> 3) & 1) * 8) * RS + warp * 8;
-    for (int kc16 = 0; kc16 < LP / 16; ++kc16) {
-      uint32_t a[2], b[2];
-      ldsm_x2(a, pb + kc16 * 16);                     // P rows 0..7, cells kc16*16 + {0..7, 8..15}
-      ldsm_x2_trans(b, vb + size_t(kc16) * 16 * RS);  // V cells kc16*16 + {0..7, 8..15}, dims 8w..8w+7
-      mma_16816(acc, a[0], 0u, a[1], 0u, b[0], b[1]);
+    // probabilities, rounded to f16 for the P.V product (P stored head-major, [head][cell]);
+    // the row sums use the rounded values
+    float psum[2] = {0.0f, 0.0f};
+    if (warp < MT) {
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const __half h = __float2half_rn(m[c] == -INFINITY ? 0.0f : expf(lg[r][c] - m[c]));
+          sP[size_t(2 * tq + c) * PS + warp * 16 + gq + 8 * r] = h;
+          psum[c] += __half2float(h);
+        }
+      }
     }
-    if (gq < G) *reinterpret_cast<float2*>(s_o + gq * D + warp * 8 + 2 * tq) = make_float2(acc[0], acc[1]);
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) psum[c] += __shfl_xor_sync(0xffffffffu, psum[c], off);
+    }
+    if (gq == 0) *reinterpret_cast<float2*>(s_rsum + warp * 8 + 2 * tq) = make_float2(psum[0], psum[1]);
+    __syncthreads();
+    if (tid < G) {
+      float mm = -INFINITY, ll = 0.0f;
+#pragma unroll
+      for (int w = 0; w < 16; ++w) {
+        mm = fmaxf(mm, s_rmax[w * 8 + tid]);
+        ll += s_rsum[w * 8 + tid];
+      }
+      s_m[tid] = mm;
+      s_l[tid] = ll;
+    }
+    // ---- unnormalised O^T = V^T P^T: warp w takes output dims [16w, 16w+16) as the 16
+    //      MMA rows (V^T tiles by transposing loads of the cell-major rows), the heads are
+    //      the 8 columns; all cells in 16-cell steps ----
+    if (warp < D / 16) {
+      float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f}, acc1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      const __half* va = sV + size_t((lane & 7) + ((lane >> 4) & 1) * 8) * RS + warp * 16 + ((lane >> 3) & 1) * 8;
+      const __half* pb = sP + size_t(lane & 7) * PS + (lane >> 3) * 8;
+      int kc16 = 0;
+      for (; kc16 + 1 < MT; kc16 += 2) {  // two accumulators (even and odd cell tiles)
+        uint32_t a[4], a1[4], b[4];
+        ldsm_x4_trans(a, va + size_t(kc16) * 16 * RS);  // V cells kc16*16 + {0..7, 8..15}, dims 16w + {0..7, 8..15}
+        ldsm_x4_trans(a1, va + size_t(kc16 + 1) * 16 * RS);
+        ldsm_x4(b, pb + kc16 * 16);                       // P heads 0..7, cells kc16*16 + {0..7, ..., 24..31}
+        mma_16816(acc, a[0], a[1], a[2], a[3], b[0], b[1]);
+        mma_16816(acc1, a1[0], a1[1], a1[2], a1[3], b[2], b[3]);
+      }
+      if (kc16 < MT) {
+        uint32_t a[4], b[2];
+        ldsm_x4_trans(a, va + size_t(kc16) * 16 * RS);
+        ldsm_x2(b, pb + kc16 * 16);
+        mma_16816(acc, a[0], a[1], a[2], a[3], b[0], b[1]);
+      }
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[c] += acc1[c];
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+          if (2 * tq + c < G) s_o[(2 * tq + c) * D + warp * 16 + gq + 8 * r] = acc[2 * r + c];
+      }
+    }
+    __syncthreads();  // s_o, s_m and s_l are complete (and pass 0's readers are done)
+    if (pass && tid == 0) QSA_TL(st, kTlAttn2, 2);  // P.V done
+    if (pass) QSA_ACYC(2);
   }
   // ---- merge: CTA r owns output pairs [r*PER, (r+1)*PER) (2 dims of one head each).
   //      Every CTA sends its (max, sum) per head and its partial of each slice into the
@@ -641,8 +720,6 @@ attn_cluster_kernel(DevState* st, const __half* __restrict__ q, const int32_t* _
   constexpr int PAIRS = G * (D / 2);
   constexpr int PER = (PAIRS + CS - 1) / CS;
   float2* s_in = reinterpret_cast<float2*>(smem + SM::in_off(Lc, CS));  // [CS][PER]
-  __syncthreads();  // s_o, s_m and s_l are complete
-  if (tid == 0) QSA_TL(st, kTlAttn2, 2);  // P.V done
   cluster_wait();   // every CTA of the cluster has started: its shared memory may be written
   if (tid == 0) QSA_TL(st, kTlAttn2, 3);
   for (int pidx = tid; pidx < PAIRS; pidx += kAcThreads) {
@@ -665,6 +742,7 @@ attn_cluster_kernel(DevState* st, const __half* __restrict__ q, const int32_t* _
   }
   cluster_arrive_relaxed();  // this CTA's data is all here; paired with the wait before exit
   if (tid == 0) QSA_TL(st, kTlAttn, kTlB);
+  QSA_ACYC(3);
   // CS lanes per output pair, lane r merging source CTA r's partial; shuffles within the
   // aligned CS-lane group combine them (max, then the weighted sums)
   static_assert(PAIRS % CS == 0 && (PER * CS) % 32 == 0 && 32 % CS == 0, "whole warps, aligned lane groups");
@@ -696,6 +774,8 @@ attn_cluster_kernel(DevState* st, const __half* __restrict__ q, const int32_t* _
   }
   cluster_wait();  // every CTA holds its data: nothing is still arriving anywhere
   if (tid == 0) QSA_TL(st, kTlAttn, kTlExit);
+  QSA_ACYC(4);
+#undef QSA_ACYC
 }
 
 template <int D, int G, int CS, bool FB, bool FP8>

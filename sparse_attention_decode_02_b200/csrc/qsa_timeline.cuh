@@ -12,7 +12,7 @@
 
 namespace qsa {
 
-enum { kTlScan = 0, kTlTopk = 1, kTlAttn = 2, kTlTopk2 = 3, kTlAttn2 = 4, kTlScan2 = 5, kTlCycles = 6, kTlTopk3 = 7, kTlScan3 = 8 };
+enum { kTlScan = 0, kTlTopk = 1, kTlAttn = 2, kTlTopk2 = 3, kTlAttn2 = 4, kTlScan2 = 5, kTlCycles = 6, kTlTopk3 = 7, kTlScan3 = 8, kTlAttnCyc = 9 };
 enum { kTlEntry = 0, kTlWait = 1, kTlA = 2, kTlB = 3, kTlExit = 4 };
 
 #ifdef QSA_TIMELINE
