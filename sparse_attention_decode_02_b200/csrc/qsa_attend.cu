@@ -453,7 +453,6 @@ attn_cluster_kernel(DevState* st, const __half* __restrict__ q, const int32_t* _
     sm100::mbar_init(&s_merge_bar, CS);
     sm100::fence_mbar_init();
   }
-  pdl_launch_dependents();
   if (tid == 0) QSA_TL(st, kTlAttn, kTlEntry);
   cluster_arrive_relaxed();  // paired with cluster_wait() before the partials are pushed
   // Two passes over the same code: pass 0 runs before the dependency wait with no cells
@@ -476,6 +475,10 @@ attn_cluster_kernel(DevState* st, const __half* __restrict__ q, const int32_t* _
     int n = 0, n_blocks = 0, ns = 0, id_spec = 0, cnt = 0;
     if (pass) {
       pdl_wait();
+      // the next kernel (in the decode step, the next layer's scan, whose prologue and L2
+      // prefetch of the pooled keys are heavy) launches now, beside this kernel's own
+      // loads and math, rather than while the selection before it runs
+      pdl_launch_dependents();
       if (tid == 0) QSA_TL(st, kTlAttn, kTlWait);
       const int n_full = ld_volatile(&st->n_ctx);
       // this thread's id, loaded in the same round trip as the counts (clamped into the
