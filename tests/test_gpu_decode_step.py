@@ -214,3 +214,83 @@ def test_early_inputs_give_identical_results(wl_name, kw):
         if step % 2:
             assert torch.equal(ga.scores, gb.scores), f"step {step}: scores"
         assert ga.state() == gb.state() == (n0 + step + 1, (n0 + step + 1) // 4, 0)
+
+
+def _layers(wl, n0, n_layers, extra=16, **cfg_kw):
+    import sparse_attention_decode_02_b200 as Q
+    qsa = Q.Qsa(H.config_of(wl, max_ctx=(n0 + extra + 3) // 4 * 4, n_layers=n_layers, **cfg_kw))
+    gs = []
+    for layer in range(n_layers):
+        g = H.GpuLayer(qsa, layer)
+        pre = synth.prefill_tokens(wl, layer, n0)
+        g.append(pre["k"], pre["v"], pre["idx"])
+        g.update()
+        gs.append(g)
+    return qsa, gs
+
+
+def _decode_step_layer(qsa, g, st):
+    d = {k: H.to_dev(x) for k, x in st.items()}
+    qsa.decode_step(g.layer, d["k"], d["v"], d["idx"], d["q_idx"], d["w"], d["q"], g.outs["sel"],
+                    g.outs["n_sel"], g.outs["out"])
+
+
+def test_back_to_back_layers_equal_synchronised_steps():
+    """Steps of three layers enqueued back to back (each layer's kernels launching while
+    the previous layer's still run, and preparing their inputs and prefetches before their
+    dependency waits) equal the same steps with a synchronisation after every call, bit
+    for bit, over block completions."""
+    wl = synth.workload("ctx64k")
+    n0, L = 8190, 3
+    qa, ga = _layers(wl, n0, L, early_inputs=1)
+    qb, gb = _layers(wl, n0, L, early_inputs=1)
+    for step in range(7):
+        sts = [synth.step_inputs(wl, layer, step) for layer in range(L)]
+        ins = [{k: H.to_dev(x) for k, x in st.items()} for st in sts]  # copied before the steps
+        torch.cuda.synchronize()
+        for layer in range(L):
+            d = ins[layer]
+            qa.decode_step(layer, d["k"], d["v"], d["idx"], d["q_idx"], d["w"], d["q"], ga[layer].outs["sel"],
+                           ga[layer].outs["n_sel"], ga[layer].outs["out"])
+        torch.cuda.synchronize()
+        for layer in range(L):
+            _decode_step_layer(qb, gb[layer], sts[layer])
+            torch.cuda.synchronize()
+        for layer in range(L):
+            a, b = ga[layer].outs, gb[layer].outs
+            na, nb = int(a["n_sel"][0]), int(b["n_sel"][0])
+            assert na == nb == wl.k_blocks
+            assert torch.equal(a["sel"][:na], b["sel"][:nb]), f"step {step} layer {layer}: selection"
+            assert torch.equal(a["out"], b["out"]), f"step {step} layer {layer}: attention output"
+            assert ga[layer].state() == gb[layer].state() == (n0 + step + 1, (n0 + step + 1) // 4, 0)
+
+
+def test_pooled_rewrite_right_before_a_step_is_seen():
+    """A pooled update enqueued right before a decode step (no synchronisation) rewrites
+    rows that the step's scan reads: the scan sees the rewritten rows, not the ones before.
+    The rows are first overwritten with a large value, so a read of them before the update
+    completed would change the selection."""
+    wl = synth.workload("ctx64k")
+    n0 = 8193
+    qa, ga, _ = _layer(wl, n0, extra=24, early_inputs=1)
+    qb, gb, _ = _layer(wl, n0, extra=24, early_inputs=1)
+    ga.update()
+    gb.update()
+    for step in range(3):
+        st = synth.step_inputs(wl, 0, step)
+        _decode_step(qa, ga, st)
+        _decode_step(qb, gb, st)
+    torch.cuda.synchronize()
+    n = n0 + 3
+    ga.buf["pooled_cache"].view(torch.int16)[: n // 4].fill_(0x7BFF)  # f16 65504
+    qa.invalidate_pooled_cache(0, 0)
+    ga.update()
+    st = synth.step_inputs(wl, 0, 3)
+    _decode_step(qa, ga, st)  # enqueued right behind the update
+    _decode_step(qb, gb, st)
+    torch.cuda.synchronize()
+    na, nb = int(ga.outs["n_sel"][0]), int(gb.outs["n_sel"][0])
+    assert na == nb
+    assert torch.equal(ga.outs["sel"][:na], gb.outs["sel"][:nb])
+    assert torch.equal(ga.outs["out"], gb.outs["out"])
+    np.testing.assert_array_equal(ga.pooled_rows(0, (n + 1) // 4), gb.pooled_rows(0, (n + 1) // 4))
