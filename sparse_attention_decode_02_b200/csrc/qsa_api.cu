@@ -480,7 +480,8 @@ qsa_status qsa_decode_step(qsa_ctx* ctx, int32_t layer, const void* k, const voi
   if (qsa_status st = ctx->cuda(launch_topk(lv, lv.scores, sel_blocks, n_sel, s, 1, 0, lv.hist, nullptr, 0, fused),
                                 "decode_step: block top-k"))
     return st;
-  return ctx->cuda(launch_attend_selected(lv, q, sel_blocks, n_sel, out, s), "decode_step: sparse attend");
+  return ctx->cuda(launch_attend_selected(lv, q, sel_blocks, n_sel, out, s, 1, nullptr, true),
+                   "decode_step: sparse attend");
 }
 
 qsa_status qsa_rollback(qsa_ctx* ctx, int32_t layer, int32_t n_keep, qsa_stream_t stream) {

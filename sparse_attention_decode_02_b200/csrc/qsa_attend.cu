@@ -413,14 +413,15 @@ __global__ void __maxnreg__(80)
 attn_cluster_kernel(DevState* st, const __half* __restrict__ q, const int32_t* __restrict__ ids,
                     const int32_t* __restrict__ n_ids, const void* __restrict__ kc_raw,
                     const void* __restrict__ vc_raw, float* __restrict__ out, int n_kv_heads, int cells_per_cta,
-                    int max_cells, int k_blocks, const float* __restrict__ kv_scales, float* __restrict__ lse_out) {
+                    int max_cells, int k_blocks, const float* __restrict__ kv_scales, float* __restrict__ lse_out,
+                    int warm) {
   const __half* __restrict__ kc = static_cast<const __half*>(kc_raw);
   const __half* __restrict__ vc = static_cast<const __half*>(vc_raw);
   using SM = AcSmem<D, G>;
   constexpr int RS = SM::RS;
   constexpr int KSTEPS = D / 16;
   constexpr int CH = D * 2 / 16;  // 16-byte chunks per row
-  static_assert(G <= 8, "the 8 rows of the MMA hold the query heads of one KV head");
+  static_assert(G <= 8, "the 8 MMA columns hold the query heads of one KV head");
   extern __shared__ __align__(16) unsigned char smem[];
   const int Lc = cells_per_cta;
   const int LP = SM::lp(Lc), PS = SM::ps(Lc);
@@ -455,12 +456,13 @@ attn_cluster_kernel(DevState* st, const __half* __restrict__ q, const int32_t* _
   }
   if (tid == 0) QSA_TL(st, kTlAttn, kTlEntry);
   cluster_arrive_relaxed();  // paired with cluster_wait() before the partials are pushed
-  // Two passes over the same code: pass 0 runs before the dependency wait with no cells
-  // (zero rows, nothing read from global memory, only this CTA's shared memory written),
-  // so that the instructions of the staging, logits and P.V phases are in the SM's
-  // instruction cache when pass 1 runs them on the selected cells. The pass number goes
-  // through a register move the compiler cannot see into, so that it keeps one copy of
-  // the loop body instead of peeling the first pass.
+  // With `warm` (the decode step, where this kernel launches while the selection still
+  // runs): two passes over the same code. Pass 0 runs before the dependency wait with no
+  // cells (zero rows, nothing read from global memory, only this CTA's shared memory
+  // written), so that the instructions of the staging, logits and P.V phases are in the
+  // SM's instruction cache when pass 1 runs them on the selected cells. The pass number
+  // goes through a register move the compiler cannot see into, so that it keeps one copy
+  // of the loop body instead of peeling the first pass.
 #ifdef QSA_TIMELINE
   long long cyc0 = 0;  // clock64 deltas from the cells known, min..max over the CTAs
 #define QSA_ACYC(pt) if (tid == 0) QSA_TL_VALUE(st, kTlAttnCyc, pt, uint32_t(clock64() - cyc0))
@@ -468,7 +470,7 @@ attn_cluster_kernel(DevState* st, const __half* __restrict__ q, const int32_t* _
 #define QSA_ACYC(pt) ((void)0)
 #endif
 #pragma unroll 1
-  for (int pass_i = 0; pass_i < 2; ++pass_i) {
+  for (int pass_i = warm ? 0 : 1; pass_i < 2; ++pass_i) {
     int pass;
     asm volatile("mov.b32 %0, %1;" : "=r"(pass) : "r"(pass_i));
     const int c0 = rank * Lc;
@@ -655,7 +657,12 @@ attn_cluster_kernel(DevState* st, const __half* __restrict__ q, const int32_t* _
       for (int r = 0; r < 2; ++r) {
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
-          const __half h = __float2half_rn(m[c] == -INFINITY ? 0.0f : expf(lg[r][c] - m[c]));
+          float p = 0.0f;  // exp(d) as 2^(d log2 e) on the MUFU unit (relative error ~2^-22)
+          if (m[c] != -INFINITY) {
+            const float x = (lg[r][c] - m[c]) * 1.4426950408889634f;
+            asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(p) : "f"(x));
+          }
+          const __half h = __float2half_rn(p);
           sP[size_t(2 * tq + c) * PS + warp * 16 + gq + 8 * r] = h;
           psum[c] += __half2float(h);
         }
@@ -668,15 +675,15 @@ attn_cluster_kernel(DevState* st, const __half* __restrict__ q, const int32_t* _
     }
     if (gq == 0) *reinterpret_cast<float2*>(s_rsum + warp * 8 + 2 * tq) = make_float2(psum[0], psum[1]);
     __syncthreads();
-    if (tid < G) {
+    if (warp == D / 16 && lane < G) {  // the heads' max and sum, on a warp without P.V work
       float mm = -INFINITY, ll = 0.0f;
 #pragma unroll
       for (int w = 0; w < 16; ++w) {
-        mm = fmaxf(mm, s_rmax[w * 8 + tid]);
-        ll += s_rsum[w * 8 + tid];
+        mm = fmaxf(mm, s_rmax[w * 8 + lane]);
+        ll += s_rsum[w * 8 + lane];
       }
-      s_m[tid] = mm;
-      s_l[tid] = ll;
+      s_m[lane] = mm;
+      s_l[lane] = ll;
     }
     // ---- unnormalised O^T = V^T P^T: warp w takes output dims [16w, 16w+16) as the 16
     //      MMA rows (V^T tiles by transposing loads of the cell-major rows), the heads are
@@ -802,7 +809,7 @@ static cudaError_t set_ac_attr(size_t smem) {
 
 template <int D, int G, int CS>
 static cudaError_t launch_ac(const LayerView& L, bool from_blocks, const void* q, const int32_t* ids,
-                             const int32_t* n_ids, float* out, cudaStream_t s, int n_queries, float* lse) {
+                             const int32_t* n_ids, float* out, cudaStream_t s, int n_queries, float* lse, int warm) {
   const int lc = L.attn_cells_per_cta;
   const size_t smem = AcSmem<D, G>::bytes(lc, CS);
   const dim3 grid(L.cfg.n_kv_heads * CS, n_queries), block(kAcThreads);
@@ -811,7 +818,7 @@ static cudaError_t launch_ac(const LayerView& L, bool from_blocks, const void* q
   const float* scl = L.kv_scales;
 #define QSA_AC_LAUNCH(FB, F8)                                                                                    \
   launch_pdl(attn_cluster_kernel<D, G, CS, FB, F8>, grid, block, smem, s, CS, L.state, (const __half*)q, ids, n_ids, \
-             (const void*)L.k_cache, (const void*)L.v_cache, out, L.cfg.n_kv_heads, lc, mc, kb, scl, lse)
+             (const void*)L.k_cache, (const void*)L.v_cache, out, L.cfg.n_kv_heads, lc, mc, kb, scl, lse, warm)
   if (from_blocks) return fp8 ? QSA_AC_LAUNCH(true, true) : QSA_AC_LAUNCH(true, false);
   return fp8 ? QSA_AC_LAUNCH(false, true) : QSA_AC_LAUNCH(false, false);
 #undef QSA_AC_LAUNCH
@@ -819,33 +826,33 @@ static cudaError_t launch_ac(const LayerView& L, bool from_blocks, const void* q
 
 template <int D, int G>
 static cudaError_t launch_ac_g(const LayerView& L, bool fb, const void* q, const int32_t* ids, const int32_t* n_ids,
-                               float* out, cudaStream_t s, int nq, float* lse) {
-  return L.attn_cluster == 16 ? launch_ac<D, G, 16>(L, fb, q, ids, n_ids, out, s, nq, lse)
-                              : launch_ac<D, G, 8>(L, fb, q, ids, n_ids, out, s, nq, lse);
+                               float* out, cudaStream_t s, int nq, float* lse, int warm) {
+  return L.attn_cluster == 16 ? launch_ac<D, G, 16>(L, fb, q, ids, n_ids, out, s, nq, lse, warm)
+                              : launch_ac<D, G, 8>(L, fb, q, ids, n_ids, out, s, nq, lse, warm);
 }
 
 template <int D>
 static cudaError_t launch_ac_d(const LayerView& L, bool fb, const void* q, const int32_t* ids, const int32_t* n_ids,
-                               float* out, cudaStream_t s, int nq, float* lse) {
+                               float* out, cudaStream_t s, int nq, float* lse, int warm) {
   switch (L.cfg.n_q_heads / L.cfg.n_kv_heads) {
-    case 1: return launch_ac_g<D, 1>(L, fb, q, ids, n_ids, out, s, nq, lse);
-    case 2: return launch_ac_g<D, 2>(L, fb, q, ids, n_ids, out, s, nq, lse);
-    case 4: return launch_ac_g<D, 4>(L, fb, q, ids, n_ids, out, s, nq, lse);
-    case 8: return launch_ac_g<D, 8>(L, fb, q, ids, n_ids, out, s, nq, lse);
+    case 1: return launch_ac_g<D, 1>(L, fb, q, ids, n_ids, out, s, nq, lse, warm);
+    case 2: return launch_ac_g<D, 2>(L, fb, q, ids, n_ids, out, s, nq, lse, warm);
+    case 4: return launch_ac_g<D, 4>(L, fb, q, ids, n_ids, out, s, nq, lse, warm);
+    case 8: return launch_ac_g<D, 8>(L, fb, q, ids, n_ids, out, s, nq, lse, warm);
     default: return cudaErrorInvalidValue;
   }
 }
 
 cudaError_t launch_attend(const LayerView& L, const void* q, const int32_t* cells, const int32_t* n_cells, float* out,
                           cudaStream_t s) {
-  return L.cfg.head_dim == 128 ? launch_ac_d<128>(L, false, q, cells, n_cells, out, s, 1, nullptr)
-                               : launch_ac_d<64>(L, false, q, cells, n_cells, out, s, 1, nullptr);
+  return L.cfg.head_dim == 128 ? launch_ac_d<128>(L, false, q, cells, n_cells, out, s, 1, nullptr, 0)
+                               : launch_ac_d<64>(L, false, q, cells, n_cells, out, s, 1, nullptr, 0);
 }
 
 cudaError_t launch_attend_selected(const LayerView& L, const void* q, const int32_t* sel, const int32_t* n_sel,
-                                   float* out, cudaStream_t s, int n_queries, float* lse) {
-  return L.cfg.head_dim == 128 ? launch_ac_d<128>(L, true, q, sel, n_sel, out, s, n_queries, lse)
-                               : launch_ac_d<64>(L, true, q, sel, n_sel, out, s, n_queries, lse);
+                                   float* out, cudaStream_t s, int n_queries, float* lse, bool warm) {
+  return L.cfg.head_dim == 128 ? launch_ac_d<128>(L, true, q, sel, n_sel, out, s, n_queries, lse, warm)
+                               : launch_ac_d<64>(L, true, q, sel, n_sel, out, s, n_queries, lse, warm);
 }
 
 // Cluster size and cells per CTA for a configuration, plus the kernel attributes they

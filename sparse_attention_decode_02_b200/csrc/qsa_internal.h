@@ -157,9 +157,11 @@ cudaError_t launch_gather(const LayerView& L, const int32_t* sel, const int32_t*
 cudaError_t launch_attend(const LayerView& L, const void* q, const int32_t* cells,
                           const int32_t* n_cells, float* out, cudaStream_t s);
 // With lse (single query): also the log-sum-exp of each head's scaled logits over its cells.
+// warm: the kernel launches well before its inputs are ready (the decode step, behind the
+// selection) and runs its code once on no cells while it waits, to cache the instructions.
 cudaError_t launch_attend_selected(const LayerView& L, const void* q, const int32_t* sel,
                                    const int32_t* n_sel, float* out, cudaStream_t s, int n_queries = 1,
-                                   float* lse = nullptr);
+                                   float* lse = nullptr, bool warm = false);
 // context-parallel step (qsa_cp.cu)
 cudaError_t launch_cp_select(const float* cand_scores, const int32_t* cand_blocks, int n_shards, int k_blocks,
                              int32_t* sel, int32_t* n_sel, cudaStream_t s);
