@@ -64,6 +64,8 @@ def parse_args():
                     help="replays of one step timed alone for the median / p10 / p90")
     ap.add_argument("--profile-case", action="store_true",
                     help="small case for ncu: 1 layer at 256k, few steps, no extras")
+    ap.add_argument("--profile-pool", action="store_true",
+                    help="case for ncu of the bulk pooled rebuild: one 256k layer pooled again --steps times")
     return ap.parse_args()
 
 
@@ -750,6 +752,39 @@ def cpu_baseline(wl, budget_s=12.0, max_steps=400):
                       f"(numpy float64, {threads} BLAS threads)"}
 
 
+def profile_pool(wl, reps):
+    """One layer at the workload's context, its pooled cache rebuilt from the raw keys `reps`
+    times (qsa_invalidate_pooled_cache + qsa_update_pooled_cache), each timed alone; the
+    rebuilt cache must equal the first one bit for bit. Prints one JSON line."""
+    import torch
+
+    import synth
+    import sparse_attention_decode_02_b200 as Q
+    cfg = Q.make_config(1, int(math.ceil((wl.n_prefill + 8) / 4) * 4), wl.d_idx, wl.n_idx_heads, wl.top_k_tokens,
+                        wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.rope_base, wl.rms_eps)
+    qsa = Q.Qsa(cfg)
+    bufs = Q.alloc_layer(cfg)
+    qsa.bind_layer(0, **bufs)
+    pre = synth.device_prefill(wl, 0)
+    qsa.append_tokens(0, pre["k"], pre["v"], pre["idx"])
+    del pre
+    qsa.update_pooled_cache(0)
+    torch.cuda.synchronize()
+    first = bufs["pooled_cache"].clone()
+    stream = torch.cuda.current_stream()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    us = []
+    for _ in range(reps):
+        qsa.invalidate_pooled_cache(0, 0)
+        a.record(stream)
+        qsa.update_pooled_cache(0)
+        b.record(stream)
+        torch.cuda.synchronize()
+        us.append(round(1e3 * a.elapsed_time(b), 2))
+    assert torch.equal(bufs["pooled_cache"], first), "rebuilt pooled cache differs"
+    print(json.dumps({"profile_pool": {"workload": wl.name, "blocks": wl.n_prefill // 4, "us_per_rebuild": us}}))
+
+
 def main_ours(args):
     import torch
 
@@ -761,6 +796,10 @@ def main_ours(args):
     barrier(world)
     wl = synth.workload(args.workload)
     K, W = args.steps, args.warmup
+    if args.profile_pool:
+        if rank == 0:
+            profile_pool(wl, K)
+        return
     if args.profile_case:
         wl = synth.workload(args.workload, n_layers=1)
         args.no_by_ctx, args.no_cpu_baseline = True, True
