@@ -391,7 +391,8 @@ qsa_status qsa_cp_select(const float* cand_scores, const int32_t* cand_blocks, i
                          int32_t* sel_blocks, int32_t* n_sel, qsa_stream_t stream);
 
 /* The shard's attention partial: over the blocks of the global selection (sel_blocks,
- * n_sel from qsa_cp_select) that fall in [block_base, block_base + n_ctx/4), plus the
+ * n_sel from qsa_cp_select, so in ascending order; other orders are not supported) that
+ * fall in [block_base, block_base + n_ctx/4), plus the
  * shard's own open tail (the last shard's), like qsa_sparse_attend_selected:
  *   out [n_q_heads][head_dim] f32: the normalised output over those cells;
  *   lse [n_q_heads] f32: log sum_c exp(q_i . K[c] / sqrt(head_dim)); -inf and out = 0 when

@@ -60,15 +60,20 @@ __device__ __forceinline__ uint32_t cp_exclusive_scan(uint32_t v, uint32_t* s_wa
 // The global top-K of n_slots = shards * K candidate slots (scores, global block ids; a slot
 // with block id -1 is empty), listed shard by shard, each shard's in ascending block order.
 // Rule: the K largest scores, ties to the lower block, output ascending; fewer than K
-// candidates: all of them. Thread t holds slots [8t, 8t + 8), so slot order is thread order.
-// A 2048-bin histogram of the keys' top 11 bits gives the bin of the K-th key; radix passes
-// over the remaining 21 bits (8, 8, 5) refine inside it, warp 0 scanning each pass's
-// digit counts; one packed prefix scan places every selected slot.
-__global__ void __launch_bounds__(kCpThreads) cp_select_kernel(const float* __restrict__ cand_scores,
-                                                               const int32_t* __restrict__ cand_blocks,
-                                                               int n_slots, int k_blocks, int32_t* __restrict__ sel,
-                                                               int32_t* __restrict__ n_sel) {
+// candidates: all of them. Thread t holds slots [8t, 8t + 8), so slot order is thread order;
+// T threads take up to 8T slots (T = 256 up to 2048 slots: the CTA-wide barriers and
+// scans of a smaller CTA are cheaper). A 2048-bin histogram of the keys' top 11 bits gives
+// the bin of the K-th key; radix passes over the remaining 21 bits (8, 8, 5) refine inside
+// it, warp 0 scanning each pass's digit counts; one packed prefix scan places every
+// selected slot.
+template <int T>
+__global__ void __launch_bounds__(T) cp_select_kernel(const float* __restrict__ cand_scores,
+                                                      const int32_t* __restrict__ cand_blocks, int n_slots,
+                                                      int k_blocks, int32_t* __restrict__ sel,
+                                                      int32_t* __restrict__ n_sel) {
   constexpr int kHB = 2048;
+  constexpr int kBinsPer = kHB / T;  // histogram bins per thread, from the top
+  static_assert(kBinsPer * T == kHB && T >= 256, "whole bins per thread; 256 digit bins per pass");
   __shared__ uint32_t s_h[kHB];
   __shared__ uint32_t s_warp[33];
   __shared__ uint32_t s_ctl[4];
@@ -85,27 +90,35 @@ __global__ void __launch_bounds__(kCpThreads) cp_select_kernel(const float* __re
     key[j] = i < n_slots ? sel::score_key(cand_scores[i]) : 0u;
     if (blk[j] >= 0) valid |= 1u << j;
   }
-  for (int i = tid; i < kHB; i += kCpThreads) s_h[i] = 0u;
+  for (int i = tid; i < kHB; i += T) s_h[i] = 0u;
   __syncthreads();
 #pragma unroll
   for (int j = 0; j < kCpPer; ++j)
     if ((valid >> j) & 1u) atomicAdd(&s_h[key[j] >> 21], 1u);
   __syncthreads();
-  // thread t holds bins 2047 - 2t and 2046 - 2t (from the top); keys above them come first
-  const uint32_t h0 = s_h[kHB - 1 - 2 * tid], h1 = s_h[kHB - 2 - 2 * tid];
+  // thread t holds bins 2047 - kBinsPer*t - q, q < kBinsPer (from the top); keys above
+  // them come first
+  uint32_t hb[kBinsPer], hsum = 0;
+#pragma unroll
+  for (int q = 0; q < kBinsPer; ++q) {
+    hb[q] = s_h[kHB - 1 - kBinsPer * tid - q];
+    hsum += hb[q];
+  }
   uint32_t total;
-  const uint32_t above = cp_exclusive_scan(h0 + h1, s_warp, &total);
+  const uint32_t above = cp_exclusive_scan(hsum, s_warp, &total);
   uint32_t prefix = 0, mask = 0, need = uint32_t(k_blocks);
   const bool all = total <= uint32_t(k_blocks);  // uniform
   if (all) {
     need = total;  // mask 0: every valid slot is "at the threshold" and taken
   } else {
-    if (above < need && above + h0 >= need) {
-      s_ctl[0] = uint32_t(kHB - 1 - 2 * tid);
-      s_ctl[1] = above;
-    } else if (above + h0 < need && above + h0 + h1 >= need) {
-      s_ctl[0] = uint32_t(kHB - 2 - 2 * tid);
-      s_ctl[1] = above + h0;
+    uint32_t acc = above;
+#pragma unroll
+    for (int q = 0; q < kBinsPer; ++q) {
+      if (acc < need && acc + hb[q] >= need) {
+        s_ctl[0] = uint32_t(kHB - 1 - kBinsPer * tid - q);
+        s_ctl[1] = acc;
+      }
+      acc += hb[q];
     }
     __syncthreads();
     prefix = s_ctl[0] << 21;
@@ -186,13 +199,14 @@ __global__ void __launch_bounds__(kCpThreads) cp_select_kernel(const float* __re
 
 // The blocks of the global selection that belong to this shard ([block_base,
 // block_base + n_ctx/4) of the global numbering), as local ids in ascending order, and
-// their count; the shard's attention reads them like its own selection.
+// their count; the shard's attention reads them like its own selection. The global
+// selection is ascending and the shard's blocks contiguous, so its entries are one run of
+// the list: an entry's position is its index less the count of entries below the shard.
 __global__ void __launch_bounds__(kCpThreads) cp_filter_kernel(DevState* st, const int32_t* __restrict__ sel_global,
                                                                const int32_t* __restrict__ n_sel_global,
                                                                int block_base, int k_blocks,
                                                                int32_t* __restrict__ sel_local,
                                                                int32_t* __restrict__ n_local) {
-  __shared__ uint32_t s_warp[33];
   const int tid = threadIdx.x;
   pdl_launch_dependents();
   pdl_wait();
@@ -200,15 +214,16 @@ __global__ void __launch_bounds__(kCpThreads) cp_filter_kernel(DevState* st, con
   int ns = *n_sel_global;
   ns = ns < 0 ? 0 : (ns > k_blocks ? k_blocks : ns);
   int b = -1;
-  bool keep = false;
+  bool keep = false, below = false;
   if (tid < ns) {
     b = sel_global[tid] - block_base;
     keep = b >= 0 && b < nb;
+    below = b < 0;
   }
-  uint32_t total;
-  const uint32_t pos = cp_exclusive_scan(keep ? 1u : 0u, s_warp, &total);
-  if (keep) sel_local[pos] = b;
-  if (tid == 0) *n_local = int32_t(total);
+  const int lo = __syncthreads_count(below);
+  const int total = __syncthreads_count(keep);
+  if (keep && tid - lo < k_blocks) sel_local[tid - lo] = b;
+  if (tid == 0) *n_local = total;
 }
 
 // out[i] = sum_r w_r o_r[i] / sum_r w_r, w_r = exp(lse_r[i] - max_r lse_r[i]) over the
@@ -238,13 +253,20 @@ __global__ void __launch_bounds__(128) cp_merge_kernel(const float* __restrict__
 
 cudaError_t launch_cp_select(const float* cand_scores, const int32_t* cand_blocks, int n_shards, int k_blocks,
                              int32_t* sel, int32_t* n_sel, cudaStream_t s) {
-  return launch_pdl(cp_select_kernel, dim3(1), dim3(kCpThreads), 0, s, 1, cand_scores, cand_blocks,
-                    n_shards * k_blocks, k_blocks, sel, n_sel);
+  const int n_slots = n_shards * k_blocks;
+  if (n_slots <= 256 * kCpPer)
+    return launch_pdl(cp_select_kernel<256>, dim3(1), dim3(256), 0, s, 1, cand_scores, cand_blocks, n_slots,
+                      k_blocks, sel, n_sel);
+  return launch_pdl(cp_select_kernel<kCpThreads>, dim3(1), dim3(kCpThreads), 0, s, 1, cand_scores, cand_blocks,
+                    n_slots, k_blocks, sel, n_sel);
 }
 
 cudaError_t launch_cp_filter(const LayerView& L, const int32_t* sel_global, const int32_t* n_sel_global,
                              int block_base, int32_t* sel_local, int32_t* n_local, cudaStream_t s) {
-  return launch_pdl(cp_filter_kernel, dim3(1), dim3(kCpThreads), 0, s, 1, L.state, sel_global, n_sel_global,
+  // one thread per entry of the global selection (k_blocks <= kCpThreads)
+  const int kb = L.cfg.top_k_tokens / kBlock;
+  const int threads = kb >= kCpThreads ? kCpThreads : (kb + 31) / 32 * 32;
+  return launch_pdl(cp_filter_kernel, dim3(1), dim3(threads), 0, s, 1, L.state, sel_global, n_sel_global,
                     block_base, L.cfg.top_k_tokens / kBlock, sel_local, n_local);
 }
 
