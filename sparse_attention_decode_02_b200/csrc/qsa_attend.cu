@@ -429,7 +429,7 @@ attn_cluster_kernel(DevState* st, const __half* __restrict__ q, const int32_t* _
   __half* sV = reinterpret_cast<__half*>(smem + SM::v_off(Lc));
   __half* sP = reinterpret_cast<__half*>(smem + SM::p_off(Lc));
   float* s_o = reinterpret_cast<float*>(smem + SM::o_off(Lc));
-  float* s_rmax = reinterpret_cast<float*>(smem + SM::red_off(Lc));   // [16 warps][8 rows]
+  float* s_rmax = reinterpret_cast<float*>(smem + SM::red_off(Lc));   // [16 warps][8 query heads]
   float* s_rsum = s_rmax + 16 * 8;
   float* s_m = reinterpret_cast<float*>(smem + SM::ml_off(Lc));       // [G], then s_l [G]
   float* s_l = s_m + G;
@@ -442,7 +442,9 @@ attn_cluster_kernel(DevState* st, const __half* __restrict__ q, const int32_t* _
   const int rank = int(cluster.block_rank());
   const int g = blockIdx.x / CS;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int gq = lane >> 2, tq = lane & 3;  // MMA fragment row (query head) and column pair
+  // m16n8k16 fragment coordinates: group gq (row gq and gq + 8 of A and D, column gq of B)
+  // and thread tq in the group (columns 2tq, 2tq + 1 of D)
+  const int gq = lane >> 2, tq = lane & 3;
   const int u = blockIdx.y, n_back = gridDim.y - 1 - blockIdx.y;
   q += size_t(u) * n_kv_heads * G * D;
   out += size_t(u) * n_kv_heads * G * D;
